@@ -1,0 +1,194 @@
+/*
+ * s4r.h -- C ABI of libs4r: S4R compressed-KV decode on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of "S^4R: Selective Sampling, Subspaces, and
+ * Sparse Reconstruction for Compressed Long-Context KV Caching"
+ * (arXiv 2608.00528), as its review page on pith.science states them:
+ *   - every non-sink token is stored as rank-r coefficients c = s . B
+ *     ("What carries the argument", Eq. 3);
+ *   - a decode step projects a sliding window of queries into the key basis,
+ *     scores every cached key coefficient in latent space with a softmax
+ *     (major comment 2, §3.2.2, Eqs. 8-10), keeps the local window plus the
+ *     top-k earlier positions (Eqs. 13-15), rebuilds only those rows from
+ *     their coefficients and runs exact attention together with the
+ *     uncompressed sink tokens (Eqs. 16-18).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers unless a comment says "host".
+ *     Every device pointer must be 16-byte aligned.
+ *   - The caller owns every buffer.  The library allocates no device memory,
+ *     keeps no per-call state between calls and may be called from several
+ *     host threads on different streams (each call with its own workspace).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work; none synchronises, except
+ *     s4r_read_device_status.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned as S4R_ERR_INVALID_ARG / S4R_ERR_UNSUPPORTED /
+ *     S4R_ERR_WORKSPACE.  A failed launch returns S4R_ERR_CUDA.  Conditions
+ *     only the device can see (a full cache on append, a length beyond the
+ *     cache capacity, a bounded wait that gave up) set a sticky status word
+ *     in the workspace, which s4r_read_device_status returns; the kernels
+ *     then skip the offending work instead of touching memory out of bounds.
+ *
+ * Layouts (row-major, innermost index last).  D' = n_heads_kv * head_dim,
+ * G = n_heads_q / n_heads_kv; query head h belongs to kv group g = h / G and
+ * uses columns g*head_dim .. (g+1)*head_dim-1 of D'.  Coefficient row i of a
+ * problem stores absolute token position n_sink + i; the first n_sink tokens
+ * are the uncompressed sinks.
+ */
+#ifndef S4R_H
+#define S4R_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  S4R_OK = 0,
+  S4R_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, inconsistent shape */
+  S4R_ERR_UNSUPPORTED = 2,  /* valid request outside the supported range */
+  S4R_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  S4R_ERR_TIMEOUT = 4,      /* device status: a bounded device-side wait gave up */
+  S4R_ERR_DEVICE = 5,       /* device status: a device-side check failed */
+  S4R_ERR_WORKSPACE = 6     /* workspace pointer null or smaller than required */
+} s4r_status;
+
+typedef enum { S4R_F32 = 0, S4R_BF16 = 1 } s4r_dtype;
+
+/* How the query window forms scoring rows (Eqs. 8-10).
+ * CONCAT (default): W*G rows; row (w, j) concatenates query head g*G + j of
+ *   every kv group g into one D'-vector, projected with the whole key basis.
+ * PER_HEAD: W*H_q rows; row (w, h) projects query head h with the head_dim
+ *   rows of the key basis that belong to its kv group. */
+typedef enum { S4R_ROWS_CONCAT = 0, S4R_ROWS_PER_HEAD = 1 } s4r_row_mode;
+
+/* Supported range (S4R_ERR_UNSUPPORTED outside it). */
+#define S4R_MAX_D_MODEL 1024    /* D' */
+#define S4R_MAX_RANK 256        /* rank_k, rank_v; multiples of 8 */
+#define S4R_MAX_HEAD_DIM 256    /* multiple of 8 */
+#define S4R_MAX_SCORE_ROWS 256  /* W*G (CONCAT) or W*H_q (PER_HEAD) */
+#define S4R_MAX_POOL_KERNEL 63  /* odd */
+
+/* ------------------------------------------------------------------ encode */
+
+/* Encode token states into coefficients, C = S . B ("What carries the
+ * argument", Eq. 3): coeffs[t][j] = sum_d states[t][d] * basis[d][j].
+ *   states  [n_tokens][d_model], row stride states_ld elements (>= d_model)
+ *   basis   [d_model][rank], contiguous
+ *   coeffs  [n_tokens][rank], row stride coeffs_ld elements (>= rank)
+ * All three have type `dtype`; accumulation is fp32 and the result is
+ * rounded to `dtype` (round to nearest even).  n_tokens == 0 is a no-op.
+ * Strides must keep every row 16-byte aligned. */
+s4r_status s4r_encode(const void *states, int64_t n_tokens, int64_t states_ld,
+                      const void *basis, int32_t d_model, int32_t rank,
+                      void *coeffs, int64_t coeffs_ld, s4r_dtype dtype, void *stream);
+
+/* Append one new token per problem to the coefficient caches (Eq. 3 applied
+ * to the token a decode step adds).  For each problem b, with n = lengths[b]
+ * read on the device:
+ *   coeff_k[b][n] = state_k[b] . basis_k[b],  coeff_v[b][n] = state_v[b] . basis_v[b],
+ *   then lengths[b] = n + 1.
+ * If n >= cache_rows the problem is skipped and the device status
+ * (S4R_ERR_DEVICE) is set in `status_workspace` (may be NULL: skip only). */
+typedef struct {
+  int32_t batch, d_model, rank_k, rank_v;
+  s4r_dtype dtype;
+  int64_t cache_rows;                 /* row capacity of each problem's caches */
+  const void *state_k, *state_v;      /* [batch][d_model] */
+  const void *basis_k, *basis_v;      /* [batch][d_model][rank] */
+  void *coeff_k, *coeff_v;            /* [batch][cache_rows][rank] */
+  int32_t *lengths;                   /* [batch] device, read and incremented */
+  void *status_workspace;             /* a decode workspace (its status word), or NULL */
+} s4r_append_args;
+
+s4r_status s4r_append(const s4r_append_args *args, void *stream);
+
+/* ------------------------------------------------------------------ decode */
+
+typedef struct {
+  int32_t batch;                      /* independent (sequence, layer) problems */
+  int32_t n_heads_q, n_heads_kv, head_dim;
+  int32_t rank_k, rank_v;
+  int32_t n_sink;                     /* s: uncompressed sink tokens per problem */
+  int32_t local_window;               /* w: newest coefficient rows always kept */
+  int32_t top_k;                      /* k: global positions chosen before the window */
+  int32_t query_window;               /* W: query rows scored per step */
+  int32_t pool_kernel;                /* 1 = off; odd kappa = max-pool of candidate scores */
+  int32_t row_mode;                   /* s4r_row_mode */
+  s4r_dtype dtype;                    /* storage type of q, coefficients, bases, sinks */
+  int64_t cache_rows;                 /* row capacity (stride) of the coefficient caches */
+  const int32_t *lengths;             /* [batch] device: L_c, coefficient rows in use */
+  const void *q;                      /* [batch][W][H_q][head_dim]; slot W-1 = current query */
+  const void *coeff_k, *coeff_v;      /* [batch][cache_rows][rank_k | rank_v] */
+  const void *basis_k, *basis_v;      /* [batch][D'][rank_k | rank_v] */
+  const void *sink_k, *sink_v;        /* [batch][n_sink][D'] */
+  float *out;                         /* [batch][H_q][head_dim] attention output */
+  int32_t *idx;                       /* [batch][top_k] chosen absolute positions,
+                                         ascending, -1 padded (window not listed) */
+  float *scores;                      /* optional [batch][cache_rows] latent scores, or NULL */
+  void *workspace;                    /* device scratch, see s4r_decode_workspace_bytes */
+  size_t workspace_bytes;
+  void *profile_events[2];            /* optional cudaEvent_t pair (or NULL): recorded on
+                                         `stream` right before and right after the
+                                         latent-scoring kernels, for timing them */
+} s4r_decode_args;
+
+/* Bytes of device workspace s4r_decode_step needs for these arguments (only
+ * the shape fields are read).  Returns 0 if the shape is invalid. */
+size_t s4r_decode_workspace_bytes(const s4r_decode_args *args);
+
+/* Number of kernel launches one s4r_decode_step with these arguments
+ * enqueues (0 if the shape is invalid). */
+int32_t s4r_decode_kernel_launches(const s4r_decode_args *args);
+
+/* Prepare a freshly allocated workspace (clears its status word and the
+ * counters that the kernels reuse).  Call once per workspace allocation. */
+s4r_status s4r_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* One decode step for every problem of the batch:
+ *   1. C_Q = Q' . B^K for the query window (rows per row_mode);
+ *   2. Z = C_Q . C_K^T / sqrt(rank_k), softmax of every row over the L_c
+ *      coefficient rows, score[i] = sum of the rows' probabilities (Eqs. 8-10);
+ *   3. idx = the top_k rows among 0 .. L_c-w-1 by score (max-pooled when
+ *      pool_kernel > 1), equal scores -> lower position (Eqs. 13-15);
+ *   4. for every query head h, exact attention of q[W-1][h] over the sinks,
+ *      the chosen rows and the last w rows, with keys c_K . B^K^T and values
+ *      c_V . B^V^T restricted to the head's kv group, logits scaled by
+ *      1/sqrt(head_dim) (Eqs. 16-18).  Rebuilt rows are kept in fp32.
+ * Arithmetic is fp32 whatever the storage type. */
+s4r_status s4r_decode_step(const s4r_decode_args *args, void *stream);
+
+/* ----------------------------------------------------------- reconstruct */
+
+/* Rebuild selected rows from coefficients, out[e][d] = sum_j coeffs[rows[e]][j]
+ * * basis[d][j] (Eq. 16).  coeffs [n_rows_total][rank] and basis
+ * [d_model][rank] have type `dtype`; rows [n] device int32 row numbers (a
+ * row < 0 or >= n_rows_total yields a zero output row); out [n][d_model]
+ * fp32. */
+s4r_status s4r_reconstruct(const void *coeffs, int64_t n_rows_total, const void *basis,
+                           int32_t d_model, int32_t rank, const int32_t *rows, int64_t n,
+                           float *out, s4r_dtype dtype, void *stream);
+
+/* ------------------------------------------------------------------ status */
+
+/* Synchronise `stream`, then return the sticky device status of `workspace`
+ * (S4R_OK, S4R_ERR_TIMEOUT or S4R_ERR_DEVICE); S4R_ERR_CUDA if the
+ * synchronisation itself failed. */
+s4r_status s4r_read_device_status(const void *workspace, void *stream);
+
+/* Reset the device status word of `workspace` (stream-ordered). */
+s4r_status s4r_clear_device_status(void *workspace, void *stream);
+
+/* Static description of a status code. */
+const char *s4r_status_string(s4r_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t s4r_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* S4R_H */

@@ -1,0 +1,309 @@
+// s4r_api.cu -- the C ABI of libs4r (declared in include/s4r.h): host-side
+// validation, workspace layout and kernel launches.  Every step of the decode
+// and encode paths runs in the kernels included below; the host only checks
+// arguments and enqueues launches on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "k_attend.cuh"
+#include "k_encode_simt.cuh"
+#include "k_project.cuh"
+#include "k_score_simt.cuh"
+#include "k_topk.cuh"
+
+using namespace s4r;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t esize(s4r_dtype dt) { return dt == S4R_BF16 ? 2 : 4; }
+
+// Byte offsets of the decode workspace regions.
+struct Layout {
+  size_t status, cq, qt, tstat, rstat, scores, pooled, part, total;
+};
+
+Layout layout_for(const Shape &s) {
+  Layout l{};
+  size_t off = 0;
+  l.status = off; off += kAlign;
+  l.cq = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_rows * s.rank_k);
+  l.qt = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * s.rank_k);
+  const size_t n_tiles = (size_t)ceil_div(s.cache_rows, kScoreTile);
+  l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
+  l.rstat = off; off += round_up(sizeof(double) * 2 * s.batch * (size_t)s.n_rows);
+  l.scores = off; off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
+  l.pooled = off; if (s.pool_kernel > 1) off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
+  l.part = off;
+  off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * att_splits(s) * (s.rank_v + 2));
+  l.total = off;
+  return l;
+}
+
+// Shape checks shared by workspace sizing and the decode step.
+s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
+  if (!a) return S4R_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->n_heads_q <= 0 || a->n_heads_kv <= 0 || a->head_dim <= 0 ||
+      a->rank_k <= 0 || a->rank_v <= 0 || a->n_sink < 0 || a->local_window < 0 ||
+      a->top_k < 0 || a->query_window <= 0 || a->pool_kernel < 1 || a->cache_rows < 0)
+    return S4R_ERR_INVALID_ARG;
+  if (a->n_heads_q % a->n_heads_kv != 0) return S4R_ERR_INVALID_ARG;
+  if (a->dtype != S4R_F32 && a->dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
+  if (a->row_mode != S4R_ROWS_CONCAT && a->row_mode != S4R_ROWS_PER_HEAD) return S4R_ERR_INVALID_ARG;
+  if (a->pool_kernel % 2 == 0) return S4R_ERR_INVALID_ARG;
+  const int64_t G = a->n_heads_q / a->n_heads_kv;
+  const int64_t Dp = (int64_t)a->n_heads_kv * a->head_dim;
+  const int64_t R = (a->row_mode == S4R_ROWS_CONCAT) ? (int64_t)a->query_window * G
+                                                    : (int64_t)a->query_window * a->n_heads_q;
+  if (a->head_dim % 8 || a->rank_k % 8 || a->rank_v % 8) return S4R_ERR_UNSUPPORTED;
+  if (a->head_dim > S4R_MAX_HEAD_DIM || Dp > S4R_MAX_D_MODEL || a->rank_k > S4R_MAX_RANK ||
+      a->rank_v > S4R_MAX_RANK || R > S4R_MAX_SCORE_ROWS || G > kAttMaxGroup ||
+      a->pool_kernel > S4R_MAX_POOL_KERNEL)
+    return S4R_ERR_UNSUPPORTED;
+  if (a->cache_rows + a->n_sink > INT32_MAX) return S4R_ERR_UNSUPPORTED;
+  s->batch = a->batch;
+  s->n_heads_q = a->n_heads_q;
+  s->n_heads_kv = a->n_heads_kv;
+  s->head_dim = a->head_dim;
+  s->rank_k = a->rank_k;
+  s->rank_v = a->rank_v;
+  s->n_sink = a->n_sink;
+  s->local_window = a->local_window;
+  s->top_k = a->top_k;
+  s->query_window = a->query_window;
+  s->pool_kernel = a->pool_kernel;
+  s->row_mode = a->row_mode;
+  s->d_model = (int32_t)Dp;
+  s->group = (int32_t)G;
+  s->n_rows = (int32_t)R;
+  s->cache_rows = a->cache_rows;
+  return S4R_OK;
+}
+
+s4r_status last_cuda() { return cudaGetLastError() == cudaSuccess ? S4R_OK : S4R_ERR_CUDA; }
+
+template <typename T>
+s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout &ly, cudaStream_t st) {
+  unsigned char *ws = static_cast<unsigned char *>(a->workspace);
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws + ly.status);
+  float *cq = reinterpret_cast<float *>(ws + ly.cq);
+  float *qt = reinterpret_cast<float *>(ws + ly.qt);
+  double *tstat = reinterpret_cast<double *>(ws + ly.tstat);
+  double *rstat = reinterpret_cast<double *>(ws + ly.rstat);
+  float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
+  float *pooled = reinterpret_cast<float *>(ws + ly.pooled);
+  float *part = reinterpret_cast<float *>(ws + ly.part);
+  const T *q = static_cast<const T *>(a->q);
+  const T *ck = static_cast<const T *>(a->coeff_k);
+  const T *cv = static_cast<const T *>(a->coeff_v);
+  const T *bk = static_cast<const T *>(a->basis_k);
+  const T *bv = static_cast<const T *>(a->basis_v);
+  const T *sk = static_cast<const T *>(a->sink_k);
+  const T *sv = static_cast<const T *>(a->sink_v);
+
+  // 1. query projection
+  {
+    dim3 grid((unsigned)ceil_div(s.n_rows + s.n_heads_q, kProjRows),
+              (unsigned)ceil_div(s.rank_k, kProjCols), (unsigned)s.batch);
+    project_kernel<T><<<grid, kProjRows * kProjCols, 0, st>>>(s, q, bk, cq, qt);
+  }
+  // 2. latent scoring
+  const unsigned n_tiles = (unsigned)ceil_div(s.cache_rows, kScoreTile);
+  if (a->profile_events[0]) cudaEventRecord(static_cast<cudaEvent_t>(a->profile_events[0]), st);
+  if (n_tiles > 0) {
+    const size_t smem = ScoreSmem::bytes(s.rank_k);
+    cudaFuncSetAttribute(score_stats_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(score_final_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    score_stats_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, tstat);
+    score_merge<<<dim3((unsigned)ceil_div(s.n_rows, 8), s.batch), 256, 0, st>>>(s, a->lengths, tstat, rstat);
+    score_final_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, rstat, scores);
+  }
+  if (a->profile_events[1]) cudaEventRecord(static_cast<cudaEvent_t>(a->profile_events[1]), st);
+  // 3. selection
+  const float *keys = scores;
+  if (s.pool_kernel > 1 && s.cache_rows > 0) {
+    pool_kernel<<<dim3((unsigned)ceil_div(s.cache_rows, 256), s.batch), 256, 0, st>>>(s, a->lengths, scores, pooled);
+    keys = pooled;
+  }
+  if (s.top_k > 0)
+    topk_kernel<<<s.batch, kTopkThreads, 0, st>>>(s, a->lengths, keys, a->idx, status);
+  // 4. rebuild + exact attention
+  {
+    const int n_split = att_splits(s);
+    attend_partial<T><<<dim3(n_split, s.n_heads_kv, s.batch), kAttThreads, 0, st>>>(
+        s, a->lengths, a->idx, ck, cv, qt, part);
+    const size_t smem = sizeof(float) * (s.rank_v + s.n_sink + 1);
+    attend_combine<T><<<dim3(s.n_heads_q, s.batch), 256, smem, st>>>(s, q, bv, sk, sv, part, a->out);
+  }
+  return last_cuda();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t s4r_decode_workspace_bytes(const s4r_decode_args *args) {
+  Shape s;
+  if (make_shape(args, &s) != S4R_OK) return 0;
+  return layout_for(s).total;
+}
+
+int32_t s4r_decode_kernel_launches(const s4r_decode_args *args) {
+  Shape s;
+  if (make_shape(args, &s) != S4R_OK) return 0;
+  if (s.batch == 0) return 0;
+  int32_t n = 1;                                  // projection
+  if (s.cache_rows > 0) n += 3;                   // scoring: stats, merge, final
+  if (s.pool_kernel > 1 && s.cache_rows > 0) n += 1;
+  if (s.top_k > 0) n += 1;
+  n += 2;                                         // attention: partial, combine
+  return n;
+}
+
+s4r_status s4r_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+  if (!workspace || workspace_bytes < kAlign || !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, kAlign, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return S4R_ERR_CUDA;
+  return S4R_OK;
+}
+
+s4r_status s4r_decode_step(const s4r_decode_args *a, void *stream) {
+  Shape s;
+  const s4r_status rc = make_shape(a, &s);
+  if (rc != S4R_OK) return rc;
+  if (s.batch == 0) return S4R_OK;
+  const void *must[] = {a->lengths, a->q, a->coeff_k, a->coeff_v, a->basis_k, a->basis_v, a->out};
+  for (const void *p : must)
+    if (!p || !aligned16(p)) return S4R_ERR_INVALID_ARG;
+  if (s.top_k > 0 && (!a->idx || !aligned16(a->idx))) return S4R_ERR_INVALID_ARG;
+  if (s.n_sink > 0 && (!a->sink_k || !a->sink_v || !aligned16(a->sink_k) || !aligned16(a->sink_v)))
+    return S4R_ERR_INVALID_ARG;
+  if (a->scores && !aligned16(a->scores)) return S4R_ERR_INVALID_ARG;
+  const Layout ly = layout_for(s);
+  if (!a->workspace || !aligned16(a->workspace) || a->workspace_bytes < ly.total) return S4R_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return a->dtype == S4R_BF16 ? decode_launch<bf16>(a, s, ly, st) : decode_launch<float>(a, s, ly, st);
+}
+
+s4r_status s4r_encode(const void *states, int64_t n_tokens, int64_t states_ld, const void *basis,
+                      int32_t d_model, int32_t rank, void *coeffs, int64_t coeffs_ld,
+                      s4r_dtype dtype, void *stream) {
+  if (dtype != S4R_F32 && dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
+  if (n_tokens < 0 || d_model <= 0 || rank <= 0 || states_ld < d_model || coeffs_ld < rank)
+    return S4R_ERR_INVALID_ARG;
+  if (n_tokens == 0) return S4R_OK;
+  if (!states || !basis || !coeffs || !aligned16(states) || !aligned16(basis) || !aligned16(coeffs))
+    return S4R_ERR_INVALID_ARG;
+  const size_t e = esize(dtype);
+  if ((states_ld * e) % 16 || (coeffs_ld * e) % 16 || ((int64_t)rank * e) % 16) return S4R_ERR_INVALID_ARG;
+  if (d_model > S4R_MAX_D_MODEL || rank > S4R_MAX_RANK) return S4R_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((unsigned)ceil_div(n_tokens, kEncTileM), (unsigned)ceil_div(rank, kEncTileN));
+  if (dtype == S4R_BF16)
+    encode_simt<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16 *>(states), n_tokens, states_ld,
+                                            static_cast<const bf16 *>(basis), d_model, rank,
+                                            static_cast<bf16 *>(coeffs), coeffs_ld);
+  else
+    encode_simt<float><<<grid, 256, 0, st>>>(static_cast<const float *>(states), n_tokens, states_ld,
+                                             static_cast<const float *>(basis), d_model, rank,
+                                             static_cast<float *>(coeffs), coeffs_ld);
+  return last_cuda();
+}
+
+s4r_status s4r_append(const s4r_append_args *a, void *stream) {
+  if (!a) return S4R_ERR_INVALID_ARG;
+  if (a->dtype != S4R_F32 && a->dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->d_model <= 0 || a->rank_k <= 0 || a->rank_v <= 0 || a->cache_rows < 0)
+    return S4R_ERR_INVALID_ARG;
+  if (a->batch == 0) return S4R_OK;
+  const void *must[] = {a->state_k, a->state_v, a->basis_k, a->basis_v, a->coeff_k, a->coeff_v, a->lengths};
+  for (const void *p : must)
+    if (!p || !aligned16(p)) return S4R_ERR_INVALID_ARG;
+  if (a->status_workspace && !aligned16(a->status_workspace)) return S4R_ERR_INVALID_ARG;
+  if (a->rank_k % 8 || a->rank_v % 8 || a->d_model % 8) return S4R_ERR_UNSUPPORTED;
+  if (a->d_model > S4R_MAX_D_MODEL || a->rank_k > S4R_MAX_RANK || a->rank_v > S4R_MAX_RANK)
+    return S4R_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = static_cast<uint32_t *>(a->status_workspace);
+  dim3 grid(a->batch, 2);
+  if (a->dtype == S4R_BF16)
+    append_kernel<bf16><<<grid, 256, 0, st>>>(
+        a->d_model, a->rank_k, a->rank_v, a->cache_rows, static_cast<const bf16 *>(a->state_k),
+        static_cast<const bf16 *>(a->state_v), static_cast<const bf16 *>(a->basis_k),
+        static_cast<const bf16 *>(a->basis_v), static_cast<bf16 *>(a->coeff_k),
+        static_cast<bf16 *>(a->coeff_v), a->lengths, status);
+  else
+    append_kernel<float><<<grid, 256, 0, st>>>(
+        a->d_model, a->rank_k, a->rank_v, a->cache_rows, static_cast<const float *>(a->state_k),
+        static_cast<const float *>(a->state_v), static_cast<const float *>(a->basis_k),
+        static_cast<const float *>(a->basis_v), static_cast<float *>(a->coeff_k),
+        static_cast<float *>(a->coeff_v), a->lengths, status);
+  append_bump_lengths<<<(unsigned)ceil_div(a->batch, 256), 256, 0, st>>>(a->batch, a->cache_rows, a->lengths);
+  return last_cuda();
+}
+
+s4r_status s4r_reconstruct(const void *coeffs, int64_t n_rows_total, const void *basis,
+                           int32_t d_model, int32_t rank, const int32_t *rows, int64_t n,
+                           float *out, s4r_dtype dtype, void *stream) {
+  if (dtype != S4R_F32 && dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
+  if (n < 0 || n_rows_total < 0 || d_model <= 0 || rank <= 0) return S4R_ERR_INVALID_ARG;
+  if (n == 0) return S4R_OK;
+  if (!coeffs || !basis || !rows || !out || !aligned16(coeffs) || !aligned16(basis) ||
+      !aligned16(rows) || !aligned16(out))
+    return S4R_ERR_INVALID_ARG;
+  if (rank % 8) return S4R_ERR_UNSUPPORTED;
+  if (d_model > S4R_MAX_D_MODEL || rank > S4R_MAX_RANK || n > INT32_MAX) return S4R_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((unsigned)n, (unsigned)ceil_div(d_model, 64));
+  if (dtype == S4R_BF16)
+    reconstruct_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16 *>(coeffs), n_rows_total,
+                                                   static_cast<const bf16 *>(basis), d_model, rank,
+                                                   rows, n, out);
+  else
+    reconstruct_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(coeffs), n_rows_total,
+                                                    static_cast<const float *>(basis), d_model, rank,
+                                                    rows, n, out);
+  return last_cuda();
+}
+
+s4r_status s4r_read_device_status(const void *workspace, void *stream) {
+  if (!workspace || !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return S4R_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return S4R_ERR_CUDA;
+  if (word & kDevStatusTimeout) return S4R_ERR_TIMEOUT;
+  if (word & kDevStatusCheck) return S4R_ERR_DEVICE;
+  return S4R_OK;
+}
+
+s4r_status s4r_clear_device_status(void *workspace, void *stream) {
+  if (!workspace || !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return S4R_ERR_CUDA;
+  return S4R_OK;
+}
+
+const char *s4r_status_string(s4r_status status) {
+  switch (status) {
+    case S4R_OK: return "ok";
+    case S4R_ERR_INVALID_ARG: return "invalid argument";
+    case S4R_ERR_UNSUPPORTED: return "unsupported shape";
+    case S4R_ERR_CUDA: return "CUDA error";
+    case S4R_ERR_TIMEOUT: return "device wait timed out";
+    case S4R_ERR_DEVICE: return "device-side check failed";
+    case S4R_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int32_t s4r_version(void) { return 100; }
+
+}  // extern "C"
