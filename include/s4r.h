@@ -133,7 +133,9 @@ typedef struct {
   size_t workspace_bytes;
   void *profile_events[2];            /* optional cudaEvent_t pair (or NULL): recorded on
                                          `stream` right before and right after the
-                                         latent-scoring kernels, for timing them */
+                                         latent-scoring kernels, for timing them; under
+                                         stream capture they become external event
+                                         record nodes of the graph */
 } s4r_decode_args;
 
 /* Bytes of device workspace s4r_decode_step needs for these arguments (only
@@ -176,10 +178,14 @@ s4r_status s4r_reconstruct(const void *coeffs, int64_t n_rows_total, const void 
 
 /* Synchronise `stream`, then return the sticky device status of `workspace`
  * (S4R_OK, S4R_ERR_TIMEOUT or S4R_ERR_DEVICE); S4R_ERR_CUDA if the
- * synchronisation itself failed. */
+ * synchronisation itself failed.  workspace == NULL reads the library-wide
+ * status of the current device, which the kernels that take no workspace
+ * (encode, reconstruct) report to. */
 s4r_status s4r_read_device_status(const void *workspace, void *stream);
 
-/* Reset the device status word of `workspace` (stream-ordered). */
+/* Reset the device status word of `workspace` (stream-ordered), or the
+ * library-wide word of the current device when workspace == NULL (this
+ * form synchronises `stream`). */
 s4r_status s4r_clear_device_status(void *workspace, void *stream);
 
 /* Static description of a status code. */

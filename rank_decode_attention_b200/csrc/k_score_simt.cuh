@@ -86,7 +86,7 @@ template <typename T>
 __global__ void __launch_bounds__(kScoreThreads)
 score_stats_simt(Shape s, const int32_t *__restrict__ lengths, const T *__restrict__ coeff_k,
                  const float *__restrict__ cq_all, double *__restrict__ tstat) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int b = blockIdx.y, r = s.rank_k;
   const int64_t L = lengths[b];
   const int64_t pos0 = (int64_t)blockIdx.x * kScoreTile;
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kScoreThreads)
 score_final_simt(Shape s, const int32_t *__restrict__ lengths, const T *__restrict__ coeff_k,
                  const float *__restrict__ cq_all, const double *__restrict__ rstat,
                  float *__restrict__ scores) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int b = blockIdx.y, r = s.rank_k;
   const int64_t L = lengths[b];
   const int64_t pos0 = (int64_t)blockIdx.x * kScoreTile;

@@ -2,6 +2,8 @@
 // validation, workspace layout and kernel launches.  Every step of the decode
 // and encode paths runs in the kernels included below; the host only checks
 // arguments and enqueues launches on the caller's stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -11,6 +13,7 @@
 #include "common.cuh"
 #include "k_attend.cuh"
 #include "k_encode_simt.cuh"
+#include "k_encode_tc.cuh"
 #include "k_project.cuh"
 #include "k_score_simt.cuh"
 #include "k_topk.cuh"
@@ -88,6 +91,48 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
 
 s4r_status last_cuda() { return cudaGetLastError() == cudaSuccess ? S4R_OK : S4R_ERR_CUDA; }
 
+// cuTensorMapEncodeTiled, resolved through the runtime (no link-time libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map, 128-byte swizzle: `inner` contiguous elements per row,
+// `outer` rows `row_bytes` apart, box of box_inner x box_outer elements.
+bool make_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core encode of bf16 states: requires rank % 32 == 0.
+s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const void *basis, int d, int r,
+                            void *coeffs, int64_t ldc, cudaStream_t st) {
+  CUtensorMap ms, mb;
+  if (!make_tmap_bf16(&ms, states, (uint64_t)d, (uint64_t)n, (uint64_t)lds * 2, kEncBK, kEncBM) ||
+      !make_tmap_bf16(&mb, basis, (uint64_t)r, (uint64_t)d, (uint64_t)r * 2, 64, kEncBK))
+    return S4R_ERR_CUDA;
+  const size_t smem = enc_smem_bytes(r);
+  cudaFuncSetAttribute(encode_tc_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  encode_tc_kernel<bf16><<<(unsigned)ceil_div(n, kEncBM), 128, smem, st>>>(ms, mb, static_cast<bf16 *>(coeffs),
+                                                                            ldc, n, d, r);
+  return last_cuda();
+}
+
 template <typename T>
 s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout &ly, cudaStream_t st) {
   unsigned char *ws = static_cast<unsigned char *>(a->workspace);
@@ -115,7 +160,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   }
   // 2. latent scoring
   const unsigned n_tiles = (unsigned)ceil_div(s.cache_rows, kScoreTile);
-  if (a->profile_events[0]) cudaEventRecord(static_cast<cudaEvent_t>(a->profile_events[0]), st);
+  if (a->profile_events[0])
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->profile_events[0]), st, cudaEventRecordExternal);
   if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
     cudaFuncSetAttribute(score_stats_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -124,7 +170,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     score_merge<<<dim3((unsigned)ceil_div(s.n_rows, 8), s.batch), 256, 0, st>>>(s, a->lengths, tstat, rstat);
     score_final_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, rstat, scores);
   }
-  if (a->profile_events[1]) cudaEventRecord(static_cast<cudaEvent_t>(a->profile_events[1]), st);
+  if (a->profile_events[1])
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->profile_events[1]), st, cudaEventRecordExternal);
   // 3. selection
   const float *keys = scores;
   if (s.pool_kernel > 1 && s.cache_rows > 0) {
@@ -204,6 +251,8 @@ s4r_status s4r_encode(const void *states, int64_t n_tokens, int64_t states_ld, c
   if ((states_ld * e) % 16 || (coeffs_ld * e) % 16 || ((int64_t)rank * e) % 16) return S4R_ERR_INVALID_ARG;
   if (d_model > S4R_MAX_D_MODEL || rank > S4R_MAX_RANK) return S4R_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == S4R_BF16 && rank % 32 == 0)
+    return encode_tc_launch(states, n_tokens, states_ld, basis, d_model, rank, coeffs, coeffs_ld, st);
   dim3 grid((unsigned)ceil_div(n_tokens, kEncTileM), (unsigned)ceil_div(rank, kEncTileN));
   if (dtype == S4R_BF16)
     encode_simt<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16 *>(states), n_tokens, states_ld,
@@ -273,11 +322,16 @@ s4r_status s4r_reconstruct(const void *coeffs, int64_t n_rows_total, const void 
 }
 
 s4r_status s4r_read_device_status(const void *workspace, void *stream) {
-  if (!workspace || !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
+  if (workspace && !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
   uint32_t word = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+  if (workspace) {
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return S4R_ERR_CUDA;
+  } else if (cudaMemcpyFromSymbolAsync(&word, g_device_status, sizeof(word), 0, cudaMemcpyDeviceToHost, st) !=
+             cudaSuccess) {
     return S4R_ERR_CUDA;
+  }
   if (cudaStreamSynchronize(st) != cudaSuccess) return S4R_ERR_CUDA;
   if (word & kDevStatusTimeout) return S4R_ERR_TIMEOUT;
   if (word & kDevStatusCheck) return S4R_ERR_DEVICE;
@@ -285,9 +339,17 @@ s4r_status s4r_read_device_status(const void *workspace, void *stream) {
 }
 
 s4r_status s4r_clear_device_status(void *workspace, void *stream) {
-  if (!workspace || !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return S4R_ERR_CUDA;
+  if (workspace && !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (workspace) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return S4R_ERR_CUDA;
+  } else {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) !=
+        cudaSuccess)
+      return S4R_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return S4R_ERR_CUDA;
+  }
   return S4R_OK;
 }
 

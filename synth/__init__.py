@@ -141,14 +141,21 @@ def sample_rows(L: int, n_sink: int, n_sample: int) -> torch.Tensor:
     return torch.cat([uniform, recent])
 
 
-def basis(X: torch.Tensor, rows: torch.Tensor, rank: int) -> torch.Tensor:
-    """Top-`rank` right singular vectors [D'][rank] of the unit-normalised sample."""
+def basis(X: torch.Tensor, rows: torch.Tensor, rank: int, gen: torch.Generator | None = None) -> torch.Tensor:
+    """Top-`rank` right singular vectors [D'][rank] of the unit-normalised sample.
+    A sample with fewer rows than `rank` (a very short prompt) is completed
+    with random orthonormal directions orthogonal to its span."""
     A = X[rows.to(X.device)]
     A = A / A.norm(dim=1, keepdim=True).clamp_min(1e-300)
     _, _, Vh = torch.linalg.svd(A, full_matrices=False)
-    if Vh.shape[0] < rank:
-        raise ValueError("sample smaller than the rank")
-    return Vh[:rank].T.contiguous()
+    V = Vh[:rank].T
+    if V.shape[1] < rank:
+        extra = torch.randn(V.shape[0], rank - V.shape[1], generator=gen, device=X.device,
+                            dtype=torch.float64)
+        extra -= V @ (V.T @ extra)
+        qm, rm = torch.linalg.qr(extra)
+        V = torch.cat([V, qm * torch.sign(torch.diagonal(rm)).unsqueeze(0)], dim=1)
+    return V.contiguous()
 
 
 def queries(n_rows: int, n_heads_q: int, head_dim: int, seed: int, device="cpu") -> torch.Tensor:
@@ -191,8 +198,8 @@ def problem_inputs(w: Workload, layer: int, seq: int, device="cpu", L: int | Non
     Xv = states(L, w.d_model, w.true_rank, w.n_sink, w.n_needles, w.needle_middle,
                 seed_of(*base, "v"), device)
     rows = sample_rows(L, w.n_sink, w.n_sample)
-    Bk = basis(Xk, rows, r)
-    Bv = basis(Xv, rows, r)
+    Bk = basis(Xk, rows, r, generator(seed_of(*base, "k-fill"), device))
+    Bv = basis(Xv, rows, r, generator(seed_of(*base, "v-fill"), device))
     nq = n_query_rows if n_query_rows is not None else w.steps + w.query_window - 1
     Q = queries(nq, w.n_heads_q, w.head_dim, seed_of(*base, "q"), device)
     return ProblemInputs(store(Xk, w.dtype), store(Xv, w.dtype), store(Bk, w.dtype),
