@@ -47,7 +47,8 @@ __device__ __forceinline__ float proj_input(const T *q, const Shape &s, int rho,
 template <typename T>
 __global__ void __launch_bounds__(kProjRows * kProjCols)
 project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k,
-               float *__restrict__ cq, float *__restrict__ qt) {
+               float *__restrict__ cq, float *__restrict__ qt, double *__restrict__ row_sum,
+               unsigned long long *__restrict__ barrier) {
   __shared__ float qs[kProjRows][kProjChunk + 1];
   __shared__ float bs[kProjChunk][kProjCols + 1];
   const int b = blockIdx.z;
@@ -57,6 +58,11 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k,
   const int r = s.rank_k, Dp = s.d_model;
   const T *qb = q + (int64_t)b * s.query_window * s.n_heads_q * s.head_dim;
   const T *Bb = basis_k + (int64_t)b * Dp * r;
+  // Reset the per-call accumulators of the tensor-core scoring kernel.
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    for (int e = threadIdx.x; e < s.n_rows; e += blockDim.x) row_sum[(int64_t)b * s.n_rows + e] = 0.0;
+    if (b == 0 && threadIdx.x == 0) *barrier = 0ull;
+  }
   double acc = 0.0;
   for (int d0 = 0; d0 < Dp; d0 += kProjChunk) {
     for (int e = threadIdx.x; e < kProjRows * kProjChunk; e += blockDim.x) {

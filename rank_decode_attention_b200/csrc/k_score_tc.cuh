@@ -1,0 +1,273 @@
+// k_score_tc.cuh -- latent relevance scoring on the tensor cores, one pass
+// over the key-coefficient cache.
+//
+// Eqs. 8-10 of S4R (review page, major comment 2, §3.2.2):
+//   z[i][row] = C_K[i] . C_Q[row] / sqrt(r),
+//   score[i]  = sum_row exp(z[i][row]) / sum_i' exp(z[i'][row]).
+//
+// Layout of the work: positions on the MMA's M (128 per tile, one TMEM lane
+// each), scoring rows on N.  C_K tiles are exact bf16, but C_Q is fp32: it is
+// split into three bf16 terms hi + mid + lo (24 significant bits) that sit
+// side by side on N (N = 3R), so each term is accumulated in its own TMEM
+// columns and the three are added in fp32 by the epilogue.  C_Q is scaled by
+// log2(e), so the epilogue works in base 2: e = 2^y with y = z log2(e).
+//
+// One cooperative launch, one CTA per pair of 128-position tiles of one
+// problem (4 warps; thread 0 issues TMA, thread 32 issues tcgen05.mma, all
+// warps run the epilogue):
+//   A. TMA both C_K tiles, build the split C_Q operand in shared memory,
+//      MMA each tile into its own 256-column TMEM region.
+//   B. per tile: y = hi + mid + lo, e = 2^y (kept in TMEM), per-row sums of e
+//      over the tile (fp64, fixed order) added atomically (fp64) into the
+//      problem's row normalisers.  A tile whose |y| exceeds 100 uses integer
+//      per-row offsets 2^(y - k) instead, so nothing overflows.
+//   C. one bounded grid barrier.
+//   D. alpha[row] = 2^k / l_row; score[i] = sum_row alpha[row] e[i][row].
+// The cache is read once; nothing but the scores and 2R doubles per problem
+// touches global memory.
+#pragma once
+#include "umma.cuh"
+
+namespace s4r {
+
+constexpr int kStcTile = 128;
+constexpr int kStcTiles = 2;          // tiles per CTA
+constexpr int kStcTmemCols = 512;
+constexpr int kStcTileCols = 256;     // TMEM columns per tile region
+constexpr float kStcRangeLimit = 100.f;
+
+__host__ __device__ constexpr int stc_kblocks(int r) { return (r + 63) / 64; }
+__host__ __device__ constexpr int stc_b_bytes(int R, int r) { return stc_kblocks(r) * 3 * R * 128; }
+__host__ __device__ constexpr int stc_a_bytes(int r) { return stc_kblocks(r) * kStcTile * 128; }
+__host__ __device__ constexpr int stc_red_bytes(int R) { return kStcTile * (R + 1) * 4; }
+constexpr int kStcControlBytes = 2048;
+constexpr int kStcMaxSmem = 232448;  // 227 KB per block on sm_100
+// dynamic shared memory: [B operand][A tile 0][A tile 1][reduction scratch unless aliased][control],
+// plus up to 1 KB lost to aligning the start to 1024 bytes.  When the scratch
+// does not fit it reuses A tile 0, which is dead once tile 0's MMAs completed.
+__host__ __device__ constexpr bool stc_red_aliased(int R, int r) {
+  return stc_b_bytes(R, r) + kStcTiles * stc_a_bytes(r) + stc_red_bytes(R) + kStcControlBytes + 1024 > kStcMaxSmem;
+}
+__host__ __device__ constexpr int stc_smem_bytes(int R, int r) {
+  return stc_b_bytes(R, r) + kStcTiles * stc_a_bytes(r) + (stc_red_aliased(R, r) ? 0 : stc_red_bytes(R)) +
+         1024 + kStcControlBytes;
+}
+
+struct StcControl {
+  uint64_t tma_full[kStcTiles];
+  uint64_t mma_done[kStcTiles];
+  uint32_t tmem_base;
+  int flag;
+  int kofs[kStcTiles][64];
+  float alpha[kStcTiles][64];
+  double half_sum[64];
+};
+static_assert(sizeof(StcControl) <= kStcControlBytes, "control block");
+static_assert(stc_smem_bytes(64, 256) <= kStcMaxSmem && stc_smem_bytes(32, 256) <= kStcMaxSmem, "smem budget");
+
+template <int R>
+__global__ void __launch_bounds__(128, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
+                const float *__restrict__ cq_all, float *__restrict__ scores, double *__restrict__ row_sum,
+                unsigned long long *__restrict__ bar, uint32_t *__restrict__ status) {
+  static_assert(R == 32 || R == 64, "scoring rows per CTA");
+  extern __shared__ __align__(1024) unsigned char stc_smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(stc_smem_raw) + 1023) & ~uintptr_t(1023));
+  const int r = s.rank_k;
+  const int nkb = stc_kblocks(r);
+  unsigned char *b_op = smem;
+  unsigned char *a_op = smem + stc_b_bytes(R, r);
+  float *red = reinterpret_cast<float *>(stc_red_aliased(R, r) ? a_op : a_op + kStcTiles * stc_a_bytes(r));
+  StcControl *ctl = reinterpret_cast<StcControl *>(a_op + kStcTiles * stc_a_bytes(r) +
+                                                   (stc_red_aliased(R, r) ? 0 : stc_red_bytes(R)));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tiles_cap = ceil_div(s.cache_rows, kStcTile);
+  const int64_t ctas_per_problem = ceil_div(tiles_cap, kStcTiles);
+  const int b = (int)(blockIdx.x / ctas_per_problem);
+  const int64_t tile0 = (blockIdx.x % ctas_per_problem) * kStcTiles;
+  const int64_t Lraw = lengths[b];
+  const int64_t L = (Lraw >= 0 && Lraw <= s.cache_rows) ? Lraw : 0;
+  int n_tiles = 0;  // active tiles of this CTA
+  for (int t = 0; t < kStcTiles; ++t)
+    if ((tile0 + t) < tiles_cap && (tile0 + t) * kStcTile < L) n_tiles = t + 1;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < kStcTiles; ++t) {
+      mbar_init(&ctl->tma_full[t], 1);
+      mbar_init(&ctl->mma_done[t], 1);
+    }
+    mbar_fence_init();
+    // A: stream this CTA's coefficient tiles.
+    for (int t = 0; t < n_tiles; ++t) {
+      mbar_arrive_expect_tx(&ctl->tma_full[t], (uint32_t)stc_a_bytes(r));
+      const int32_t row = (int32_t)((int64_t)b * s.cache_rows + (tile0 + t) * kStcTile);
+      for (int kb = 0; kb < nkb; ++kb)
+        tma_load_2d(a_op + t * stc_a_bytes(r) + kb * (kStcTile * 128), &tmap_ck, &ctl->tma_full[t], kb * 64, row);
+    }
+  }
+  if (warp == 0) tmem_alloc(&ctl->tmem_base, kStcTmemCols);
+  // Build the split query operand: row n = term * R + i, K-major, 128B swizzle.
+  {
+    const float *cq = cq_all + (int64_t)b * s.n_rows * r;
+    const int kpad = nkb * 64;
+    for (int e = threadIdx.x; e < R * kpad; e += blockDim.x) {
+      const int i = e / kpad, k = e - i * kpad;
+      double x = 0.0;
+      if (i < s.n_rows && k < r) x = (double)cq[(int64_t)i * r + k] * 1.4426950408889634;  // log2(e)
+      const bf16 hi = __double2bfloat16(x);
+      const double r1 = x - (double)__bfloat162float(hi);
+      const bf16 mid = __double2bfloat16(r1);
+      const bf16 lo = __double2bfloat16(r1 - (double)__bfloat162float(mid));
+      unsigned char *blk = b_op + (k >> 6) * (3 * R * 128);
+      const int kk = k & 63;
+      *reinterpret_cast<bf16 *>(blk + sw128_offset(i, kk)) = hi;
+      *reinterpret_cast<bf16 *>(blk + sw128_offset(R + i, kk)) = mid;
+      *reinterpret_cast<bf16 *>(blk + sw128_offset(2 * R + i, kk)) = lo;
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  bool ok = true;
+
+  if (threadIdx.x == 32) {
+    // MMA issuer: D_t[128 x 3R] = A_t[128 x r] . B[3R x r]^T
+    const uint32_t idesc = idesc_bf16_f32(128, 3 * R, 0, 0);
+    const uint32_t b_base = smem_u32(b_op);
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      ok = mbar_wait(&ctl->tma_full[t], 0, status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(a_op + t * stc_a_bytes(r));
+      for (int kb = 0; kb < nkb; ++kb)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = sdesc_sw128(a_base + kb * (kStcTile * 128) + ks * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + kb * (3 * R * 128) + ks * 32, 16, 1024);
+          umma_f16(tmem + t * kStcTileCols, ad, bd, idesc, (kb | ks) ? 1u : 0u);
+        }
+      umma_commit(&ctl->mma_done[t]);
+    }
+  }
+  __syncwarp();
+
+  // B: per-tile exponentials and row sums.
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int p = threadIdx.x;  // position within the tile
+  constexpr int TPR = 128 / R;  // threads per row in the reductions
+  for (int t = 0; t < n_tiles; ++t) {
+    ok = mbar_wait(&ctl->mma_done[t], 0, status) && ok;
+    tc_fence_after();
+    const int64_t pos = (tile0 + t) * kStcTile + p;
+    const bool valid = pos < L;
+    const uint32_t col0 = tmem + lane_base + t * kStcTileCols;
+    float amax = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < R / 32; ++c) {
+      uint32_t hi[32], mid[32], lo[32];
+      tmem_ld32(col0 + c * 32, hi);
+      tmem_ld32(col0 + R + c * 32, mid);
+      tmem_ld32(col0 + 2 * R + c * 32, lo);
+      tmem_wait_ld();
+      uint32_t ev[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float y = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
+        hi[j] = __float_as_uint(y);
+        amax = valid ? fmaxf(amax, fabsf(y)) : amax;
+        const float e = valid ? ex2_approx(y) : 0.f;
+        ev[j] = __float_as_uint(e);
+        red[p * (R + 1) + c * 32 + j] = e;
+      }
+      tmem_st32(col0 + c * 32, hi);      // y
+      tmem_st32(col0 + R + c * 32, ev);  // e
+      tmem_wait_st();
+    }
+    const bool wide = __syncthreads_or(amax > kStcRangeLimit) != 0;
+    if (wide) {
+      // Rare path: per-row integer offsets k = floor(max_i y) for this tile.
+      for (int c = 0; c < R / 32; ++c) {
+        uint32_t yv[32];
+        tmem_ld32(col0 + c * 32, yv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) red[p * (R + 1) + c * 32 + j] = valid ? __uint_as_float(yv[j]) : -INFINITY;
+      }
+      __syncthreads();
+      if (threadIdx.x < R) {
+        float m = -INFINITY;
+        for (int q = 0; q < kStcTile; ++q) m = fmaxf(m, red[q * (R + 1) + threadIdx.x]);
+        ctl->kofs[t][threadIdx.x] = (m == -INFINITY) ? 0 : (int)floorf(m);
+      }
+      __syncthreads();
+      for (int c = 0; c < R / 32; ++c) {
+        uint32_t yv[32], ev[32];
+        tmem_ld32(col0 + c * 32, yv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float e = valid ? ex2_approx(__uint_as_float(yv[j]) - (float)ctl->kofs[t][c * 32 + j]) : 0.f;
+          ev[j] = __float_as_uint(e);
+          red[p * (R + 1) + c * 32 + j] = e;
+        }
+        tmem_st32(col0 + R + c * 32, ev);
+        tmem_wait_st();
+      }
+    } else if (threadIdx.x < R) {
+      ctl->kofs[t][threadIdx.x] = 0;
+    }
+    __syncthreads();
+    // Row sums over the tile's 128 positions: TPR threads per row, fp64, fixed order.
+    {
+      const int row = threadIdx.x % R, part = threadIdx.x / R;
+      double acc = 0.0;
+      for (int q = part * (kStcTile / TPR); q < (part + 1) * (kStcTile / TPR); ++q) acc += (double)red[q * (R + 1) + row];
+      if (part > 0) ctl->half_sum[row] = 0.0;
+      __syncthreads();
+      for (int pp = 1; pp < TPR; ++pp) {
+        if (part == pp) ctl->half_sum[row] += acc;
+        __syncthreads();
+      }
+      if (part == 0 && row < s.n_rows) {
+        const double l = acc + (TPR > 1 ? ctl->half_sum[row] : 0.0);
+        atomicAdd(&row_sum[(int64_t)b * s.n_rows + row], ldexp(l, ctl->kofs[t][row]));
+      }
+    }
+    __syncthreads();
+  }
+
+  // C: every tile of every problem has added its row sums.
+  const bool bar_ok = grid_barrier(bar, status, &ctl->flag);
+
+  // D: scores.
+  if (threadIdx.x < R) {
+    const int row = threadIdx.x;
+    const double l = (row < s.n_rows && bar_ok) ? __ldcg(&row_sum[(int64_t)b * s.n_rows + row]) : 0.0;
+    for (int t = 0; t < n_tiles; ++t)
+      ctl->alpha[t][row] = (l > 0.0) ? (float)(ldexp(1.0, ctl->kofs[t][row]) / l) : 0.f;
+  }
+  __syncthreads();
+  for (int t = 0; t < n_tiles; ++t) {
+    const int64_t pos = (tile0 + t) * kStcTile + p;
+    const uint32_t col0 = tmem + lane_base + t * kStcTileCols;
+    float acc = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < R / 32; ++c) {
+      uint32_t ev[32];
+      tmem_ld32(col0 + R + c * 32, ev);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc = fmaf(ctl->alpha[t][c * 32 + j], __uint_as_float(ev[j]), acc);
+    }
+    if (pos < L) scores[(int64_t)b * s.cache_rows + pos] = acc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kStcTmemCols);
+  (void)lane;
+}
+
+}  // namespace s4r

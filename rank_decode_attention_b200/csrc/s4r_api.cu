@@ -16,6 +16,7 @@
 #include "k_encode_tc.cuh"
 #include "k_project.cuh"
 #include "k_score_simt.cuh"
+#include "k_score_tc.cuh"
 #include "k_topk.cuh"
 
 using namespace s4r;
@@ -29,18 +30,21 @@ inline size_t esize(s4r_dtype dt) { return dt == S4R_BF16 ? 2 : 4; }
 
 // Byte offsets of the decode workspace regions.
 struct Layout {
-  size_t status, cq, qt, tstat, rstat, scores, pooled, part, total;
+  size_t status, barrier, cq, qt, tstat, rstat, rowsum, scores, pooled, part, total;
 };
 
 Layout layout_for(const Shape &s) {
   Layout l{};
   size_t off = 0;
-  l.status = off; off += kAlign;
+  l.status = off;
+  l.barrier = off + 64;
+  off += kAlign;
   l.cq = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_rows * s.rank_k);
   l.qt = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * s.rank_k);
   const size_t n_tiles = (size_t)ceil_div(s.cache_rows, kScoreTile);
   l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
   l.rstat = off; off += round_up(sizeof(double) * 2 * s.batch * (size_t)s.n_rows);
+  l.rowsum = off; off += round_up(sizeof(double) * s.batch * (size_t)s.n_rows);
   l.scores = off; off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.pooled = off; if (s.pool_kernel > 1) off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.part = off;
@@ -133,6 +137,66 @@ s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const vo
   return last_cuda();
 }
 
+// Which latent-scoring kernel a decode call uses.
+struct ScorePlan {
+  bool tc = false;   // tensor-core single-pass kernel (else fp64 CUDA-core passes)
+  int R = 0;         // rows per problem (template argument of the TC kernel)
+  int grid = 0;
+  size_t smem = 0;
+};
+
+template <int R>
+bool tc_fits(int rank, int grid, size_t *smem_out) {
+  const size_t smem = (size_t)stc_smem_bytes(R, rank);
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  if (cudaFuncSetAttribute(score_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return false;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, 128, smem) != cudaSuccess) return false;
+  *smem_out = smem;
+  return grid <= per_sm * sms;
+}
+
+ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
+  ScorePlan p;
+  if (dt != S4R_BF16 || s.cache_rows == 0 || s.batch == 0) return p;
+  if (s.n_rows != 32 && s.n_rows != 64) return p;
+  if ((int64_t)s.batch * s.cache_rows >= INT32_MAX) return p;
+  const int64_t grid = (int64_t)s.batch * ceil_div(ceil_div(s.cache_rows, kStcTile), kStcTiles);
+  if (grid > 4096) return p;
+  size_t smem = 0;
+  const bool fits = s.n_rows == 64 ? tc_fits<64>(s.rank_k, (int)grid, &smem) : tc_fits<32>(s.rank_k, (int)grid, &smem);
+  if (!fits) {
+    cudaGetLastError();
+    return p;
+  }
+  p.tc = true;
+  p.R = s.n_rows;
+  p.grid = (int)grid;
+  p.smem = smem;
+  return p;
+}
+
+template <int R>
+s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s, const int32_t *lengths,
+                           const float *cq, float *scores, double *rowsum, unsigned long long *bar, uint32_t *status,
+                           cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cq, scores, rowsum, bar, status) == cudaSuccess
+             ? S4R_OK
+             : S4R_ERR_CUDA;
+}
+
 template <typename T>
 s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout &ly, cudaStream_t st) {
   unsigned char *ws = static_cast<unsigned char *>(a->workspace);
@@ -141,6 +205,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   float *qt = reinterpret_cast<float *>(ws + ly.qt);
   double *tstat = reinterpret_cast<double *>(ws + ly.tstat);
   double *rstat = reinterpret_cast<double *>(ws + ly.rstat);
+  double *rowsum = reinterpret_cast<double *>(ws + ly.rowsum);
+  unsigned long long *bar = reinterpret_cast<unsigned long long *>(ws + ly.barrier);
   float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
   float *pooled = reinterpret_cast<float *>(ws + ly.pooled);
   float *part = reinterpret_cast<float *>(ws + ly.part);
@@ -156,13 +222,22 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   {
     dim3 grid((unsigned)ceil_div(s.n_rows + s.n_heads_q, kProjRows),
               (unsigned)ceil_div(s.rank_k, kProjCols), (unsigned)s.batch);
-    project_kernel<T><<<grid, kProjRows * kProjCols, 0, st>>>(s, q, bk, cq, qt);
+    project_kernel<T><<<grid, kProjRows * kProjCols, 0, st>>>(s, q, bk, cq, qt, rowsum, bar);
   }
   // 2. latent scoring
   const unsigned n_tiles = (unsigned)ceil_div(s.cache_rows, kScoreTile);
   if (a->profile_events[0])
     cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->profile_events[0]), st, cudaEventRecordExternal);
-  if (n_tiles > 0) {
+  const ScorePlan plan = plan_scoring(s, a->dtype);
+  if (plan.tc) {
+    CUtensorMap tmap;
+    if (!make_tmap_bf16(&tmap, ck, (uint64_t)s.rank_k, (uint64_t)s.batch * s.cache_rows, (uint64_t)s.rank_k * 2, 64,
+                        kStcTile))
+      return S4R_ERR_CUDA;
+    const s4r_status rc = plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cq, scores, rowsum, bar, status, st)
+                                       : launch_score_tc<32>(plan, tmap, s, a->lengths, cq, scores, rowsum, bar, status, st);
+    if (rc != S4R_OK) return rc;
+  } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
     cudaFuncSetAttribute(score_stats_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaFuncSetAttribute(score_final_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -206,7 +281,8 @@ int32_t s4r_decode_kernel_launches(const s4r_decode_args *args) {
   if (make_shape(args, &s) != S4R_OK) return 0;
   if (s.batch == 0) return 0;
   int32_t n = 1;                                  // projection
-  if (s.cache_rows > 0) n += 3;                   // scoring: stats, merge, final
+  if (plan_scoring(s, args->dtype).tc) n += 1;    // scoring: one tensor-core pass
+  else if (s.cache_rows > 0) n += 3;              // scoring: stats, merge, final
   if (s.pool_kernel > 1 && s.cache_rows > 0) n += 1;
   if (s.top_k > 0) n += 1;
   n += 2;                                         // attention: partial, combine

@@ -109,6 +109,54 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Store 32 consecutive 32-bit columns of the warp's 32 lanes (inverse of tmem_ld32).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// 2^x on the special-function unit (max relative error about 2 ulp).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Grid-wide barrier for a cooperative launch.  `ctr` is zeroed by an earlier
+// launch on the same stream; every CTA adds one arrival and waits (bounded)
+// until all gridDim.x CTAs have arrived.  Returns false on timeout.
+__device__ __forceinline__ bool grid_barrier(unsigned long long *ctr, uint32_t *status, int *flag_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    atomicAdd(ctr, 1ull);
+    const long long t0 = clock64();
+    while (true) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+      if (v >= (unsigned long long)gridDim.x) break;
+      if (clock64() - t0 > kWaitCycles) {
+        set_status(status, kDevStatusTimeout);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    *flag_smem = ok;
+  }
+  __syncthreads();
+  return *flag_smem != 0;
+}
 
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
 // lane (base lane + t), columns col .. col+31.
