@@ -146,8 +146,9 @@ size_t s4r_decode_workspace_bytes(const s4r_decode_args *args);
  * enqueues (0 if the shape is invalid). */
 int32_t s4r_decode_kernel_launches(const s4r_decode_args *args);
 
-/* Prepare a freshly allocated workspace (clears its status word and the
- * counters that the kernels reuse).  Call once per workspace allocation. */
+/* Prepare a freshly allocated workspace: zeroes all of it (status word,
+ * counters and accumulators that the kernels reuse and leave zeroed after
+ * each call).  Call once per workspace allocation, before its first use. */
 s4r_status s4r_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* One decode step for every problem of the batch:

@@ -12,26 +12,47 @@
 // rows of the basis that belong to group g.  Nothing is rounded to the
 // storage type; all arithmetic is fp32.
 //
-// attend_partial: CTA (split, g, b) runs an online softmax over a slice of
-//   the selected rows for the G heads of group g and writes (m, l, acc[r_v]).
-// attend_combine: CTA (h, b) merges the slices with the sink logits and maps
-//   the latent accumulator back through B^V[g].
+// One launch, CTA (split, g, problem), 128 threads:
+//   1. cp.async the split's selected C_K / C_V rows (<= 64) into shared memory;
+//   2. logits of the G heads of group g, their softmax partials (max, sum) and
+//      the latent value sums acc[j][:] = sum_e p[j][e] c_V[e];
+//   3. write the partial; the last CTA of the group (atomic ticket) merges all
+//      splits with the sink logits, maps acc through B^V[g] and writes out.
 #pragma once
 #include "common.cuh"
 #include "k_topk.cuh"
+#include "umma.cuh"
 
 namespace s4r {
 
 constexpr int kAttThreads = 128;      // 4 warps
 constexpr int kAttEntries = 64;       // selected rows per split
 constexpr int kAttMaxGroup = 8;       // G <= 8
-constexpr int kAttMaxRankLane = 8;    // rank / 32 <= 8
+constexpr int kAttMaxSinks = 16;      // sinks merged by the combining CTA
 
 __host__ __device__ inline int64_t att_max_selected(const Shape &s) {
   return (int64_t)s.top_k + s.local_window;
 }
 __host__ __device__ inline int att_splits(const Shape &s) {
   return (int)ceil_div(att_max_selected(s) > 0 ? att_max_selected(s) : 1, kAttEntries);
+}
+// Row pitch (elements) of staged rows: 16-byte multiples whose 4-byte-word
+// stride is 4 (mod 8), so the 16-byte reads of 8 consecutive rows fall in
+// distinct bank quads.
+__host__ __device__ inline int att_pitch(int n, int esize) {
+  int words = (n * esize) / 4;
+  while (words % 8 != 4) words += 4;
+  return words * 4 / esize;
+}
+__host__ __device__ inline size_t att_stage_bytes(const Shape &s, int esize) {
+  const size_t rows = (size_t)kAttEntries * (att_pitch(s.rank_k, esize) + att_pitch(s.rank_v, esize)) * esize;
+  const size_t bv = (size_t)s.head_dim * att_pitch(s.rank_v, esize) * esize;
+  return rows > bv ? rows : bv;
+}
+__host__ inline size_t att_smem_bytes(const Shape &s, int esize) {
+  return att_stage_bytes(s, esize) +
+         sizeof(float) * (size_t)(kAttMaxGroup * s.rank_k + kAttMaxGroup * kAttEntries + 4 * kAttMaxGroup +
+                                  kAttMaxGroup * s.rank_v + kAttMaxGroup * kAttMaxSinks);
 }
 
 // Row number of selected entry e (top-k list first, then the window).
@@ -41,171 +62,207 @@ __device__ __forceinline__ int64_t att_entry_row(const int32_t *idx_b, int64_t n
   return L - n_win + (e - n_top);
 }
 
+// Dot product of n (a multiple of 8) fp32 values with n storage values, 16-byte reads.
+template <typename T>
+__device__ __forceinline__ float dot_f32_store(const float *a, const T *x, int n) {
+  constexpr int V = Vec16<T>::n;
+  float acc = 0.f;
+  for (int k = 0; k < n; k += V) {
+    float xv[V];
+    load16(x + k, xv);
+#pragma unroll
+    for (int u = 0; u < V; ++u) acc = fmaf(a[k + u], xv[u], acc);
+  }
+  return acc;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kAttThreads)
-attend_partial(Shape s, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
-               const T *__restrict__ coeff_k, const T *__restrict__ coeff_v,
-               const float *__restrict__ qt_all, float *__restrict__ part) {
-  __shared__ float q_s[kAttMaxGroup][S4R_MAX_RANK];
-  __shared__ float m_s[4][kAttMaxGroup], l_s[4][kAttMaxGroup];
-  __shared__ float acc_s[4][kAttMaxGroup][S4R_MAX_RANK];
+attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
+              const T *__restrict__ coeff_k, const T *__restrict__ coeff_v, const float *__restrict__ qt_all,
+              const T *__restrict__ q, const T *__restrict__ basis_v, const T *__restrict__ sink_k,
+              const T *__restrict__ sink_v, float *__restrict__ part, unsigned int *__restrict__ tickets,
+              float *__restrict__ out) {
+  extern __shared__ __align__(16) unsigned char att_smem[];
+  constexpr int V = Vec16<T>::n;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int G = s.group, rk = s.rank_k, rv = s.rank_v;
+  const int n_split = gridDim.x;
+  const int G = s.group, rk = s.rank_k, rv = s.rank_v, dh = s.head_dim, Dp = s.d_model, ns = s.n_sink;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int pk = att_pitch(rk, sizeof(T)), pv = att_pitch(rv, sizeof(T));
+  T *ck_s = reinterpret_cast<T *>(att_smem);
+  T *cv_s = ck_s + kAttEntries * pk;
+  float *q_s = reinterpret_cast<float *>(att_smem + att_stage_bytes(s, sizeof(T)));  // [G][rk]
+  float *p_s = q_s + kAttMaxGroup * rk;                               // [G][64]
+  float *ml_s = p_s + kAttMaxGroup * kAttEntries;                     // [G][4]
+  float *acc_s = ml_s + 4 * kAttMaxGroup;                             // [G][rv]
+  float *sw_s = acc_s + kAttMaxGroup * rv;                            // [G][kAttMaxSinks]
+  __shared__ int64_t rows_s[kAttEntries];
+  __shared__ int last_flag;
+
   const int64_t L = valid_length(lengths[b], s.cache_rows);
   const int64_t n_top = smin<int64_t>(s.top_k, n_candidates(L, s.local_window));
   const int64_t n_win = smin<int64_t>(s.local_window, L);
   const int64_t n_sel = n_top + n_win;
   const int64_t e0 = (int64_t)split * kAttEntries;
-  const int64_t e1 = smin<int64_t>(n_sel, e0 + kAttEntries);
-  for (int e = threadIdx.x; e < G * rk; e += blockDim.x) {
-    const int j = e / rk, k = e - j * rk;
-    q_s[j][k] = qt_all[((int64_t)b * s.n_heads_q + g * G + j) * rk + k];
-  }
-  __syncthreads();
-  float m[kAttMaxGroup], l[kAttMaxGroup], acc[kAttMaxGroup][kAttMaxRankLane];
-#pragma unroll
-  for (int j = 0; j < kAttMaxGroup; ++j) {
-    m[j] = -INFINITY; l[j] = 0.f;
-#pragma unroll
-    for (int u = 0; u < kAttMaxRankLane; ++u) acc[j][u] = 0.f;
-  }
+  const int n_e = (int)smax<int64_t>(0, smin<int64_t>(kAttEntries, n_sel - e0));
   const int32_t *idx_b = idx + (int64_t)b * s.top_k;
   const T *ckb = coeff_k + (int64_t)b * s.cache_rows * rk;
   const T *cvb = coeff_v + (int64_t)b * s.cache_rows * rv;
-  for (int64_t e = e0 + wid; e < e1; e += 4) {
-    const int64_t row = att_entry_row(idx_b, n_top, L, n_win, e, s.n_sink);
-    if (row < 0 || row >= L) continue;  // idx entries come from the top-k kernel
-    float ck[kAttMaxRankLane];
-#pragma unroll
-    for (int u = 0; u < kAttMaxRankLane; ++u) {
-      const int k = lane + 32 * u;
-      ck[u] = (k < rk) ? to_f(ckb[row * rk + k]) : 0.f;
+
+  // 1. stage the split's rows; an entry outside [0, L) (which the top-k
+  //    kernel never produces) is skipped with logit -inf.
+  for (int e = threadIdx.x; e < kAttEntries; e += blockDim.x) {
+    int64_t row = -1;
+    if (e < n_e) {
+      row = att_entry_row(idx_b, n_top, L, n_win, e0 + e, s.n_sink);
+      if (row < 0 || row >= L) row = -1;
     }
-    float cv[kAttMaxRankLane];
-#pragma unroll
-    for (int u = 0; u < kAttMaxRankLane; ++u) {
-      const int k = lane + 32 * u;
-      cv[u] = (k < rv) ? to_f(cvb[row * rv + k]) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < kAttMaxGroup; ++j) {
-      if (j >= G) break;
-      float d = 0.f;
-#pragma unroll
-      for (int u = 0; u < kAttMaxRankLane; ++u) {
-        const int k = lane + 32 * u;
-        if (k < rk) d = fmaf(q_s[j][k], ck[u], d);
+    rows_s[e] = row;
+  }
+  __syncthreads();
+  {
+    const int ck_chunks = rk / V, cv_chunks = rv / V;
+    for (int t = threadIdx.x; t < n_e * (ck_chunks + cv_chunks); t += blockDim.x) {
+      const int e = t / (ck_chunks + cv_chunks), c = t - e * (ck_chunks + cv_chunks);
+      const int64_t row = rows_s[e];
+      if (row < 0) {  // keep skipped rows finite: their weights are zero
+        T *dst = (c < ck_chunks) ? ck_s + e * pk + c * V : cv_s + e * pv + (c - ck_chunks) * V;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        continue;
       }
-      const float logit = warp_sum(d);
-      const float nm = fmaxf(m[j], logit);
-      const float scale = __expf(m[j] - nm);
-      const float p = __expf(logit - nm);
-      l[j] = l[j] * scale + p;
-#pragma unroll
-      for (int u = 0; u < kAttMaxRankLane; ++u) acc[j][u] = acc[j][u] * scale + p * cv[u];
-      m[j] = nm;
+      if (c < ck_chunks)
+        cp_async16(ck_s + e * pk + c * V, ckb + row * rk + c * V);
+      else
+        cp_async16(cv_s + e * pv + (c - ck_chunks) * V, cvb + row * rv + (c - ck_chunks) * V);
     }
   }
-  // Combine the 4 warps.
-#pragma unroll
-  for (int j = 0; j < kAttMaxGroup; ++j) {
-    if (j >= G) break;
-    if (lane == 0) { m_s[wid][j] = m[j]; l_s[wid][j] = l[j]; }
-#pragma unroll
-    for (int u = 0; u < kAttMaxRankLane; ++u) {
-      const int k = lane + 32 * u;
-      if (k < rv) acc_s[wid][j][k] = acc[j][u];
+  for (int t = threadIdx.x; t < G * rk; t += blockDim.x) {
+    const int j = t / rk, k = t - j * rk;
+    q_s[j * rk + k] = qt_all[((int64_t)b * s.n_heads_q + g * G + j) * rk + k];
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // 2a. logits of (head j, entry e) pairs.
+  for (int t = threadIdx.x; t < G * kAttEntries; t += blockDim.x) {
+    const int j = t / kAttEntries, e = t - j * kAttEntries;
+    float l = -INFINITY;
+    if (e < n_e && rows_s[e] >= 0) l = dot_f32_store(q_s + j * rk, ck_s + e * pk, rk);
+    p_s[j * kAttEntries + e] = l;
+  }
+  __syncthreads();
+  // 2b. softmax partial per head: warp w takes heads w, w+4.
+  for (int j = wid; j < G; j += 4) {
+    const float l0 = p_s[j * kAttEntries + lane], l1 = p_s[j * kAttEntries + lane + 32];
+    const float m = warp_max(fmaxf(l0, l1));
+    const float p0 = (m == -INFINITY) ? 0.f : __expf(l0 - m);
+    const float p1 = (m == -INFINITY) ? 0.f : __expf(l1 - m);
+    const float l = warp_sum(p0 + p1);
+    p_s[j * kAttEntries + lane] = p0;
+    p_s[j * kAttEntries + lane + 32] = p1;
+    if (lane == 0) {
+      ml_s[j * 4] = m;
+      ml_s[j * 4 + 1] = l;
     }
   }
   __syncthreads();
-  const int n_split = gridDim.x;
-  for (int e = threadIdx.x; e < G * (rv + 2); e += blockDim.x) {
-    const int j = e / (rv + 2), k = e - j * (rv + 2);
-    float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, m_s[w][j]);
-    float v = 0.f;
-    if (k == 0) {
-      v = M;
-    } else {
-      for (int w = 0; w < 4; ++w) {
-        const float f = (m_s[w][j] == -INFINITY) ? 0.f : __expf(m_s[w][j] - M);
-        v += f * ((k == 1) ? l_s[w][j] : acc_s[w][j][k - 2]);
-      }
+  // 2c. latent value sums, one column k per thread.
+  for (int k = threadIdx.x; k < rv; k += blockDim.x) {
+    float acc[kAttMaxGroup];
+#pragma unroll
+    for (int j = 0; j < kAttMaxGroup; ++j) acc[j] = 0.f;
+    for (int e = 0; e < n_e; ++e) {
+      const float v = to_f(cv_s[e * pv + k]);
+#pragma unroll
+      for (int j = 0; j < kAttMaxGroup; ++j)
+        if (j < G) acc[j] = fmaf(p_s[j * kAttEntries + e], v, acc[j]);
     }
-    const int h = g * G + j;
-    part[(((int64_t)b * s.n_heads_q + h) * n_split + split) * (rv + 2) + k] = v;
+#pragma unroll
+    for (int j = 0; j < kAttMaxGroup; ++j)
+      if (j < G) part[(((int64_t)b * s.n_heads_q + g * G + j) * n_split + split) * (rv + 2) + 2 + k] = acc[j];
   }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(256)
-attend_combine(Shape s, const T *__restrict__ q, const T *__restrict__ basis_v,
-               const T *__restrict__ sink_k, const T *__restrict__ sink_v,
-               const float *__restrict__ part, float *__restrict__ out) {
-  extern __shared__ float cs[];  // [rv] latent accumulator, then [n_sink] sink weights
-  __shared__ float red[8];
-  __shared__ float sh_M, sh_den;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int G = s.group, g = h / G, dh = s.head_dim, rv = s.rank_v, Dp = s.d_model;
-  const int ns = s.n_sink, n_split = att_splits(s);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  float *acc_s = cs;
-  float *sw = cs + rv;
-  const T *qh = q + (((int64_t)b * s.query_window + s.query_window - 1) * s.n_heads_q + h) * dh;
-  const float *pb = part + ((int64_t)b * s.n_heads_q + h) * n_split * (rv + 2);
-  // Sink logits, one warp per sink.
+  if (threadIdx.x < G) {
+    float *pp = part + (((int64_t)b * s.n_heads_q + g * G + threadIdx.x) * n_split + split) * (rv + 2);
+    pp[0] = ml_s[threadIdx.x * 4];
+    pp[1] = ml_s[threadIdx.x * 4 + 1];
+  }
+  // 3. the last split CTA of this (problem, group) merges.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int t = atomicAdd(&tickets[(int64_t)b * s.n_heads_kv + g], 1u);
+    last_flag = (t == (unsigned int)n_split - 1);
+  }
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+  // Stage B^V[g] (d_h rows x rv) over the row buffers.
+  T *bv_s = ck_s;
+  const T *Bv = basis_v + (int64_t)b * Dp * rv + (int64_t)g * dh * rv;
+  for (int t = threadIdx.x; t < dh * (rv / V); t += blockDim.x) {
+    const int e = t / (rv / V), c = t - e * (rv / V);
+    cp_async16(bv_s + e * pv + c * V, Bv + (int64_t)e * rv + c * V);
+  }
+  // Sink logits: one warp per (head, sink).
   const float qscale = rsqrtf((float)dh);
-  for (int t = wid; t < ns; t += nw) {
-    const T *kr = sink_k + ((int64_t)b * ns + t) * Dp + (int64_t)g * dh;
+  for (int t = wid; t < G * ns; t += 4) {
+    const int j = t / ns, tk = t - j * ns;
+    const T *qh = q + (((int64_t)b * s.query_window + s.query_window - 1) * s.n_heads_q + g * G + j) * dh;
+    const T *kr = sink_k + ((int64_t)b * ns + tk) * Dp + (int64_t)g * dh;
     float d = 0.f;
     for (int e = lane; e < dh; e += 32) d = fmaf(to_f(qh[e]), to_f(kr[e]), d);
     d = warp_sum(d);
-    if (lane == 0) sw[t] = d * qscale;
+    if (lane == 0) sw_s[j * kAttMaxSinks + tk] = d * qscale;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  // Merge statistics per head: warp w takes heads w, w+4.
+  for (int j = wid; j < G; j += 4) {
+    const float *pb = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2);
     float M = -INFINITY;
-    for (int t = 0; t < ns; ++t) M = fmaxf(M, sw[t]);
-    for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, pb[sp * (rv + 2)]);
+    for (int sp = lane; sp < n_split; sp += 32) M = fmaxf(M, __ldcg(pb + sp * (rv + 2)));
+    for (int tk = lane; tk < ns; tk += 32) M = fmaxf(M, sw_s[j * kAttMaxSinks + tk]);
+    M = warp_max(M);
     float den = 0.f;
-    for (int t = 0; t < ns; ++t) den += __expf(sw[t] - M);
-    for (int sp = 0; sp < n_split; ++sp) {
-      const float ms = pb[sp * (rv + 2)];
-      if (ms != -INFINITY) den += pb[sp * (rv + 2) + 1] * __expf(ms - M);
+    for (int sp = lane; sp < n_split; sp += 32) {
+      const float ms = __ldcg(pb + sp * (rv + 2));
+      if (ms != -INFINITY) den += __ldcg(pb + sp * (rv + 2) + 1) * __expf(ms - M);
     }
-    sh_M = M;
-    sh_den = den;
+    for (int tk = lane; tk < ns; tk += 32) den += __expf(sw_s[j * kAttMaxSinks + tk] - M);
+    den = warp_sum(den);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    if (lane == 0) {
+      ml_s[j * 4 + 2] = M;
+      ml_s[j * 4 + 3] = inv;
+    }
+    __syncwarp();
+    for (int tk = lane; tk < ns; tk += 32)
+      sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
   }
   __syncthreads();
-  const float M = sh_M;
-  const float inv = (sh_den > 0.f) ? 1.f / sh_den : 0.f;
-  for (int k = threadIdx.x; k < rv; k += blockDim.x) {
+  // Latent accumulator per head: acc[j][k] = sum_split w_split acc_split[k].
+  for (int t = threadIdx.x; t < G * rv; t += blockDim.x) {
+    const int j = t / rv, k = t - j * rv;
+    const float *pb = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2);
+    const float M = ml_s[j * 4 + 2], inv = ml_s[j * 4 + 3];
     float a = 0.f;
     for (int sp = 0; sp < n_split; ++sp) {
-      const float ms = pb[sp * (rv + 2)];
-      if (ms != -INFINITY) a += pb[sp * (rv + 2) + 2 + k] * __expf(ms - M);
+      const float ms = __ldcg(pb + sp * (rv + 2));
+      if (ms != -INFINITY) a = fmaf(__expf(ms - M), __ldcg(pb + sp * (rv + 2) + 2 + k), a);
     }
-    acc_s[k] = a * inv;
+    acc_s[j * rv + k] = a * inv;
   }
+  cp_async_wait_all();
   __syncthreads();
-  for (int t = threadIdx.x; t < ns; t += blockDim.x) sw[t] = __expf(sw[t] - M) * inv;
-  __syncthreads();
-  (void)red;
-  // out[h][e] = sum_k acc[k] B^V[g*dh + e][k] + sum_t w_t sink_v[t][g*dh + e]; one warp per e.
-  const T *Bv = basis_v + (int64_t)b * Dp * rv;
-  for (int e = wid; e < dh; e += nw) {
-    const T *brow = Bv + (int64_t)(g * dh + e) * rv;
-    float d = 0.f;
-    for (int k = lane; k < rv; k += 32) d = fmaf(acc_s[k], to_f(brow[k]), d);
-    d = warp_sum(d);
-    if (lane == 0) {
-      float sv = 0.f;
-      for (int t = 0; t < ns; ++t)
-        sv = fmaf(sw[t], to_f(sink_v[((int64_t)b * ns + t) * Dp + (int64_t)g * dh + e]), sv);
-      out[((int64_t)b * s.n_heads_q + h) * dh + e] = d + sv;
-    }
+  // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e].
+  for (int t = threadIdx.x; t < G * dh; t += blockDim.x) {
+    const int j = t / dh, e = t - j * dh;
+    float o = dot_f32_store(acc_s + j * rv, bv_s + e * pv, rv);
+    for (int tk = 0; tk < ns; ++tk)
+      o = fmaf(sw_s[j * kAttMaxSinks + tk], to_f(sink_v[((int64_t)b * ns + tk) * Dp + (int64_t)g * dh + e]), o);
+    out[((int64_t)b * s.n_heads_q + g * G + j) * dh + e] = o;
   }
+  if (threadIdx.x == 0) tickets[(int64_t)b * s.n_heads_kv + g] = 0u;
 }
 
 // Rebuild rows explicitly: out[e][d] = sum_j C[rows[e]][j] B[d][j] (fp32).

@@ -2,94 +2,166 @@
 //
 // "Core claim" of the S4R review page: at decoding, queries are projected into
 // the key subspace; the sliding query window is then scored in latent space
-// (Eqs. 8-10).  One launch produces, per problem,
-//   cq[R][r_k]   scoring rows C_Q, already multiplied by 1/sqrt(r_k), and
-//   qt[H_q][r_k] the current query (window slot W-1) of every head projected
-//                with the head_dim rows of its kv group's key-basis slice,
-//                multiplied by 1/sqrt(head_dim) -- the absorbed form of the
-//                exact-attention logits q . (c B^T) = (q B) . c.
-// Output rows rho < R are scoring rows, rows R .. R+H_q-1 are the qt rows.
-// Products of two storage values are exact in fp32; each 64-term chunk is
-// summed in fp32 and the chunks in fp64, so the result is the fp64 dot
-// product rounded once to fp32 (up to the chunk rounding).
+// (Eqs. 8-10).  Every per-head projection
+//     p[w][h][c] = q[w][h] . B^K[g*d_h : (g+1)*d_h][c],   g = h / G,
+// is computed once (CTA (g, 64-column block, problem)), and from it
+//   * CONCAT rows:   C_Q[w*G + j] = sum_g p[w][g*G + j]   (row = Q'[w][j] . B^K)
+//   * PER_HEAD rows: C_Q[w*H_q + h] = p[w][h]
+//   * qt[h] = p[W-1][h] / sqrt(d_h), the current query in latent form for the
+//     absorbed exact-attention logits q . (c B^T) = (q B) . c.
+// Products of two storage values are exact in fp32; each dot product sums
+// 64-term fp32 chunks in fp64, and the group sum is an fp64 atomic sum.
+// The last CTA of a column block (an atomic ticket) scales the fp64 rows by
+// 1/sqrt(r_k) and writes
+//   * cq  [R][r_k] fp32 (natural-log units), read by the CUDA-core scoring;
+//   * cqs  the shared-memory image of the tensor-core operand: C_Q * log2(e)
+//     split into three bf16 terms hi + mid + lo (rows term*R + i), K-major,
+//     128-byte swizzled, one 3R x 64 block per 64 columns,
+// and clears its fp64 accumulators and ticket for the next call.
 #pragma once
 #include "common.cuh"
+#include "umma.cuh"
 
 namespace s4r {
 
-constexpr int kProjRows = 8;    // output rows per CTA
-constexpr int kProjCols = 32;   // rank columns per CTA
-constexpr int kProjChunk = 64;  // D' rows staged per iteration
+constexpr int kProjThreads = 256;
+constexpr int kProjColBlock = 64;   // columns per CTA (= one 128-byte swizzle row of bf16)
+constexpr int kProjRowBlock = 64;   // per-head rows (w, j) staged at once
 
-// Value of input row `rho` at model column d (0 outside the row's support).
-template <typename T>
-__device__ __forceinline__ float proj_input(const T *q, const Shape &s, int rho, int d) {
-  const int dh = s.head_dim, G = s.group, Hq = s.n_heads_q;
-  const int g = d / dh, t = d - g * dh;
-  int w, h;
-  if (rho < s.n_rows) {
-    if (s.row_mode == S4R_ROWS_CONCAT) {
-      w = rho / G;
-      h = g * G + (rho - w * G);
-    } else {
-      w = rho / Hq;
-      h = rho - w * Hq;
-      if (h / G != g) return 0.f;
-    }
-  } else {
-    w = s.query_window - 1;
-    h = rho - s.n_rows;
-    if (h / G != g) return 0.f;
-  }
-  return to_f(q[((int64_t)w * Hq + h) * dh + t]);
-}
+// Shared-memory image of the split C_Q operand: bytes per 64-column block.
+__host__ __device__ constexpr int cqs_block_bytes(int R) { return 3 * R * 128; }
 
 template <typename T>
-__global__ void __launch_bounds__(kProjRows * kProjCols)
-project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k,
-               float *__restrict__ cq, float *__restrict__ qt, double *__restrict__ row_sum,
+__global__ void __launch_bounds__(kProjThreads)
+project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, float *__restrict__ cq,
+               unsigned char *__restrict__ cqs, float *__restrict__ qt, double *__restrict__ cq64,
+               unsigned int *__restrict__ tickets, double *__restrict__ row_sum,
                unsigned long long *__restrict__ barrier) {
-  __shared__ float qs[kProjRows][kProjChunk + 1];
-  __shared__ float bs[kProjChunk][kProjCols + 1];
-  const int b = blockIdx.z;
-  const int row0 = blockIdx.x * kProjRows, col0 = blockIdx.y * kProjCols;
-  const int tx = threadIdx.x % kProjCols, ty = threadIdx.x / kProjCols;
-  const int n_out = s.n_rows + s.n_heads_q;
-  const int r = s.rank_k, Dp = s.d_model;
-  const T *qb = q + (int64_t)b * s.query_window * s.n_heads_q * s.head_dim;
-  const T *Bb = basis_k + (int64_t)b * Dp * r;
+  __shared__ float qs[kProjRowBlock][65];            // per-head query rows of group g, 64 of d_h
+  __shared__ float bs[64][kProjColBlock + 1];        // basis slice, 64 rows of d_h
+  __shared__ int last_flag;
+  const int g = blockIdx.x, cb = blockIdx.y, b = blockIdx.z;
+  const int G = s.group, W = s.query_window, Hq = s.n_heads_q, dh = s.head_dim, r = s.rank_k;
+  const int R = s.n_rows;
+  const int c0 = cb * kProjColBlock;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16: 4 rows x 4 cols each
+  const T *qb = q + (int64_t)b * W * Hq * dh;
+  const T *Bb = basis_k + (int64_t)b * s.d_model * r;
+  double *cq64b = cq64 + (int64_t)b * R * r;
   // Reset the per-call accumulators of the tensor-core scoring kernel.
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
-    for (int e = threadIdx.x; e < s.n_rows; e += blockDim.x) row_sum[(int64_t)b * s.n_rows + e] = 0.0;
+  if (g == 0 && cb == 0) {
+    for (int e = threadIdx.x; e < R; e += blockDim.x) row_sum[(int64_t)b * R + e] = 0.0;
     if (b == 0 && threadIdx.x == 0) *barrier = 0ull;
   }
-  double acc = 0.0;
-  for (int d0 = 0; d0 < Dp; d0 += kProjChunk) {
-    for (int e = threadIdx.x; e < kProjRows * kProjChunk; e += blockDim.x) {
-      const int rr = e / kProjChunk, dd = e % kProjChunk;
-      const int rho = row0 + rr, d = d0 + dd;
-      qs[rr][dd] = (rho < n_out && d < Dp) ? proj_input(qb, s, rho, d) : 0.f;
-    }
-    for (int e = threadIdx.x; e < kProjChunk * kProjCols; e += blockDim.x) {
-      const int dd = e / kProjCols, cc = e % kProjCols;
-      const int d = d0 + dd, c = col0 + cc;
-      bs[dd][cc] = (d < Dp && c < r) ? to_f(Bb[(int64_t)d * r + c]) : 0.f;
-    }
-    __syncthreads();
-    float part = 0.f;
+  const int n_prow = W * G;  // per-head rows (w, j) of this group
+  for (int pr0 = 0; pr0 < n_prow; pr0 += kProjRowBlock) {
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int t0 = 0; t0 < dh; t0 += 64) {
+      const int tn = smin(64, dh - t0);
+      __syncthreads();
+      // 16 independent loads per thread for each operand (fully unrolled).
+#pragma unroll
+      for (int u = 0; u < (kProjRowBlock * 64) / kProjThreads; ++u) {
+        const int e = threadIdx.x + u * kProjThreads;
+        const int pr = e >> 6, t = e & 63;
+        const int row = pr0 + pr;
+        float v = 0.f;
+        if (row < n_prow && t < tn) {
+          const int w = row / G, j = row - w * G;
+          v = to_f(qb[((int64_t)w * Hq + g * G + j) * dh + t0 + t]);
+        }
+        qs[pr][t] = v;
+      }
+#pragma unroll
+      for (int u = 0; u < (64 * kProjColBlock) / kProjThreads; ++u) {
+        const int e = threadIdx.x + u * kProjThreads;
+        const int t = e >> 6, c = e & 63;
+        bs[t][c] = (t < tn && c0 + c < r) ? to_f(Bb[(int64_t)(g * dh + t0 + t) * r + c0 + c]) : 0.f;
+      }
+      __syncthreads();
+      float part[4][4] = {};
 #pragma unroll 8
-    for (int dd = 0; dd < kProjChunk; ++dd) part = fmaf(qs[ty][dd], bs[dd][tx], part);
-    acc += (double)part;
-    __syncthreads();
+      for (int k = 0; k < 64; ++k) {
+        float a[4], bb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = qs[ty + 16 * i][k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bb[j] = bs[k][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], bb[j], part[i][j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = pr0 + ty + 16 * i;
+      if (row >= n_prow) continue;
+      const int w = row / G, j = row - w * G, h = g * G + j;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int c = c0 + tx + 16 * jj;
+        if (c >= r) continue;
+        const double v = acc[i][jj];
+        if (w == W - 1) qt[((int64_t)b * Hq + h) * r + c] = (float)(v / sqrt((double)dh));
+        if (s.row_mode == S4R_ROWS_CONCAT)
+          atomicAdd(&cq64b[(int64_t)(w * G + j) * r + c], v);
+        else
+          cq64b[(int64_t)(w * Hq + h) * r + c] = v;
+      }
+    }
   }
-  const int rho = row0 + ty, c = col0 + tx;
-  if (rho >= n_out || c >= r) return;
-  if (rho < s.n_rows) {
-    cq[((int64_t)b * s.n_rows + rho) * r + c] = (float)(acc / sqrt((double)r));
-  } else {
-    const int h = rho - s.n_rows;
-    qt[((int64_t)b * s.n_heads_q + h) * r + c] = (float)(acc / sqrt((double)s.head_dim));
+  // Ticket: the last of the H_kv group CTAs of this column block finishes the rows.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int t = atomicAdd(&tickets[(int64_t)b * gridDim.y + cb], 1u);
+    last_flag = (t == gridDim.x - 1);
   }
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+  const double scale = 1.0 / sqrt((double)r);
+  unsigned char *blk = cqs + ((int64_t)b * gridDim.y + cb) * cqs_block_bytes(R);
+  constexpr int kU = 4;  // loads in flight per thread
+  for (int e0 = 0; e0 < R * kProjColBlock; e0 += kU * kProjThreads) {
+    double xs[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int e = e0 + u * kProjThreads + threadIdx.x;
+      const int i = e / kProjColBlock, c = c0 + (e - i * kProjColBlock);
+      xs[u] = (e < R * kProjColBlock && c < r) ? __ldcg(&cq64b[(int64_t)i * r + c]) : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int e = e0 + u * kProjThreads + threadIdx.x;
+      if (e >= R * kProjColBlock) continue;
+      const int i = e / kProjColBlock, kk = e - i * kProjColBlock;
+      const int c = c0 + kk;
+      const double x = xs[u] * scale;
+      if (c < r) {
+        cq64b[(int64_t)i * r + c] = 0.0;
+        cq[((int64_t)b * R + i) * r + c] = (float)x;
+      }
+      const double y = x * 1.4426950408889634;  // log2(e)
+      const bf16 hi = __double2bfloat16(y);
+      const double r1 = y - (double)__bfloat162float(hi);
+      const bf16 mid = __double2bfloat16(r1);
+      const bf16 lo = __double2bfloat16(r1 - (double)__bfloat162float(mid));
+      *reinterpret_cast<bf16 *>(blk + sw128_offset(i, kk)) = hi;
+      *reinterpret_cast<bf16 *>(blk + sw128_offset(R + i, kk)) = mid;
+      *reinterpret_cast<bf16 *>(blk + sw128_offset(2 * R + i, kk)) = lo;
+    }
+  }
+  if (threadIdx.x == 0) tickets[(int64_t)b * gridDim.y + cb] = 0u;
 }
 
 }  // namespace s4r

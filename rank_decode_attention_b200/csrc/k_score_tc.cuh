@@ -15,8 +15,9 @@
 // One cooperative launch, one CTA per pair of 128-position tiles of one
 // problem (4 warps; thread 0 issues TMA, thread 32 issues tcgen05.mma, all
 // warps run the epilogue):
-//   A. TMA both C_K tiles, build the split C_Q operand in shared memory,
-//      MMA each tile into its own 256-column TMEM region.
+//   A. bulk-copy the split C_Q operand (prepared by the projection kernel in
+//      its shared-memory image), TMA both C_K tiles, MMA each tile into its
+//      own 256-column TMEM region.
 //   B. per tile: y = hi + mid + lo, e = 2^y (kept in TMEM), per-row sums of e
 //      over the tile (fp64, fixed order) added atomically (fp64) into the
 //      problem's row normalisers.  A tile whose |y| exceeds 100 uses integer
@@ -54,6 +55,7 @@ __host__ __device__ constexpr int stc_smem_bytes(int R, int r) {
 }
 
 struct StcControl {
+  uint64_t b_full;
   uint64_t tma_full[kStcTiles];
   uint64_t mma_done[kStcTiles];
   uint32_t tmem_base;
@@ -68,7 +70,7 @@ static_assert(stc_smem_bytes(64, 256) <= kStcMaxSmem && stc_smem_bytes(32, 256) 
 template <int R>
 __global__ void __launch_bounds__(128, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
-                const float *__restrict__ cq_all, float *__restrict__ scores, double *__restrict__ row_sum,
+                const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
                 unsigned long long *__restrict__ bar, uint32_t *__restrict__ status) {
   static_assert(R == 32 || R == 64, "scoring rows per CTA");
   extern __shared__ __align__(1024) unsigned char stc_smem_raw[];
@@ -93,11 +95,17 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     if ((tile0 + t) < tiles_cap && (tile0 + t) * kStcTile < L) n_tiles = t + 1;
 
   if (threadIdx.x == 0) {
+    mbar_init(&ctl->b_full, 1);
     for (int t = 0; t < kStcTiles; ++t) {
       mbar_init(&ctl->tma_full[t], 1);
       mbar_init(&ctl->mma_done[t], 1);
     }
     mbar_fence_init();
+    // The split query operand, already in its shared-memory image.
+    mbar_arrive_expect_tx(&ctl->b_full, (uint32_t)stc_b_bytes(R, r));
+    const unsigned char *src = cqs + (int64_t)b * stc_b_bytes(R, r);
+    for (int kb = 0; kb < nkb; ++kb)
+      bulk_load(b_op + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128, &ctl->b_full);
     // A: stream this CTA's coefficient tiles.
     for (int t = 0; t < n_tiles; ++t) {
       mbar_arrive_expect_tx(&ctl->tma_full[t], (uint32_t)stc_a_bytes(r));
@@ -107,26 +115,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     }
   }
   if (warp == 0) tmem_alloc(&ctl->tmem_base, kStcTmemCols);
-  // Build the split query operand: row n = term * R + i, K-major, 128B swizzle.
-  {
-    const float *cq = cq_all + (int64_t)b * s.n_rows * r;
-    const int kpad = nkb * 64;
-    for (int e = threadIdx.x; e < R * kpad; e += blockDim.x) {
-      const int i = e / kpad, k = e - i * kpad;
-      double x = 0.0;
-      if (i < s.n_rows && k < r) x = (double)cq[(int64_t)i * r + k] * 1.4426950408889634;  // log2(e)
-      const bf16 hi = __double2bfloat16(x);
-      const double r1 = x - (double)__bfloat162float(hi);
-      const bf16 mid = __double2bfloat16(r1);
-      const bf16 lo = __double2bfloat16(r1 - (double)__bfloat162float(mid));
-      unsigned char *blk = b_op + (k >> 6) * (3 * R * 128);
-      const int kk = k & 63;
-      *reinterpret_cast<bf16 *>(blk + sw128_offset(i, kk)) = hi;
-      *reinterpret_cast<bf16 *>(blk + sw128_offset(R + i, kk)) = mid;
-      *reinterpret_cast<bf16 *>(blk + sw128_offset(2 * R + i, kk)) = lo;
-    }
-  }
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -137,6 +125,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     // MMA issuer: D_t[128 x 3R] = A_t[128 x r] . B[3R x r]^T
     const uint32_t idesc = idesc_bf16_f32(128, 3 * R, 0, 0);
     const uint32_t b_base = smem_u32(b_op);
+    if (n_tiles > 0) ok = mbar_wait(&ctl->b_full, 0, status);
     for (int t = 0; t < n_tiles && ok; ++t) {
       ok = mbar_wait(&ctl->tma_full[t], 0, status);
       if (!ok) break;

@@ -65,10 +65,26 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_t
   return before;
 }
 
+constexpr int kTopkSmemKeys = 40960;  // keys staged in shared memory (160 KB) when they fit
+constexpr int kTopkBins = 2048;
+__host__ inline size_t topk_smem_bytes(int64_t cache_rows) {
+  return sizeof(uint32_t) * (size_t)smin<int64_t>(cache_rows, kTopkSmemKeys);
+}
+
+// Histogram update aggregated across the lanes of a warp that share a bin
+// (scores of one problem share their high bits, so plain atomics serialise).
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t bin, bool active) {
+  const uint32_t key = active ? bin : 0xffffffffu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, key);
+  const int leader = __ffs(peers) - 1;
+  if (active && (threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restrict__ keys_all,
             int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
-  __shared__ uint32_t hist[256];
+  extern __shared__ __align__(16) uint32_t topk_keys_s[];
+  __shared__ uint32_t hist[kTopkBins];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t sh_total, sh_digit, sh_above;
   const int b = blockIdx.x;
@@ -78,7 +94,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
   const int64_t nc = n_candidates(L, s.local_window);
   const int k = s.top_k;
   int32_t *out = idx + (int64_t)b * k;
-  const uint32_t *keys = reinterpret_cast<const uint32_t *>(keys_all + (int64_t)b * s.cache_rows);
+  const uint32_t *gkeys = reinterpret_cast<const uint32_t *>(keys_all + (int64_t)b * s.cache_rows);
   const int64_t need = smin<int64_t>(k, nc);
   for (int e = threadIdx.x; e < k; e += blockDim.x)
     if (e >= need) out[e] = -1;
@@ -87,43 +103,84 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
     for (int64_t i = threadIdx.x; i < nc; i += blockDim.x) out[i] = (int32_t)(s.n_sink + i);
     return;
   }
-  // Radix select of the need-th largest key.
+  // Stage the keys in shared memory when they fit (16-byte loads, all in flight).
+  const bool staged = nc <= kTopkSmemKeys;
+  if (staged) {
+    const int64_t n4 = nc / 4;
+    const uint4 *src4 = reinterpret_cast<const uint4 *>(gkeys);
+    uint4 *dst4 = reinterpret_cast<uint4 *>(topk_keys_s);
+    for (int64_t i0 = 0; i0 < n4; i0 += 4 * kTopkThreads) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
+        if (i < n4) v[u] = __ldcg(src4 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
+        if (i < n4) dst4[i] = v[u];
+      }
+    }
+    for (int64_t i = n4 * 4 + threadIdx.x; i < nc; i += blockDim.x) topk_keys_s[i] = __ldcg(gkeys + i);
+    __syncthreads();
+  }
+  const uint32_t *keys = staged ? topk_keys_s : gkeys;
+  // Radix select of the need-th largest key: digits of 11, 11 and 10 bits.
   uint32_t prefix = 0, mask = 0;
   uint32_t remaining = (uint32_t)need;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int e = threadIdx.x; e < 256; e += blockDim.x) hist[e] = 0;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = shifts[pass];
+    const uint32_t nb = 1u << widths[pass], dmask = nb - 1u;
+    for (int e = threadIdx.x; e < (int)nb; e += blockDim.x) hist[e] = 0;
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < nc; i += blockDim.x) {
-      const uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    for (int64_t i0 = 0; i0 < nc; i0 += 4 * (int64_t)blockDim.x) {
+      uint32_t kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // loads first, so up to 4 are in flight
+        const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
+        kv[u] = (i < nc) ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
+        const bool act = (i < nc) && ((kv[u] & mask) == prefix);
+        hist_add(hist, (kv[u] >> shift) & dmask, act);
+      }
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-      // Warp 0 walks the digits from the top, 8 per lane.
+      // Warp 0 walks the bins from the top; lane l owns nb/32 consecutive bins.
       const int lane = threadIdx.x;
-      uint32_t cnt[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
+      const int per = (int)nb / 32;
+      uint32_t sum = 0;
+      for (int j = 0; j < per; ++j) sum += hist[nb - 1 - (lane * per + j)];
       uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      uint32_t run = incl - sum;  // keys in higher digits than this lane's first
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (run < remaining && run + cnt[j] >= remaining) {
-          sh_digit = 255u - (uint32_t)(lane * 8 + j);
-          sh_above = run;
+      uint32_t run = incl - sum;
+      if (run < remaining && incl >= remaining) {
+        for (int j = 0; j < per; ++j) {
+          const uint32_t bin = nb - 1 - (uint32_t)(lane * per + j);
+          const uint32_t c = hist[bin];
+          if (run + c >= remaining) {
+            sh_digit = bin;
+            sh_above = run;
+            break;
+          }
+          run += c;
         }
-        run += cnt[j];
       }
     }
     __syncthreads();
     remaining -= sh_above;
     prefix |= sh_digit << shift;
-    mask |= 255u << shift;
+    mask |= dmask << shift;
     __syncthreads();
   }
   const uint32_t tau = prefix;

@@ -30,7 +30,7 @@ inline size_t esize(s4r_dtype dt) { return dt == S4R_BF16 ? 2 : 4; }
 
 // Byte offsets of the decode workspace regions.
 struct Layout {
-  size_t status, barrier, cq, qt, tstat, rstat, rowsum, scores, pooled, part, total;
+  size_t status, barrier, cq, cqs, cq64, tickets, att_tickets, qt, tstat, rstat, rowsum, scores, pooled, part, total;
 };
 
 Layout layout_for(const Shape &s) {
@@ -40,6 +40,11 @@ Layout layout_for(const Shape &s) {
   l.barrier = off + 64;
   off += kAlign;
   l.cq = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_rows * s.rank_k);
+  const size_t n_cb = (size_t)ceil_div(s.rank_k, kProjColBlock);
+  l.cqs = off; off += round_up((size_t)s.batch * n_cb * cqs_block_bytes(s.n_rows));
+  l.cq64 = off; off += round_up(sizeof(double) * s.batch * (size_t)s.n_rows * s.rank_k);
+  l.tickets = off; off += round_up(sizeof(unsigned int) * s.batch * n_cb);
+  l.att_tickets = off; off += round_up(sizeof(unsigned int) * s.batch * (size_t)s.n_heads_kv);
   l.qt = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * s.rank_k);
   const size_t n_tiles = (size_t)ceil_div(s.cache_rows, kScoreTile);
   l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
@@ -74,6 +79,7 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
       a->pool_kernel > S4R_MAX_POOL_KERNEL)
     return S4R_ERR_UNSUPPORTED;
   if (a->cache_rows + a->n_sink > INT32_MAX) return S4R_ERR_UNSUPPORTED;
+  if (a->n_sink > kAttMaxSinks) return S4R_ERR_UNSUPPORTED;
   s->batch = a->batch;
   s->n_heads_q = a->n_heads_q;
   s->n_heads_kv = a->n_heads_kv;
@@ -90,6 +96,7 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
   s->group = (int32_t)G;
   s->n_rows = (int32_t)R;
   s->cache_rows = a->cache_rows;
+  if (att_smem_bytes(*s, a->dtype == S4R_BF16 ? 2 : 4) > 232448) return S4R_ERR_UNSUPPORTED;
   return S4R_OK;
 }
 
@@ -180,7 +187,7 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
 
 template <int R>
 s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s, const int32_t *lengths,
-                           const float *cq, float *scores, double *rowsum, unsigned long long *bar, uint32_t *status,
+                           const unsigned char *cqs, float *scores, double *rowsum, unsigned long long *bar, uint32_t *status,
                            cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
@@ -192,7 +199,7 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cq, scores, rowsum, bar, status) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status) == cudaSuccess
              ? S4R_OK
              : S4R_ERR_CUDA;
 }
@@ -206,6 +213,10 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   double *tstat = reinterpret_cast<double *>(ws + ly.tstat);
   double *rstat = reinterpret_cast<double *>(ws + ly.rstat);
   double *rowsum = reinterpret_cast<double *>(ws + ly.rowsum);
+  unsigned char *cqs = ws + ly.cqs;
+  double *cq64 = reinterpret_cast<double *>(ws + ly.cq64);
+  unsigned int *tickets = reinterpret_cast<unsigned int *>(ws + ly.tickets);
+  unsigned int *att_tickets = reinterpret_cast<unsigned int *>(ws + ly.att_tickets);
   unsigned long long *bar = reinterpret_cast<unsigned long long *>(ws + ly.barrier);
   float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
   float *pooled = reinterpret_cast<float *>(ws + ly.pooled);
@@ -220,9 +231,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
 
   // 1. query projection
   {
-    dim3 grid((unsigned)ceil_div(s.n_rows + s.n_heads_q, kProjRows),
-              (unsigned)ceil_div(s.rank_k, kProjCols), (unsigned)s.batch);
-    project_kernel<T><<<grid, kProjRows * kProjCols, 0, st>>>(s, q, bk, cq, qt, rowsum, bar);
+    dim3 grid((unsigned)s.n_heads_kv, (unsigned)ceil_div(s.rank_k, kProjColBlock), (unsigned)s.batch);
+    project_kernel<T><<<grid, kProjThreads, 0, st>>>(s, q, bk, cq, cqs, qt, cq64, tickets, rowsum, bar);
   }
   // 2. latent scoring
   const unsigned n_tiles = (unsigned)ceil_div(s.cache_rows, kScoreTile);
@@ -234,8 +244,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     if (!make_tmap_bf16(&tmap, ck, (uint64_t)s.rank_k, (uint64_t)s.batch * s.cache_rows, (uint64_t)s.rank_k * 2, 64,
                         kStcTile))
       return S4R_ERR_CUDA;
-    const s4r_status rc = plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cq, scores, rowsum, bar, status, st)
-                                       : launch_score_tc<32>(plan, tmap, s, a->lengths, cq, scores, rowsum, bar, status, st);
+    const s4r_status rc = plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, bar, status, st)
+                                       : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, bar, status, st);
     if (rc != S4R_OK) return rc;
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
@@ -253,15 +263,17 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     pool_kernel<<<dim3((unsigned)ceil_div(s.cache_rows, 256), s.batch), 256, 0, st>>>(s, a->lengths, scores, pooled);
     keys = pooled;
   }
-  if (s.top_k > 0)
-    topk_kernel<<<s.batch, kTopkThreads, 0, st>>>(s, a->lengths, keys, a->idx, status);
-  // 4. rebuild + exact attention
+  if (s.top_k > 0) {
+    const size_t smem = topk_smem_bytes(s.cache_rows);
+    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    topk_kernel<<<s.batch, kTopkThreads, smem, st>>>(s, a->lengths, keys, a->idx, status);
+  }
+  // 4. rebuild + exact attention (the last CTA of each kv group merges)
   {
-    const int n_split = att_splits(s);
-    attend_partial<T><<<dim3(n_split, s.n_heads_kv, s.batch), kAttThreads, 0, st>>>(
-        s, a->lengths, a->idx, ck, cv, qt, part);
-    const size_t smem = sizeof(float) * (s.rank_v + s.n_sink + 1);
-    attend_combine<T><<<dim3(s.n_heads_q, s.batch), 256, smem, st>>>(s, q, bv, sk, sv, part, a->out);
+    const size_t smem = att_smem_bytes(s, sizeof(T));
+    cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attend_kernel<T><<<dim3(att_splits(s), s.n_heads_kv, s.batch), kAttThreads, smem, st>>>(
+        s, a->lengths, a->idx, ck, cv, qt, q, bv, sk, sv, part, att_tickets, a->out);
   }
   return last_cuda();
 }
@@ -285,13 +297,13 @@ int32_t s4r_decode_kernel_launches(const s4r_decode_args *args) {
   else if (s.cache_rows > 0) n += 3;              // scoring: stats, merge, final
   if (s.pool_kernel > 1 && s.cache_rows > 0) n += 1;
   if (s.top_k > 0) n += 1;
-  n += 2;                                         // attention: partial, combine
+  n += 1;                                         // attention (fused combine)
   return n;
 }
 
 s4r_status s4r_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
   if (!workspace || workspace_bytes < kAlign || !aligned16(workspace)) return S4R_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(workspace, 0, kAlign, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return S4R_ERR_CUDA;
   return S4R_OK;
 }
