@@ -71,6 +71,9 @@ typedef enum { S4R_ROWS_CONCAT = 0, S4R_ROWS_PER_HEAD = 1 } s4r_row_mode;
 #define S4R_MAX_HEAD_DIM 256    /* multiple of 8 */
 #define S4R_MAX_SCORE_ROWS 256  /* W*G (CONCAT) or W*H_q (PER_HEAD) */
 #define S4R_MAX_POOL_KERNEL 63  /* odd */
+#define S4R_MAX_GROUP 8         /* G = n_heads_q / n_heads_kv */
+#define S4R_MAX_SINKS 16        /* n_sink */
+#define S4R_MAX_SELECTED 8192   /* top_k + local_window */
 
 /* ------------------------------------------------------------------ encode */
 
@@ -191,6 +194,11 @@ s4r_status s4r_clear_device_status(void *workspace, void *stream);
 
 /* Static description of a status code. */
 const char *s4r_status_string(s4r_status status);
+
+/* Human-readable description of the last S4R_ERR_CUDA returned on the
+ * calling host thread (which step failed and the CUDA error name); "" if
+ * none.  The string stays valid until the next failing call on the thread. */
+const char *s4r_last_error(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int32_t s4r_version(void);

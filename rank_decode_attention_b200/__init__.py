@@ -28,7 +28,9 @@ _DTYPE = {torch.float32: S4R_F32, torch.bfloat16: S4R_BF16}
 
 class S4RError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {s4r_status_string(status)} (status {status})")
+        detail = s4r_last_error() if status == S4R_ERR_CUDA else ""
+        super().__init__(f"{what}: {s4r_status_string(status)} (status {status})"
+                         + (f" -- {detail}" if detail else ""))
         self.status = status
 
 
@@ -75,6 +77,7 @@ SIGNATURES = {
     "s4r_clear_device_status": (ctypes.c_int, [_vp, _vp]),
     "s4r_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "s4r_version": (_i32, []),
+    "s4r_last_error": (ctypes.c_char_p, []),
 }
 
 _lib = None
@@ -119,6 +122,10 @@ def _check(status: int, what: str) -> int:
 
 def s4r_status_string(status: int) -> str:
     return lib().s4r_status_string(status).decode()
+
+
+def s4r_last_error() -> str:
+    return (lib().s4r_last_error() or b"").decode()
 
 
 def s4r_version() -> int:

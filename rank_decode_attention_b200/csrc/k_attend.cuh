@@ -12,7 +12,7 @@
 // rows of the basis that belong to group g.  Nothing is rounded to the
 // storage type; all arithmetic is fp32.
 //
-// One launch, CTA (split, g, problem), 128 threads:
+// One launch, CTA (split, g, problem), 256 threads:
 //   1. cp.async the split's selected C_K / C_V rows (<= 64) into shared memory;
 //   2. logits of the G heads of group g, their softmax partials (max, sum) and
 //      the latent value sums acc[j][:] = sum_e p[j][e] c_V[e];
@@ -25,7 +25,8 @@
 
 namespace s4r {
 
-constexpr int kAttThreads = 128;      // 4 warps
+constexpr int kAttThreads = 256;      // 8 warps
+constexpr int kAttMaxSplits = 128;    // (top_k + local_window) <= 128 * 64
 constexpr int kAttEntries = 64;       // selected rows per split
 constexpr int kAttMaxGroup = 8;       // G <= 8
 constexpr int kAttMaxSinks = 16;      // sinks merged by the combining CTA
@@ -52,7 +53,8 @@ __host__ __device__ inline size_t att_stage_bytes(const Shape &s, int esize) {
 __host__ inline size_t att_smem_bytes(const Shape &s, int esize) {
   return att_stage_bytes(s, esize) +
          sizeof(float) * (size_t)(kAttMaxGroup * s.rank_k + kAttMaxGroup * kAttEntries + 4 * kAttMaxGroup +
-                                  kAttMaxGroup * s.rank_v + kAttMaxGroup * kAttMaxSinks);
+                                  kAttMaxGroup * s.rank_v + kAttMaxGroup * kAttMaxSinks +
+                                  kAttMaxGroup * kAttMaxSplits);
 }
 
 // Row number of selected entry e (top-k list first, then the window).
@@ -97,6 +99,7 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   float *ml_s = p_s + kAttMaxGroup * kAttEntries;                     // [G][4]
   float *acc_s = ml_s + 4 * kAttMaxGroup;                             // [G][rv]
   float *sw_s = acc_s + kAttMaxGroup * rv;                            // [G][kAttMaxSinks]
+  float *f_s = sw_s + kAttMaxGroup * kAttMaxSinks;                    // [G][kAttMaxSplits]
   __shared__ int64_t rows_s[kAttEntries];
   __shared__ int last_flag;
 
@@ -152,8 +155,8 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
     p_s[j * kAttEntries + e] = l;
   }
   __syncthreads();
-  // 2b. softmax partial per head: warp w takes heads w, w+4.
-  for (int j = wid; j < G; j += 4) {
+  // 2b. softmax partial per head: warp w takes head w.
+  for (int j = wid; j < G; j += kAttThreads / 32) {
     const float l0 = p_s[j * kAttEntries + lane], l1 = p_s[j * kAttEntries + lane + 32];
     const float m = warp_max(fmaxf(l0, l1));
     const float p0 = (m == -INFINITY) ? 0.f : __expf(l0 - m);
@@ -206,7 +209,7 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   }
   // Sink logits: one warp per (head, sink).
   const float qscale = rsqrtf((float)dh);
-  for (int t = wid; t < G * ns; t += 4) {
+  for (int t = wid; t < G * ns; t += kAttThreads / 32) {
     const int j = t / ns, tk = t - j * ns;
     const T *qh = q + (((int64_t)b * s.query_window + s.query_window - 1) * s.n_heads_q + g * G + j) * dh;
     const T *kr = sink_k + ((int64_t)b * ns + tk) * Dp + (int64_t)g * dh;
@@ -216,41 +219,56 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
     if (lane == 0) sw_s[j * kAttMaxSinks + tk] = d * qscale;
   }
   __syncthreads();
-  // Merge statistics per head: warp w takes heads w, w+4.
-  for (int j = wid; j < G; j += 4) {
+  // Merge statistics per head (warp w takes head w): weights of the splits
+  // f[j][sp] = exp(m_sp - M) / den and of the sinks, into shared memory.
+  for (int j = wid; j < G; j += kAttThreads / 32) {
     const float *pb = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2);
+    float ms[kAttMaxSplits / 32], ls[kAttMaxSplits / 32];
     float M = -INFINITY;
-    for (int sp = lane; sp < n_split; sp += 32) M = fmaxf(M, __ldcg(pb + sp * (rv + 2)));
+#pragma unroll
+    for (int u = 0; u < kAttMaxSplits / 32; ++u) {
+      const int sp = lane + 32 * u;
+      ms[u] = sp < n_split ? __ldcg(pb + sp * (rv + 2)) : -INFINITY;
+      ls[u] = sp < n_split ? __ldcg(pb + sp * (rv + 2) + 1) : 0.f;
+      M = fmaxf(M, ms[u]);
+    }
     for (int tk = lane; tk < ns; tk += 32) M = fmaxf(M, sw_s[j * kAttMaxSinks + tk]);
     M = warp_max(M);
     float den = 0.f;
-    for (int sp = lane; sp < n_split; sp += 32) {
-      const float ms = __ldcg(pb + sp * (rv + 2));
-      if (ms != -INFINITY) den += __ldcg(pb + sp * (rv + 2) + 1) * __expf(ms - M);
+#pragma unroll
+    for (int u = 0; u < kAttMaxSplits / 32; ++u) {
+      ms[u] = (ms[u] == -INFINITY) ? 0.f : __expf(ms[u] - M);
+      den += ls[u] * ms[u];
     }
     for (int tk = lane; tk < ns; tk += 32) den += __expf(sw_s[j * kAttMaxSinks + tk] - M);
     den = warp_sum(den);
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    if (lane == 0) {
-      ml_s[j * 4 + 2] = M;
-      ml_s[j * 4 + 3] = inv;
+#pragma unroll
+    for (int u = 0; u < kAttMaxSplits / 32; ++u) {
+      const int sp = lane + 32 * u;
+      if (sp < n_split) f_s[j * kAttMaxSplits + sp] = ms[u] * inv;
     }
     __syncwarp();
     for (int tk = lane; tk < ns; tk += 32)
       sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
   }
   __syncthreads();
-  // Latent accumulator per head: acc[j][k] = sum_split w_split acc_split[k].
+  // Latent accumulator per head: acc[j][k] = sum_split f[j][split] acc_split[k];
+  // the split loads are independent, four in flight.
   for (int t = threadIdx.x; t < G * rv; t += blockDim.x) {
     const int j = t / rv, k = t - j * rv;
-    const float *pb = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2);
-    const float M = ml_s[j * 4 + 2], inv = ml_s[j * 4 + 3];
+    const float *pb = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2) + 2 + k;
     float a = 0.f;
-    for (int sp = 0; sp < n_split; ++sp) {
-      const float ms = __ldcg(pb + sp * (rv + 2));
-      if (ms != -INFINITY) a = fmaf(__expf(ms - M), __ldcg(pb + sp * (rv + 2) + 2 + k), a);
+    int sp = 0;
+    for (; sp + 4 <= n_split; sp += 4) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldcg(pb + (sp + u) * (rv + 2));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a = fmaf(f_s[j * kAttMaxSplits + sp + u], v[u], a);
     }
-    acc_s[j * rv + k] = a * inv;
+    for (; sp < n_split; ++sp) a = fmaf(f_s[j * kAttMaxSplits + sp], __ldcg(pb + sp * (rv + 2)), a);
+    acc_s[j * rv + k] = a;
   }
   cp_async_wait_all();
   __syncthreads();

@@ -4,7 +4,7 @@
 // the key subspace; the sliding query window is then scored in latent space
 // (Eqs. 8-10).  Every per-head projection
 //     p[w][h][c] = q[w][h] . B^K[g*d_h : (g+1)*d_h][c],   g = h / G,
-// is computed once (CTA (g, 64-column block, problem)), and from it
+// is computed once (CTA (g, 64-column block, 16-row block, problem)), and from it
 //   * CONCAT rows:   C_Q[w*G + j] = sum_g p[w][g*G + j]   (row = Q'[w][j] . B^K)
 //   * PER_HEAD rows: C_Q[w*H_q + h] = p[w][h]
 //   * qt[h] = p[W-1][h] / sqrt(d_h), the current query in latent form for the
@@ -24,9 +24,9 @@
 
 namespace s4r {
 
-constexpr int kProjThreads = 256;
+constexpr int kProjThreads = 128;
 constexpr int kProjColBlock = 64;   // columns per CTA (= one 128-byte swizzle row of bf16)
-constexpr int kProjRowBlock = 64;   // per-head rows (w, j) staged at once
+constexpr int kProjRowBlock = 16;   // per-head rows (w, j) per CTA
 
 // Shared-memory image of the split C_Q operand: bytes per 64-column block.
 __host__ __device__ constexpr int cqs_block_bytes(int R) { return 3 * R * 128; }
@@ -37,101 +37,112 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
                unsigned char *__restrict__ cqs, float *__restrict__ qt, double *__restrict__ cq64,
                unsigned int *__restrict__ tickets, double *__restrict__ row_sum,
                unsigned long long *__restrict__ barrier) {
-  __shared__ float qs[kProjRowBlock][65];            // per-head query rows of group g, 64 of d_h
+  __shared__ float qs[kProjRowBlock][65];            // per-head query rows, 64 of d_h
   __shared__ float bs[64][kProjColBlock + 1];        // basis slice, 64 rows of d_h
   __shared__ int last_flag;
-  const int g = blockIdx.x, cb = blockIdx.y, b = blockIdx.z;
+  const int g = blockIdx.x, cb = blockIdx.y;
+  const int n_rb = (int)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
+  const int rb = blockIdx.z % n_rb, b = blockIdx.z / n_rb;
   const int G = s.group, W = s.query_window, Hq = s.n_heads_q, dh = s.head_dim, r = s.rank_k;
   const int R = s.n_rows;
   const int c0 = cb * kProjColBlock;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16: 4 rows x 4 cols each
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 8: 2 rows x 4 cols each
   const T *qb = q + (int64_t)b * W * Hq * dh;
   const T *Bb = basis_k + (int64_t)b * s.d_model * r;
   double *cq64b = cq64 + (int64_t)b * R * r;
   // Reset the per-call accumulators of the tensor-core scoring kernel.
-  if (g == 0 && cb == 0) {
+  if (g == 0 && cb == 0 && rb == 0) {
     for (int e = threadIdx.x; e < R; e += blockDim.x) row_sum[(int64_t)b * R + e] = 0.0;
     if (b == 0 && threadIdx.x == 0) *barrier = 0ull;
   }
   const int n_prow = W * G;  // per-head rows (w, j) of this group
-  for (int pr0 = 0; pr0 < n_prow; pr0 += kProjRowBlock) {
-    double acc[4][4];
+  const int pr0 = rb * kProjRowBlock;
+  double acc[2][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int t0 = 0; t0 < dh; t0 += 64) {
-      const int tn = smin(64, dh - t0);
-      __syncthreads();
-      // 16 independent loads per thread for each operand (fully unrolled).
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  for (int t0 = 0; t0 < dh; t0 += 64) {
+    const int tn = smin(64, dh - t0);
+    __syncthreads();
+    // All loads of the chunk are independent and issued before any use.
+    float qv[(kProjRowBlock * 64) / kProjThreads], bv[(64 * kProjColBlock) / kProjThreads];
 #pragma unroll
-      for (int u = 0; u < (kProjRowBlock * 64) / kProjThreads; ++u) {
-        const int e = threadIdx.x + u * kProjThreads;
-        const int pr = e >> 6, t = e & 63;
-        const int row = pr0 + pr;
-        float v = 0.f;
-        if (row < n_prow && t < tn) {
-          const int w = row / G, j = row - w * G;
-          v = to_f(qb[((int64_t)w * Hq + g * G + j) * dh + t0 + t]);
-        }
-        qs[pr][t] = v;
+    for (int u = 0; u < (kProjRowBlock * 64) / kProjThreads; ++u) {
+      const int e = threadIdx.x + u * kProjThreads;
+      const int pr = e >> 6, t = e & 63;
+      const int row = pr0 + pr;
+      qv[u] = 0.f;
+      if (row < n_prow && t < tn) {
+        const int w = row / G, j = row - w * G;
+        qv[u] = to_f(qb[((int64_t)w * Hq + g * G + j) * dh + t0 + t]);
       }
-#pragma unroll
-      for (int u = 0; u < (64 * kProjColBlock) / kProjThreads; ++u) {
-        const int e = threadIdx.x + u * kProjThreads;
-        const int t = e >> 6, c = e & 63;
-        bs[t][c] = (t < tn && c0 + c < r) ? to_f(Bb[(int64_t)(g * dh + t0 + t) * r + c0 + c]) : 0.f;
-      }
-      __syncthreads();
-      float part[4][4] = {};
-#pragma unroll 8
-      for (int k = 0; k < 64; ++k) {
-        float a[4], bb[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = qs[ty + 16 * i][k];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) bb[j] = bs[k][tx + 16 * j];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], bb[j], part[i][j]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = pr0 + ty + 16 * i;
-      if (row >= n_prow) continue;
-      const int w = row / G, j = row - w * G, h = g * G + j;
+    for (int u = 0; u < (64 * kProjColBlock) / kProjThreads; ++u) {
+      const int e = threadIdx.x + u * kProjThreads;
+      const int t = e >> 6, c = e & 63;
+      bv[u] = (t < tn && c0 + c < r) ? to_f(Bb[(int64_t)(g * dh + t0 + t) * r + c0 + c]) : 0.f;
+    }
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int c = c0 + tx + 16 * jj;
-        if (c >= r) continue;
-        const double v = acc[i][jj];
-        if (w == W - 1) qt[((int64_t)b * Hq + h) * r + c] = (float)(v / sqrt((double)dh));
-        if (s.row_mode == S4R_ROWS_CONCAT)
-          atomicAdd(&cq64b[(int64_t)(w * G + j) * r + c], v);
-        else
-          cq64b[(int64_t)(w * Hq + h) * r + c] = v;
-      }
+    for (int u = 0; u < (kProjRowBlock * 64) / kProjThreads; ++u) {
+      const int e = threadIdx.x + u * kProjThreads;
+      qs[e >> 6][e & 63] = qv[u];
+    }
+#pragma unroll
+    for (int u = 0; u < (64 * kProjColBlock) / kProjThreads; ++u) {
+      const int e = threadIdx.x + u * kProjThreads;
+      bs[e >> 6][e & 63] = bv[u];
+    }
+    __syncthreads();
+    float part[2][4] = {};
+#pragma unroll 16
+    for (int k = 0; k < 64; ++k) {
+      float a[2], bb[4];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) a[i] = qs[ty + 8 * i][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bb[j] = bs[k][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], bb[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int row = pr0 + ty + 8 * i;
+    if (row >= n_prow) continue;
+    const int w = row / G, j = row - w * G, h = g * G + j;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int c = c0 + tx + 16 * jj;
+      if (c >= r) continue;
+      const double v = acc[i][jj];
+      if (w == W - 1) qt[((int64_t)b * Hq + h) * r + c] = (float)(v / sqrt((double)dh));
+      if (s.row_mode == S4R_ROWS_CONCAT)
+        atomicAdd(&cq64b[(int64_t)(w * G + j) * r + c], v);
+      else
+        cq64b[(int64_t)(w * Hq + h) * r + c] = v;
     }
   }
-  // Ticket: the last of the H_kv group CTAs of this column block finishes the rows.
+  // Ticket: the last of the (group, row block) CTAs of this column block finishes the rows.
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned int t = atomicAdd(&tickets[(int64_t)b * gridDim.y + cb], 1u);
-    last_flag = (t == gridDim.x - 1);
+    last_flag = (t == gridDim.x * (unsigned int)n_rb - 1);
   }
   __syncthreads();
   if (!last_flag) return;
   __threadfence();
   const double scale = 1.0 / sqrt((double)r);
   unsigned char *blk = cqs + ((int64_t)b * gridDim.y + cb) * cqs_block_bytes(R);
-  constexpr int kU = 4;  // loads in flight per thread
+  constexpr int kU = 8;  // loads in flight per thread
   for (int e0 = 0; e0 < R * kProjColBlock; e0 += kU * kProjThreads) {
     double xs[kU];
 #pragma unroll

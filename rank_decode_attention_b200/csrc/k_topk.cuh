@@ -66,24 +66,40 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_t
 }
 
 constexpr int kTopkSmemKeys = 40960;  // keys staged in shared memory (160 KB) when they fit
-constexpr int kTopkBins = 2048;
+constexpr int kTopkBins = 256;     // 8-bit digits, 4 passes
+constexpr int kTopkWarps = kTopkThreads / 32;
 __host__ inline size_t topk_smem_bytes(int64_t cache_rows) {
   return sizeof(uint32_t) * (size_t)smin<int64_t>(cache_rows, kTopkSmemKeys);
 }
 
-// Histogram update aggregated across the lanes of a warp that share a bin
-// (scores of one problem share their high bits, so plain atomics serialise).
-__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t bin, bool active) {
-  const uint32_t key = active ? bin : 0xffffffffu;
-  const uint32_t peers = __match_any_sync(0xffffffffu, key);
-  const int leader = __ffs(peers) - 1;
-  if (active && (threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+// One histogram pass over the keys into the calling warp's private
+// histogram (scores of one problem share their high bits, so a single shared
+// histogram would serialise every warp on a few bins).  `keys` is either the
+// shared-memory copy or the global row; both are read with plain loads of
+// their own address space.
+template <bool kShared>
+__device__ __forceinline__ void hist_pass(const uint32_t *keys, int64_t nc, uint32_t mask, uint32_t prefix,
+                                          int shift, uint32_t *whist) {
+  for (int64_t i0 = 0; i0 < nc; i0 += 4 * (int64_t)blockDim.x) {
+    uint32_t kv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
+      kv[u] = (i < nc) ? (kShared ? keys[i] : __ldcg(keys + i)) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
+      if (i < nc && (kv[u] & mask) == prefix) atomicAdd(&whist[(kv[u] >> shift) & 255u], 1u);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restrict__ keys_all,
             int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) uint32_t topk_keys_s[];
+  __shared__ uint32_t whist[kTopkWarps][kTopkBins];
   __shared__ uint32_t hist[kTopkBins];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t sh_total, sh_digit, sh_above;
@@ -106,9 +122,13 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
   // Stage the keys in shared memory when they fit (16-byte loads, all in flight).
   const bool staged = nc <= kTopkSmemKeys;
   if (staged) {
-    const int64_t n4 = nc / 4;
-    const uint4 *src4 = reinterpret_cast<const uint4 *>(gkeys);
-    uint4 *dst4 = reinterpret_cast<uint4 *>(topk_keys_s);
+    // Row b starts at b * cache_rows floats, which need not be 16-byte
+    // aligned: copy the head up to the first aligned key one by one, the
+    // aligned middle with 16-byte loads, and the tail one by one.
+    const int64_t head = smin<int64_t>(nc, (int64_t)((16u - (reinterpret_cast<uintptr_t>(gkeys) & 15u)) & 15u) / 4);
+    const int64_t n4 = (nc - head) / 4;
+    const uint4 *src4 = reinterpret_cast<const uint4 *>(gkeys + head);
+    for (int64_t i = threadIdx.x; i < head; i += blockDim.x) topk_keys_s[i] = __ldcg(gkeys + i);
     for (int64_t i0 = 0; i0 < n4; i0 += 4 * kTopkThreads) {
       uint4 v[4];
 #pragma unroll
@@ -119,44 +139,39 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
-        if (i < n4) dst4[i] = v[u];
+        if (i < n4) {
+          uint32_t *d = topk_keys_s + head + 4 * i;   // shared copy may be unaligned too: scalar stores
+          d[0] = v[u].x; d[1] = v[u].y; d[2] = v[u].z; d[3] = v[u].w;
+        }
       }
     }
-    for (int64_t i = n4 * 4 + threadIdx.x; i < nc; i += blockDim.x) topk_keys_s[i] = __ldcg(gkeys + i);
+    for (int64_t i = head + 4 * n4 + threadIdx.x; i < nc; i += blockDim.x) topk_keys_s[i] = __ldcg(gkeys + i);
     __syncthreads();
   }
-  const uint32_t *keys = staged ? topk_keys_s : gkeys;
-  // Radix select of the need-th largest key: digits of 11, 11 and 10 bits.
+  // Radix select of the need-th largest key, 8-bit digits from the top.
   uint32_t prefix = 0, mask = 0;
   uint32_t remaining = (uint32_t)need;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const uint32_t nb = 1u << widths[pass], dmask = nb - 1u;
-    for (int e = threadIdx.x; e < (int)nb; e += blockDim.x) hist[e] = 0;
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int j = 0; j < kTopkBins / 32; ++j) whist[wid][lane + 32 * j] = 0;
+    __syncwarp();
+    if (staged)
+      hist_pass<true>(topk_keys_s, nc, mask, prefix, shift, whist[wid]);
+    else
+      hist_pass<false>(gkeys, nc, mask, prefix, shift, whist[wid]);
     __syncthreads();
-    for (int64_t i0 = 0; i0 < nc; i0 += 4 * (int64_t)blockDim.x) {
-      uint32_t kv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {  // loads first, so up to 4 are in flight
-        const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
-        kv[u] = (i < nc) ? keys[i] : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
-        const bool act = (i < nc) && ((kv[u] & mask) == prefix);
-        hist_add(hist, (kv[u] >> shift) & dmask, act);
-      }
+    if (threadIdx.x < kTopkBins) {
+      uint32_t c = 0;
+      for (int w = 0; w < kTopkWarps; ++w) c += whist[w][threadIdx.x];
+      hist[threadIdx.x] = c;
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-      // Warp 0 walks the bins from the top; lane l owns nb/32 consecutive bins.
-      const int lane = threadIdx.x;
-      const int per = (int)nb / 32;
-      uint32_t sum = 0;
-      for (int j = 0; j < per; ++j) sum += hist[nb - 1 - (lane * per + j)];
+      // Warp 0 walks the digits from the top, 8 per lane.
+      uint32_t cnt[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
       uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -164,23 +179,19 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
         if (lane >= o) incl += y;
       }
       uint32_t run = incl - sum;
-      if (run < remaining && incl >= remaining) {
-        for (int j = 0; j < per; ++j) {
-          const uint32_t bin = nb - 1 - (uint32_t)(lane * per + j);
-          const uint32_t c = hist[bin];
-          if (run + c >= remaining) {
-            sh_digit = bin;
-            sh_above = run;
-            break;
-          }
-          run += c;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (run < remaining && run + cnt[j] >= remaining) {
+          sh_digit = 255u - (uint32_t)(lane * 8 + j);
+          sh_above = run;
         }
+        run += cnt[j];
       }
     }
     __syncthreads();
     remaining -= sh_above;
     prefix |= sh_digit << shift;
-    mask |= dmask << shift;
+    mask |= 255u << shift;
     __syncthreads();
   }
   const uint32_t tau = prefix;
@@ -191,7 +202,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
   const int64_t i1 = smin<int64_t>(nc, i0 + chunk);
   uint32_t n_gt = 0, n_eq = 0;
   for (int64_t i = i0; i < i1; ++i) {
-    const uint32_t key = keys[i];
+    const uint32_t key = staged ? topk_keys_s[i] : __ldcg(gkeys + i);
     n_gt += key > tau;
     n_eq += key == tau;
   }
@@ -200,7 +211,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
   const uint32_t out_before = block_excl_scan(n_gt + eq_take, warp_tot, &sh_total);
   uint32_t pos = out_before, eq_seen = 0;
   for (int64_t i = i0; i < i1; ++i) {
-    const uint32_t key = keys[i];
+    const uint32_t key = staged ? topk_keys_s[i] : __ldcg(gkeys + i);
     bool take = key > tau;
     if (key == tau) { take = eq_seen < eq_take; ++eq_seen; }
     if (take && pos < (uint32_t)k) out[pos++] = (int32_t)(s.n_sink + i);

@@ -8,6 +8,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
@@ -20,6 +21,10 @@
 #include "k_topk.cuh"
 
 using namespace s4r;
+
+static_assert(S4R_MAX_GROUP <= kAttMaxGroup && S4R_MAX_SINKS <= kAttMaxSinks &&
+                  S4R_MAX_SELECTED <= kAttMaxSplits * kAttEntries,
+              "header limits must fit the attention kernel");
 
 namespace {
 
@@ -75,11 +80,11 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
                                                     : (int64_t)a->query_window * a->n_heads_q;
   if (a->head_dim % 8 || a->rank_k % 8 || a->rank_v % 8) return S4R_ERR_UNSUPPORTED;
   if (a->head_dim > S4R_MAX_HEAD_DIM || Dp > S4R_MAX_D_MODEL || a->rank_k > S4R_MAX_RANK ||
-      a->rank_v > S4R_MAX_RANK || R > S4R_MAX_SCORE_ROWS || G > kAttMaxGroup ||
+      a->rank_v > S4R_MAX_RANK || R > S4R_MAX_SCORE_ROWS || G > S4R_MAX_GROUP ||
       a->pool_kernel > S4R_MAX_POOL_KERNEL)
     return S4R_ERR_UNSUPPORTED;
   if (a->cache_rows + a->n_sink > INT32_MAX) return S4R_ERR_UNSUPPORTED;
-  if (a->n_sink > kAttMaxSinks) return S4R_ERR_UNSUPPORTED;
+  if (a->n_sink > S4R_MAX_SINKS || (int64_t)a->top_k + a->local_window > S4R_MAX_SELECTED) return S4R_ERR_UNSUPPORTED;
   s->batch = a->batch;
   s->n_heads_q = a->n_heads_q;
   s->n_heads_kv = a->n_heads_kv;
@@ -100,7 +105,19 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
   return S4R_OK;
 }
 
-s4r_status last_cuda() { return cudaGetLastError() == cudaSuccess ? S4R_OK : S4R_ERR_CUDA; }
+// Description of the last failure on this host thread (s4r_last_error).
+thread_local char g_last_error[256] = "";
+
+s4r_status fail(const char *what, cudaError_t err) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what, cudaGetErrorName(err), cudaGetErrorString(err));
+  return S4R_ERR_CUDA;
+}
+// Status of the launches enqueued since the previous check, labelled `what`.
+s4r_status check_launch(const char *what) {
+  const cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? S4R_OK : fail(what, err);
+}
+s4r_status last_cuda() { return check_launch("kernel launch"); }
 
 // cuTensorMapEncodeTiled, resolved through the runtime (no link-time libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -199,9 +216,8 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status) == cudaSuccess
-             ? S4R_OK
-             : S4R_ERR_CUDA;
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status);
+  return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (cooperative launch)", err);
 }
 
 template <typename T>
@@ -231,8 +247,10 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
 
   // 1. query projection
   {
-    dim3 grid((unsigned)s.n_heads_kv, (unsigned)ceil_div(s.rank_k, kProjColBlock), (unsigned)s.batch);
+    const unsigned n_rb = (unsigned)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
+    dim3 grid((unsigned)s.n_heads_kv, (unsigned)ceil_div(s.rank_k, kProjColBlock), n_rb * (unsigned)s.batch);
     project_kernel<T><<<grid, kProjThreads, 0, st>>>(s, q, bk, cq, cqs, qt, cq64, tickets, rowsum, bar);
+    if (check_launch("project_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
   // 2. latent scoring
   const unsigned n_tiles = (unsigned)ceil_div(s.cache_rows, kScoreTile);
@@ -242,8 +260,10 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   if (plan.tc) {
     CUtensorMap tmap;
     if (!make_tmap_bf16(&tmap, ck, (uint64_t)s.rank_k, (uint64_t)s.batch * s.cache_rows, (uint64_t)s.rank_k * 2, 64,
-                        kStcTile))
+                        kStcTile)) {
+      snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed for the key-coefficient cache");
       return S4R_ERR_CUDA;
+    }
     const s4r_status rc = plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, bar, status, st)
                                        : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, bar, status, st);
     if (rc != S4R_OK) return rc;
@@ -254,6 +274,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     score_stats_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, tstat);
     score_merge<<<dim3((unsigned)ceil_div(s.n_rows, 8), s.batch), 256, 0, st>>>(s, a->lengths, tstat, rstat);
     score_final_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, rstat, scores);
+    if (check_launch("score (CUDA-core passes)") != S4R_OK) return S4R_ERR_CUDA;
   }
   if (a->profile_events[1])
     cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->profile_events[1]), st, cudaEventRecordExternal);
@@ -267,6 +288,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     const size_t smem = topk_smem_bytes(s.cache_rows);
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     topk_kernel<<<s.batch, kTopkThreads, smem, st>>>(s, a->lengths, keys, a->idx, status);
+    if (check_launch("topk_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
   // 4. rebuild + exact attention (the last CTA of each kv group merges)
   {
@@ -274,6 +296,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attend_kernel<T><<<dim3(att_splits(s), s.n_heads_kv, s.batch), kAttThreads, smem, st>>>(
         s, a->lengths, a->idx, ck, cv, qt, q, bv, sk, sv, part, att_tickets, a->out);
+    if (check_launch("attend_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
   return last_cuda();
 }
@@ -455,5 +478,7 @@ const char *s4r_status_string(s4r_status status) {
 }
 
 int32_t s4r_version(void) { return 100; }
+
+const char *s4r_last_error(void) { return g_last_error; }
 
 }  // extern "C"
