@@ -253,22 +253,42 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
   }
   __syncthreads();
-  // Latent accumulator per head: acc[j][k] = sum_split f[j][split] acc_split[k];
-  // the split loads are independent, four in flight.
-  for (int t = threadIdx.x; t < G * rv; t += blockDim.x) {
-    const int j = t / rv, k = t - j * rv;
-    const float *pb = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2) + 2 + k;
-    float a = 0.f;
-    int sp = 0;
-    for (; sp + 4 <= n_split; sp += 4) {
-      float v[4];
+  // Latent accumulator per head: acc[j][k] = sum_split f[j][split] acc_split[k].
+  // Each thread owns up to kOut outputs and reads their split values in
+  // rounds of 4 splits, so kOut * 4 independent loads are in flight.
+  {
+    constexpr int kOut = 4;
+    const int n_out = G * rv;
+    for (int t0 = 0; t0 < n_out; t0 += kOut * kAttThreads) {
+      const float *src[kOut];
+      float a[kOut];
+      int jj[kOut];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldcg(pb + (sp + u) * (rv + 2));
+      for (int o = 0; o < kOut; ++o) {
+        const int t = t0 + o * kAttThreads + threadIdx.x;
+        const int j = (t < n_out) ? t / rv : 0, k = (t < n_out) ? t - j * rv : 0;
+        jj[o] = j;
+        src[o] = part + ((int64_t)b * s.n_heads_q + g * G + j) * n_split * (rv + 2) + 2 + k;
+        a[o] = 0.f;
+      }
+      for (int sp = 0; sp < n_split; sp += 4) {
+        float v[kOut][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) a = fmaf(f_s[j * kAttMaxSplits + sp + u], v[u], a);
+        for (int o = 0; o < kOut; ++o)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) v[o][u] = (sp + u < n_split) ? __ldcg(src[o] + (sp + u) * (rv + 2)) : 0.f;
+#pragma unroll
+        for (int o = 0; o < kOut; ++o)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (sp + u < n_split) a[o] = fmaf(f_s[jj[o] * kAttMaxSplits + sp + u], v[o][u], a[o]);
+      }
+#pragma unroll
+      for (int o = 0; o < kOut; ++o) {
+        const int t = t0 + o * kAttThreads + threadIdx.x;
+        if (t < n_out) acc_s[t] = a[o];   // acc_s[j * rv + k] == acc_s[t]
+      }
     }
-    for (; sp < n_split; ++sp) a = fmaf(f_s[j * kAttMaxSplits + sp], __ldcg(pb + sp * (rv + 2)), a);
-    acc_s[j * rv + k] = a;
   }
   cp_async_wait_all();
   __syncthreads();

@@ -37,8 +37,8 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
                unsigned char *__restrict__ cqs, float *__restrict__ qt, double *__restrict__ cq64,
                unsigned int *__restrict__ tickets, double *__restrict__ row_sum,
                unsigned long long *__restrict__ barrier) {
-  __shared__ float qs[kProjRowBlock][65];            // per-head query rows, 64 of d_h
-  __shared__ float bs[64][kProjColBlock + 1];        // basis slice, 64 rows of d_h
+  __shared__ float qs[kProjRowBlock][129];           // per-head query rows, 128 of d_h
+  __shared__ float bs[128][kProjColBlock + 1];       // basis slice, 128 rows of d_h
   __shared__ int last_flag;
   const int g = blockIdx.x, cb = blockIdx.y;
   const int n_rb = (int)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
@@ -62,15 +62,16 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-  for (int t0 = 0; t0 < dh; t0 += 64) {
-    const int tn = smin(64, dh - t0);
+  for (int t0 = 0; t0 < dh; t0 += 128) {
+    const int tn = smin(128, dh - t0);
     __syncthreads();
-    // All loads of the chunk are independent and issued before any use.
-    float qv[(kProjRowBlock * 64) / kProjThreads], bv[(64 * kProjColBlock) / kProjThreads];
+    // Every load of the 128-wide slice is issued before any is used.
+    constexpr int kQU = (kProjRowBlock * 128) / kProjThreads, kBU = (128 * kProjColBlock) / kProjThreads;
+    float qv[kQU], bv[kBU];
 #pragma unroll
-    for (int u = 0; u < (kProjRowBlock * 64) / kProjThreads; ++u) {
+    for (int u = 0; u < kQU; ++u) {
       const int e = threadIdx.x + u * kProjThreads;
-      const int pr = e >> 6, t = e & 63;
+      const int pr = e >> 7, t = e & 127;
       const int row = pr0 + pr;
       qv[u] = 0.f;
       if (row < n_prow && t < tn) {
@@ -79,39 +80,43 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
       }
     }
 #pragma unroll
-    for (int u = 0; u < (64 * kProjColBlock) / kProjThreads; ++u) {
+    for (int u = 0; u < kBU; ++u) {
       const int e = threadIdx.x + u * kProjThreads;
       const int t = e >> 6, c = e & 63;
       bv[u] = (t < tn && c0 + c < r) ? to_f(Bb[(int64_t)(g * dh + t0 + t) * r + c0 + c]) : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < (kProjRowBlock * 64) / kProjThreads; ++u) {
+    for (int u = 0; u < kQU; ++u) {
       const int e = threadIdx.x + u * kProjThreads;
-      qs[e >> 6][e & 63] = qv[u];
+      qs[e >> 7][e & 127] = qv[u];
     }
 #pragma unroll
-    for (int u = 0; u < (64 * kProjColBlock) / kProjThreads; ++u) {
+    for (int u = 0; u < kBU; ++u) {
       const int e = threadIdx.x + u * kProjThreads;
       bs[e >> 6][e & 63] = bv[u];
     }
     __syncthreads();
-    float part[2][4] = {};
+    // Two 64-term fp32 chunks, each added to the fp64 accumulators.
+#pragma unroll
+    for (int h0 = 0; h0 < 128; h0 += 64) {
+      float part[2][4] = {};
 #pragma unroll 16
-    for (int k = 0; k < 64; ++k) {
-      float a[2], bb[4];
+      for (int k = h0; k < h0 + 64; ++k) {
+        float a[2], bb[4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) a[i] = qs[ty + 8 * i][k];
+        for (int i = 0; i < 2; ++i) a[i] = qs[ty + 8 * i][k];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bb[j] = bs[k][tx + 16 * j];
+        for (int j = 0; j < 4; ++j) bb[j] = bs[k][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], bb[j], part[i][j]);
+      }
 #pragma unroll
       for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], bb[j], part[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
   }
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
@@ -142,7 +147,7 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   __threadfence();
   const double scale = 1.0 / sqrt((double)r);
   unsigned char *blk = cqs + ((int64_t)b * gridDim.y + cb) * cqs_block_bytes(R);
-  constexpr int kU = 8;  // loads in flight per thread
+  constexpr int kU = 16;  // loads in flight per thread
   for (int e0 = 0; e0 < R * kProjColBlock; e0 += kU * kProjThreads) {
     double xs[kU];
 #pragma unroll
@@ -162,11 +167,15 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
         cq64b[(int64_t)i * r + c] = 0.0;
         cq[((int64_t)b * R + i) * r + c] = (float)x;
       }
-      const double y = x * 1.4426950408889634;  // log2(e)
-      const bf16 hi = __double2bfloat16(y);
-      const double r1 = y - (double)__bfloat162float(hi);
-      const bf16 mid = __double2bfloat16(r1);
-      const bf16 lo = __double2bfloat16(r1 - (double)__bfloat162float(mid));
+      // y = x log2(e) as y1 + y2 (fp32 pair, |y2| <= ulp(y1)/2), then three
+      // bf16 terms whose residuals are exact fp32 differences.
+      const double y = x * 1.4426950408889634;
+      const float y1 = (float)y;
+      const float y2 = (float)(y - (double)y1);
+      const bf16 hi = __float2bfloat16_rn(y1);
+      const float r1 = (y1 - __bfloat162float(hi)) + y2;
+      const bf16 mid = __float2bfloat16_rn(r1);
+      const bf16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
       *reinterpret_cast<bf16 *>(blk + sw128_offset(i, kk)) = hi;
       *reinterpret_cast<bf16 *>(blk + sw128_offset(R + i, kk)) = mid;
       *reinterpret_cast<bf16 *>(blk + sw128_offset(2 * R + i, kk)) = lo;

@@ -73,13 +73,15 @@ __host__ inline size_t topk_smem_bytes(int64_t cache_rows) {
 }
 
 // One histogram pass over the keys into the calling warp's private
-// histogram (scores of one problem share their high bits, so a single shared
-// histogram would serialise every warp on a few bins).  `keys` is either the
-// shared-memory copy or the global row; both are read with plain loads of
-// their own address space.
+// histogram.  Scores of one problem share their high bits, so atomics on a
+// shared histogram serialise; instead each warp loops over the distinct
+// digits present among its 32 lanes (one ballot per digit, usually one to
+// three in the high passes, and few keys are still active in the low
+// passes) and lane 0 alone updates the warp's histogram.
 template <bool kShared>
 __device__ __forceinline__ void hist_pass(const uint32_t *keys, int64_t nc, uint32_t mask, uint32_t prefix,
                                           int shift, uint32_t *whist) {
+  const int lane = threadIdx.x & 31;
   for (int64_t i0 = 0; i0 < nc; i0 += 4 * (int64_t)blockDim.x) {
     uint32_t kv[4];
 #pragma unroll
@@ -90,7 +92,15 @@ __device__ __forceinline__ void hist_pass(const uint32_t *keys, int64_t nc, uint
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int64_t i = i0 + u * (int64_t)blockDim.x + threadIdx.x;
-      if (i < nc && (kv[u] & mask) == prefix) atomicAdd(&whist[(kv[u] >> shift) & 255u], 1u);
+      const bool act = (i < nc) && ((kv[u] & mask) == prefix);
+      const uint32_t d = (kv[u] >> shift) & 255u;
+      uint32_t pending = __ballot_sync(0xffffffffu, act);
+      while (pending) {
+        const uint32_t dd = __shfl_sync(0xffffffffu, d, __ffs(pending) - 1);
+        const uint32_t same = __ballot_sync(0xffffffffu, d == dd) & pending;
+        if (lane == 0) whist[dd] += (uint32_t)__popc(same);
+        pending &= ~same;
+      }
     }
   }
 }
