@@ -20,6 +20,7 @@
 // and clears its fp64 accumulators and ticket for the next call.
 #pragma once
 #include "common.cuh"
+#include "k_score_tc.cuh"
 #include "umma.cuh"
 
 namespace s4r {
@@ -36,7 +37,7 @@ __global__ void __launch_bounds__(kProjThreads)
 project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, float *__restrict__ cq,
                unsigned char *__restrict__ cqs, float *__restrict__ qt, double *__restrict__ cq64,
                unsigned int *__restrict__ tickets, double *__restrict__ row_sum,
-               unsigned long long *__restrict__ barrier) {
+               unsigned int *__restrict__ barrier) {
   __shared__ float qs[kProjRowBlock][129];           // per-head query rows, 128 of d_h
   __shared__ float bs[128][kProjColBlock + 1];       // basis slice, 128 rows of d_h
   __shared__ int last_flag;
@@ -52,8 +53,8 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   double *cq64b = cq64 + (int64_t)b * R * r;
   // Reset the per-call accumulators of the tensor-core scoring kernel.
   if (g == 0 && cb == 0 && rb == 0) {
-    for (int e = threadIdx.x; e < R; e += blockDim.x) row_sum[(int64_t)b * R + e] = 0.0;
-    if (b == 0 && threadIdx.x == 0) *barrier = 0ull;
+    for (int e = threadIdx.x; e < kStcSumSlots * R; e += blockDim.x) row_sum[(int64_t)b * kStcSumSlots * R + e] = 0.0;
+    if (b == 0 && threadIdx.x < kBarWords) barrier[threadIdx.x] = 0u;
   }
   const int n_prow = W * G;  // per-head rows (w, j) of this group
   const int pr0 = rb * kProjRowBlock;

@@ -36,6 +36,7 @@ constexpr int kStcTiles = 2;          // tiles per CTA
 constexpr int kStcTmemCols = 512;
 constexpr int kStcTileCols = 256;     // TMEM columns per tile region
 constexpr float kStcRangeLimit = 100.f;
+constexpr int kStcSumSlots = 16;      // row-sum atomics spread over 16 copies per row
 
 __host__ __device__ constexpr int stc_kblocks(int r) { return (r + 63) / 64; }
 __host__ __device__ constexpr int stc_b_bytes(int R, int r) { return stc_kblocks(r) * 3 * R * 128; }
@@ -71,7 +72,7 @@ template <int R>
 __global__ void __launch_bounds__(128, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
                 const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
-                unsigned long long *__restrict__ bar, uint32_t *__restrict__ status) {
+                unsigned int *__restrict__ bar, uint32_t *__restrict__ status) {
   static_assert(R == 32 || R == 64, "scoring rows per CTA");
   extern __shared__ __align__(1024) unsigned char stc_smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -222,7 +223,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       }
       if (part == 0 && row < s.n_rows) {
         const double l = acc + (TPR > 1 ? ctl->half_sum[row] : 0.0);
-        atomicAdd(&row_sum[(int64_t)b * s.n_rows + row], ldexp(l, ctl->kofs[t][row]));
+        atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + blockIdx.x % kStcSumSlots) * s.n_rows + row],
+                  ldexp(l, ctl->kofs[t][row]));
       }
     }
     __syncthreads();
@@ -231,12 +233,22 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   // C: every tile of every problem has added its row sums.
   const bool bar_ok = grid_barrier(bar, status, &ctl->flag);
 
-  // D: scores.
+  // D: scores.  l_row = sum of the row's slots (fixed order).
   if (threadIdx.x < R) {
     const int row = threadIdx.x;
-    const double l = (row < s.n_rows && bar_ok) ? __ldcg(&row_sum[(int64_t)b * s.n_rows + row]) : 0.0;
-    for (int t = 0; t < n_tiles; ++t)
-      ctl->alpha[t][row] = (l > 0.0) ? (float)(ldexp(1.0, ctl->kofs[t][row]) / l) : 0.f;
+    double l = 0.0;
+    if (row < s.n_rows && bar_ok) {
+      double part[kStcSumSlots];
+#pragma unroll
+      for (int q = 0; q < kStcSumSlots; ++q) part[q] = __ldcg(&row_sum[((int64_t)b * kStcSumSlots + q) * s.n_rows + row]);
+#pragma unroll
+      for (int q = 0; q < kStcSumSlots; ++q) l += part[q];
+    }
+    const double inv = (l > 0.0) ? 1.0 / l : 0.0;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int k = ctl->kofs[t][row];
+      ctl->alpha[t][row] = (k == 0) ? (float)inv : (float)ldexp(inv, k);
+    }
   }
   __syncthreads();
   for (int t = 0; t < n_tiles; ++t) {

@@ -54,7 +54,7 @@ Layout layout_for(const Shape &s) {
   const size_t n_tiles = (size_t)ceil_div(s.cache_rows, kScoreTile);
   l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
   l.rstat = off; off += round_up(sizeof(double) * 2 * s.batch * (size_t)s.n_rows);
-  l.rowsum = off; off += round_up(sizeof(double) * s.batch * (size_t)s.n_rows);
+  l.rowsum = off; off += round_up(sizeof(double) * s.batch * (size_t)kStcSumSlots * s.n_rows);
   l.scores = off; off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.pooled = off; if (s.pool_kernel > 1) off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.part = off;
@@ -204,7 +204,7 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
 
 template <int R>
 s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s, const int32_t *lengths,
-                           const unsigned char *cqs, float *scores, double *rowsum, unsigned long long *bar, uint32_t *status,
+                           const unsigned char *cqs, float *scores, double *rowsum, unsigned int *bar, uint32_t *status,
                            cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
@@ -233,7 +233,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   double *cq64 = reinterpret_cast<double *>(ws + ly.cq64);
   unsigned int *tickets = reinterpret_cast<unsigned int *>(ws + ly.tickets);
   unsigned int *att_tickets = reinterpret_cast<unsigned int *>(ws + ly.att_tickets);
-  unsigned long long *bar = reinterpret_cast<unsigned long long *>(ws + ly.barrier);
+  unsigned int *bar = reinterpret_cast<unsigned int *>(ws + ly.barrier);
   float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
   float *pooled = reinterpret_cast<float *>(ws + ly.pooled);
   float *part = reinterpret_cast<float *>(ws + ly.part);
