@@ -63,7 +63,6 @@ struct StcControl {
   int flag;
   int kofs[kStcTiles][64];
   float alpha[kStcTiles][64];
-  double half_sum[64];
 };
 static_assert(sizeof(StcControl) <= kStcControlBytes, "control block");
 static_assert(stc_smem_bytes(64, 256) <= kStcMaxSmem && stc_smem_bytes(32, 256) <= kStcMaxSmem, "smem budget");
@@ -210,19 +209,21 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       ctl->kofs[t][threadIdx.x] = 0;
     }
     __syncthreads();
-    // Row sums over the tile's 128 positions: TPR threads per row, fp64, fixed order.
+    // Row sums over the tile's 128 positions: TPR threads per row, four
+    // independent fp32 partial sums each (fp64 arithmetic would stall the
+    // tensor pipe), combined in a fixed order and added in fp64.
     {
       const int row = threadIdx.x % R, part = threadIdx.x / R;
-      double acc = 0.0;
-      for (int q = part * (kStcTile / TPR); q < (part + 1) * (kStcTile / TPR); ++q) acc += (double)red[q * (R + 1) + row];
-      if (part > 0) ctl->half_sum[row] = 0.0;
+      constexpr int kPer = kStcTile / TPR;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int q = 0; q < kPer; ++q) a4[q & 3] += red[(part * kPer + q) * (R + 1) + row];
+      const float mine = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      red[p * (R + 1) + R] = mine;   // column R of the scratch is free
       __syncthreads();
-      for (int pp = 1; pp < TPR; ++pp) {
-        if (part == pp) ctl->half_sum[row] += acc;
-        __syncthreads();
-      }
       if (part == 0 && row < s.n_rows) {
-        const double l = acc + (TPR > 1 ? ctl->half_sum[row] : 0.0);
+        double l = 0.0;
+        for (int pp = 0; pp < TPR; ++pp) l += (double)red[(pp * R + row) * (R + 1) + R];
         atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + blockIdx.x % kStcSumSlots) * s.n_rows + row],
                   ldexp(l, ctl->kofs[t][row]));
       }
@@ -233,7 +234,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   // C: every tile of every problem has added its row sums.
   const bool bar_ok = grid_barrier(bar, status, &ctl->flag);
 
-  // D: scores.  l_row = sum of the row's slots (fixed order).
+  // D: scores.  l_row = sum of the row's slots (fixed order), then its
+  // fp32 reciprocal.
   if (threadIdx.x < R) {
     const int row = threadIdx.x;
     double l = 0.0;
@@ -244,10 +246,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
 #pragma unroll
       for (int q = 0; q < kStcSumSlots; ++q) l += part[q];
     }
-    const double inv = (l > 0.0) ? 1.0 / l : 0.0;
+    const float inv = (l > 0.0) ? 1.f / (float)l : 0.f;
     for (int t = 0; t < n_tiles; ++t) {
       const int k = ctl->kofs[t][row];
-      ctl->alpha[t][row] = (k == 0) ? (float)inv : (float)ldexp(inv, k);
+      ctl->alpha[t][row] = (k == 0) ? inv : ldexpf(inv, k);
     }
   }
   __syncthreads();

@@ -66,12 +66,15 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_t
 }
 
 constexpr int kTopkSmemKeys = 32768;  // keys staged in shared memory (128 KB) when they fit
+// Staged key i lives at word i + i/32: a thread walking its own contiguous
+// chunk of 32 keys then never shares a bank with the other lanes of its warp.
+__host__ __device__ __forceinline__ int64_t kpad(int64_t i) { return i + (i >> 5); }
 constexpr int kTopkBins = 256;         // 8-bit digits
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkSample = 1024;      // sampled keys that bracket the threshold
 constexpr int kTopkCand = 8192;        // capacity of the in-bracket candidate list
 __host__ inline size_t topk_smem_bytes(int64_t cache_rows) {
-  return sizeof(uint32_t) * ((size_t)smin<int64_t>(cache_rows, kTopkSmemKeys) + kTopkCand);
+  return sizeof(uint32_t) * ((size_t)kpad(smin<int64_t>(cache_rows, kTopkSmemKeys)) + 1 + kTopkCand);
 }
 
 struct TopkShared {
@@ -137,7 +140,7 @@ __device__ void radix_select_small(const uint32_t *vals, int n, uint32_t need, T
 
 template <bool kShared>
 __device__ __forceinline__ uint32_t key_at(const uint32_t *keys, int64_t i) {
-  return kShared ? keys[i] : __ldcg(keys + i);
+  return kShared ? keys[kpad(i)] : __ldcg(keys + i);
 }
 
 // Threshold of the top `need` keys: a sorted-free sample brackets it, one
@@ -295,7 +298,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
     for (int64_t i = threadIdx.x; i < nc; i += blockDim.x) out[i] = (int32_t)(s.n_sink + i);
     return;
   }
-  const int64_t n_stage = smin<int64_t>(s.cache_rows, kTopkSmemKeys);
+  const int64_t n_stage = kpad(smin<int64_t>(s.cache_rows, kTopkSmemKeys)) + 1;
   uint32_t *keys_s = topk_dyn;
   uint32_t *cand = topk_dyn + n_stage;
   if (nc <= kTopkSmemKeys) {
@@ -305,7 +308,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
     const int64_t head = smin<int64_t>(nc, (int64_t)((16u - (reinterpret_cast<uintptr_t>(gkeys) & 15u)) & 15u) / 4);
     const int64_t n4 = (nc - head) / 4;
     const uint4 *src4 = reinterpret_cast<const uint4 *>(gkeys + head);
-    for (int64_t i = threadIdx.x; i < head; i += blockDim.x) keys_s[i] = __ldcg(gkeys + i);
+    for (int64_t i = threadIdx.x; i < head; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i);
     for (int64_t i0 = 0; i0 < n4; i0 += 4 * kTopkThreads) {
       uint4 v[4];
 #pragma unroll
@@ -317,12 +320,15 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
       for (int u = 0; u < 4; ++u) {
         const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
         if (i < n4) {
-          uint32_t *d = keys_s + head + 4 * i;   // the shared copy may be unaligned too: scalar stores
-          d[0] = v[u].x; d[1] = v[u].y; d[2] = v[u].z; d[3] = v[u].w;
+          const int64_t j = head + 4 * i;
+          keys_s[kpad(j)] = v[u].x;
+          keys_s[kpad(j + 1)] = v[u].y;
+          keys_s[kpad(j + 2)] = v[u].z;
+          keys_s[kpad(j + 3)] = v[u].w;
         }
       }
     }
-    for (int64_t i = head + 4 * n4 + threadIdx.x; i < nc; i += blockDim.x) keys_s[i] = __ldcg(gkeys + i);
+    for (int64_t i = head + 4 * n4 + threadIdx.x; i < nc; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i);
     __syncthreads();
     select_top<true>(keys_s, nc, (uint32_t)need, s.n_sink, out, k, sh, cand);
   } else {

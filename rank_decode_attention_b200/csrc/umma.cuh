@@ -145,34 +145,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Grid-wide barrier for a cooperative launch, two levels to keep atomics
-// uncontended.  `bar` points at kBarWords zeroed words (an earlier launch on
-// the same stream zeroes them): 16 group counters, a top counter and a flag.
-// CTA c arrives on group c % 16; the last CTA of a group arrives on the top
-// counter, and the last group sets the flag, which every CTA polls (bounded).
+// Grid-wide barrier for a cooperative launch.  `bar` points at kBarWords
+// words that an earlier launch on the same stream zeroed; every CTA adds one
+// arrival to bar[0] and waits (bounded) until all gridDim.x CTAs arrived.
 // Returns false on timeout.
-constexpr int kBarGroups = 16;
-constexpr int kBarWords = kBarGroups + 2;
+constexpr int kBarWords = 2;
 __device__ __forceinline__ bool grid_barrier(unsigned int *bar, uint32_t *status, int *flag_smem) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    const unsigned int n = gridDim.x, grp = blockIdx.x % kBarGroups;
-    const unsigned int n_groups = n < kBarGroups ? n : kBarGroups;
-    const unsigned int in_grp = (n - grp + kBarGroups - 1) / kBarGroups;
     __threadfence();
-    if (atomicAdd(&bar[grp], 1u) == in_grp - 1) {
-      __threadfence();
-      if (atomicAdd(&bar[kBarGroups], 1u) == n_groups - 1) {
-        __threadfence();
-        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(bar + kBarGroups + 1), "r"(1u) : "memory");
-      }
-    }
+    atomicAdd(bar, 1u);
     const long long t0 = clock64();
     while (true) {
       unsigned int v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar + kBarGroups + 1) : "memory");
-      if (v != 0u) break;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (v >= gridDim.x) break;
       if (clock64() - t0 > kWaitCycles) {
         set_status(status, kDevStatusTimeout);
         ok = 0;
