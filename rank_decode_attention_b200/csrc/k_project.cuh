@@ -38,9 +38,12 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
                unsigned char *__restrict__ cqs, float *__restrict__ qt, double *__restrict__ cq64,
                unsigned int *__restrict__ tickets, double *__restrict__ row_sum,
                unsigned int *__restrict__ barrier) {
-  __shared__ float qs[kProjRowBlock][129];           // per-head query rows, 128 of d_h
-  __shared__ float bs[128][kProjColBlock + 1];       // basis slice, 128 rows of d_h
+  // Raw storage-type slices, copied with 16-byte cp.async (all in flight at once).
+  __shared__ __align__(16) T qraw[kProjRowBlock][128];          // per-head query rows, 128 of d_h
+  __shared__ __align__(16) T braw[128][kProjColBlock + 16 / sizeof(T)];  // basis slice (padded rows)
   __shared__ int last_flag;
+  constexpr int V = Vec16<T>::n;
+  constexpr int kBPitch = kProjColBlock + 16 / (int)sizeof(T);
   const int g = blockIdx.x, cb = blockIdx.y;
   const int n_rb = (int)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
   const int rb = blockIdx.z % n_rb, b = blockIdx.z / n_rb;
@@ -64,38 +67,29 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
   for (int t0 = 0; t0 < dh; t0 += 128) {
-    const int tn = smin(128, dh - t0);
+    const int tn = smin(128, dh - t0);  // a multiple of 8
     __syncthreads();
-    // Every load of the 128-wide slice is issued before any is used.
-    constexpr int kQU = (kProjRowBlock * 128) / kProjThreads, kBU = (128 * kProjColBlock) / kProjThreads;
-    float qv[kQU], bv[kBU];
-#pragma unroll
-    for (int u = 0; u < kQU; ++u) {
-      const int e = threadIdx.x + u * kProjThreads;
-      const int pr = e >> 7, t = e & 127;
+    // Query rows: kProjRowBlock x tn elements; basis slice: tn x 64 columns.
+    for (int e = threadIdx.x; e < kProjRowBlock * (128 / V); e += blockDim.x) {
+      const int pr = e / (128 / V), cc = e - pr * (128 / V);
       const int row = pr0 + pr;
-      qv[u] = 0.f;
-      if (row < n_prow && t < tn) {
+      T *dst = &qraw[pr][cc * V];
+      if (row < n_prow && cc * V < tn) {
         const int w = row / G, j = row - w * G;
-        qv[u] = to_f(qb[((int64_t)w * Hq + g * G + j) * dh + t0 + t]);
+        cp_async16(dst, qb + ((int64_t)w * Hq + g * G + j) * dh + t0 + cc * V);
+      } else {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-#pragma unroll
-    for (int u = 0; u < kBU; ++u) {
-      const int e = threadIdx.x + u * kProjThreads;
-      const int t = e >> 6, c = e & 63;
-      bv[u] = (t < tn && c0 + c < r) ? to_f(Bb[(int64_t)(g * dh + t0 + t) * r + c0 + c]) : 0.f;
+    for (int e = threadIdx.x; e < 128 * (kProjColBlock / V); e += blockDim.x) {
+      const int t = e / (kProjColBlock / V), cc = e - t * (kProjColBlock / V);
+      T *dst = &braw[t][cc * V];
+      if (t < tn && c0 + cc * V < r)   // r % 8 == 0, so a chunk never straddles r
+        cp_async16(dst, Bb + (int64_t)(g * dh + t0 + t) * r + c0 + cc * V);
+      else
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
-#pragma unroll
-    for (int u = 0; u < kQU; ++u) {
-      const int e = threadIdx.x + u * kProjThreads;
-      qs[e >> 7][e & 127] = qv[u];
-    }
-#pragma unroll
-    for (int u = 0; u < kBU; ++u) {
-      const int e = threadIdx.x + u * kProjThreads;
-      bs[e >> 6][e & 63] = bv[u];
-    }
+    cp_async_wait_all();
     __syncthreads();
     // Two 64-term fp32 chunks, each added to the fp64 accumulators.
 #pragma unroll
@@ -105,9 +99,9 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
       for (int k = h0; k < h0 + 64; ++k) {
         float a[2], bb[4];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) a[i] = qs[ty + 8 * i][k];
+        for (int i = 0; i < 2; ++i) a[i] = to_f(qraw[ty + 8 * i][k]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) bb[j] = bs[k][tx + 16 * j];
+        for (int j = 0; j < 4; ++j) bb[j] = to_f(braw[k][tx + 16 * j]);
 #pragma unroll
         for (int i = 0; i < 2; ++i)
 #pragma unroll

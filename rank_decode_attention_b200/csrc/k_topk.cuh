@@ -71,8 +71,9 @@ constexpr int kTopkSmemKeys = 32768;  // keys staged in shared memory (128 KB) w
 __host__ __device__ __forceinline__ int64_t kpad(int64_t i) { return i + (i >> 5); }
 constexpr int kTopkBins = 256;         // 8-bit digits
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkSample = 1024;      // sampled keys that bracket the threshold
-constexpr int kTopkCand = 8192;        // capacity of the in-bracket candidate list
+constexpr int kTopkSample = 256;       // sampled keys that bracket the threshold
+constexpr int kTopkSeg = 256;          // in-bracket candidates kept per warp
+constexpr int kTopkCand = kTopkWarps * kTopkSeg;
 __host__ inline size_t topk_smem_bytes(int64_t cache_rows) {
   return sizeof(uint32_t) * ((size_t)kpad(smin<int64_t>(cache_rows, kTopkSmemKeys)) + 1 + kTopkCand);
 }
@@ -81,165 +82,179 @@ struct TopkShared {
   uint32_t whist[kTopkWarps][kTopkBins];
   uint32_t hist[kTopkBins];
   uint32_t sample[kTopkSample];
+  uint32_t seg_count[kTopkWarps];
+  uint32_t seg_above[kTopkWarps];
   uint32_t warp_tot[32];
-  uint32_t total, digit, above, n_cand, n_above;
+  uint32_t total, digit, above, t_hi, t_lo, cmin, cmax;
 };
-
-// Exact radix select over a short shared-memory array: the value tau of the
-// need-th largest element (1 <= need <= n) and how many elements equal to tau
-// belong to the top `need`.  Per-warp histograms; contention stays small
-// because n is small.
-__device__ void radix_select_small(const uint32_t *vals, int n, uint32_t need, TopkShared &sh, uint32_t *tau_out,
-                                   uint32_t *take_eq_out) {
-  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t prefix = 0, mask = 0, remaining = need;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-    for (int j = 0; j < kTopkBins / 32; ++j) sh.whist[wid][lane + 32 * j] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t v = vals[i];
-      if ((v & mask) == prefix) atomicAdd(&sh.whist[wid][(v >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (threadIdx.x < kTopkBins) {
-      uint32_t c = 0;
-      for (int w = 0; w < kTopkWarps; ++w) c += sh.whist[w][threadIdx.x];
-      sh.hist[threadIdx.x] = c;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      uint32_t cnt[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t run = incl - sum;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (run < remaining && run + cnt[j] >= remaining) {
-          sh.digit = 255u - (uint32_t)(lane * 8 + j);
-          sh.above = run;
-        }
-        run += cnt[j];
-      }
-    }
-    __syncthreads();
-    remaining -= sh.above;
-    prefix |= sh.digit << shift;
-    mask |= 255u << shift;
-    __syncthreads();
-  }
-  *tau_out = prefix;
-  *take_eq_out = remaining;
-}
 
 template <bool kShared>
 __device__ __forceinline__ uint32_t key_at(const uint32_t *keys, int64_t i) {
   return kShared ? keys[kpad(i)] : __ldcg(keys + i);
 }
 
-// Threshold of the top `need` keys: a sorted-free sample brackets it, one
-// comparison pass counts the keys above the bracket and collects those inside
-// it, and an exact radix select on the collected keys finishes.  Returns false
-// if the bracket missed or overflowed the candidate list (the caller then
-// selects on all keys).
-template <bool kShared>
-__device__ bool bracket_select(const uint32_t *keys, int64_t nc, uint32_t need, TopkShared &sh, uint32_t *cand,
-                               uint32_t *tau, uint32_t *take_eq) {
-  const int lane = threadIdx.x & 31;
-  // Sample and two of its order statistics around the expected rank.
-  const int M = kTopkSample;
-  for (int i = threadIdx.x; i < M; i += blockDim.x) sh.sample[i] = key_at<kShared>(keys, (int64_t)i * nc / M);
+// One radix pass: histogram of digit (v >> shift) & 255 over the values that
+// match `prefix` under `mask`, then the digit holding the `remaining`-th
+// largest.  `value(i)` returns (valid, v) for slot i < n_slots.
+template <typename ValueFn>
+__device__ void radix_pass(ValueFn value, int64_t n_slots, int shift, uint32_t mask, uint32_t &prefix,
+                           uint32_t &remaining, TopkShared &sh) {
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < kTopkBins / 32; ++j) sh.whist[wid][lane + 32 * j] = 0;
   __syncthreads();
-  const double q = (double)need * M / (double)nc;
-  const double delta = 4.0 * sqrt(q + 1.0) + 8.0;
-  const int r_hi = (int)fmax(1.0, floor(q - delta));       // rank (1-based) of the upper bracket end
-  const int r_lo = (int)fmin((double)M, ceil(q + delta));   // rank of the lower bracket end
-  uint32_t t_hi = 0xffffffffu, t_lo = 0u, dummy;
-  if (q - delta >= 1.0) radix_select_small(sh.sample, M, (uint32_t)r_hi, sh, &t_hi, &dummy);
-  if (q + delta <= (double)M) radix_select_small(sh.sample, M, (uint32_t)r_lo, sh, &t_lo, &dummy);
-  // Count keys strictly above t_hi and collect keys in [t_lo, t_hi].
-  if (threadIdx.x == 0) { sh.n_cand = 0; sh.n_above = 0; }
+  for (int64_t i = threadIdx.x; i < n_slots; i += blockDim.x) {
+    bool ok;
+    const uint32_t v = value(i, ok);
+    if (ok && (v & mask) == prefix) atomicAdd(&sh.whist[wid][(v >> shift) & 255u], 1u);
+  }
   __syncthreads();
-  uint32_t above = 0;
-  for (int64_t i0 = 0; i0 < nc; i0 += blockDim.x) {
-    const int64_t i = i0 + threadIdx.x;
-    const uint32_t v = (i < nc) ? key_at<kShared>(keys, i) : 0u;
-    const bool valid = i < nc;
-    above += (valid && v > t_hi);
-    const bool in = valid && v <= t_hi && v >= t_lo;
-    const uint32_t ball = __ballot_sync(0xffffffffu, in);
-    uint32_t base = 0;
-    if (lane == 0 && ball) base = atomicAdd(&sh.n_cand, (uint32_t)__popc(ball));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    if (in) {
-      const uint32_t slot = base + __popc(ball & ((1u << lane) - 1u));
-      if (slot < kTopkCand) cand[slot] = v;
+  if (threadIdx.x < kTopkBins) {
+    uint32_t c = 0;
+#pragma unroll 8
+    for (int w = 0; w < kTopkWarps; ++w) c += sh.whist[w][threadIdx.x];
+    sh.hist[threadIdx.x] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t cnt[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t run = incl - sum;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (run < remaining && run + cnt[j] >= remaining) {
+        sh.digit = 255u - (uint32_t)(lane * 8 + j);
+        sh.above = run;
+      }
+      run += cnt[j];
     }
   }
-  above = warp_sum_u32(above);
-  if (lane == 0 && above) atomicAdd(&sh.n_above, above);
   __syncthreads();
-  const uint32_t n_above = sh.n_above, n_cand = sh.n_cand;
-  if (!(n_above < need && need <= n_above + n_cand) || n_cand > (uint32_t)kTopkCand) return false;
-  radix_select_small(cand, (int)n_cand, need - n_above, sh, tau, take_eq);
-  return true;
+  remaining -= sh.above;
+  prefix |= sh.digit << shift;
+  __syncthreads();
 }
 
-// Exact radix select over all keys (fallback).
-template <bool kShared>
-__device__ void radix_select_all(const uint32_t *keys, int64_t nc, uint32_t need, TopkShared &sh, uint32_t *tau,
-                                 uint32_t *take_eq) {
-  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Exact radix select of the need-th largest value; passes start below the
+// leading bits that every value shares (known from lo_all/hi_all, the
+// minimum and maximum).  Returns tau and how many values equal to tau are in
+// the top `need`.
+template <typename ValueFn>
+__device__ void radix_select(ValueFn value, int64_t n_slots, uint32_t need, uint32_t lo_all, uint32_t hi_all,
+                             TopkShared &sh, uint32_t *tau, uint32_t *take_eq) {
+  const uint32_t diff = lo_all ^ hi_all;
+  int top = 31;
+  while (top >= 0 && !((diff >> top) & 1u)) --top;  // highest differing bit, -1 if all equal
   uint32_t prefix = 0, mask = 0, remaining = need;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-    for (int j = 0; j < kTopkBins / 32; ++j) sh.whist[wid][lane + 32 * j] = 0;
-    __syncthreads();
-    for (int64_t i = threadIdx.x; i < nc; i += blockDim.x) {
-      const uint32_t v = key_at<kShared>(keys, i);
-      if ((v & mask) == prefix) atomicAdd(&sh.whist[wid][(v >> shift) & 255u], 1u);
+  if (top < 31) {
+    const uint32_t common = (top < 0) ? 0xffffffffu : ~((2u << top) - 1u);
+    prefix = lo_all & common;
+    mask = common;
+  }
+  if (top >= 0) {
+    // digits whose 8-bit window covers bits top..0, aligned to multiples of 8
+    for (int shift = (top / 8) * 8; shift >= 0; shift -= 8) {
+      radix_pass(value, n_slots, shift, mask, prefix, remaining, sh);
+      mask |= 255u << shift;
     }
-    __syncthreads();
-    if (threadIdx.x < kTopkBins) {
-      uint32_t c = 0;
-      for (int w = 0; w < kTopkWarps; ++w) c += sh.whist[w][threadIdx.x];
-      sh.hist[threadIdx.x] = c;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      uint32_t cnt[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t run = incl - sum;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (run < remaining && run + cnt[j] >= remaining) {
-          sh.digit = 255u - (uint32_t)(lane * 8 + j);
-          sh.above = run;
-        }
-        run += cnt[j];
-      }
-    }
-    __syncthreads();
-    remaining -= sh.above;
-    prefix |= sh.digit << shift;
-    mask |= 255u << shift;
-    __syncthreads();
   }
   *tau = prefix;
   *take_eq = remaining;
+}
+
+__device__ __forceinline__ void block_minmax(uint32_t lo, uint32_t hi, TopkShared &sh) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (threadIdx.x == 0) { sh.cmin = 0xffffffffu; sh.cmax = 0u; }
+  __syncthreads();
+  if (lane == 0) { atomicMin(&sh.cmin, lo); atomicMax(&sh.cmax, hi); }
+  __syncthreads();
+}
+
+// Threshold of the top `need` keys: a 256-key sample, ranked by counting,
+// brackets it; one comparison pass counts the keys above the bracket and
+// collects those inside it into per-warp segments; an exact radix select on
+// the collected keys finishes.  Returns false if the bracket missed or a
+// segment overflowed (the caller then selects on all keys).
+template <bool kShared>
+__device__ bool bracket_select(const uint32_t *keys, int64_t nc, uint32_t need, TopkShared &sh, uint32_t *cand,
+                               uint32_t *tau, uint32_t *take_eq) {
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = kTopkSample;
+  if (threadIdx.x < M) sh.sample[threadIdx.x] = key_at<kShared>(keys, (int64_t)threadIdx.x * nc / M);
+  const double q = (double)need * M / (double)nc;
+  const double delta = 4.0 * sqrt(q + 1.0) + 8.0;
+  const int r_hi = (int)floor(q - delta);   // 1-based ranks of the bracket ends
+  const int r_lo = (int)ceil(q + delta);
+  if (threadIdx.x == 0) {
+    sh.t_hi = 0xffffffffu;
+    sh.t_lo = 0u;
+  }
+  __syncthreads();
+  if (threadIdx.x < M) {
+    // rank (0 = largest) by counting; equal keys ordered by sample index
+    const uint32_t v = sh.sample[threadIdx.x];
+    int rank = 0;
+#pragma unroll 8
+    for (int j = 0; j < M; ++j) {
+      const uint32_t u = sh.sample[j];
+      rank += (u > v) || (u == v && j < (int)threadIdx.x);
+    }
+    if (r_hi >= 1 && rank == r_hi - 1) sh.t_hi = v;
+    if (r_lo <= M && rank == r_lo - 1) sh.t_lo = v;
+  }
+  __syncthreads();
+  const uint32_t t_hi = sh.t_hi, t_lo = sh.t_lo;
+  // Count keys strictly above t_hi and collect keys in [t_lo, t_hi].
+  uint32_t above = 0, seg = 0, cmin = 0xffffffffu, cmax = 0u;
+  uint32_t *mine = cand + wid * kTopkSeg;
+  for (int64_t i0 = 0; i0 < nc; i0 += blockDim.x) {
+    const int64_t i = i0 + threadIdx.x;
+    const bool valid = i < nc;
+    const uint32_t v = valid ? key_at<kShared>(keys, i) : 0u;
+    above += (valid && v > t_hi);
+    const bool in = valid && v <= t_hi && v >= t_lo;
+    const uint32_t ball = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      const uint32_t slot = seg + __popc(ball & ((1u << lane) - 1u));
+      if (slot < kTopkSeg) mine[slot] = v;
+      cmin = min(cmin, v);
+      cmax = max(cmax, v);
+    }
+    seg += __popc(ball);
+  }
+  above = warp_sum_u32(above);
+  if (lane == 0) {
+    sh.seg_count[wid] = seg;
+    sh.seg_above[wid] = above;
+  }
+  block_minmax(cmin, cmax, sh);   // includes a __syncthreads
+  uint32_t n_above = 0, n_cand = 0;
+  bool overflow = false;
+  for (int w = 0; w < kTopkWarps; ++w) {
+    n_above += sh.seg_above[w];
+    n_cand += sh.seg_count[w];
+    overflow |= sh.seg_count[w] > (uint32_t)kTopkSeg;
+  }
+  if (overflow || !(n_above < need && need <= n_above + n_cand)) return false;
+  auto value = [&](int64_t i, bool &ok) -> uint32_t {
+    const int w = (int)(i / kTopkSeg), e = (int)(i - (int64_t)w * kTopkSeg);
+    ok = e < (int)sh.seg_count[w];
+    return ok ? cand[i] : 0u;
+  };
+  radix_select(value, (int64_t)kTopkCand, need - n_above, sh.cmin, sh.cmax, sh, tau, take_eq);
+  return true;
 }
 
 // Stable compaction in index order: every key > tau and the first take_eq
@@ -247,7 +262,7 @@ __device__ void radix_select_all(const uint32_t *keys, int64_t nc, uint32_t need
 template <bool kShared>
 __device__ void compact_selected(const uint32_t *keys, int64_t nc, uint32_t tau, uint32_t take_eq, int32_t n_sink,
                                  int32_t *out, int k, TopkShared &sh) {
-  const int64_t chunk = ceil_div(nc, blockDim.x);
+  const int chunk = (int)ceil_div(nc, blockDim.x);
   const int64_t i0 = smin<int64_t>(nc, (int64_t)threadIdx.x * chunk);
   const int64_t i1 = smin<int64_t>(nc, i0 + chunk);
   uint32_t n_gt = 0, n_eq = 0;
@@ -272,8 +287,13 @@ template <bool kShared>
 __device__ void select_top(const uint32_t *keys, int64_t nc, uint32_t need, int32_t n_sink, int32_t *out, int k,
                            TopkShared &sh, uint32_t *cand) {
   uint32_t tau = 0, take_eq = 0;
-  if (nc <= 2 * kTopkSample || !bracket_select<kShared>(keys, nc, need, sh, cand, &tau, &take_eq))
-    radix_select_all<kShared>(keys, nc, need, sh, &tau, &take_eq);
+  if (nc <= 4 * kTopkSample || !bracket_select<kShared>(keys, nc, need, sh, cand, &tau, &take_eq)) {
+    auto value = [&](int64_t i, bool &ok) -> uint32_t {
+      ok = true;
+      return key_at<kShared>(keys, i);
+    };
+    radix_select(value, nc, need, 0u, 0xffffffffu, sh, &tau, &take_eq);
+  }
   compact_selected<kShared>(keys, nc, tau, take_eq, n_sink, out, k, sh);
 }
 
