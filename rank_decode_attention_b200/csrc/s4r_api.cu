@@ -22,8 +22,7 @@
 
 using namespace s4r;
 
-static_assert(S4R_MAX_GROUP <= kAttMaxGroup && S4R_MAX_SINKS <= kAttMaxSinks &&
-                  S4R_MAX_SELECTED <= kAttMaxSplits * kAttEntries,
+static_assert(S4R_MAX_GROUP <= kAttMaxGroup && S4R_MAX_SINKS <= kAttMaxSinks && S4R_MAX_RANK <= kAttThreads,
               "header limits must fit the attention kernel");
 
 namespace {
@@ -35,7 +34,7 @@ inline size_t esize(s4r_dtype dt) { return dt == S4R_BF16 ? 2 : 4; }
 
 // Byte offsets of the decode workspace regions.
 struct Layout {
-  size_t status, barrier, cq, cqs, cq64, tickets, att_tickets, qt, tstat, rstat, rowsum, scores, pooled, part, total;
+  size_t status, barrier, cq, cqs, qt, tstat, rstat, rowsum, scores, pooled, total;
 };
 
 Layout layout_for(const Shape &s) {
@@ -47,9 +46,6 @@ Layout layout_for(const Shape &s) {
   l.cq = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_rows * s.rank_k);
   const size_t n_cb = (size_t)ceil_div(s.rank_k, kProjColBlock);
   l.cqs = off; off += round_up((size_t)s.batch * n_cb * cqs_block_bytes(s.n_rows));
-  l.cq64 = off; off += round_up(sizeof(double) * s.batch * (size_t)s.n_rows * s.rank_k);
-  l.tickets = off; off += round_up(sizeof(unsigned int) * s.batch * n_cb);
-  l.att_tickets = off; off += round_up(sizeof(unsigned int) * s.batch * (size_t)s.n_heads_kv);
   l.qt = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * s.rank_k);
   const size_t n_tiles = (size_t)ceil_div(s.cache_rows, kScoreTile);
   l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
@@ -57,8 +53,6 @@ Layout layout_for(const Shape &s) {
   l.rowsum = off; off += round_up(sizeof(double) * s.batch * (size_t)kStcSumSlots * s.n_rows);
   l.scores = off; off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.pooled = off; if (s.pool_kernel > 1) off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
-  l.part = off;
-  off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * att_splits(s) * (s.rank_v + 2));
   l.total = off;
   return l;
 }
@@ -230,13 +224,9 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   double *rstat = reinterpret_cast<double *>(ws + ly.rstat);
   double *rowsum = reinterpret_cast<double *>(ws + ly.rowsum);
   unsigned char *cqs = ws + ly.cqs;
-  double *cq64 = reinterpret_cast<double *>(ws + ly.cq64);
-  unsigned int *tickets = reinterpret_cast<unsigned int *>(ws + ly.tickets);
-  unsigned int *att_tickets = reinterpret_cast<unsigned int *>(ws + ly.att_tickets);
   unsigned int *bar = reinterpret_cast<unsigned int *>(ws + ly.barrier);
   float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
   float *pooled = reinterpret_cast<float *>(ws + ly.pooled);
-  float *part = reinterpret_cast<float *>(ws + ly.part);
   const T *q = static_cast<const T *>(a->q);
   const T *ck = static_cast<const T *>(a->coeff_k);
   const T *cv = static_cast<const T *>(a->coeff_v);
@@ -248,8 +238,20 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   // 1. query projection
   {
     const unsigned n_rb = (unsigned)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
-    dim3 grid((unsigned)s.n_heads_kv, (unsigned)ceil_div(s.rank_k, kProjColBlock), n_rb * (unsigned)s.batch);
-    project_kernel<T><<<grid, kProjThreads, 0, st>>>(s, q, bk, cq, cqs, qt, cq64, tickets, rowsum, bar);
+    const unsigned n_rank = (unsigned)proj_cluster(s.n_heads_kv);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_rank, (unsigned)ceil_div(s.rank_k, kProjColBlock), n_rb * (unsigned)s.batch);
+    cfg.blockDim = dim3(kProjThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = n_rank;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, project_kernel<T>, s, q, bk, cq, cqs, qt, rowsum, bar);
+    if (err != cudaSuccess) return fail("project_kernel (cluster launch)", err);
     if (check_launch("project_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
   // 2. latent scoring
@@ -290,12 +292,12 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     topk_kernel<<<s.batch, kTopkThreads, smem, st>>>(s, a->lengths, keys, a->idx, status);
     if (check_launch("topk_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
-  // 4. rebuild + exact attention (the last CTA of each kv group merges)
+  // 4. rebuild + exact attention (one cluster of CTAs per kv group)
   {
     const size_t smem = att_smem_bytes(s, sizeof(T));
     cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attend_kernel<T><<<dim3(att_splits(s), s.n_heads_kv, s.batch), kAttThreads, smem, st>>>(
-        s, a->lengths, a->idx, ck, cv, qt, q, bv, sk, sv, part, att_tickets, a->out);
+    attend_kernel<T><<<dim3(kAttCluster, s.n_heads_kv, s.batch), kAttThreads, smem, st>>>(
+        s, a->lengths, a->idx, ck, cv, qt, q, bv, sk, sv, a->out);
     if (check_launch("attend_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
   return last_cuda();
