@@ -108,6 +108,7 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   float *sw_s = acc_s + kAttMaxGroup * rv;                  // [G][kAttMaxSinks]
   float *f_s = sw_s + kAttMaxGroup * kAttMaxSinks;          // [G][kAttCluster]
   __shared__ int64_t rows_s[kAttEntries];
+  __shared__ __align__(8) uint64_t stage_bar;
 
   const int64_t L = valid_length(lengths[b], s.cache_rows);
   const int64_t n_top = smin<int64_t>(s.top_k, n_candidates(L, s.local_window));
@@ -124,6 +125,10 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
     const int j = t / rk, k = t - j * rk;
     q_s[j * rk + k] = qt_all[((int64_t)b * s.n_heads_q + g * G + j) * rk + k];
   }
+  if (threadIdx.x == 0) {
+    mbar_init(&stage_bar, 1);
+    mbar_fence_init();
+  }
   if (threadIdx.x < G) {
     ml_s[threadIdx.x * 4] = -INFINITY;   // running max
     ml_s[threadIdx.x * 4 + 1] = 0.f;     // running sum
@@ -133,6 +138,7 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   for (int j = 0; j < kAttMaxGroup; ++j) acc[j] = 0.f;
   const int kcol = threadIdx.x;  // latent value column owned by this thread (< rv)
 
+  uint32_t phase = 0;
   for (int64_t c0 = e_begin; c0 < e_end; c0 += kAttEntries) {
     const int n_e = (int)smin<int64_t>(kAttEntries, e_end - c0);
     __syncthreads();  // previous chunk fully consumed
@@ -145,23 +151,29 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       rows_s[e] = row;
     }
     __syncthreads();
-    {
-      const int ck_chunks = rk / V, cv_chunks = rv / V;
-      for (int t = threadIdx.x; t < n_e * (ck_chunks + cv_chunks); t += blockDim.x) {
-        const int e = t / (ck_chunks + cv_chunks), c = t - e * (ck_chunks + cv_chunks);
-        const int64_t row = rows_s[e];
-        T *dst = (c < ck_chunks) ? ck_s + e * pk + c * V : cv_s + e * pv + (c - ck_chunks) * V;
-        if (row < 0) {  // keep skipped rows finite: their weights are zero
-          *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-          continue;
-        }
-        if (c < ck_chunks)
-          cp_async16(dst, ckb + row * rk + c * V);
-        else
-          cp_async16(dst, cvb + row * rv + (c - ck_chunks) * V);
+    // One bulk copy per row and operand (rows are 16-byte multiples), all
+    // completing on stage_bar; skipped rows are zeroed by plain stores.
+    if (threadIdx.x == 0) {
+      uint32_t bytes = 0;
+      for (int e = 0; e < n_e; ++e)
+        if (rows_s[e] >= 0) bytes += (uint32_t)((rk + rv) * sizeof(T));
+      mbar_arrive_expect_tx(&stage_bar, bytes);
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * n_e) {
+      const int e = threadIdx.x % n_e;
+      const bool is_v = threadIdx.x >= n_e;
+      const int64_t row = rows_s[e];
+      T *dst = is_v ? cv_s + e * pv : ck_s + e * pk;
+      const int n = is_v ? rv : rk;
+      if (row >= 0) {
+        bulk_load(dst, is_v ? cvb + row * rv : ckb + row * rk, (uint32_t)(n * sizeof(T)), &stage_bar);
+      } else {
+        for (int c = 0; c < n; c += V) *reinterpret_cast<uint4 *>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    cp_async_wait_all();
+    mbar_wait(&stage_bar, phase, nullptr);
+    phase ^= 1u;
     __syncthreads();
     // logits of (head j, entry e) pairs
     for (int t = threadIdx.x; t < G * kAttEntries; t += blockDim.x) {
@@ -218,10 +230,10 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   const T *Bv = basis_v + (int64_t)b * Dp * rv + (int64_t)g * dh * rv;
   if (rank == 0) {
     // Stage B^V[g] (d_h rows x rv) over the row buffers while the cluster syncs.
-    for (int t = threadIdx.x; t < dh * (rv / V); t += blockDim.x) {
-      const int e = t / (rv / V), c = t - e * (rv / V);
-      cp_async16(bv_s + e * pv + c * V, Bv + (int64_t)e * rv + c * V);
-    }
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&stage_bar, (uint32_t)(dh * rv * sizeof(T)));
+    __syncthreads();
+    for (int e = threadIdx.x; e < dh; e += blockDim.x)
+      bulk_load(bv_s + e * pv, Bv + (int64_t)e * rv, (uint32_t)(rv * sizeof(T)), &stage_bar);
   }
   cluster_sync();  // every partial is in place
   if (rank == 0) {
@@ -271,7 +283,7 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       for (int r = 0; r < kAttCluster; ++r) a = fmaf(f_s[j * kAttCluster + r], v[r], a);
       acc_s[t] = a;
     }
-    cp_async_wait_all();
+    mbar_wait(&stage_bar, phase, nullptr);
     __syncthreads();
     // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e].
     for (int t = threadIdx.x; t < G * dh; t += blockDim.x) {

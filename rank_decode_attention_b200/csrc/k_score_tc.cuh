@@ -13,14 +13,14 @@
 // log2(e), so the epilogue works in base 2: e = 2^y with y = z log2(e).
 //
 // One cooperative launch, one CTA per pair of 128-position tiles of one
-// problem (4 warps; thread 0 issues TMA, thread 32 issues tcgen05.mma, all
-// warps run the epilogue):
+// problem (5 warps: warps 0-3 run the epilogue, one per 32 TMEM lanes; one
+// thread of warp 4 issues the TMA copies and the tcgen05.mma):
 //   A. bulk-copy the split C_Q operand (prepared by the projection kernel in
 //      its shared-memory image), TMA both C_K tiles, MMA each tile into its
 //      own 256-column TMEM region.
 //   B. per tile: y = hi + mid + lo, e = 2^y (kept in TMEM), per-row sums of e
-//      over the tile (fp64, fixed order) added atomically (fp64) into the
-//      problem's row normalisers.  A tile whose |y| exceeds 100 uses integer
+//      over the tile (fp32 partials, fixed order); one fp64 atomic per row
+//      and CTA adds them to the problem's row normalisers (16 slots per row).  A tile whose |y| exceeds 100 uses integer
 //      per-row offsets 2^(y - k) instead, so nothing overflows.
 //   C. one bounded grid barrier.
 //   D. alpha[row] = 2^k / l_row; score[i] = sum_row alpha[row] e[i][row].
@@ -57,18 +57,21 @@ __host__ __device__ constexpr int stc_smem_bytes(int R, int r) {
 
 struct StcControl {
   uint64_t b_full;
-  uint64_t tma_full[kStcTiles];
+  uint64_t tma_full[kStcTiles][4];   // per (tile, 64-wide K-block)
   uint64_t mma_done[kStcTiles];
   uint32_t tmem_base;
   int flag;
   int kofs[kStcTiles][64];
   float alpha[kStcTiles][64];
+  float tile_sum[kStcTiles][64];
 };
 static_assert(sizeof(StcControl) <= kStcControlBytes, "control block");
 static_assert(stc_smem_bytes(64, 256) <= kStcMaxSmem && stc_smem_bytes(32, 256) <= kStcMaxSmem, "smem budget");
 
+constexpr int kStcThreads = 160;  // warps 0-3: epilogue (one TMEM lane each); warp 4: TMA + MMA issue
+
 template <int R>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kStcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
                 const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
                 unsigned int *__restrict__ bar, uint32_t *__restrict__ status) {
@@ -83,7 +86,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   float *red = reinterpret_cast<float *>(stc_red_aliased(R, r) ? a_op : a_op + kStcTiles * stc_a_bytes(r));
   StcControl *ctl = reinterpret_cast<StcControl *>(a_op + kStcTiles * stc_a_bytes(r) +
                                                    (stc_red_aliased(R, r) ? 0 : stc_red_bytes(R)));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const bool epi = warp < 4;
   const int64_t tiles_cap = ceil_div(s.cache_rows, kStcTile);
   const int64_t ctas_per_problem = ceil_div(tiles_cap, kStcTiles);
   const int b = (int)(blockIdx.x / ctas_per_problem);
@@ -94,10 +98,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   for (int t = 0; t < kStcTiles; ++t)
     if ((tile0 + t) < tiles_cap && (tile0 + t) * kStcTile < L) n_tiles = t + 1;
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 128) {
     mbar_init(&ctl->b_full, 1);
     for (int t = 0; t < kStcTiles; ++t) {
-      mbar_init(&ctl->tma_full[t], 1);
+      for (int kb = 0; kb < 4; ++kb) mbar_init(&ctl->tma_full[t][kb], 1);
       mbar_init(&ctl->mma_done[t], 1);
     }
     mbar_fence_init();
@@ -106,12 +110,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     const unsigned char *src = cqs + (int64_t)b * stc_b_bytes(R, r);
     for (int kb = 0; kb < nkb; ++kb)
       bulk_load(b_op + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128, &ctl->b_full);
-    // A: stream this CTA's coefficient tiles.
+    // A: stream this CTA's coefficient tiles, one barrier per K-block.
     for (int t = 0; t < n_tiles; ++t) {
-      mbar_arrive_expect_tx(&ctl->tma_full[t], (uint32_t)stc_a_bytes(r));
       const int32_t row = (int32_t)((int64_t)b * s.cache_rows + (tile0 + t) * kStcTile);
-      for (int kb = 0; kb < nkb; ++kb)
-        tma_load_2d(a_op + t * stc_a_bytes(r) + kb * (kStcTile * 128), &tmap_ck, &ctl->tma_full[t], kb * 64, row);
+      for (int kb = 0; kb < nkb; ++kb) {
+        mbar_arrive_expect_tx(&ctl->tma_full[t][kb], (uint32_t)(kStcTile * 128));
+        tma_load_2d(a_op + t * stc_a_bytes(r) + kb * (kStcTile * 128), &tmap_ck, &ctl->tma_full[t][kb], kb * 64, row);
+      }
     }
   }
   if (warp == 0) tmem_alloc(&ctl->tmem_base, kStcTmemCols);
@@ -121,70 +126,74 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   const uint32_t tmem = ctl->tmem_base;
   bool ok = true;
 
-  if (threadIdx.x == 32) {
+  if (threadIdx.x == 128) {
     // MMA issuer: D_t[128 x 3R] = A_t[128 x r] . B[3R x r]^T
     const uint32_t idesc = idesc_bf16_f32(128, 3 * R, 0, 0);
     const uint32_t b_base = smem_u32(b_op);
     if (n_tiles > 0) ok = mbar_wait(&ctl->b_full, 0, status);
     for (int t = 0; t < n_tiles && ok; ++t) {
-      ok = mbar_wait(&ctl->tma_full[t], 0, status);
-      if (!ok) break;
-      tc_fence_after();
       const uint32_t a_base = smem_u32(a_op + t * stc_a_bytes(r));
-      for (int kb = 0; kb < nkb; ++kb)
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        ok = mbar_wait(&ctl->tma_full[t][kb], 0, status);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t ad = sdesc_sw128(a_base + kb * (kStcTile * 128) + ks * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(b_base + kb * (3 * R * 128) + ks * 32, 16, 1024);
           umma_f16(tmem + t * kStcTileCols, ad, bd, idesc, (kb | ks) ? 1u : 0u);
         }
+      }
       umma_commit(&ctl->mma_done[t]);
     }
   }
   __syncwarp();
 
-  // B: per-tile exponentials and row sums.
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const int p = threadIdx.x;  // position within the tile
+  // B: per-tile exponentials and row sums (warps 0-3; warp 4 only joins the barriers).
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const int p = threadIdx.x;  // position within the tile (epilogue warps)
   constexpr int TPR = 128 / R;  // threads per row in the reductions
   for (int t = 0; t < n_tiles; ++t) {
-    ok = mbar_wait(&ctl->mma_done[t], 0, status) && ok;
-    tc_fence_after();
     const int64_t pos = (tile0 + t) * kStcTile + p;
-    const bool valid = pos < L;
+    const bool valid = epi && pos < L;
     const uint32_t col0 = tmem + lane_base + t * kStcTileCols;
     float amax = 0.f;
+    if (epi) {
+      ok = mbar_wait(&ctl->mma_done[t], 0, status) && ok;
+      tc_fence_after();
 #pragma unroll 1
-    for (int c = 0; c < R / 32; ++c) {
-      uint32_t hi[32], mid[32], lo[32];
-      tmem_ld32(col0 + c * 32, hi);
-      tmem_ld32(col0 + R + c * 32, mid);
-      tmem_ld32(col0 + 2 * R + c * 32, lo);
-      tmem_wait_ld();
-      uint32_t ev[32];
+      for (int c = 0; c < R / 32; ++c) {
+        uint32_t hi[32], mid[32], lo[32];
+        tmem_ld32(col0 + c * 32, hi);
+        tmem_ld32(col0 + R + c * 32, mid);
+        tmem_ld32(col0 + 2 * R + c * 32, lo);
+        tmem_wait_ld();
+        uint32_t ev[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float y = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
-        hi[j] = __float_as_uint(y);
-        amax = valid ? fmaxf(amax, fabsf(y)) : amax;
-        const float e = valid ? ex2_approx(y) : 0.f;
-        ev[j] = __float_as_uint(e);
-        red[p * (R + 1) + c * 32 + j] = e;
+        for (int j = 0; j < 32; ++j) {
+          const float y = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
+          hi[j] = __float_as_uint(y);
+          amax = valid ? fmaxf(amax, fabsf(y)) : amax;
+          const float e = valid ? ex2_approx(y) : 0.f;
+          ev[j] = __float_as_uint(e);
+          red[p * (R + 1) + c * 32 + j] = e;
+        }
+        tmem_st32(col0 + c * 32, hi);      // y
+        tmem_st32(col0 + R + c * 32, ev);  // e
+        tmem_wait_st();
       }
-      tmem_st32(col0 + c * 32, hi);      // y
-      tmem_st32(col0 + R + c * 32, ev);  // e
-      tmem_wait_st();
     }
     const bool wide = __syncthreads_or(amax > kStcRangeLimit) != 0;
     if (wide) {
       // Rare path: per-row integer offsets k = floor(max_i y) for this tile.
-      for (int c = 0; c < R / 32; ++c) {
-        uint32_t yv[32];
-        tmem_ld32(col0 + c * 32, yv);
-        tmem_wait_ld();
+      if (epi)
+        for (int c = 0; c < R / 32; ++c) {
+          uint32_t yv[32];
+          tmem_ld32(col0 + c * 32, yv);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) red[p * (R + 1) + c * 32 + j] = valid ? __uint_as_float(yv[j]) : -INFINITY;
-      }
+          for (int j = 0; j < 32; ++j) red[p * (R + 1) + c * 32 + j] = valid ? __uint_as_float(yv[j]) : -INFINITY;
+        }
       __syncthreads();
       if (threadIdx.x < R) {
         float m = -INFINITY;
@@ -192,43 +201,56 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
         ctl->kofs[t][threadIdx.x] = (m == -INFINITY) ? 0 : (int)floorf(m);
       }
       __syncthreads();
-      for (int c = 0; c < R / 32; ++c) {
-        uint32_t yv[32], ev[32];
-        tmem_ld32(col0 + c * 32, yv);
-        tmem_wait_ld();
+      if (epi)
+        for (int c = 0; c < R / 32; ++c) {
+          uint32_t yv[32], ev[32];
+          tmem_ld32(col0 + c * 32, yv);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float e = valid ? ex2_approx(__uint_as_float(yv[j]) - (float)ctl->kofs[t][c * 32 + j]) : 0.f;
-          ev[j] = __float_as_uint(e);
-          red[p * (R + 1) + c * 32 + j] = e;
+          for (int j = 0; j < 32; ++j) {
+            const float e = valid ? ex2_approx(__uint_as_float(yv[j]) - (float)ctl->kofs[t][c * 32 + j]) : 0.f;
+            ev[j] = __float_as_uint(e);
+            red[p * (R + 1) + c * 32 + j] = e;
+          }
+          tmem_st32(col0 + R + c * 32, ev);
+          tmem_wait_st();
         }
-        tmem_st32(col0 + R + c * 32, ev);
-        tmem_wait_st();
-      }
     } else if (threadIdx.x < R) {
       ctl->kofs[t][threadIdx.x] = 0;
     }
     __syncthreads();
     // Row sums over the tile's 128 positions: TPR threads per row, four
-    // independent fp32 partial sums each (fp64 arithmetic would stall the
-    // tensor pipe), combined in a fixed order and added in fp64.
+    // independent fp32 partial sums each, combined in a fixed order.
     {
       const int row = threadIdx.x % R, part = threadIdx.x / R;
       constexpr int kPer = kStcTile / TPR;
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+      float mine = 0.f;
+      if (epi) {
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-      for (int q = 0; q < kPer; ++q) a4[q & 3] += red[(part * kPer + q) * (R + 1) + row];
-      const float mine = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-      red[p * (R + 1) + R] = mine;   // column R of the scratch is free
+        for (int q = 0; q < kPer; ++q) a4[q & 3] += red[(part * kPer + q) * (R + 1) + row];
+        mine = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      }
       __syncthreads();
-      if (part == 0 && row < s.n_rows) {
-        double l = 0.0;
-        for (int pp = 0; pp < TPR; ++pp) l += (double)red[(pp * R + row) * (R + 1) + R];
-        atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + blockIdx.x % kStcSumSlots) * s.n_rows + row],
-                  ldexp(l, ctl->kofs[t][row]));
+      if (epi) red[p * (R + 1) + R] = mine;   // column R of the scratch is free
+      __syncthreads();
+      if (epi && part == 0) {
+        float l = 0.f;
+        for (int pp = 0; pp < TPR; ++pp) l += red[(pp * R + row) * (R + 1) + R];
+        ctl->tile_sum[t][row] = l;
       }
     }
     __syncthreads();
+  }
+  // One fp64 atomic per row and CTA (both tiles belong to the same problem).
+  if (threadIdx.x < R && threadIdx.x < s.n_rows && n_tiles > 0) {
+    const int row = threadIdx.x;
+    double l = 0.0;
+    for (int t = 0; t < n_tiles; ++t) {
+      const double v = (double)ctl->tile_sum[t][row];
+      l += ctl->kofs[t][row] ? ldexp(v, ctl->kofs[t][row]) : v;
+    }
+    atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + blockIdx.x % kStcSumSlots) * s.n_rows + row], l);
   }
 
   // C: every tile of every problem has added its row sums.
@@ -253,24 +275,24 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     }
   }
   __syncthreads();
-  for (int t = 0; t < n_tiles; ++t) {
-    const int64_t pos = (tile0 + t) * kStcTile + p;
-    const uint32_t col0 = tmem + lane_base + t * kStcTileCols;
-    float acc = 0.f;
+  if (epi)
+    for (int t = 0; t < n_tiles; ++t) {
+      const int64_t pos = (tile0 + t) * kStcTile + p;
+      const uint32_t col0 = tmem + lane_base + t * kStcTileCols;
+      float acc = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < R / 32; ++c) {
-      uint32_t ev[32];
-      tmem_ld32(col0 + R + c * 32, ev);
-      tmem_wait_ld();
+      for (int c = 0; c < R / 32; ++c) {
+        uint32_t ev[32];
+        tmem_ld32(col0 + R + c * 32, ev);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc = fmaf(ctl->alpha[t][c * 32 + j], __uint_as_float(ev[j]), acc);
+        for (int j = 0; j < 32; ++j) acc = fmaf(ctl->alpha[t][c * 32 + j], __uint_as_float(ev[j]), acc);
+      }
+      if (pos < L) scores[(int64_t)b * s.cache_rows + pos] = acc;
     }
-    if (pos < L) scores[(int64_t)b * s.cache_rows + pos] = acc;
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kStcTmemCols);
-  (void)lane;
 }
 
 }  // namespace s4r

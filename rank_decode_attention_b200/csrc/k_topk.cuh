@@ -68,7 +68,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_t
 constexpr int kTopkSmemKeys = 32768;  // keys staged in shared memory (128 KB) when they fit
 // Staged key i lives at word i + i/32: a thread walking its own contiguous
 // chunk of 32 keys then never shares a bank with the other lanes of its warp.
-__host__ __device__ __forceinline__ int64_t kpad(int64_t i) { return i + (i >> 5); }
+__host__ __device__ __forceinline__ int kpad(int i) { return i + (i >> 5); }
 constexpr int kTopkBins = 256;         // 8-bit digits
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkSample = 256;       // sampled keys that bracket the threshold
@@ -89,7 +89,7 @@ struct TopkShared {
 };
 
 template <bool kShared>
-__device__ __forceinline__ uint32_t key_at(const uint32_t *keys, int64_t i) {
+__device__ __forceinline__ uint32_t key_at(const uint32_t *keys, int i) {
   return kShared ? keys[kpad(i)] : __ldcg(keys + i);
 }
 
@@ -97,13 +97,13 @@ __device__ __forceinline__ uint32_t key_at(const uint32_t *keys, int64_t i) {
 // match `prefix` under `mask`, then the digit holding the `remaining`-th
 // largest.  `value(i)` returns (valid, v) for slot i < n_slots.
 template <typename ValueFn>
-__device__ void radix_pass(ValueFn value, int64_t n_slots, int shift, uint32_t mask, uint32_t &prefix,
+__device__ __forceinline__ void radix_pass(ValueFn value, int n_slots, int shift, uint32_t mask, uint32_t &prefix,
                            uint32_t &remaining, TopkShared &sh) {
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < kTopkBins / 32; ++j) sh.whist[wid][lane + 32 * j] = 0;
   __syncthreads();
-  for (int64_t i = threadIdx.x; i < n_slots; i += blockDim.x) {
+  for (int i = threadIdx.x; i < n_slots; i += blockDim.x) {
     bool ok;
     const uint32_t v = value(i, ok);
     if (ok && (v & mask) == prefix) atomicAdd(&sh.whist[wid][(v >> shift) & 255u], 1u);
@@ -147,7 +147,7 @@ __device__ void radix_pass(ValueFn value, int64_t n_slots, int shift, uint32_t m
 // minimum and maximum).  Returns tau and how many values equal to tau are in
 // the top `need`.
 template <typename ValueFn>
-__device__ void radix_select(ValueFn value, int64_t n_slots, uint32_t need, uint32_t lo_all, uint32_t hi_all,
+__device__ __forceinline__ void radix_select(ValueFn value, int n_slots, uint32_t need, uint32_t lo_all, uint32_t hi_all,
                              TopkShared &sh, uint32_t *tau, uint32_t *take_eq) {
   const uint32_t diff = lo_all ^ hi_all;
   int top = 31;
@@ -188,11 +188,11 @@ __device__ __forceinline__ void block_minmax(uint32_t lo, uint32_t hi, TopkShare
 // the collected keys finishes.  Returns false if the bracket missed or a
 // segment overflowed (the caller then selects on all keys).
 template <bool kShared>
-__device__ bool bracket_select(const uint32_t *keys, int64_t nc, uint32_t need, TopkShared &sh, uint32_t *cand,
+__device__ __forceinline__ bool bracket_select(const uint32_t *keys, int nc, uint32_t need, TopkShared &sh, uint32_t *cand,
                                uint32_t *tau, uint32_t *take_eq) {
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = kTopkSample;
-  if (threadIdx.x < M) sh.sample[threadIdx.x] = key_at<kShared>(keys, (int64_t)threadIdx.x * nc / M);
+  if (threadIdx.x < M) sh.sample[threadIdx.x] = key_at<kShared>(keys, (int)(((int64_t)threadIdx.x * nc) / M));
   const double q = (double)need * M / (double)nc;
   const double delta = 4.0 * sqrt(q + 1.0) + 8.0;
   const int r_hi = (int)floor(q - delta);   // 1-based ranks of the bracket ends
@@ -219,8 +219,8 @@ __device__ bool bracket_select(const uint32_t *keys, int64_t nc, uint32_t need, 
   // Count keys strictly above t_hi and collect keys in [t_lo, t_hi].
   uint32_t above = 0, seg = 0, cmin = 0xffffffffu, cmax = 0u;
   uint32_t *mine = cand + wid * kTopkSeg;
-  for (int64_t i0 = 0; i0 < nc; i0 += blockDim.x) {
-    const int64_t i = i0 + threadIdx.x;
+  for (int i0 = 0; i0 < nc; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
     const bool valid = i < nc;
     const uint32_t v = valid ? key_at<kShared>(keys, i) : 0u;
     above += (valid && v > t_hi);
@@ -248,25 +248,25 @@ __device__ bool bracket_select(const uint32_t *keys, int64_t nc, uint32_t need, 
     overflow |= sh.seg_count[w] > (uint32_t)kTopkSeg;
   }
   if (overflow || !(n_above < need && need <= n_above + n_cand)) return false;
-  auto value = [&](int64_t i, bool &ok) -> uint32_t {
-    const int w = (int)(i / kTopkSeg), e = (int)(i - (int64_t)w * kTopkSeg);
+  auto value = [&](int i, bool &ok) -> uint32_t {
+    const int w = i / kTopkSeg, e = i - w * kTopkSeg;
     ok = e < (int)sh.seg_count[w];
     return ok ? cand[i] : 0u;
   };
-  radix_select(value, (int64_t)kTopkCand, need - n_above, sh.cmin, sh.cmax, sh, tau, take_eq);
+  radix_select(value, kTopkCand, need - n_above, sh.cmin, sh.cmax, sh, tau, take_eq);
   return true;
 }
 
 // Stable compaction in index order: every key > tau and the first take_eq
 // keys == tau, written as absolute positions.
 template <bool kShared>
-__device__ void compact_selected(const uint32_t *keys, int64_t nc, uint32_t tau, uint32_t take_eq, int32_t n_sink,
+__device__ __forceinline__ void compact_selected(const uint32_t *keys, int nc, uint32_t tau, uint32_t take_eq, int32_t n_sink,
                                  int32_t *out, int k, TopkShared &sh) {
-  const int chunk = (int)ceil_div(nc, blockDim.x);
-  const int64_t i0 = smin<int64_t>(nc, (int64_t)threadIdx.x * chunk);
-  const int64_t i1 = smin<int64_t>(nc, i0 + chunk);
+  const int chunk = (nc + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int i0 = min(nc, (int)threadIdx.x * chunk);
+  const int i1 = min(nc, i0 + chunk);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int64_t i = i0; i < i1; ++i) {
+  for (int i = i0; i < i1; ++i) {
     const uint32_t key = key_at<kShared>(keys, i);
     n_gt += key > tau;
     n_eq += key == tau;
@@ -275,7 +275,7 @@ __device__ void compact_selected(const uint32_t *keys, int64_t nc, uint32_t tau,
   const uint32_t eq_take = (eq_before >= take_eq) ? 0u : min(n_eq, take_eq - eq_before);
   const uint32_t out_before = block_excl_scan(n_gt + eq_take, sh.warp_tot, &sh.total);
   uint32_t pos = out_before, eq_seen = 0;
-  for (int64_t i = i0; i < i1; ++i) {
+  for (int i = i0; i < i1; ++i) {
     const uint32_t key = key_at<kShared>(keys, i);
     bool take = key > tau;
     if (key == tau) { take = eq_seen < eq_take; ++eq_seen; }
@@ -284,11 +284,11 @@ __device__ void compact_selected(const uint32_t *keys, int64_t nc, uint32_t tau,
 }
 
 template <bool kShared>
-__device__ void select_top(const uint32_t *keys, int64_t nc, uint32_t need, int32_t n_sink, int32_t *out, int k,
+__device__ __forceinline__ void select_top(const uint32_t *keys, int nc, uint32_t need, int32_t n_sink, int32_t *out, int k,
                            TopkShared &sh, uint32_t *cand) {
   uint32_t tau = 0, take_eq = 0;
   if (nc <= 4 * kTopkSample || !bracket_select<kShared>(keys, nc, need, sh, cand, &tau, &take_eq)) {
-    auto value = [&](int64_t i, bool &ok) -> uint32_t {
+    auto value = [&](int i, bool &ok) -> uint32_t {
       ok = true;
       return key_at<kShared>(keys, i);
     };
@@ -318,7 +318,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
     for (int64_t i = threadIdx.x; i < nc; i += blockDim.x) out[i] = (int32_t)(s.n_sink + i);
     return;
   }
-  const int64_t n_stage = kpad(smin<int64_t>(s.cache_rows, kTopkSmemKeys)) + 1;
+  const int n_stage = kpad((int)smin<int64_t>(s.cache_rows, kTopkSmemKeys)) + 1;
   uint32_t *keys_s = topk_dyn;
   uint32_t *cand = topk_dyn + n_stage;
   if (nc <= kTopkSmemKeys) {
@@ -328,7 +328,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
     const int64_t head = smin<int64_t>(nc, (int64_t)((16u - (reinterpret_cast<uintptr_t>(gkeys) & 15u)) & 15u) / 4);
     const int64_t n4 = (nc - head) / 4;
     const uint4 *src4 = reinterpret_cast<const uint4 *>(gkeys + head);
-    for (int64_t i = threadIdx.x; i < head; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i);
+    for (int i = threadIdx.x; i < (int)head; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i);
     for (int64_t i0 = 0; i0 < n4; i0 += 4 * kTopkThreads) {
       uint4 v[4];
 #pragma unroll
@@ -340,7 +340,7 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
       for (int u = 0; u < 4; ++u) {
         const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
         if (i < n4) {
-          const int64_t j = head + 4 * i;
+          const int j = (int)(head + 4 * i);
           keys_s[kpad(j)] = v[u].x;
           keys_s[kpad(j + 1)] = v[u].y;
           keys_s[kpad(j + 2)] = v[u].z;
@@ -348,11 +348,11 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
         }
       }
     }
-    for (int64_t i = head + 4 * n4 + threadIdx.x; i < nc; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i);
+    for (int i = (int)(head + 4 * n4) + threadIdx.x; i < (int)nc; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i);
     __syncthreads();
-    select_top<true>(keys_s, nc, (uint32_t)need, s.n_sink, out, k, sh, cand);
+    select_top<true>(keys_s, (int)nc, (uint32_t)need, s.n_sink, out, k, sh, cand);
   } else {
-    select_top<false>(gkeys, nc, (uint32_t)need, s.n_sink, out, k, sh, cand);
+    select_top<false>(gkeys, (int)nc, (uint32_t)need, s.n_sink, out, k, sh, cand);
   }
 }
 

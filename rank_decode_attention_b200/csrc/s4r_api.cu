@@ -171,7 +171,8 @@ bool tc_fits(int rank, int grid, size_t *smem_out) {
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
   if (cudaFuncSetAttribute(score_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return false;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, 128, smem) != cudaSuccess) return false;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, kStcThreads, smem) != cudaSuccess)
+    return false;
   *smem_out = smem;
   return grid <= per_sm * sms;
 }
@@ -202,7 +203,7 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
                            cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(kStcThreads);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
