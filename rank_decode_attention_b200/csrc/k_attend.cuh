@@ -12,10 +12,10 @@
 // rows of the basis that belong to group g.  Nothing is rounded to the
 // storage type; all arithmetic is fp32.
 //
-// One launch; the kAttCluster CTAs of a (kv group g, problem) form a thread
-// block cluster, 256 threads each:
+// One launch; the CTAs of a (kv group g, problem) form a thread block
+// cluster (16 CTAs, or 8 where 16 cannot be scheduled), 256 threads each:
 //   1. CTA rank c takes an equal share of the selected rows and walks it in
-//      chunks of 64: cp.async the chunk's C_K / C_V rows, logits of the G
+//      chunks of 128 rows (64 for fp32 storage): cp.async the chunk's C_K / C_V rows, logits of the G
 //      heads of group g, online softmax (running max, sum) and the latent
 //      value sums acc[j][:] += p[j][e] c_V[e];
 //   2. its partial (m, l, acc) stays in its shared memory; after a cluster
@@ -31,8 +31,9 @@
 namespace s4r {
 
 constexpr int kAttThreads = 256;      // 8 warps
-constexpr int kAttCluster = 8;        // CTAs per (kv group, problem)
-constexpr int kAttEntries = 64;       // selected rows per chunk
+constexpr int kAttCluster = 16;       // most CTAs per (kv group, problem); the launch may use 8
+constexpr int kAttEntriesMax = 128;   // selected rows per chunk (bf16 storage; 64 for fp32)
+template <typename T> __host__ __device__ constexpr int att_entries() { return sizeof(T) == 2 ? 128 : 64; }
 constexpr int kAttMaxGroup = 8;       // G <= 8
 constexpr int kAttMaxSinks = 16;      // sinks merged by rank 0
 
@@ -45,13 +46,13 @@ __host__ __device__ inline int att_pitch(int n, int esize) {
   return words * 4 / esize;
 }
 __host__ __device__ inline size_t att_stage_bytes(const Shape &s, int esize) {
-  const size_t rows = (size_t)kAttEntries * (att_pitch(s.rank_k, esize) + att_pitch(s.rank_v, esize)) * esize;
+  const size_t rows = (size_t)(esize == 2 ? 128 : 64) * (att_pitch(s.rank_k, esize) + att_pitch(s.rank_v, esize)) * esize;
   const size_t bv = (size_t)s.head_dim * att_pitch(s.rank_v, esize) * esize;
   return rows > bv ? rows : bv;
 }
 __host__ __device__ inline size_t att_float_words(const Shape &s) {
   return (size_t)kAttMaxGroup * s.rank_k          // q_s
-         + (size_t)kAttMaxGroup * kAttEntries     // p_s
+         + (size_t)kAttMaxGroup * kAttEntriesMax  // p_s
          + (size_t)kAttMaxGroup * 4               // ml_s: m, l, chunk scale, merged inverse
          + (size_t)kAttMaxGroup * (s.rank_v + 2)  // part_s: this CTA's m, l, acc[rv] per head
          + (size_t)kAttMaxGroup * s.rank_v        // acc_s (rank 0)
@@ -85,7 +86,7 @@ __device__ __forceinline__ float dot_f32_store(const float *a, const T *x, int n
 }
 
 template <typename T>
-__global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThreads)
+__global__ void __launch_bounds__(kAttThreads)
 attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
               const T *__restrict__ coeff_k, const T *__restrict__ coeff_v, const float *__restrict__ qt_all,
               const T *__restrict__ q, const T *__restrict__ basis_v, const T *__restrict__ sink_k,
@@ -93,28 +94,30 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   extern __shared__ __align__(16) unsigned char att_smem[];
   constexpr int V = Vec16<T>::n;
   constexpr int kWarps = kAttThreads / 32;
+  constexpr int kAttEntries = att_entries<T>();
   const int g = blockIdx.y, b = blockIdx.z;
   const uint32_t rank = cluster_ctarank();
+  const int n_ranks = (int)gridDim.x;   // the launch makes gridDim.x CTAs one cluster
   const int G = s.group, rk = s.rank_k, rv = s.rank_v, dh = s.head_dim, Dp = s.d_model, ns = s.n_sink;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int pk = att_pitch(rk, sizeof(T)), pv = att_pitch(rv, sizeof(T));
   T *ck_s = reinterpret_cast<T *>(att_smem);
   T *cv_s = ck_s + kAttEntries * pk;
   float *q_s = reinterpret_cast<float *>(att_smem + att_stage_bytes(s, sizeof(T)));  // [G][rk]
-  float *p_s = q_s + kAttMaxGroup * rk;                     // [G][64] logits, then weights
+  float *p_s = q_s + kAttMaxGroup * rk;                     // [G][entries] logits, then weights
   float *ml_s = p_s + kAttMaxGroup * kAttEntries;           // [G][4]
   float *part_s = ml_s + kAttMaxGroup * 4;                  // [G][rv + 2]
   float *acc_s = part_s + kAttMaxGroup * (rv + 2);          // [G][rv]
   float *sw_s = acc_s + kAttMaxGroup * rv;                  // [G][kAttMaxSinks]
   float *f_s = sw_s + kAttMaxGroup * kAttMaxSinks;          // [G][kAttCluster]
-  __shared__ int64_t rows_s[kAttEntries];
+  __shared__ int64_t rows_s[kAttEntriesMax];
   __shared__ __align__(8) uint64_t stage_bar;
 
   const int64_t L = valid_length(lengths[b], s.cache_rows);
   const int64_t n_top = smin<int64_t>(s.top_k, n_candidates(L, s.local_window));
   const int64_t n_win = smin<int64_t>(s.local_window, L);
   const int64_t n_sel = n_top + n_win;
-  const int64_t per = ceil_div(n_sel, kAttCluster);
+  const int64_t per = ceil_div(n_sel, n_ranks);
   const int64_t e_begin = smin<int64_t>(n_sel, (int64_t)rank * per);
   const int64_t e_end = smin<int64_t>(n_sel, e_begin + per);
   const int32_t *idx_b = idx + (int64_t)b * s.top_k;
@@ -183,16 +186,26 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       p_s[j * kAttEntries + e] = l;
     }
     __syncthreads();
-    // online softmax update per head (warp j)
+    // online softmax update per head (warp j), kAttEntries / 32 entries per lane
     for (int j = wid; j < G; j += kWarps) {
-      const float l0 = p_s[j * kAttEntries + lane], l1 = p_s[j * kAttEntries + lane + 32];
+      constexpr int kPer = kAttEntries / 32;
+      float lv[kPer];
+      float mc = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        lv[u] = p_s[j * kAttEntries + lane + 32 * u];
+        mc = fmaxf(mc, lv[u]);
+      }
       const float m_old = ml_s[j * 4];
-      const float m_new = fmaxf(m_old, warp_max(fmaxf(l0, l1)));
-      const float p0 = (m_new == -INFINITY) ? 0.f : __expf(l0 - m_new);
-      const float p1 = (m_new == -INFINITY) ? 0.f : __expf(l1 - m_new);
-      const float csum = warp_sum(p0 + p1);
-      p_s[j * kAttEntries + lane] = p0;
-      p_s[j * kAttEntries + lane + 32] = p1;
+      const float m_new = fmaxf(m_old, warp_max(mc));
+      float csum = 0.f;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const float pu = (m_new == -INFINITY) ? 0.f : __expf(lv[u] - m_new);
+        p_s[j * kAttEntries + lane + 32 * u] = pu;
+        csum += pu;
+      }
+      csum = warp_sum(csum);
       if (lane == 0) {
         const float scale = (m_old == -INFINITY) ? 0.f : __expf(m_old - m_new);
         ml_s[j * 4] = m_new;
@@ -249,10 +262,10 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       if (lane == 0) sw_s[j * kAttMaxSinks + tk] = d * qscale;
     }
     __syncthreads();
-    // Merge weights per head (warp j): ranks r = lanes 0..7.
+    // Merge weights per head (warp j): ranks r = lanes 0 .. n_ranks-1.
     for (int j = wid; j < G; j += kWarps) {
       float mr = -INFINITY, lr = 0.f;
-      if (lane < kAttCluster) {
+      if (lane < n_ranks) {
         const uint32_t base = cluster_map(part_s + j * (rv + 2), (uint32_t)lane);
         mr = ld_cluster_f32(base);
         lr = ld_cluster_f32(base + 4);
@@ -265,7 +278,7 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       for (int tk = lane; tk < ns; tk += 32) den += __expf(sw_s[j * kAttMaxSinks + tk] - M);
       den = warp_sum(den);
       const float inv = den > 0.f ? 1.f / den : 0.f;
-      if (lane < kAttCluster) f_s[j * kAttCluster + lane] = fr * inv;
+      if (lane < n_ranks) f_s[j * kAttCluster + lane] = fr * inv;
       __syncwarp();
       for (int tk = lane; tk < ns; tk += 32)
         sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
@@ -277,10 +290,11 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
       float v[kAttCluster];
 #pragma unroll
       for (int r = 0; r < kAttCluster; ++r)
-        v[r] = ld_cluster_f32(cluster_map(part_s + j * (rv + 2) + 2 + k, (uint32_t)r));
+        v[r] = (r < n_ranks) ? ld_cluster_f32(cluster_map(part_s + j * (rv + 2) + 2 + k, (uint32_t)r)) : 0.f;
       float a = 0.f;
 #pragma unroll
-      for (int r = 0; r < kAttCluster; ++r) a = fmaf(f_s[j * kAttCluster + r], v[r], a);
+      for (int r = 0; r < kAttCluster; ++r)
+        if (r < n_ranks) a = fmaf(f_s[j * kAttCluster + r], v[r], a);
       acc_s[t] = a;
     }
     mbar_wait(&stage_bar, phase, nullptr);

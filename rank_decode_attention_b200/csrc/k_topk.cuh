@@ -12,6 +12,7 @@
 // order takes every key > tau and the lowest-index keys == tau.
 #pragma once
 #include "common.cuh"
+#include "umma.cuh"
 
 namespace s4r {
 
@@ -354,6 +355,307 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
   } else {
     select_top<false>(gkeys, (int)nc, (uint32_t)need, s.n_sink, out, k, sh, cand);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Cluster variant: the kTopkCl CTAs of a cluster split one problem's keys.
+// Each CTA stages its contiguous share in shared memory and contributes 32
+// sampled keys; every CTA ranks the 256 samples (read through distributed
+// shared memory) the same way, collects its in-bracket keys, and rank 0
+// radix-selects the exact threshold among all ranks' candidates.  A cluster
+// prefix of the per-rank counts then gives each rank its output offset for
+// the stable compaction.  Falls back to rank 0 selecting over every key
+// (read through distributed shared memory) if the bracket misses.
+constexpr int kTopkCl = 8;                       // CTAs per problem
+constexpr int kTopkClThreads = 512;
+constexpr int kTopkClWarps = kTopkClThreads / 32;
+constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
+constexpr int kTopkClSeg = 256;                  // candidates per warp
+constexpr int kTopkClCand = 8192;                // candidates rank 0 gathers at most
+__host__ inline size_t topk_cl_smem_bytes() {
+  return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1 + kTopkClWarps * kTopkClSeg + kTopkClCand);
+}
+
+struct TopkClShared {
+  uint32_t whist[kTopkClWarps][kTopkBins];
+  uint32_t hist[kTopkBins];
+  uint32_t sample[32];               // this rank's samples (read by all ranks)
+  uint32_t all_sample[kTopkSample];
+  uint32_t seg_count[kTopkClWarps];
+  uint32_t seg_above[kTopkClWarps];
+  uint32_t warp_tot[32];
+  uint32_t total, digit, above, t_hi, t_lo, cmin, cmax;
+  uint32_t n_above, n_cand;          // this rank's totals (read by rank 0)
+  uint32_t tau, take_eq, ok;         // rank 0's result (read by all ranks)
+  uint32_t n_gt, n_eq;               // this rank's compaction counts (read by all ranks)
+};
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+template <typename Tp>
+__device__ __forceinline__ uint32_t remote_u32(const Tp *p, uint32_t rank) {
+  return ld_cluster_u32(cluster_map(p, rank));
+}
+
+// Block-wide radix pass / select for blockDim-sized CTAs of the cluster kernel.
+template <typename ValueFn>
+__device__ __forceinline__ void cl_radix_pass(ValueFn value, int n_slots, int shift, uint32_t mask, uint32_t &prefix,
+                                              uint32_t &remaining, TopkClShared &sh) {
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < kTopkBins / 32; ++j) sh.whist[wid][lane + 32 * j] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_slots; i += blockDim.x) {
+    bool ok;
+    const uint32_t v = value(i, ok);
+    if (ok && (v & mask) == prefix) atomicAdd(&sh.whist[wid][(v >> shift) & 255u], 1u);
+  }
+  __syncthreads();
+  if (threadIdx.x < kTopkBins) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kTopkClWarps; ++w) c += sh.whist[w][threadIdx.x];
+    sh.hist[threadIdx.x] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t cnt[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t run = incl - sum;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (run < remaining && run + cnt[j] >= remaining) {
+        sh.digit = 255u - (uint32_t)(lane * 8 + j);
+        sh.above = run;
+      }
+      run += cnt[j];
+    }
+  }
+  __syncthreads();
+  remaining -= sh.above;
+  prefix |= sh.digit << shift;
+  __syncthreads();
+}
+template <typename ValueFn>
+__device__ __forceinline__ void cl_radix_select(ValueFn value, int n_slots, uint32_t need, uint32_t lo_all,
+                                                uint32_t hi_all, TopkClShared &sh, uint32_t *tau, uint32_t *take_eq) {
+  const uint32_t diff = lo_all ^ hi_all;
+  int top = 31;
+  while (top >= 0 && !((diff >> top) & 1u)) --top;
+  uint32_t prefix = 0, mask = 0, remaining = need;
+  if (top < 31) {
+    const uint32_t common = (top < 0) ? 0xffffffffu : ~((2u << top) - 1u);
+    prefix = lo_all & common;
+    mask = common;
+  }
+  if (top >= 0)
+    for (int shift = (top / 8) * 8; shift >= 0; shift -= 8) {
+      cl_radix_pass(value, n_slots, shift, mask, prefix, remaining, sh);
+      mask |= 255u << shift;
+    }
+  *tau = prefix;
+  *take_eq = remaining;
+}
+
+__global__ void __cluster_dims__(kTopkCl, 1, 1) __launch_bounds__(kTopkClThreads)
+topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restrict__ keys_all,
+                    int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
+  extern __shared__ __align__(16) uint32_t tcl_dyn[];
+  __shared__ TopkClShared sh;
+  uint32_t *keys_s = tcl_dyn;                                   // this rank's keys (padded)
+  uint32_t *seg = tcl_dyn + kpad(kTopkClKeys) + 1;              // per-warp candidate segments
+  uint32_t *gath = seg + kTopkClWarps * kTopkClSeg;             // rank 0: all candidates
+  const uint32_t rank = cluster_ctarank();
+  const int b = blockIdx.y;
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t Lraw = lengths[b];
+  if (rank == 0 && threadIdx.x == 0 && (Lraw < 0 || Lraw > s.cache_rows)) set_status(status, kDevStatusCheck);
+  const int64_t L = valid_length(Lraw, s.cache_rows);
+  const int nc = (int)n_candidates(L, s.local_window);
+  const int k = s.top_k;
+  int32_t *out = idx + (int64_t)b * k;
+  const uint32_t *gkeys = reinterpret_cast<const uint32_t *>(keys_all + (int64_t)b * s.cache_rows);
+  const int need = min(k, nc);
+  // Trivial cases: every rank takes the same branch (uniform), no cluster barrier used.
+  if (need == 0 || need == nc) {
+    for (int e = (int)rank * blockDim.x + threadIdx.x; e < k; e += kTopkCl * blockDim.x)
+      out[e] = (e < nc) ? (int32_t)(s.n_sink + e) : -1;
+    return;
+  }
+  for (int e = need + (int)rank * blockDim.x + threadIdx.x; e < k; e += kTopkCl * blockDim.x) out[e] = -1;
+  const int chunk = (nc + kTopkCl - 1) / kTopkCl;
+  const int i_begin = min(nc, (int)rank * chunk), i_end = min(nc, i_begin + chunk);
+  const int my_n = i_end - i_begin;
+  for (int i = threadIdx.x; i < my_n; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i_begin + i);
+  __syncthreads();
+  // 32 samples of this rank's share, then all 256 (same order on every rank).
+  if (threadIdx.x < 32)
+    sh.sample[threadIdx.x] = my_n > 0 ? keys_s[kpad((int)(((int64_t)threadIdx.x * my_n) / 32))] : 0u;
+  cluster_sync();
+  if (threadIdx.x < kTopkSample) sh.all_sample[threadIdx.x] = remote_u32(&sh.sample[threadIdx.x & 31], threadIdx.x >> 5);
+  if (threadIdx.x == 0) { sh.t_hi = 0xffffffffu; sh.t_lo = 0u; }
+  __syncthreads();
+  {
+    const double q = (double)need * kTopkSample / (double)nc;
+    const double delta = 4.0 * sqrt(q + 1.0) + 8.0;
+    const int r_hi = (int)floor(q - delta), r_lo = (int)ceil(q + delta);
+    if (threadIdx.x < kTopkSample) {
+      const uint32_t v = sh.all_sample[threadIdx.x];
+      int rnk = 0;
+#pragma unroll 8
+      for (int j = 0; j < kTopkSample; ++j) {
+        const uint32_t u = sh.all_sample[j];
+        rnk += (u > v) || (u == v && j < (int)threadIdx.x);
+      }
+      if (r_hi >= 1 && rnk == r_hi - 1) sh.t_hi = v;
+      if (r_lo <= kTopkSample && rnk == r_lo - 1) sh.t_lo = v;
+    }
+  }
+  __syncthreads();
+  const uint32_t t_hi = sh.t_hi, t_lo = sh.t_lo;
+  // Count this rank's keys above the bracket and collect those inside it.
+  uint32_t above = 0, cnt = 0, cmin = 0xffffffffu, cmax = 0u;
+  uint32_t *mine = seg + wid * kTopkClSeg;
+  for (int i0 = 0; i0 < my_n; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const bool valid = i < my_n;
+    const uint32_t v = valid ? keys_s[kpad(i)] : 0u;
+    above += (valid && v > t_hi);
+    const bool in = valid && v <= t_hi && v >= t_lo;
+    const uint32_t ball = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      const uint32_t slot = cnt + __popc(ball & ((1u << lane) - 1u));
+      if (slot < kTopkClSeg) mine[slot] = v;
+      cmin = min(cmin, v);
+      cmax = max(cmax, v);
+    }
+    cnt += __popc(ball);
+  }
+  above = warp_sum_u32(above);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
+    cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+  }
+  if (threadIdx.x == 0) { sh.cmin = 0xffffffffu; sh.cmax = 0u; }
+  __syncthreads();
+  if (lane == 0) {
+    sh.seg_count[wid] = cnt;
+    sh.seg_above[wid] = above;
+    atomicMin(&sh.cmin, cmin);
+    atomicMax(&sh.cmax, cmax);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t na = 0, ncd = 0;
+    for (int w = 0; w < kTopkClWarps; ++w) {
+      na += sh.seg_above[w];
+      ncd += (sh.seg_count[w] > (uint32_t)kTopkClSeg) ? 0x40000000u : sh.seg_count[w];  // overflow poisons
+    }
+    sh.n_above = na;
+    sh.n_cand = ncd;
+  }
+  cluster_sync();
+  if (rank == 0) {
+    uint32_t n_above = 0, n_cand = 0, lo = 0xffffffffu, hi = 0u;
+    for (uint32_t c = 0; c < kTopkCl; ++c) {
+      n_above += remote_u32(&sh.n_above, c);
+      n_cand += remote_u32(&sh.n_cand, c);
+      lo = min(lo, remote_u32(&sh.cmin, c));
+      hi = max(hi, remote_u32(&sh.cmax, c));
+    }
+    const bool bracket_ok = n_cand < (uint32_t)kTopkClCand && n_above < (uint32_t)need &&
+                            (uint32_t)need <= n_above + n_cand;
+    uint32_t tau = 0, take_eq = 0;
+    if (bracket_ok) {
+      // Gather the candidates (rank-major, warp segments dense) into rank 0.
+      __shared__ uint32_t seg_off[kTopkCl * kTopkClWarps + 1];
+      if (threadIdx.x < kTopkCl * kTopkClWarps)   // all remote counts in one parallel round
+        seg_off[threadIdx.x + 1] = remote_u32(&sh.seg_count[threadIdx.x % kTopkClWarps],
+                                              (uint32_t)(threadIdx.x / kTopkClWarps));
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        seg_off[0] = 0;
+        for (int i = 1; i <= kTopkCl * kTopkClWarps; ++i) seg_off[i] += seg_off[i - 1];
+      }
+      __syncthreads();
+      for (int sgi = wid; sgi < kTopkCl * kTopkClWarps; sgi += kTopkClWarps) {
+        const int c = sgi / kTopkClWarps, w = sgi - c * kTopkClWarps;
+        const uint32_t o = seg_off[sgi], n = seg_off[sgi + 1] - o;
+        for (uint32_t e = lane; e < n; e += 32) gath[o + e] = remote_u32(seg + w * kTopkClSeg + e, (uint32_t)c);
+      }
+      __syncthreads();
+      auto value = [&](int i, bool &ok) -> uint32_t {
+        ok = true;
+        return gath[i];
+      };
+      cl_radix_select(value, (int)n_cand, (uint32_t)need - n_above, lo, hi, sh, &tau, &take_eq);
+    } else {
+      // Exact select over every key of every rank (read remotely).
+      auto value = [&](int i, bool &ok) -> uint32_t {
+        ok = true;
+        const int c = i / chunk;
+        return remote_u32(keys_s + kpad(i - c * chunk), (uint32_t)c);
+      };
+      cl_radix_select(value, nc, (uint32_t)need, 0u, 0xffffffffu, sh, &tau, &take_eq);
+    }
+    if (threadIdx.x == 0) {
+      sh.tau = tau;
+      sh.take_eq = take_eq;
+    }
+  }
+  cluster_sync();
+  const uint32_t tau = remote_u32(&sh.tau, 0), take_eq = remote_u32(&sh.take_eq, 0);
+  // Per-thread contiguous chunk counts, then the rank's totals.
+  const int per = (my_n + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int j0 = min(my_n, (int)threadIdx.x * per), j1 = min(my_n, j0 + per);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int i = j0; i < j1; ++i) {
+    const uint32_t key = keys_s[kpad(i)];
+    n_gt += key > tau;
+    n_eq += key == tau;
+  }
+  const uint32_t eq_before_local = block_excl_scan(n_eq, sh.warp_tot, &sh.total);
+  const uint32_t eq_total = sh.total;
+  const uint32_t gt_before_local = block_excl_scan(n_gt, sh.warp_tot, &sh.total);
+  const uint32_t gt_total = sh.total;
+  if (threadIdx.x == 0) { sh.n_gt = gt_total; sh.n_eq = eq_total; }
+  cluster_sync();
+  __shared__ uint32_t rank_gt[kTopkCl], rank_eq[kTopkCl];
+  if (threadIdx.x < kTopkCl) {
+    rank_gt[threadIdx.x] = remote_u32(&sh.n_gt, threadIdx.x);
+    rank_eq[threadIdx.x] = remote_u32(&sh.n_eq, threadIdx.x);
+  }
+  __syncthreads();
+  uint32_t eq_before_rank = 0, out_before_rank = 0;
+  for (uint32_t c = 0; c < rank; ++c) {
+    const uint32_t gt_c = rank_gt[c], eq_c = rank_eq[c];
+    const uint32_t take_c = (eq_before_rank >= take_eq) ? 0u : min(eq_c, take_eq - eq_before_rank);
+    out_before_rank += gt_c + take_c;
+    eq_before_rank += eq_c;
+  }
+  // Within the rank: equal keys taken in index order up to take_eq overall.
+  const uint32_t eq_before = eq_before_rank + eq_before_local;
+  const uint32_t eq_take = (eq_before >= take_eq) ? 0u : min(n_eq, take_eq - eq_before);
+  const uint32_t take_before_local = block_excl_scan(eq_take, sh.warp_tot, &sh.total);
+  uint32_t pos = out_before_rank + gt_before_local + take_before_local, eq_seen = 0;
+  for (int i = j0; i < j1; ++i) {
+    const uint32_t key = keys_s[kpad(i)];
+    bool take = key > tau;
+    if (key == tau) { take = eq_seen < eq_take; ++eq_seen; }
+    if (take && pos < (uint32_t)k) out[pos++] = (int32_t)(s.n_sink + i_begin + i);
+  }
+  cluster_sync();  // no rank leaves while another may still read its shared memory
 }
 
 }  // namespace s4r
