@@ -64,7 +64,9 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        # S4R_ORACLE_LIB: load another build of this source instead (the
+        # mutation test points it at copies with planted mistakes).
+        lib = ctypes.CDLL(os.environ.get("S4R_ORACLE_LIB") or build())
         P = ctypes.POINTER(_Problem)
         dp = ctypes.c_void_p
         lib.s4r_oracle_encode.argtypes = [dp, ctypes.c_int64, ctypes.c_int32, dp, ctypes.c_int32, dp]
