@@ -12,8 +12,8 @@
 // rows of the basis that belong to group g.  Nothing is rounded to the
 // storage type; all arithmetic is fp32.
 //
-// One launch; the CTAs of a (kv group g, problem) form a thread block
-// cluster (16 CTAs, or 8 where 16 cannot be scheduled), 256 threads each:
+// One launch; the kAttCluster CTAs of a (kv group g, problem) form a thread
+// block cluster, 256 threads each:
 //   1. CTA rank c takes an equal share of the selected rows and walks it in
 //      chunks of 128 rows (64 for fp32 storage): cp.async the chunk's C_K / C_V rows, logits of the G
 //      heads of group g, online softmax (running max, sum) and the latent
@@ -31,7 +31,7 @@
 namespace s4r {
 
 constexpr int kAttThreads = 256;      // 8 warps
-constexpr int kAttCluster = 16;       // most CTAs per (kv group, problem); the launch may use 8
+constexpr int kAttCluster = 8;        // CTAs per (kv group, problem)
 constexpr int kAttEntriesMax = 128;   // selected rows per chunk (bf16 storage; 64 for fp32)
 template <typename T> __host__ __device__ constexpr int att_entries() { return sizeof(T) == 2 ? 128 : 64; }
 constexpr int kAttMaxGroup = 8;       // G <= 8

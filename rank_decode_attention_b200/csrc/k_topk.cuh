@@ -39,7 +39,8 @@ __global__ void pool_kernel(Shape s, const int32_t *__restrict__ lengths,
   }
 }
 
-// Inclusive block scan of one value per thread (kTopkThreads threads).
+// Exclusive block scan of one value per thread (any multiple of 32 threads,
+// at most 1024); *total receives the block total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_tot, uint32_t *total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint32_t x = v;
@@ -51,7 +52,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_t
   if (lane == 31) warp_tot[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    uint32_t t = warp_tot[lane];
+    uint32_t t = (lane < (int)(blockDim.x >> 5)) ? warp_tot[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
@@ -371,7 +372,8 @@ constexpr int kTopkClThreads = 512;
 constexpr int kTopkClWarps = kTopkClThreads / 32;
 constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
 constexpr int kTopkClSeg = 256;                  // candidates per warp
-constexpr int kTopkClCand = 8192;                // candidates rank 0 gathers at most
+constexpr int kTopkClPerRank = 2048;             // candidate slots per rank in rank 0's buffer
+constexpr int kTopkClCand = kTopkCl * kTopkClPerRank;
 __host__ inline size_t topk_cl_smem_bytes() {
   return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1 + kTopkClWarps * kTopkClSeg + kTopkClCand);
 }
@@ -386,6 +388,7 @@ struct TopkClShared {
   uint32_t warp_tot[32];
   uint32_t total, digit, above, t_hi, t_lo, cmin, cmax;
   uint32_t n_above, n_cand;          // this rank's totals (read by rank 0)
+  uint32_t warp_off[kTopkClWarps];   // this rank's candidate offset per warp
   uint32_t tau, take_eq, ok;         // rank 0's result (read by all ranks)
   uint32_t n_gt, n_eq;               // this rank's compaction counts (read by all ranks)
 };
@@ -560,10 +563,20 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
     uint32_t na = 0, ncd = 0;
     for (int w = 0; w < kTopkClWarps; ++w) {
       na += sh.seg_above[w];
+      sh.warp_off[w] = ncd;
       ncd += (sh.seg_count[w] > (uint32_t)kTopkClSeg) ? 0x40000000u : sh.seg_count[w];  // overflow poisons
     }
     sh.n_above = na;
     sh.n_cand = ncd;
+  }
+  __syncthreads();
+  // Push this rank's candidates into its slots of rank 0's buffer (remote
+  // stores, made visible by the cluster barrier below).
+  if (sh.n_cand <= (uint32_t)kTopkClPerRank) {
+    const uint32_t n_w = min(sh.seg_count[wid], (uint32_t)kTopkClSeg);
+    const uint32_t base = cluster_map(gath + rank * kTopkClPerRank + sh.warp_off[wid], 0u);
+    for (uint32_t e = lane; e < n_w; e += 32)
+      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(base + 4 * e), "r"(mine[e]) : "memory");
   }
   cluster_sync();
   if (rank == 0) {
@@ -574,32 +587,22 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       lo = min(lo, remote_u32(&sh.cmin, c));
       hi = max(hi, remote_u32(&sh.cmax, c));
     }
-    const bool bracket_ok = n_cand < (uint32_t)kTopkClCand && n_above < (uint32_t)need &&
-                            (uint32_t)need <= n_above + n_cand;
+    __shared__ uint32_t rank_cand[kTopkCl];
+    bool per_rank_ok = true;
+    if (threadIdx.x == 0)
+      for (int c = 0; c < kTopkCl; ++c) rank_cand[c] = remote_u32(&sh.n_cand, (uint32_t)c);
+    __syncthreads();
+    for (int c = 0; c < kTopkCl; ++c) per_rank_ok &= rank_cand[c] <= (uint32_t)kTopkClPerRank;
+    const bool bracket_ok = per_rank_ok && n_above < (uint32_t)need && (uint32_t)need <= n_above + n_cand;
     uint32_t tau = 0, take_eq = 0;
     if (bracket_ok) {
-      // Gather the candidates (rank-major, warp segments dense) into rank 0.
-      __shared__ uint32_t seg_off[kTopkCl * kTopkClWarps + 1];
-      if (threadIdx.x < kTopkCl * kTopkClWarps)   // all remote counts in one parallel round
-        seg_off[threadIdx.x + 1] = remote_u32(&sh.seg_count[threadIdx.x % kTopkClWarps],
-                                              (uint32_t)(threadIdx.x / kTopkClWarps));
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        seg_off[0] = 0;
-        for (int i = 1; i <= kTopkCl * kTopkClWarps; ++i) seg_off[i] += seg_off[i - 1];
-      }
-      __syncthreads();
-      for (int sgi = wid; sgi < kTopkCl * kTopkClWarps; sgi += kTopkClWarps) {
-        const int c = sgi / kTopkClWarps, w = sgi - c * kTopkClWarps;
-        const uint32_t o = seg_off[sgi], n = seg_off[sgi + 1] - o;
-        for (uint32_t e = lane; e < n; e += 32) gath[o + e] = remote_u32(seg + w * kTopkClSeg + e, (uint32_t)c);
-      }
-      __syncthreads();
+      // Candidates sit in fixed per-rank slots of gath.
       auto value = [&](int i, bool &ok) -> uint32_t {
-        ok = true;
-        return gath[i];
+        const int c = i / kTopkClPerRank, e = i - c * kTopkClPerRank;
+        ok = e < (int)rank_cand[c];
+        return ok ? gath[i] : 0u;
       };
-      cl_radix_select(value, (int)n_cand, (uint32_t)need - n_above, lo, hi, sh, &tau, &take_eq);
+      cl_radix_select(value, kTopkClCand, (uint32_t)need - n_above, lo, hi, sh, &tau, &take_eq);
     } else {
       // Exact select over every key of every rank (read remotely).
       auto value = [&](int i, bool &ok) -> uint32_t {

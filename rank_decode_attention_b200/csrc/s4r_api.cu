@@ -303,31 +303,18 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   {
     const size_t smem = att_smem_bytes(s, sizeof(T));
     cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)kAttCluster, (unsigned)s.n_heads_kv, (unsigned)s.batch);
     cfg.blockDim = dim3(kAttThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)kAttCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // 16 CTAs per cluster when the GPU can place such clusters, else 8.
-    int n_ranks = 8;
-    for (int cand : {kAttCluster, 8}) {
-      cfg.gridDim = dim3((unsigned)cand, (unsigned)s.n_heads_kv, (unsigned)s.batch);
-      attr[0].val.clusterDim.x = (unsigned)cand;
-      int n_clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&n_clusters, attend_kernel<T>, &cfg) == cudaSuccess && n_clusters > 0) {
-        n_ranks = cand;
-        break;
-      }
-      cudaGetLastError();
-    }
-    cfg.gridDim = dim3((unsigned)n_ranks, (unsigned)s.n_heads_kv, (unsigned)s.batch);
-    attr[0].val.clusterDim.x = (unsigned)n_ranks;
     const cudaError_t err = cudaLaunchKernelEx(&cfg, attend_kernel<T>, s, a->lengths, a->idx, ck, cv, qt, q, bv, sk,
                                                sv, a->out);
     if (err != cudaSuccess) return fail("attend_kernel (cluster launch)", err);
