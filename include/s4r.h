@@ -167,6 +167,31 @@ s4r_status s4r_workspace_init(void *workspace, size_t workspace_bytes, void *str
  * Arithmetic is fp32 whatever the storage type. */
 s4r_status s4r_decode_step(const s4r_decode_args *args, void *stream);
 
+/* ------------------------------------------------- decode without alloc */
+
+/* Library extension: the S4R paper has no counterpart to this entry point.
+ *
+ * The same decode step as s4r_decode_step, for callers that cannot allocate
+ * or own device memory for a workspace (a host program that manages no
+ * device memory, or an engine that has handed all free HBM to its cache pool
+ * and may not allocate while serving).  Instead of args->workspace (ignored,
+ * may be NULL) it uses a scratch array of S4R_NOALLOC_SCRATCH_BYTES compiled
+ * into the library, one per device.  It allocates nothing.
+ *   - Shapes whose s4r_decode_workspace_bytes exceeds
+ *     S4R_NOALLOC_SCRATCH_BYTES are rejected with S4R_ERR_UNSUPPORTED before
+ *     anything is enqueued; s4r_last_error names both sizes.
+ *   - The first call on a device (current device at call time) looks up the
+ *     array and zeroes it synchronously; make that first call before any
+ *     stream capture or other work that must not be synchronised.
+ *   - Every call on a device shares the one array.  Calls that may overlap
+ *     in time (other streams or host threads) race on it and give wrong
+ *     results; order them on one stream or synchronise between them.
+ *   - Device-side conditions (a bounded wait that gave up, a bad length) go
+ *     to the library-wide status of the device: read them with
+ *     s4r_read_device_status(NULL, stream). */
+#define S4R_NOALLOC_SCRATCH_BYTES (4u << 20)
+s4r_status s4r_decode_step_noalloc(const s4r_decode_args *args, void *stream);
+
 /* ----------------------------------------------------------- reconstruct */
 
 /* Rebuild selected rows from coefficients, out[e][d] = sum_j coeffs[rows[e]][j]

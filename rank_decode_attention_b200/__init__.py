@@ -72,6 +72,7 @@ SIGNATURES = {
     "s4r_decode_kernel_launches": (_i32, [ctypes.POINTER(DecodeArgs)]),
     "s4r_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "s4r_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeArgs), _vp]),
+    "s4r_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(DecodeArgs), _vp]),
     "s4r_reconstruct": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i32, _vp, _i64, _vp, ctypes.c_int, _vp]),
     "s4r_read_device_status": (ctypes.c_int, [_vp, _vp]),
     "s4r_clear_device_status": (ctypes.c_int, [_vp, _vp]),
@@ -196,6 +197,13 @@ def s4r_workspace_init(workspace: torch.Tensor, stream=None) -> int:
 def s4r_decode_step(args: DecodeArgs, stream=None) -> int:
     """One decode step for every problem (see include/s4r.h)."""
     return _check(lib().s4r_decode_step(ctypes.byref(args), _stream(stream)), "s4r_decode_step")
+
+
+def s4r_decode_step_noalloc(args: DecodeArgs, stream=None) -> int:
+    """The decode step on the library's fixed per-device scratch array (no
+    workspace, nothing allocated; see include/s4r.h for its limits)."""
+    return _check(lib().s4r_decode_step_noalloc(ctypes.byref(args), _stream(stream)),
+                  "s4r_decode_step_noalloc")
 
 
 def s4r_reconstruct(coeffs: torch.Tensor, basis: torch.Tensor, rows: torch.Tensor,

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "k_attend.cuh"
@@ -504,3 +505,83 @@ int32_t s4r_version(void) { return 100; }
 const char *s4r_last_error(void) { return g_last_error; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any allocation.
+//
+// Some callers cannot hand the library a workspace: a host program that
+// manages no device memory of its own, or an engine that has given every free
+// byte of HBM to its cache pool and must not allocate again while serving.
+// For them the decode step can run on a scratch array compiled into the
+// library, one per device.  It holds at most S4R_NOALLOC_SCRATCH_BYTES, so
+// only shapes whose workspace fits are accepted.  Every call on a device
+// shares this one array: two calls that overlap in time (other streams, other
+// host threads) overwrite each other's scratch, so callers must order them.
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[S4R_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Moves a device-side status the call recorded in the scratch array into the
+// library-wide status word of the device, and zeroes the scratch word so the
+// next call starts clean.
+__global__ void noalloc_fold_status(uint32_t *scratch_status) {
+  const uint32_t w = *scratch_status;
+  if (w) atomicOr(&g_device_status, w);
+  *scratch_status = 0u;
+}
+
+// Address of this device's scratch array.  The first call on a device looks
+// the symbol up and zeroes the array (synchronously); later calls only read
+// the cached pointer.
+s4r_status noalloc_scratch(void **out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail("cudaGetDevice", err);
+  if (dev < 0 || dev >= kNoallocMaxDevices) {
+    snprintf(g_last_error, sizeof(g_last_error), "device ordinal %d beyond the no-alloc table", dev);
+    return S4R_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess) return fail("cudaGetSymbolAddress(no-alloc scratch)", err);
+    err = cudaMemset(p, 0, S4R_NOALLOC_SCRATCH_BYTES);
+    if (err == cudaSuccess) err = cudaDeviceSynchronize();
+    if (err != cudaSuccess) return fail("clearing the no-alloc scratch", err);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return S4R_OK;
+}
+
+}  // namespace
+
+extern "C" s4r_status s4r_decode_step_noalloc(const s4r_decode_args *a, void *stream) {
+  Shape s;
+  const s4r_status rc = make_shape(a, &s);
+  if (rc != S4R_OK) return rc;
+  if (s.batch == 0) return S4R_OK;
+  const Layout ly = layout_for(s);
+  if (ly.total > (size_t)S4R_NOALLOC_SCRATCH_BYTES) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "s4r_decode_step_noalloc: these shapes need %zu bytes of scratch, the fixed array holds %zu",
+             ly.total, (size_t)S4R_NOALLOC_SCRATCH_BYTES);
+    return S4R_ERR_UNSUPPORTED;
+  }
+  void *scratch = nullptr;
+  const s4r_status sr = noalloc_scratch(&scratch);
+  if (sr != S4R_OK) return sr;
+  s4r_decode_args local = *a;
+  local.workspace = scratch;
+  local.workspace_bytes = S4R_NOALLOC_SCRATCH_BYTES;
+  const s4r_status dr = s4r_decode_step(&local, stream);
+  if (dr != S4R_OK) return dr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  noalloc_fold_status<<<1, 1, 0, st>>>(reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(scratch) + ly.status));
+  return check_launch("noalloc_fold_status");
+}
