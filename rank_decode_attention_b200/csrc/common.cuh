@@ -83,4 +83,14 @@ __device__ __forceinline__ int64_t n_candidates(int64_t L, int32_t w) {
   return c > 0 ? c : 0;
 }
 
+// Programmatic dependent launch.  The kernels of a decode call are launched
+// so that each may start while its predecessor in the stream drains.
+// pdl_wait blocks until the preceding grid has completed and its writes are
+// visible; a kernel calls it before touching anything that grid (or any
+// earlier work) may still write.  pdl_trigger, called after the wait, lets
+// the next grid start its own prologue.  Both are no-ops for a kernel that
+// was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace s4r

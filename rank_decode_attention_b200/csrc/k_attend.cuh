@@ -14,15 +14,20 @@
 //
 // One launch; the kAttCluster CTAs of a (kv group g, problem) form a thread
 // block cluster, 256 threads each:
-//   1. CTA rank c takes an equal share of the selected rows and walks it in
-//      chunks of 128 rows (64 for fp32 storage): cp.async the chunk's C_K / C_V rows, logits of the G
-//      heads of group g, online softmax (running max, sum) and the latent
-//      value sums acc[j][:] += p[j][e] c_V[e];
-//   2. its partial (m, l, acc) stays in its shared memory; after a cluster
-//      barrier rank 0 reads the other ranks' partials through distributed
-//      shared memory, merges them with the sink logits, maps acc through
-//      B^V[g] and writes out; a second cluster barrier keeps the partials
-//      alive until rank 0 is done.
+//   0. before waiting for the top-k kernel, each CTA starts bulk copies of
+//      the rows of B^V[g] its share of the output needs (an input);
+//   1. CTA rank c takes an equal share of the selected rows, bulk-copies
+//      their C_K / C_V rows into shared memory (all at once when they fit,
+//      else in chunks), computes the logits of the G heads of group g, an
+//      online softmax (running max, sum) and the latent value sums
+//      acc[j][:] += p[j][e] c_V[e]; it also computes the sink logits of the
+//      heads it will finish;
+//   2. its partial (m, l, acc) stays in its shared memory.  After a cluster
+//      barrier every CTA finishes its own slice of the output, (head j,
+//      column e) pairs: it merges the ranks' partials of head j (read through
+//      distributed shared memory) with the sink terms and maps the merged acc
+//      through its staged rows of B^V[g].  A second cluster barrier keeps the
+//      partials alive until every CTA is done.
 #pragma once
 #include "common.cuh"
 #include "k_topk.cuh"
@@ -32,10 +37,10 @@ namespace s4r {
 
 constexpr int kAttThreads = 256;      // 8 warps
 constexpr int kAttCluster = 8;        // CTAs per (kv group, problem)
-constexpr int kAttEntriesMax = 128;   // selected rows per chunk (bf16 storage; 64 for fp32)
-template <typename T> __host__ __device__ constexpr int att_entries() { return sizeof(T) == 2 ? 128 : 64; }
+constexpr int kAttEntriesMax = 256;   // selected rows staged at once per CTA
 constexpr int kAttMaxGroup = 8;       // G <= 8
-constexpr int kAttMaxSinks = 16;      // sinks merged by rank 0
+constexpr int kAttMaxSinks = 16;
+constexpr size_t kAttSmemBudget = 224 * 1024;  // dynamic; leaves room for the static rows and barriers
 
 // Row pitch (elements) of staged rows: 16-byte multiples whose 4-byte-word
 // stride is 4 (mod 8), so the 16-byte reads of 8 consecutive rows fall in
@@ -45,22 +50,61 @@ __host__ __device__ inline int att_pitch(int n, int esize) {
   while (words % 8 != 4) words += 4;
   return words * 4 / esize;
 }
-__host__ __device__ inline size_t att_stage_bytes(const Shape &s, int esize) {
-  const size_t rows = (size_t)(esize == 2 ? 128 : 64) * (att_pitch(s.rank_k, esize) + att_pitch(s.rank_v, esize)) * esize;
-  const size_t bv = (size_t)s.head_dim * att_pitch(s.rank_v, esize) * esize;
-  return rows > bv ? rows : bv;
+
+// Output items of a cluster rank: (head j, column e) pairs t = j*d_h + e in
+// [t0, t1), needing rows e_lo .. e_hi-1 of B^V[g] (all d_h rows if the
+// range spans two heads).
+struct AttItems {
+  int t0, t1, e_lo, e_hi;
+};
+__host__ __device__ inline AttItems att_items(int G, int dh, int n_ranks, int rank) {
+  const int total = G * dh, per = (total + n_ranks - 1) / n_ranks;
+  AttItems it;
+  it.t0 = rank * per < total ? rank * per : total;
+  it.t1 = it.t0 + per < total ? it.t0 + per : total;
+  if (it.t1 <= it.t0) {
+    it.e_lo = it.e_hi = 0;
+  } else if (it.t0 / dh == (it.t1 - 1) / dh) {
+    it.e_lo = it.t0 % dh;
+    it.e_hi = (it.t1 - 1) % dh + 1;
+  } else {
+    it.e_lo = 0;
+    it.e_hi = dh;
+  }
+  return it;
 }
-__host__ __device__ inline size_t att_float_words(const Shape &s) {
+
+// Launch plan: rows staged per pass (a multiple of 32) and B^V rows staged.
+struct AttPlan {
+  int e_cap, bv_rows;
+};
+__host__ __device__ inline size_t att_float_words(const Shape &s, int e_cap, int bv_rows) {
   return (size_t)kAttMaxGroup * s.rank_k          // q_s
-         + (size_t)kAttMaxGroup * kAttEntriesMax  // p_s
-         + (size_t)kAttMaxGroup * 4               // ml_s: m, l, chunk scale, merged inverse
+         + (size_t)kAttMaxGroup * e_cap           // p_s: [entry][kAttMaxGroup]
+         + (size_t)s.n_sink * bv_rows             // sv_s: sink values of this CTA's output columns
+         + (size_t)kAttMaxGroup * 4               // ml_s: m, l, chunk scale
          + (size_t)kAttMaxGroup * (s.rank_v + 2)  // part_s: this CTA's m, l, acc[rv] per head
-         + (size_t)kAttMaxGroup * s.rank_v        // acc_s (rank 0)
-         + (size_t)kAttMaxGroup * kAttMaxSinks    // sw_s
+         + (size_t)kAttMaxGroup * s.rank_v        // acc_s: merged acc of the heads this CTA finishes
+         + (size_t)kAttMaxGroup * kAttMaxSinks    // sw_s: sink logits, then weights
          + (size_t)kAttMaxGroup * kAttCluster;    // f_s: merge weights of the ranks
 }
-__host__ inline size_t att_smem_bytes(const Shape &s, int esize) {
-  return att_stage_bytes(s, esize) + sizeof(float) * att_float_words(s);
+__host__ __device__ inline size_t att_smem_bytes(const Shape &s, int esize, const AttPlan &pl) {
+  const size_t rows = (size_t)pl.e_cap * (att_pitch(s.rank_k, esize) + att_pitch(s.rank_v, esize)) * esize;
+  const size_t bv = (size_t)pl.bv_rows * att_pitch(s.rank_v, esize) * esize;
+  return rows + bv + sizeof(float) * att_float_words(s, pl.e_cap, pl.bv_rows);
+}
+__host__ inline AttPlan att_plan(const Shape &s, int esize) {
+  AttPlan pl;
+  pl.bv_rows = 0;
+  for (int c = 0; c < kAttCluster; ++c) {
+    const AttItems it = att_items(s.group, s.head_dim, kAttCluster, c);
+    pl.bv_rows = it.e_hi - it.e_lo > pl.bv_rows ? it.e_hi - it.e_lo : pl.bv_rows;
+  }
+  const int64_t per = ceil_div((int64_t)s.top_k + s.local_window, kAttCluster);
+  int e = (int)smin<int64_t>(kAttEntriesMax, smax<int64_t>(32, (per + 31) / 32 * 32));
+  pl.e_cap = e;
+  while (pl.e_cap > 32 && att_smem_bytes(s, esize, pl) > kAttSmemBudget) pl.e_cap -= 32;
+  return pl;
 }
 
 // Row number of selected entry e (top-k list first, then the window).
@@ -87,31 +131,75 @@ __device__ __forceinline__ float dot_f32_store(const float *a, const T *x, int n
 
 template <typename T>
 __global__ void __launch_bounds__(kAttThreads)
-attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
+attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
               const T *__restrict__ coeff_k, const T *__restrict__ coeff_v, const float *__restrict__ qt_all,
               const T *__restrict__ q, const T *__restrict__ basis_v, const T *__restrict__ sink_k,
               const T *__restrict__ sink_v, float *__restrict__ out) {
   extern __shared__ __align__(16) unsigned char att_smem[];
   constexpr int V = Vec16<T>::n;
   constexpr int kWarps = kAttThreads / 32;
-  constexpr int kAttEntries = att_entries<T>();
+  const int E = pl.e_cap;
   const int g = blockIdx.y, b = blockIdx.z;
   const uint32_t rank = cluster_ctarank();
   const int n_ranks = (int)gridDim.x;   // the launch makes gridDim.x CTAs one cluster
   const int G = s.group, rk = s.rank_k, rv = s.rank_v, dh = s.head_dim, Dp = s.d_model, ns = s.n_sink;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pk = att_pitch(rk, sizeof(T)), pv = att_pitch(rv, sizeof(T));
   T *ck_s = reinterpret_cast<T *>(att_smem);
-  T *cv_s = ck_s + kAttEntries * pk;
-  float *q_s = reinterpret_cast<float *>(att_smem + att_stage_bytes(s, sizeof(T)));  // [G][rk]
-  float *p_s = q_s + kAttMaxGroup * rk;                     // [G][entries] logits, then weights
-  float *ml_s = p_s + kAttMaxGroup * kAttEntries;           // [G][4]
+  T *cv_s = ck_s + (size_t)E * pk;
+  T *bv_s = cv_s + (size_t)E * pv;
+  float *q_s = reinterpret_cast<float *>(bv_s + (size_t)pl.bv_rows * pv);  // [G][rk]
+  float *p_s = q_s + kAttMaxGroup * rk;                     // [E][kAttMaxGroup] logits, then weights
+  float *sv_s = p_s + kAttMaxGroup * E;                     // [ns][e_hi - e_lo] sink values
+  float *ml_s = sv_s + (size_t)ns * pl.bv_rows;             // [G][4]
   float *part_s = ml_s + kAttMaxGroup * 4;                  // [G][rv + 2]
   float *acc_s = part_s + kAttMaxGroup * (rv + 2);          // [G][rv]
   float *sw_s = acc_s + kAttMaxGroup * rv;                  // [G][kAttMaxSinks]
   float *f_s = sw_s + kAttMaxGroup * kAttMaxSinks;          // [G][kAttCluster]
   __shared__ int64_t rows_s[kAttEntriesMax];
-  __shared__ __align__(8) uint64_t stage_bar;
+  __shared__ __align__(8) uint64_t stage_bar, bv_bar;
+
+  // 0. This CTA's output items and their rows of B^V[g] (inputs: the copies
+  // start before the wait for the top-k kernel).
+  const AttItems it = att_items(G, dh, n_ranks, (int)rank);
+  const T *Bv = basis_v + (int64_t)b * Dp * rv + (int64_t)g * dh * rv;
+  if (threadIdx.x == 0) {
+    mbar_init(&stage_bar, 1);
+    mbar_init(&bv_bar, 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(&bv_bar, (uint32_t)((it.e_hi - it.e_lo) * rv * sizeof(T)));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < it.e_hi - it.e_lo; e += blockDim.x)
+    bulk_load(bv_s + (size_t)e * pv, Bv + (int64_t)(it.e_lo + e) * rv, (uint32_t)(rv * sizeof(T)), &bv_bar);
+  const int j_lo = it.t1 > it.t0 ? it.t0 / dh : 0, j_hi = it.t1 > it.t0 ? (it.t1 - 1) / dh + 1 : 0;
+  // The latent query (written by the projection kernel, which completed
+  // before the top-k kernel started), the sink values of this CTA's output
+  // columns and the sink logits of its heads: none of it depends on the
+  // top-k kernel, so it is prepared while that kernel runs.
+  for (int t = threadIdx.x; t < G * rk; t += blockDim.x) {
+    const int j = t / rk, k = t - j * rk;
+    q_s[j * rk + k] = __ldcg(qt_all + ((int64_t)b * s.n_heads_q + g * G + j) * rk + k);
+  }
+  for (int t = threadIdx.x; t < ns * (it.e_hi - it.e_lo); t += blockDim.x) {
+    const int tk = t / (it.e_hi - it.e_lo), e = t - tk * (it.e_hi - it.e_lo);
+    sv_s[t] = to_f(sink_v[((int64_t)b * ns + tk) * Dp + (int64_t)g * dh + it.e_lo + e]);
+  }
+  {
+    const float qscale = rsqrtf((float)dh);
+    const int nh = j_hi - j_lo;
+    for (int t = wid; t < nh * ns; t += kWarps) {
+      const int j = j_lo + t / ns, tk = t % ns;
+      const T *qh = q + (((int64_t)b * s.query_window + s.query_window - 1) * s.n_heads_q + g * G + j) * dh;
+      const T *kr = sink_k + ((int64_t)b * ns + tk) * Dp + (int64_t)g * dh;
+      float d = 0.f;
+      for (int e = lane; e < dh; e += 32) d = fmaf(to_f(qh[e]), to_f(kr[e]), d);
+      d = warp_sum(d);
+      if (lane == 0) sw_s[j * kAttMaxSinks + tk] = d * qscale;
+    }
+  }
+  pdl_wait();      // idx comes from the preceding kernel
+  pdl_trigger();
 
   const int64_t L = valid_length(lengths[b], s.cache_rows);
   const int64_t n_top = smin<int64_t>(s.top_k, n_candidates(L, s.local_window));
@@ -123,15 +211,6 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   const int32_t *idx_b = idx + (int64_t)b * s.top_k;
   const T *ckb = coeff_k + (int64_t)b * s.cache_rows * rk;
   const T *cvb = coeff_v + (int64_t)b * s.cache_rows * rv;
-
-  for (int t = threadIdx.x; t < G * rk; t += blockDim.x) {
-    const int j = t / rk, k = t - j * rk;
-    q_s[j * rk + k] = qt_all[((int64_t)b * s.n_heads_q + g * G + j) * rk + k];
-  }
-  if (threadIdx.x == 0) {
-    mbar_init(&stage_bar, 1);
-    mbar_fence_init();
-  }
   if (threadIdx.x < G) {
     ml_s[threadIdx.x * 4] = -INFINITY;   // running max
     ml_s[threadIdx.x * 4 + 1] = 0.f;     // running sum
@@ -142,32 +221,29 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
   const int kcol = threadIdx.x;  // latent value column owned by this thread (< rv)
 
   uint32_t phase = 0;
-  for (int64_t c0 = e_begin; c0 < e_end; c0 += kAttEntries) {
-    const int n_e = (int)smin<int64_t>(kAttEntries, e_end - c0);
+  for (int64_t c0 = e_begin; c0 < e_end; c0 += E) {
+    const int n_e = (int)smin<int64_t>(E, e_end - c0);
     __syncthreads();  // previous chunk fully consumed
-    for (int e = threadIdx.x; e < kAttEntries; e += blockDim.x) {
+    int live = 0;     // E <= blockDim.x: at most one entry per thread
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
       int64_t row = -1;
       if (e < n_e) {
         row = att_entry_row(idx_b, n_top, L, n_win, c0 + e, s.n_sink);
         if (row < 0 || row >= L) row = -1;  // never produced by the top-k kernel
       }
       rows_s[e] = row;
+      live = row >= 0;
     }
-    __syncthreads();
     // One bulk copy per row and operand (rows are 16-byte multiples), all
     // completing on stage_bar; skipped rows are zeroed by plain stores.
-    if (threadIdx.x == 0) {
-      uint32_t bytes = 0;
-      for (int e = 0; e < n_e; ++e)
-        if (rows_s[e] >= 0) bytes += (uint32_t)((rk + rv) * sizeof(T));
-      mbar_arrive_expect_tx(&stage_bar, bytes);
-    }
+    const int n_live = __syncthreads_count(live);
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&stage_bar, (uint32_t)(n_live * (rk + rv) * sizeof(T)));
     __syncthreads();
-    if (threadIdx.x < 2 * n_e) {
-      const int e = threadIdx.x % n_e;
-      const bool is_v = threadIdx.x >= n_e;
+    for (int t = threadIdx.x; t < 2 * n_e; t += blockDim.x) {
+      const int e = t % n_e;
+      const bool is_v = t >= n_e;
       const int64_t row = rows_s[e];
-      T *dst = is_v ? cv_s + e * pv : ck_s + e * pk;
+      T *dst = is_v ? cv_s + (size_t)e * pv : ck_s + (size_t)e * pk;
       const int n = is_v ? rv : rk;
       if (row >= 0) {
         bulk_load(dst, is_v ? cvb + row * rv : ckb + row * rk, (uint32_t)(n * sizeof(T)), &stage_bar);
@@ -178,32 +254,59 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
     mbar_wait(&stage_bar, phase, nullptr);
     phase ^= 1u;
     __syncthreads();
-    // logits of (head j, entry e) pairs
-    for (int t = threadIdx.x; t < G * kAttEntries; t += blockDim.x) {
-      const int j = t / kAttEntries, e = t - j * kAttEntries;
-      float l = -INFINITY;
-      if (e < n_e && rows_s[e] >= 0) l = dot_f32_store(q_s + j * rk, ck_s + e * pk, rk);
-      p_s[j * kAttEntries + e] = l;
+    // logits: the thread of entry e computes all G heads, reading its key
+    // row once and the latent queries as broadcast float4s
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      float l0[kAttMaxGroup], l1[kAttMaxGroup];
+#pragma unroll
+      for (int j = 0; j < kAttMaxGroup; ++j) l0[j] = l1[j] = 0.f;
+      const bool ok = e < n_e && rows_s[e] >= 0;
+      if (ok) {
+        const T *kr = ck_s + (size_t)e * pk;
+        for (int k = 0; k < rk; k += V) {
+          float xv[V];
+          load16(kr + k, xv);
+#pragma unroll
+          for (int j = 0; j < kAttMaxGroup; ++j) {
+            if (j < G) {
+#pragma unroll
+              for (int u = 0; u < V; u += 4) {
+                const float4 qv = *reinterpret_cast<const float4 *>(q_s + j * rk + k + u);
+                l0[j] = fmaf(qv.x, xv[u], l0[j]);
+                l1[j] = fmaf(qv.y, xv[u + 1], l1[j]);
+                l0[j] = fmaf(qv.z, xv[u + 2], l0[j]);
+                l1[j] = fmaf(qv.w, xv[u + 3], l1[j]);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kAttMaxGroup; ++j)
+        if (j < G) p_s[e * kAttMaxGroup + j] = ok ? l0[j] + l1[j] : -INFINITY;
     }
     __syncthreads();
-    // online softmax update per head (warp j), kAttEntries / 32 entries per lane
+    // online softmax update per head (warp j), E / 32 entries per lane
     for (int j = wid; j < G; j += kWarps) {
-      constexpr int kPer = kAttEntries / 32;
-      float lv[kPer];
+      constexpr int kPerMax = kAttEntriesMax / 32;
+      const int n_per = E / 32;
+      float lv[kPerMax];
       float mc = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        lv[u] = p_s[j * kAttEntries + lane + 32 * u];
+      for (int u = 0; u < kPerMax; ++u) {
+        lv[u] = u < n_per ? p_s[(lane + 32 * u) * kAttMaxGroup + j] : -INFINITY;
         mc = fmaxf(mc, lv[u]);
       }
       const float m_old = ml_s[j * 4];
       const float m_new = fmaxf(m_old, warp_max(mc));
       float csum = 0.f;
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const float pu = (m_new == -INFINITY) ? 0.f : __expf(lv[u] - m_new);
-        p_s[j * kAttEntries + lane + 32 * u] = pu;
-        csum += pu;
+      for (int u = 0; u < kPerMax; ++u) {
+        if (u < n_per) {
+          const float pu = (m_new == -INFINITY) ? 0.f : __expf(lv[u] - m_new);
+          p_s[(lane + 32 * u) * kAttMaxGroup + j] = pu;
+          csum += pu;
+        }
       }
       csum = warp_sum(csum);
       if (lane == 0) {
@@ -222,14 +325,23 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
         acc[j] *= sc[j];
       }
       for (int e = 0; e < n_e; ++e) {
-        const float v = to_f(cv_s[e * pv + kcol]);
-#pragma unroll
-        for (int j = 0; j < kAttMaxGroup; ++j)
-          if (j < G) acc[j] = fmaf(p_s[j * kAttEntries + e], v, acc[j]);
+        const float v = to_f(cv_s[(size_t)e * pv + kcol]);
+        const float4 pa = *reinterpret_cast<const float4 *>(p_s + e * kAttMaxGroup);
+        acc[0] = fmaf(pa.x, v, acc[0]);
+        acc[1] = fmaf(pa.y, v, acc[1]);
+        acc[2] = fmaf(pa.z, v, acc[2]);
+        acc[3] = fmaf(pa.w, v, acc[3]);
+        if (G > 4) {
+          const float4 pb = *reinterpret_cast<const float4 *>(p_s + e * kAttMaxGroup + 4);
+          acc[4] = fmaf(pb.x, v, acc[4]);
+          acc[5] = fmaf(pb.y, v, acc[5]);
+          acc[6] = fmaf(pb.z, v, acc[6]);
+          acc[7] = fmaf(pb.w, v, acc[7]);
+        }
       }
     }
   }
-  // This CTA's partial, kept in shared memory for rank 0.
+  // This CTA's partial, kept in shared memory for the other ranks.
   if (kcol < rv)
 #pragma unroll
     for (int j = 0; j < kAttMaxGroup; ++j)
@@ -239,76 +351,53 @@ attend_kernel(Shape s, const int32_t *__restrict__ lengths, const int32_t *__res
     part_s[threadIdx.x * (rv + 2)] = ml_s[threadIdx.x * 4];
     part_s[threadIdx.x * (rv + 2) + 1] = ml_s[threadIdx.x * 4 + 1];
   }
-  T *bv_s = ck_s;
-  const T *Bv = basis_v + (int64_t)b * Dp * rv + (int64_t)g * dh * rv;
-  if (rank == 0) {
-    // Stage B^V[g] (d_h rows x rv) over the row buffers while the cluster syncs.
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(&stage_bar, (uint32_t)(dh * rv * sizeof(T)));
-    __syncthreads();
-    for (int e = threadIdx.x; e < dh; e += blockDim.x)
-      bulk_load(bv_s + e * pv, Bv + (int64_t)e * rv, (uint32_t)(rv * sizeof(T)), &stage_bar);
-  }
   cluster_sync();  // every partial is in place
-  if (rank == 0) {
-    // Sink logits: one warp per (head, sink).
-    const float qscale = rsqrtf((float)dh);
-    for (int t = wid; t < G * ns; t += kWarps) {
-      const int j = t / ns, tk = t - j * ns;
-      const T *qh = q + (((int64_t)b * s.query_window + s.query_window - 1) * s.n_heads_q + g * G + j) * dh;
-      const T *kr = sink_k + ((int64_t)b * ns + tk) * Dp + (int64_t)g * dh;
-      float d = 0.f;
-      for (int e = lane; e < dh; e += 32) d = fmaf(to_f(qh[e]), to_f(kr[e]), d);
-      d = warp_sum(d);
-      if (lane == 0) sw_s[j * kAttMaxSinks + tk] = d * qscale;
+  // Merge weights of the heads this CTA finishes (warp per head; ranks = lanes).
+  for (int j = j_lo + wid; j < j_hi; j += kWarps) {
+    float mr = -INFINITY, lr = 0.f;
+    if (lane < n_ranks) {
+      const uint32_t base = cluster_map(part_s + j * (rv + 2), (uint32_t)lane);
+      mr = ld_cluster_f32(base);
+      lr = ld_cluster_f32(base + 4);
     }
-    __syncthreads();
-    // Merge weights per head (warp j): ranks r = lanes 0 .. n_ranks-1.
-    for (int j = wid; j < G; j += kWarps) {
-      float mr = -INFINITY, lr = 0.f;
-      if (lane < n_ranks) {
-        const uint32_t base = cluster_map(part_s + j * (rv + 2), (uint32_t)lane);
-        mr = ld_cluster_f32(base);
-        lr = ld_cluster_f32(base + 4);
-      }
-      float M = mr;
-      for (int tk = lane; tk < ns; tk += 32) M = fmaxf(M, sw_s[j * kAttMaxSinks + tk]);
-      M = warp_max(M);
-      const float fr = (mr == -INFINITY) ? 0.f : __expf(mr - M);
-      float den = lr * fr;
-      for (int tk = lane; tk < ns; tk += 32) den += __expf(sw_s[j * kAttMaxSinks + tk] - M);
-      den = warp_sum(den);
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-      if (lane < n_ranks) f_s[j * kAttCluster + lane] = fr * inv;
-      __syncwarp();
-      for (int tk = lane; tk < ns; tk += 32)
-        sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
-    }
-    __syncthreads();
-    // acc[j][k] = sum_r f[j][r] acc_r[j][k], read through distributed shared memory.
-    for (int t = threadIdx.x; t < G * rv; t += blockDim.x) {
-      const int j = t / rv, k = t - j * rv;
-      float v[kAttCluster];
-#pragma unroll
-      for (int r = 0; r < kAttCluster; ++r)
-        v[r] = (r < n_ranks) ? ld_cluster_f32(cluster_map(part_s + j * (rv + 2) + 2 + k, (uint32_t)r)) : 0.f;
-      float a = 0.f;
-#pragma unroll
-      for (int r = 0; r < kAttCluster; ++r)
-        if (r < n_ranks) a = fmaf(f_s[j * kAttCluster + r], v[r], a);
-      acc_s[t] = a;
-    }
-    mbar_wait(&stage_bar, phase, nullptr);
-    __syncthreads();
-    // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e].
-    for (int t = threadIdx.x; t < G * dh; t += blockDim.x) {
-      const int j = t / dh, e = t - j * dh;
-      float o = dot_f32_store(acc_s + j * rv, bv_s + e * pv, rv);
-      for (int tk = 0; tk < ns; ++tk)
-        o = fmaf(sw_s[j * kAttMaxSinks + tk], to_f(sink_v[((int64_t)b * ns + tk) * Dp + (int64_t)g * dh + e]), o);
-      out[((int64_t)b * s.n_heads_q + g * G + j) * dh + e] = o;
-    }
+    float M = mr;
+    for (int tk = lane; tk < ns; tk += 32) M = fmaxf(M, sw_s[j * kAttMaxSinks + tk]);
+    M = warp_max(M);
+    const float fr = (mr == -INFINITY) ? 0.f : __expf(mr - M);
+    float den = lr * fr;
+    for (int tk = lane; tk < ns; tk += 32) den += __expf(sw_s[j * kAttMaxSinks + tk] - M);
+    den = warp_sum(den);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    if (lane < n_ranks) f_s[j * kAttCluster + lane] = fr * inv;
+    __syncwarp();
+    for (int tk = lane; tk < ns; tk += 32)
+      sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
   }
-  cluster_sync();  // rank 0 has read every partial
+  __syncthreads();
+  // acc[j][k] = sum_r f[j][r] acc_r[j][k], read through distributed shared memory.
+  for (int t = threadIdx.x; t < (j_hi - j_lo) * rv; t += blockDim.x) {
+    const int j = j_lo + t / rv, k = t % rv;
+    float v[kAttCluster];
+#pragma unroll
+    for (int r = 0; r < kAttCluster; ++r)
+      v[r] = (r < n_ranks) ? ld_cluster_f32(cluster_map(part_s + j * (rv + 2) + 2 + k, (uint32_t)r)) : 0.f;
+    float a = 0.f;
+#pragma unroll
+    for (int r = 0; r < kAttCluster; ++r)
+      if (r < n_ranks) a = fmaf(f_s[j * kAttCluster + r], v[r], a);
+    acc_s[j * rv + k] = a;
+  }
+  mbar_wait(&bv_bar, 0, nullptr);
+  __syncthreads();
+  // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e].
+  for (int t = it.t0 + (int)threadIdx.x; t < it.t1; t += blockDim.x) {
+    const int j = t / dh, e = t - j * dh;
+    float o = dot_f32_store(acc_s + j * rv, bv_s + (size_t)(e - it.e_lo) * pv, rv);
+    for (int tk = 0; tk < ns; ++tk)
+      o = fmaf(sw_s[j * kAttMaxSinks + tk], sv_s[tk * (it.e_hi - it.e_lo) + (e - it.e_lo)], o);
+    out[((int64_t)b * s.n_heads_q + g * G + j) * dh + e] = o;
+  }
+  cluster_sync();  // every CTA has read the partials it needs
 }
 
 // Rebuild rows explicitly: out[e][d] = sum_j C[rows[e]][j] B[d][j] (fp32).

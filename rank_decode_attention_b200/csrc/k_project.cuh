@@ -63,6 +63,8 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   __shared__ __align__(16) T qraw[kProjRowBlock][128];                  // per-head query rows, 128 of d_h
   __shared__ __align__(16) T braw[128][kProjColBlock + 16 / sizeof(T)];  // basis slice (padded rows)
   constexpr int V = Vec16<T>::n;
+  pdl_wait();      // the previous call's kernels may still read this workspace
+  pdl_trigger();
   const int rank = (int)blockIdx.x, n_rank = (int)gridDim.x, cb = blockIdx.y;
   const int n_rb = (int)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
   const int rb = blockIdx.z % n_rb, b = blockIdx.z / n_rb;

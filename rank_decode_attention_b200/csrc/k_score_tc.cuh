@@ -105,12 +105,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       mbar_init(&ctl->mma_done[t], 1);
     }
     mbar_fence_init();
-    // The split query operand, already in its shared-memory image.
-    mbar_arrive_expect_tx(&ctl->b_full, (uint32_t)stc_b_bytes(R, r));
-    const unsigned char *src = cqs + (int64_t)b * stc_b_bytes(R, r);
-    for (int kb = 0; kb < nkb; ++kb)
-      bulk_load(b_op + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128, &ctl->b_full);
-    // A: stream this CTA's coefficient tiles, one barrier per K-block.
+    // A: stream this CTA's coefficient tiles, one barrier per K-block.  No
+    // kernel of a decode call writes the cache, so these copies start before
+    // the wait for the projection kernel.
     for (int t = 0; t < n_tiles; ++t) {
       const int32_t row = (int32_t)((int64_t)b * s.cache_rows + (tile0 + t) * kStcTile);
       for (int kb = 0; kb < nkb; ++kb) {
@@ -120,6 +117,17 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     }
   }
   if (warp == 0) tmem_alloc(&ctl->tmem_base, kStcTmemCols);
+  // Everything below may read what the projection kernel wrote (the split
+  // query operand, the zeroed row sums and barrier words).
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 128) {
+    // The split query operand, already in its shared-memory image.
+    mbar_arrive_expect_tx(&ctl->b_full, (uint32_t)stc_b_bytes(R, r));
+    const unsigned char *src = cqs + (int64_t)b * stc_b_bytes(R, r);
+    for (int kb = 0; kb < nkb; ++kb)
+      bulk_load(b_op + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128, &ctl->b_full);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -304,6 +304,8 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
             int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) uint32_t topk_dyn[];
   __shared__ TopkShared sh;
+  pdl_wait();      // scores come from the preceding kernel
+  pdl_trigger();
   const int b = blockIdx.x;
   const int64_t Lraw = lengths[b];
   if (threadIdx.x == 0 && (Lraw < 0 || Lraw > s.cache_rows)) set_status(status, kDevStatusCheck);
@@ -478,6 +480,8 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   uint32_t *keys_s = tcl_dyn;                                   // this rank's keys (padded)
   uint32_t *seg = tcl_dyn + kpad(kTopkClKeys) + 1;              // per-warp candidate segments
   uint32_t *gath = seg + kTopkClWarps * kTopkClSeg;             // rank 0: all candidates
+  pdl_wait();      // scores come from the preceding kernel
+  pdl_trigger();
   const uint32_t rank = cluster_ctarank();
   const int b = blockIdx.y;
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;

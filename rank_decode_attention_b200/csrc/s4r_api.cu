@@ -96,7 +96,10 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
   s->group = (int32_t)G;
   s->n_rows = (int32_t)R;
   s->cache_rows = a->cache_rows;
-  if (att_smem_bytes(*s, a->dtype == S4R_BF16 ? 2 : 4) > 232448) return S4R_ERR_UNSUPPORTED;
+  {
+    const int es = a->dtype == S4R_BF16 ? 2 : 4;
+    if (att_smem_bytes(*s, es, att_plan(*s, es)) > kAttSmemBudget) return S4R_ERR_UNSUPPORTED;
+  }
   return S4R_OK;
 }
 
@@ -113,6 +116,20 @@ s4r_status check_launch(const char *what) {
   return err == cudaSuccess ? S4R_OK : fail(what, err);
 }
 s4r_status last_cuda() { return check_launch("kernel launch"); }
+
+// Launch attribute that lets a kernel start while the previous kernel in the
+// stream drains (its CTAs wait in pdl_wait before reading that kernel's
+// output).  Every decode kernel launched with it calls pdl_wait first.
+inline cudaLaunchAttribute pdl_attr() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+// Whether the cooperative scoring launch accepts the attribute above
+// (-1 not tried yet, 0 no, 1 yes).
+int g_coop_pdl = -1;
 
 // cuTensorMapEncodeTiled, resolved through the runtime (no link-time libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -207,12 +224,25 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
   cfg.blockDim = dim3(kStcThreads);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1] = pdl_attr();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status);
+  cfg.numAttrs = g_coop_pdl == 0 ? 1 : 2;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status);
+  if (cfg.numAttrs == 2 && g_coop_pdl < 0) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cap);
+    if (err == cudaSuccess) {
+      g_coop_pdl = 1;
+    } else if (cap == cudaStreamCaptureStatusNone) {
+      cudaGetLastError();   // not supported together: launch without it from now on
+      g_coop_pdl = 0;
+      cfg.numAttrs = 1;
+      err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status);
+    }
+  }
   return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (cooperative launch)", err);
 }
 
@@ -245,13 +275,14 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     cfg.gridDim = dim3(n_rank, (unsigned)ceil_div(s.rank_k, kProjColBlock), n_rb * (unsigned)s.batch);
     cfg.blockDim = dim3(kProjThreads);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = n_rank;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const cudaError_t err = cudaLaunchKernelEx(&cfg, project_kernel<T>, s, q, bk, cq, cqs, qt, rowsum, bar);
     if (err != cudaSuccess) return fail("project_kernel (cluster launch)", err);
     if (check_launch("project_kernel") != S4R_OK) return S4R_ERR_CUDA;
@@ -292,31 +323,51 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     if (s.cache_rows <= (int64_t)kTopkCl * kTopkClKeys) {
       const size_t smem = topk_cl_smem_bytes();
       cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      topk_cluster_kernel<<<dim3(kTopkCl, s.batch), kTopkClThreads, smem, st>>>(s, a->lengths, keys, a->idx, status);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kTopkCl, (unsigned)s.batch);
+      cfg.blockDim = dim3(kTopkClThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1] = {pdl_attr()};
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t err = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, s, a->lengths, keys, a->idx, status);
+      if (err != cudaSuccess) return fail("topk_cluster_kernel (cluster launch)", err);
     } else {
       const size_t smem = topk_smem_bytes(s.cache_rows);
       cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      topk_kernel<<<s.batch, kTopkThreads, smem, st>>>(s, a->lengths, keys, a->idx, status);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)s.batch);
+      cfg.blockDim = dim3(kTopkThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1] = {pdl_attr()};
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t err = cudaLaunchKernelEx(&cfg, topk_kernel, s, a->lengths, keys, a->idx, status);
+      if (err != cudaSuccess) return fail("topk_kernel", err);
     }
     if (check_launch("topk_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
   // 4. rebuild + exact attention (one cluster of CTAs per kv group)
   {
-    const size_t smem = att_smem_bytes(s, sizeof(T));
+    const AttPlan pl = att_plan(s, (int)sizeof(T));
+    const size_t smem = att_smem_bytes(s, (int)sizeof(T), pl);
     cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)kAttCluster, (unsigned)s.n_heads_kv, (unsigned)s.batch);
     cfg.blockDim = dim3(kAttThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)kAttCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t err = cudaLaunchKernelEx(&cfg, attend_kernel<T>, s, a->lengths, a->idx, ck, cv, qt, q, bv, sk,
+    cfg.numAttrs = 2;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, attend_kernel<T>, s, pl, a->lengths, a->idx, ck, cv, qt, q, bv, sk,
                                                sv, a->out);
     if (err != cudaSuccess) return fail("attend_kernel (cluster launch)", err);
     if (check_launch("attend_kernel") != S4R_OK) return S4R_ERR_CUDA;
