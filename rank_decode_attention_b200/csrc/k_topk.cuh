@@ -361,99 +361,73 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
 }
 
 // ---------------------------------------------------------------------------
-// Cluster variant: the kTopkCl CTAs of a cluster split one problem's keys.
-// Each CTA stages its contiguous share in shared memory and contributes 32
-// sampled keys; every CTA ranks the 256 samples (read through distributed
-// shared memory) the same way, collects its in-bracket keys, and rank 0
-// radix-selects the exact threshold among all ranks' candidates.  A cluster
-// prefix of the per-rank counts then gives each rank its output offset for
-// the stable compaction.  Falls back to rank 0 selecting over every key
-// (read through distributed shared memory) if the bracket misses.
+// Cluster variant: the kTopkCl CTAs of a cluster split one problem's
+// candidates into contiguous shares held in shared memory.  The threshold
+// key tau is found by a radix select on the float bit patterns, one 8-bit
+// digit per pass from the exponent down:
+//   * every rank histograms its keys that match the digits chosen so far and
+//     stores the histogram into every rank (distributed shared memory); after
+//     a cluster barrier each rank sums the ranks' histograms and takes the
+//     same decision: the digit of tau, and every rank's keys in higher bins
+//     (which are > tau);
+//   * once the chosen bin holds at most kTopkGather keys, the ranks store
+//     those keys into every rank instead (rank by rank, so each key's rank is
+//     known from its position) and each rank resolves tau among them alone;
+//   * a bin that is taken whole ends the search (tau = its lower bound - 1).
+// Every rank then knows every rank's counts of keys > tau and == tau, hence
+// its own output offset; a stable compaction in index order writes the
+// rank's keys > tau and its share of the keys == tau (lower positions first).
 constexpr int kTopkCl = 8;                       // CTAs per problem
 constexpr int kTopkClThreads = 512;
 constexpr int kTopkClWarps = kTopkClThreads / 32;
 constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
-constexpr int kTopkClSeg = 256;                  // candidates per warp
-constexpr int kTopkClPerRank = 2048;             // candidate slots per rank in rank 0's buffer
-constexpr int kTopkClCand = kTopkCl * kTopkClPerRank;
-__host__ inline size_t topk_cl_smem_bytes() {
-  return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1 + kTopkClWarps * kTopkClSeg + kTopkClCand);
-}
+constexpr int kTopkGather = 1024;                // keys of the final bin gathered into every rank
+__host__ inline size_t topk_cl_smem_bytes() { return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1); }
 
 struct TopkClShared {
-  uint32_t whist[kTopkClWarps][kTopkBins];
-  uint32_t hist[kTopkBins];
-  uint32_t sample[32];               // this rank's samples (read by all ranks)
-  uint32_t all_sample[kTopkSample];
-  uint32_t seg_count[kTopkClWarps];
-  uint32_t seg_above[kTopkClWarps];
+  uint32_t hist[kTopkBins];                 // summed histogram of the current pass
+  uint32_t lhist[4][kTopkBins];             // this rank's histogram (warp w adds into copy w % 4)
+  uint32_t g_hist[2][kTopkCl][kTopkBins];   // every rank's histogram (stored by that rank), two passes in flight
+  uint32_t gbuf[kTopkGather];               // gathered keys of the final bin, rank segments in rank order
+  uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau so far / in the chosen bin
   uint32_t warp_tot[32];
-  uint32_t total, digit, above, t_hi, t_lo, cmin, cmax;
-  uint32_t n_above, n_cand;          // this rank's totals (read by rank 0)
-  uint32_t warp_off[kTopkClWarps];   // this rank's candidate offset per warp
-  uint32_t tau, take_eq, ok;         // rank 0's result (read by all ranks)
-  uint32_t n_gt, n_eq;               // this rank's compaction counts (read by all ranks)
+  uint32_t total, digit, above, gcount;
+  // The threshold, how many keys equal to it are taken overall, and this
+  // rank's output offset and equal keys before it.
+  uint32_t tau, take_eq, out_before, eq_before;
 };
 
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-template <typename Tp>
-__device__ __forceinline__ uint32_t remote_u32(const Tp *p, uint32_t rank) {
-  return ld_cluster_u32(cluster_map(p, rank));
+// Warp 0: the digit (from the top) whose bin holds the remaining-th largest
+// key of sh.hist, and how many keys lie in higher bins.
+__device__ __forceinline__ void cl_pick_digit(TopkClShared &sh, uint32_t remaining) {
+  const int lane = threadIdx.x & 31;
+  uint32_t cnt[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t run = incl - sum;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (run < remaining && run + cnt[j] >= remaining) {
+      sh.digit = 255u - (uint32_t)(lane * 8 + j);
+      sh.above = run;
+    }
+    run += cnt[j];
+  }
 }
 
-// Block-wide radix pass / select for blockDim-sized CTAs of the cluster kernel.
+// Block-wide radix select over n values of this CTA (value(i)): tau is the
+// need-th largest and take_eq how many keys equal to it are among the need
+// largest.  lo_all / hi_all bound the values (their common bits are skipped).
 template <typename ValueFn>
-__device__ __forceinline__ void cl_radix_pass(ValueFn value, int n_slots, int shift, uint32_t mask, uint32_t &prefix,
-                                              uint32_t &remaining, TopkClShared &sh) {
-  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int j = 0; j < kTopkBins / 32; ++j) sh.whist[wid][lane + 32 * j] = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < n_slots; i += blockDim.x) {
-    bool ok;
-    const uint32_t v = value(i, ok);
-    if (ok && (v & mask) == prefix) atomicAdd(&sh.whist[wid][(v >> shift) & 255u], 1u);
-  }
-  __syncthreads();
-  if (threadIdx.x < kTopkBins) {
-    uint32_t c = 0;
-#pragma unroll
-    for (int w = 0; w < kTopkClWarps; ++w) c += sh.whist[w][threadIdx.x];
-    sh.hist[threadIdx.x] = c;
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    uint32_t cnt[8], sum = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    uint32_t run = incl - sum;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (run < remaining && run + cnt[j] >= remaining) {
-        sh.digit = 255u - (uint32_t)(lane * 8 + j);
-        sh.above = run;
-      }
-      run += cnt[j];
-    }
-  }
-  __syncthreads();
-  remaining -= sh.above;
-  prefix |= sh.digit << shift;
-  __syncthreads();
-}
-template <typename ValueFn>
-__device__ __forceinline__ void cl_radix_select(ValueFn value, int n_slots, uint32_t need, uint32_t lo_all,
+__device__ __forceinline__ void cl_radix_select(ValueFn value, int n, uint32_t need, uint32_t lo_all,
                                                 uint32_t hi_all, TopkClShared &sh, uint32_t *tau, uint32_t *take_eq) {
+  const int lane = threadIdx.x & 31;
   const uint32_t diff = lo_all ^ hi_all;
   int top = 31;
   while (top >= 0 && !((diff >> top) & 1u)) --top;
@@ -465,21 +439,33 @@ __device__ __forceinline__ void cl_radix_select(ValueFn value, int n_slots, uint
   }
   if (top >= 0)
     for (int shift = (top / 8) * 8; shift >= 0; shift -= 8) {
-      cl_radix_pass(value, n_slots, shift, mask, prefix, remaining, sh);
+      for (int j = threadIdx.x; j < kTopkBins; j += blockDim.x) sh.hist[j] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t v = value(i);
+        const bool in = (v & mask) == prefix;
+        const uint32_t bin = in ? (v >> shift) & 255u : 0xffffffffu;
+        const uint32_t peers = __match_any_sync(__activemask(), bin);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
+      __syncthreads();
+      remaining -= sh.above;
+      prefix |= sh.digit << shift;
       mask |= 255u << shift;
+      __syncthreads();   // digit / above are rewritten by the next pass
     }
   *tau = prefix;
   *take_eq = remaining;
 }
 
-__global__ void __cluster_dims__(kTopkCl, 1, 1) __launch_bounds__(kTopkClThreads)
+__global__ void __cluster_dims__(kTopkCl, 1, 1) __launch_bounds__(kTopkClThreads, 1)
 topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restrict__ keys_all,
                     int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) uint32_t tcl_dyn[];
   __shared__ TopkClShared sh;
   uint32_t *keys_s = tcl_dyn;                                   // this rank's keys (padded)
-  uint32_t *seg = tcl_dyn + kpad(kTopkClKeys) + 1;              // per-warp candidate segments
-  uint32_t *gath = seg + kTopkClWarps * kTopkClSeg;             // rank 0: all candidates
   pdl_wait();      // scores come from the preceding kernel
   pdl_trigger();
   const uint32_t rank = cluster_ctarank();
@@ -503,127 +489,165 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   const int chunk = (nc + kTopkCl - 1) / kTopkCl;
   const int i_begin = min(nc, (int)rank * chunk), i_end = min(nc, i_begin + chunk);
   const int my_n = i_end - i_begin;
-  for (int i = threadIdx.x; i < my_n; i += blockDim.x) keys_s[kpad(i)] = __ldcg(gkeys + i_begin + i);
+  // Asynchronous 4-byte copies: every load of the share is in flight at once.
+  for (int i = threadIdx.x; i < my_n; i += blockDim.x)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(keys_s + kpad(i))),
+                 "l"(gkeys + i_begin + i)
+                 : "memory");
+  for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
+  if (threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) sh.gcount = 0u;
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  // 32 samples of this rank's share, then all 256 (same order on every rank).
-  if (threadIdx.x < 32)
-    sh.sample[threadIdx.x] = my_n > 0 ? keys_s[kpad((int)(((int64_t)threadIdx.x * my_n) / 32))] : 0u;
+
+  // This rank's histogram of the keys matching (prefix, mask) at digit
+  // `shift`, stored into slot `buf` of every rank.  Scores are >= 0, so
+  // their bit patterns order like the values and bit 31 is clear.
+  auto histogram_and_store = [&](uint32_t prefix, uint32_t mask, int shift, int buf) {
+    for (int i = threadIdx.x; i < my_n; i += blockDim.x) {
+      const uint32_t v = keys_s[kpad(i)];
+      if ((v & mask) == prefix) atomicAdd(&sh.lhist[wid & 3][(v >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < kTopkBins) {
+      const uint32_t h = sh.lhist[0][threadIdx.x] + sh.lhist[1][threadIdx.x] + sh.lhist[2][threadIdx.x] +
+                         sh.lhist[3][threadIdx.x];
+      sh.lhist[0][threadIdx.x] = h;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < kTopkBins * kTopkCl; t += blockDim.x) {
+      const int bin = t & (kTopkBins - 1), dst = t / kTopkBins;
+      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(&sh.g_hist[buf][rank][bin], (uint32_t)dst)),
+                   "r"(sh.lhist[0][bin])
+                   : "memory");
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
+  };
+
+  uint32_t prefix = 0u, mask = 0x80000000u, remaining = (uint32_t)need;
+  uint32_t tau = 0u, take_eq = 0u;
+  histogram_and_store(prefix, mask, 23, 0);
   cluster_sync();
-  if (threadIdx.x < kTopkSample) sh.all_sample[threadIdx.x] = remote_u32(&sh.sample[threadIdx.x & 31], threadIdx.x >> 5);
-  if (threadIdx.x == 0) { sh.t_hi = 0xffffffffu; sh.t_lo = 0u; }
-  __syncthreads();
-  {
-    const double q = (double)need * kTopkSample / (double)nc;
-    const double delta = 4.0 * sqrt(q + 1.0) + 8.0;
-    const int r_hi = (int)floor(q - delta), r_lo = (int)ceil(q + delta);
-    if (threadIdx.x < kTopkSample) {
-      const uint32_t v = sh.all_sample[threadIdx.x];
-      int rnk = 0;
-#pragma unroll 8
-      for (int j = 0; j < kTopkSample; ++j) {
-        const uint32_t u = sh.all_sample[j];
-        rnk += (u > v) || (u == v && j < (int)threadIdx.x);
-      }
-      if (r_hi >= 1 && rnk == r_hi - 1) sh.t_hi = v;
-      if (r_lo <= kTopkSample && rnk == r_lo - 1) sh.t_lo = v;
+  for (int pass = 0;; ++pass) {
+    const int buf = pass & 1, shift = pass < 3 ? 23 - 8 * pass : 0;   // 23, 15, 7, 0
+    if (pass > 0) {
+      histogram_and_store(prefix, mask, shift, buf);
+      cluster_sync();
     }
-  }
-  __syncthreads();
-  const uint32_t t_hi = sh.t_hi, t_lo = sh.t_lo;
-  // Count this rank's keys above the bracket and collect those inside it.
-  uint32_t above = 0, cnt = 0, cmin = 0xffffffffu, cmax = 0u;
-  uint32_t *mine = seg + wid * kTopkClSeg;
-  for (int i0 = 0; i0 < my_n; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const bool valid = i < my_n;
-    const uint32_t v = valid ? keys_s[kpad(i)] : 0u;
-    above += (valid && v > t_hi);
-    const bool in = valid && v <= t_hi && v >= t_lo;
-    const uint32_t ball = __ballot_sync(0xffffffffu, in);
-    if (in) {
-      const uint32_t slot = cnt + __popc(ball & ((1u << lane) - 1u));
-      if (slot < kTopkClSeg) mine[slot] = v;
-      cmin = min(cmin, v);
-      cmax = max(cmax, v);
-    }
-    cnt += __popc(ball);
-  }
-  above = warp_sum_u32(above);
+    // Every rank holds every rank's histogram and takes the same decisions.
+    if (threadIdx.x < kTopkBins) {
+      uint32_t h = 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
-    cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
-  }
-  if (threadIdx.x == 0) { sh.cmin = 0xffffffffu; sh.cmax = 0u; }
-  __syncthreads();
-  if (lane == 0) {
-    sh.seg_count[wid] = cnt;
-    sh.seg_above[wid] = above;
-    atomicMin(&sh.cmin, cmin);
-    atomicMax(&sh.cmax, cmax);
+      for (int c = 0; c < kTopkCl; ++c) h += sh.g_hist[buf][c][threadIdx.x];
+      sh.hist[threadIdx.x] = h;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
+    __syncthreads();
+    const uint32_t d = sh.digit, in_bin = sh.hist[d];
+    remaining -= sh.above;
+    if (threadIdx.x < kTopkBins) {
+#pragma unroll
+      for (int c = 0; c < kTopkCl; ++c) {
+        const uint32_t g = __reduce_add_sync(0xffffffffu, (uint32_t)threadIdx.x > d ? sh.g_hist[buf][c][threadIdx.x] : 0u);
+        if (lane == 0 && g) atomicAdd(&sh.gt_acc[c], g);
+      }
+    }
+    if (threadIdx.x < kTopkCl) sh.eq_acc[threadIdx.x] = sh.g_hist[buf][threadIdx.x][d];
+    prefix |= d << shift;
+    mask |= 255u << shift;
+    __syncthreads();
+    if (in_bin == remaining && prefix != 0u) {
+      // Every key of the bin is taken: they are exactly the keys >= prefix
+      // within it, so tau = prefix - 1 and no equal key is rationed.
+      if (threadIdx.x < kTopkCl) {
+        sh.gt_acc[threadIdx.x] += sh.eq_acc[threadIdx.x];
+        sh.eq_acc[threadIdx.x] = 0u;
+      }
+      tau = prefix - 1u;
+      take_eq = 0u;
+      break;
+    }
+    if (pass == 3) {
+      tau = prefix;        // all 31 bits resolved: eq_acc counts the keys == tau
+      take_eq = remaining;
+      break;
+    }
+    if (in_bin <= (uint32_t)kTopkGather) {
+      // Gather the bin's keys into every rank, rank by rank.
+      uint32_t seg[kTopkCl + 1];
+      seg[0] = 0u;
+#pragma unroll
+      for (int c = 0; c < kTopkCl; ++c) seg[c + 1] = seg[c] + sh.eq_acc[c];
+      uint32_t my_off = 0u;
+#pragma unroll
+      for (int c = 0; c < kTopkCl; ++c) my_off = (uint32_t)c == rank ? seg[c] : my_off;
+      for (int i0 = 0; i0 < my_n; i0 += blockDim.x) {
+        const int i = i0 + threadIdx.x;
+        const uint32_t v = i < my_n ? keys_s[kpad(i)] : 0u;
+        const bool in = i < my_n && (v & mask) == prefix;
+        const uint32_t ball = __ballot_sync(0xffffffffu, in);
+        if (ball == 0u) continue;
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(&sh.gcount, (uint32_t)__popc(ball));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (in) {
+          const uint32_t pos = my_off + base + __popc(ball & ((1u << lane) - 1u));
+#pragma unroll
+          for (int dst = 0; dst < kTopkCl; ++dst)
+            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(&sh.gbuf[pos], (uint32_t)dst)), "r"(v)
+                         : "memory");
+        }
+      }
+      cluster_sync();
+      // tau among the gathered keys, then every rank's keys > tau and == tau.
+      const uint32_t lo_b = prefix, hi_b = prefix | ~mask;
+      auto value = [&](int i) -> uint32_t { return sh.gbuf[i]; };
+      cl_radix_select(value, (int)in_bin, remaining, lo_b, hi_b, sh, &tau, &take_eq);
+      uint32_t gt_c[kTopkCl], eq_c[kTopkCl];
+#pragma unroll
+      for (int c = 0; c < kTopkCl; ++c) gt_c[c] = eq_c[c] = 0u;
+      for (uint32_t i = threadIdx.x; i < in_bin; i += blockDim.x) {
+        const uint32_t v = sh.gbuf[i];
+#pragma unroll
+        for (int c = 0; c < kTopkCl; ++c) {
+          const bool mine_c = i >= seg[c] && i < seg[c + 1];
+          gt_c[c] += mine_c && v > tau;
+          eq_c[c] += mine_c && v == tau;
+        }
+      }
+      if (threadIdx.x < kTopkCl) sh.eq_acc[threadIdx.x] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int c = 0; c < kTopkCl; ++c) {
+        const uint32_t g = __reduce_add_sync(0xffffffffu, gt_c[c]);
+        const uint32_t e = __reduce_add_sync(0xffffffffu, eq_c[c]);
+        if (lane == 0) {
+          if (g) atomicAdd(&sh.gt_acc[c], g);
+          if (e) atomicAdd(&sh.eq_acc[c], e);
+        }
+      }
+      break;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t na = 0, ncd = 0;
-    for (int w = 0; w < kTopkClWarps; ++w) {
-      na += sh.seg_above[w];
-      sh.warp_off[w] = ncd;
-      ncd += (sh.seg_count[w] > (uint32_t)kTopkClSeg) ? 0x40000000u : sh.seg_count[w];  // overflow poisons
+    uint32_t out_before = 0, eq_before = 0;
+    for (uint32_t c = 0; c < rank; ++c) {
+      const uint32_t eq2 = sh.eq_acc[c];
+      const uint32_t take2 = (eq_before >= take_eq) ? 0u : min(eq2, take_eq - eq_before);
+      out_before += sh.gt_acc[c] + take2;
+      eq_before += eq2;
     }
-    sh.n_above = na;
-    sh.n_cand = ncd;
+    sh.out_before = out_before;
+    sh.eq_before = eq_before;
   }
   __syncthreads();
-  // Push this rank's candidates into its slots of rank 0's buffer (remote
-  // stores, made visible by the cluster barrier below).
-  if (sh.n_cand <= (uint32_t)kTopkClPerRank) {
-    const uint32_t n_w = min(sh.seg_count[wid], (uint32_t)kTopkClSeg);
-    const uint32_t base = cluster_map(gath + rank * kTopkClPerRank + sh.warp_off[wid], 0u);
-    for (uint32_t e = lane; e < n_w; e += 32)
-      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(base + 4 * e), "r"(mine[e]) : "memory");
-  }
-  cluster_sync();
-  if (rank == 0) {
-    uint32_t n_above = 0, n_cand = 0, lo = 0xffffffffu, hi = 0u;
-    for (uint32_t c = 0; c < kTopkCl; ++c) {
-      n_above += remote_u32(&sh.n_above, c);
-      n_cand += remote_u32(&sh.n_cand, c);
-      lo = min(lo, remote_u32(&sh.cmin, c));
-      hi = max(hi, remote_u32(&sh.cmax, c));
-    }
-    __shared__ uint32_t rank_cand[kTopkCl];
-    bool per_rank_ok = true;
-    if (threadIdx.x == 0)
-      for (int c = 0; c < kTopkCl; ++c) rank_cand[c] = remote_u32(&sh.n_cand, (uint32_t)c);
-    __syncthreads();
-    for (int c = 0; c < kTopkCl; ++c) per_rank_ok &= rank_cand[c] <= (uint32_t)kTopkClPerRank;
-    const bool bracket_ok = per_rank_ok && n_above < (uint32_t)need && (uint32_t)need <= n_above + n_cand;
-    uint32_t tau = 0, take_eq = 0;
-    if (bracket_ok) {
-      // Candidates sit in fixed per-rank slots of gath.
-      auto value = [&](int i, bool &ok) -> uint32_t {
-        const int c = i / kTopkClPerRank, e = i - c * kTopkClPerRank;
-        ok = e < (int)rank_cand[c];
-        return ok ? gath[i] : 0u;
-      };
-      cl_radix_select(value, kTopkClCand, (uint32_t)need - n_above, lo, hi, sh, &tau, &take_eq);
-    } else {
-      // Exact select over every key of every rank (read remotely).
-      auto value = [&](int i, bool &ok) -> uint32_t {
-        ok = true;
-        const int c = i / chunk;
-        return remote_u32(keys_s + kpad(i - c * chunk), (uint32_t)c);
-      };
-      cl_radix_select(value, nc, (uint32_t)need, 0u, 0xffffffffu, sh, &tau, &take_eq);
-    }
-    if (threadIdx.x == 0) {
-      sh.tau = tau;
-      sh.take_eq = take_eq;
-    }
-  }
-  cluster_sync();
-  const uint32_t tau = remote_u32(&sh.tau, 0), take_eq = remote_u32(&sh.take_eq, 0);
-  // Per-thread contiguous chunk counts, then the rank's totals.
+  const uint32_t out_before_rank = sh.out_before, eq_before_rank = sh.eq_before;
+  // Per-thread contiguous chunks: one scan of (n_gt << 16 | n_eq), which
+  // cannot carry between the halves because a rank holds < 65536 keys.
+  static_assert(kTopkClKeys < 65536, "packed counts");
   const int per = (my_n + (int)blockDim.x - 1) / (int)blockDim.x;
   const int j0 = min(my_n, (int)threadIdx.x * per), j1 = min(my_n, j0 + per);
   uint32_t n_gt = 0, n_eq = 0;
@@ -632,29 +656,12 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
     n_gt += key > tau;
     n_eq += key == tau;
   }
-  const uint32_t eq_before_local = block_excl_scan(n_eq, sh.warp_tot, &sh.total);
-  const uint32_t eq_total = sh.total;
-  const uint32_t gt_before_local = block_excl_scan(n_gt, sh.warp_tot, &sh.total);
-  const uint32_t gt_total = sh.total;
-  if (threadIdx.x == 0) { sh.n_gt = gt_total; sh.n_eq = eq_total; }
-  cluster_sync();
-  __shared__ uint32_t rank_gt[kTopkCl], rank_eq[kTopkCl];
-  if (threadIdx.x < kTopkCl) {
-    rank_gt[threadIdx.x] = remote_u32(&sh.n_gt, threadIdx.x);
-    rank_eq[threadIdx.x] = remote_u32(&sh.n_eq, threadIdx.x);
-  }
-  __syncthreads();
-  uint32_t eq_before_rank = 0, out_before_rank = 0;
-  for (uint32_t c = 0; c < rank; ++c) {
-    const uint32_t gt_c = rank_gt[c], eq_c = rank_eq[c];
-    const uint32_t take_c = (eq_before_rank >= take_eq) ? 0u : min(eq_c, take_eq - eq_before_rank);
-    out_before_rank += gt_c + take_c;
-    eq_before_rank += eq_c;
-  }
-  // Within the rank: equal keys taken in index order up to take_eq overall.
-  const uint32_t eq_before = eq_before_rank + eq_before_local;
-  const uint32_t eq_take = (eq_before >= take_eq) ? 0u : min(n_eq, take_eq - eq_before);
-  const uint32_t take_before_local = block_excl_scan(eq_take, sh.warp_tot, &sh.total);
+  const uint32_t packed_before = block_excl_scan((n_gt << 16) | n_eq, sh.warp_tot, &sh.total);
+  const uint32_t eq_before_local = packed_before & 0xffffu, gt_before_local = packed_before >> 16;
+  // Equal keys still to take when this rank starts, and this thread's share.
+  const uint32_t avail = take_eq > eq_before_rank ? take_eq - eq_before_rank : 0u;
+  const uint32_t take_before_local = min(avail, eq_before_local);
+  const uint32_t eq_take = avail > eq_before_local ? min(n_eq, avail - eq_before_local) : 0u;
   uint32_t pos = out_before_rank + gt_before_local + take_before_local, eq_seen = 0;
   for (int i = j0; i < j1; ++i) {
     const uint32_t key = keys_s[kpad(i)];
@@ -662,7 +669,8 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
     if (key == tau) { take = eq_seen < eq_take; ++eq_seen; }
     if (take && pos < (uint32_t)k) out[pos++] = (int32_t)(s.n_sink + i_begin + i);
   }
-  cluster_sync();  // no rank leaves while another may still read its shared memory
+  // Each rank's distributed accesses ended at its last cluster barrier, so
+  // no rank waits for the others before leaving.
 }
 
 }  // namespace s4r

@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from problems import check_batch, make_batch, run_gpu
 
@@ -91,3 +92,37 @@ def test_device_status_on_bad_length():
     assert res["status"] == s4r.S4R_ERR_DEVICE
     assert torch.isfinite(res["out"]).all()
     assert (res["idx"][1] == -1).all()
+
+
+def _run_exact_idx(batch):
+    """Run the batch and also require the index sets to equal the oracle's
+    exactly: these cases are built so that ties are decided by position."""
+    res = run_gpu(batch)
+    assert res["status"] == 0, f"device status {res['status']}"
+    check_batch(batch, res)
+    for b in range(batch.batch):
+        _, idx_ref, _ = oracle.decode_step(batch.oracle_problem(b))
+        assert np.array_equal(res["idx"][b].numpy(), idx_ref), f"problem {b}: tie order differs"
+    return res
+
+
+def test_all_scores_tied_take_lowest_positions():
+    # Zero key coefficients: every logit is 0, every score equal, so the top-k
+    # is the k lowest candidate positions (and every rank's candidate buffer
+    # overflows, which sends the cluster select to its exact path).
+    batch = make_batch(W1, lengths=[20000, 9000], top_k=512, tag="tied")
+    batch.coeff_k.zero_()
+    res = _run_exact_idx(batch)
+    for b in range(2):
+        assert np.array_equal(res["idx"][b].numpy(), 4 + np.arange(512))
+
+
+@pytest.mark.parametrize("top_k", [1000, 4000])
+def test_three_distinct_rows_tie_across_ranks(top_k):
+    # Key rows repeat three vectors, so the scores take three values and the
+    # threshold value is shared by thousands of keys spread over the cluster.
+    batch = make_batch(W1, lengths=[9000], top_k=top_k, tag="three")
+    g = torch.Generator().manual_seed(7)
+    pats = synth.store(torch.randn(3, batch.coeff_k.shape[2], generator=g, dtype=torch.float64) * 0.5, "bf16")
+    batch.coeff_k[0, :9000] = pats[torch.arange(9000) % 3]
+    _run_exact_idx(batch)
