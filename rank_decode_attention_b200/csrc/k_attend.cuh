@@ -74,6 +74,10 @@ __host__ __device__ inline AttItems att_items(int G, int dh, int n_ranks, int ra
   return it;
 }
 
+// Float counts of shared-memory regions are kept multiples of 4 (16 bytes),
+// so every region starts 16-byte aligned.
+__host__ __device__ inline size_t att_round4(size_t n) { return (n + 3) / 4 * 4; }
+
 // Launch plan: rows staged per pass (a multiple of 32) and B^V rows staged.
 struct AttPlan {
   int e_cap, bv_rows;
@@ -81,12 +85,15 @@ struct AttPlan {
 __host__ __device__ inline size_t att_float_words(const Shape &s, int e_cap, int bv_rows) {
   return (size_t)kAttMaxGroup * s.rank_k          // q_s
          + (size_t)kAttMaxGroup * e_cap           // p_s: [entry][kAttMaxGroup]
-         + (size_t)s.n_sink * bv_rows             // sv_s: sink values of this CTA's output columns
+         + att_round4((size_t)s.n_sink * bv_rows)  // sv_s: sink values of this CTA's output columns
+         + (size_t)8 * att_pitch(s.rank_k, 2)     // qb_s: [16][pitch] bf16 split query (tensor-core B operand)
          + (size_t)kAttMaxGroup * 4               // ml_s: m, l, chunk scale
-         + (size_t)kAttMaxGroup * (s.rank_v + 2)  // part_s: this CTA's m, l, acc[rv] per head
-         + (size_t)kAttMaxGroup * s.rank_v        // acc_s: merged acc of the heads this CTA finishes
+         + (size_t)kAttMaxGroup * (s.rank_v + 4)  // part_s: this CTA's (m, l, -, -, acc[rv]) per head
+         + (size_t)2 * kAttCluster * (s.rank_v + 4)  // recv_s: every rank's partial of the <= 2 heads finished here
+         + (size_t)2 * s.rank_v                   // acc_s: merged acc of those heads
          + (size_t)kAttMaxGroup * kAttMaxSinks    // sw_s: sink logits, then weights
-         + (size_t)kAttMaxGroup * kAttCluster;    // f_s: merge weights of the ranks
+         + (size_t)2 * kAttCluster                // f_s: merge weights of the ranks
+         + (size_t)8 * att_pitch(e_cap, 2);       // pb_s: [16][pitch] bf16 split weights (tensor-core B operand)
 }
 __host__ __device__ inline size_t att_smem_bytes(const Shape &s, int esize, const AttPlan &pl) {
   const size_t rows = (size_t)pl.e_cap * (att_pitch(s.rank_k, esize) + att_pitch(s.rank_v, esize)) * esize;
@@ -130,7 +137,7 @@ __device__ __forceinline__ float dot_f32_store(const float *a, const T *x, int n
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kAttThreads)
+__global__ void __launch_bounds__(kAttThreads, 1)
 attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
               const T *__restrict__ coeff_k, const T *__restrict__ coeff_v, const float *__restrict__ qt_all,
               const T *__restrict__ q, const T *__restrict__ basis_v, const T *__restrict__ sink_k,
@@ -151,11 +158,17 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
   float *q_s = reinterpret_cast<float *>(bv_s + (size_t)pl.bv_rows * pv);  // [G][rk]
   float *p_s = q_s + kAttMaxGroup * rk;                     // [E][kAttMaxGroup] logits, then weights
   float *sv_s = p_s + kAttMaxGroup * E;                     // [ns][e_hi - e_lo] sink values
-  float *ml_s = sv_s + (size_t)ns * pl.bv_rows;             // [G][4]
-  float *part_s = ml_s + kAttMaxGroup * 4;                  // [G][rv + 2]
-  float *acc_s = part_s + kAttMaxGroup * (rv + 2);          // [G][rv]
-  float *sw_s = acc_s + kAttMaxGroup * rv;                  // [G][kAttMaxSinks]
-  float *f_s = sw_s + kAttMaxGroup * kAttMaxSinks;          // [G][kAttCluster]
+  bf16 *qb_s = reinterpret_cast<bf16 *>(sv_s + att_round4((size_t)ns * pl.bv_rows));  // [16][pq]
+  const int pq = att_pitch(rk, 2);
+  float *ml_s = reinterpret_cast<float *>(qb_s + 16 * pq);  // [G][4]
+  const int pr = rv + 4;                                    // partial row: m, l, -, -, acc[rv]
+  float *part_s = ml_s + kAttMaxGroup * 4;                  // [G][pr]
+  float *recv_s = part_s + kAttMaxGroup * pr;               // [2][kAttCluster][pr]
+  float *acc_s = recv_s + 2 * kAttCluster * pr;             // [2][rv]
+  float *sw_s = acc_s + 2 * rv;                             // [G][kAttMaxSinks]
+  float *f_s = sw_s + kAttMaxGroup * kAttMaxSinks;          // [2][kAttCluster]
+  bf16 *pb_s = reinterpret_cast<bf16 *>(f_s + 2 * kAttCluster);  // [16][ppb]
+  const int ppb = att_pitch(E, 2);
   __shared__ int64_t rows_s[kAttEntriesMax];
   __shared__ __align__(8) uint64_t stage_bar, bv_bar;
 
@@ -180,6 +193,18 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
   for (int t = threadIdx.x; t < G * rk; t += blockDim.x) {
     const int j = t / rk, k = t - j * rk;
     q_s[j * rk + k] = __ldcg(qt_all + ((int64_t)b * s.n_heads_q + g * G + j) * rk + k);
+  }
+  // Tensor-core operand of the logits: column n = 2j + term holds head j's
+  // latent query as two bf16 terms (hi, lo) whose sum keeps ~16 bits.
+  for (int t = threadIdx.x; t < 16 * rk; t += blockDim.x) {
+    const int n = t / rk, k = t - n * rk, j = n >> 1;
+    float v = 0.f;
+    if (j < G) {
+      const float x = __ldcg(qt_all + ((int64_t)b * s.n_heads_q + g * G + j) * rk + k);
+      const float hi = __bfloat162float(__float2bfloat16_rn(x));
+      v = (n & 1) ? x - hi : hi;
+    }
+    qb_s[n * pq + k] = __float2bfloat16_rn(v);
   }
   for (int t = threadIdx.x; t < ns * (it.e_hi - it.e_lo); t += blockDim.x) {
     const int tk = t / (it.e_hi - it.e_lo), e = t - tk * (it.e_hi - it.e_lo);
@@ -219,6 +244,18 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
 #pragma unroll
   for (int j = 0; j < kAttMaxGroup; ++j) acc[j] = 0.f;
   const int kcol = threadIdx.x;  // latent value column owned by this thread (< rv)
+  // Tensor-core path of the latent value sums (bf16 storage): acc^T[k][n] =
+  // sum_e C_V[e][k] W[e][n], W column n = 2j + term holding head j's
+  // weights as two bf16 terms; warp w owns the 16-column tiles w, w + 8.
+  const bool tc_acc = sizeof(T) == 2 && rv % 16 == 0;
+  const int n_nt = (2 * G + 7) / 8;
+  float accf[2][2][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int d = 0; d < 4; ++d) accf[a][c][d] = 0.f;
 
   uint32_t phase = 0;
   for (int64_t c0 = e_begin; c0 < e_end; c0 += E) {
@@ -239,10 +276,10 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
     const int n_live = __syncthreads_count(live);
     if (threadIdx.x == 0) mbar_arrive_expect_tx(&stage_bar, (uint32_t)(n_live * (rk + rv) * sizeof(T)));
     __syncthreads();
-    for (int t = threadIdx.x; t < 2 * n_e; t += blockDim.x) {
-      const int e = t % n_e;
-      const bool is_v = t >= n_e;
-      const int64_t row = rows_s[e];
+    for (int t = threadIdx.x; t < 2 * E; t += blockDim.x) {
+      const int e = t % E;
+      const bool is_v = t >= E;
+      const int64_t row = e < n_e ? rows_s[e] : -1;
       T *dst = is_v ? cv_s + (size_t)e * pv : ck_s + (size_t)e * pk;
       const int n = is_v ? rv : rk;
       if (row >= 0) {
@@ -254,6 +291,39 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
     mbar_wait(&stage_bar, phase, nullptr);
     phase ^= 1u;
     __syncthreads();
+    if (sizeof(T) == 2 && rk % 16 == 0) {
+      // logits on the tensor cores: per warp, 16-entry tiles of
+      // C_K[16 x rk] . Qsplit[rk x 8] (mma m16n8k16, bf16 in, fp32 out); the
+      // accumulator of row e, column 2j + term is split over lanes
+      // (g = lane / 4 rows, t = lane % 4 column pairs).
+      const int gq = lane >> 2, tq = lane & 3;
+      const int n_nt = (2 * G + 7) / 8;
+      for (int mt = wid; mt < E / 16; mt += kWarps) {
+        const int e0 = mt * 16 + gq, e1 = e0 + 8;
+        const uint32_t *a_lo = reinterpret_cast<const uint32_t *>(ck_s + (size_t)e0 * pk) + tq;
+        const uint32_t *a_hi = reinterpret_cast<const uint32_t *>(ck_s + (size_t)e1 * pk) + tq;
+        const bool ok0 = e0 < n_e && rows_s[e0] >= 0, ok1 = e1 < n_e && rows_s[e1] >= 0;
+        for (int nt = 0; nt < n_nt; ++nt) {
+          const uint32_t *bq = reinterpret_cast<const uint32_t *>(qb_s + (size_t)(nt * 8 + gq) * pq) + tq;
+          float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll 4
+          for (int ks = 0; ks < rk / 16; ++ks) {
+            const uint32_t a0 = a_lo[ks * 8], a1 = a_hi[ks * 8], a2 = a_lo[ks * 8 + 4], a3 = a_hi[ks * 8 + 4];
+            const uint32_t b0 = bq[ks * 8], b1 = bq[ks * 8 + 4];
+            asm volatile(
+                "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                "{%0,%1,%2,%3};"
+                : "+f"(c0), "+f"(c1), "+f"(c2), "+f"(c3)
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+          }
+          const int j = nt * 4 + tq;   // columns 2j, 2j + 1: the two terms of head j
+          if (j < G) {
+            p_s[e0 * kAttMaxGroup + j] = ok0 ? c0 + c1 : -INFINITY;
+            p_s[e1 * kAttMaxGroup + j] = ok1 ? c2 + c3 : -INFINITY;
+          }
+        }
+      }
+    } else
     // logits: the thread of entry e computes all G heads, reading its key
     // row once and the latent queries as broadcast float4s
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -317,13 +387,59 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
       }
     }
     __syncthreads();
-    if (kcol < rv) {
+    if (tc_acc) {
+      // Split weights into the B operand, then one m16n8k16 per (tile, 16 entries).
+      for (int t = threadIdx.x; t < 16 * E; t += blockDim.x) {
+        const int n = t / E, e = t - n * E, j = n >> 1;
+        const float pv_ = j < G ? p_s[e * kAttMaxGroup + j] : 0.f;
+        const float hi = __bfloat162float(__float2bfloat16_rn(pv_));
+        pb_s[n * ppb + e] = __float2bfloat16_rn((n & 1) ? pv_ - hi : hi);
+      }
+      __syncthreads();
+      const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int mt = wid + a * kWarps;
+        if (mt < rv / 16) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int j = c * 4 + tq;
+            const float sc = (c < n_nt && j < G) ? ml_s[j * 4 + 2] : 0.f;
+#pragma unroll
+            for (int d = 0; d < 4; ++d) accf[a][c][d] *= sc;
+          }
+          for (int ks = 0; ks < E / 16; ++ks) {
+            // A = C_V^T tile: four 8x8 blocks (entries x columns) loaded transposed.
+            const int m = lane >> 3;
+            const int e = ks * 16 + ((m & 2) ? 8 : 0) + (lane & 7);
+            const int c0 = mt * 16 + ((m & 1) ? 8 : 0);
+            uint32_t a0, a1, a2, a3;
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                         : "r"(smem_u32(cv_s + (size_t)e * pv + c0)));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              if (c < n_nt) {
+                const uint32_t *bw = reinterpret_cast<const uint32_t *>(pb_s + (size_t)(c * 8 + gq) * ppb + ks * 16) + tq;
+                const uint32_t b0 = bw[0], b1 = bw[4];
+                asm volatile(
+                    "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                    "{%0,%1,%2,%3};"
+                    : "+f"(accf[a][c][0]), "+f"(accf[a][c][1]), "+f"(accf[a][c][2]), "+f"(accf[a][c][3])
+                    : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+              }
+            }
+          }
+        }
+      }
+    } else if (kcol < rv) {
       float sc[kAttMaxGroup];
 #pragma unroll
       for (int j = 0; j < kAttMaxGroup; ++j) {
         sc[j] = (j < G) ? ml_s[j * 4 + 2] : 0.f;
         acc[j] *= sc[j];
       }
+#pragma unroll 4
       for (int e = 0; e < n_e; ++e) {
         const float v = to_f(cv_s[(size_t)e * pv + kcol]);
         const float4 pa = *reinterpret_cast<const float4 *>(p_s + e * kAttMaxGroup);
@@ -341,24 +457,55 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
       }
     }
   }
-  // This CTA's partial, kept in shared memory for the other ranks.
-  if (kcol < rv)
+  // This CTA's partial (m, l, acc) of every head, then stored into the CTAs
+  // that finish each head.
+  if (tc_acc) {
+    const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const int mt = wid + a * kWarps;
+      if (mt < rv / 16) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int j = c * 4 + tq;
+          if (c < n_nt && j < G) {
+            part_s[j * pr + 4 + mt * 16 + gq] = accf[a][c][0] + accf[a][c][1];
+            part_s[j * pr + 4 + mt * 16 + gq + 8] = accf[a][c][2] + accf[a][c][3];
+          }
+        }
+      }
+    }
+  } else if (kcol < rv) {
 #pragma unroll
     for (int j = 0; j < kAttMaxGroup; ++j)
-      if (j < G) part_s[j * (rv + 2) + 2 + kcol] = acc[j];
-  __syncthreads();
-  if (threadIdx.x < G) {
-    part_s[threadIdx.x * (rv + 2)] = ml_s[threadIdx.x * 4];
-    part_s[threadIdx.x * (rv + 2) + 1] = ml_s[threadIdx.x * 4 + 1];
+      if (j < G) part_s[j * pr + 4 + kcol] = acc[j];
   }
-  cluster_sync();  // every partial is in place
+  if (threadIdx.x < G) {
+    part_s[threadIdx.x * pr] = ml_s[threadIdx.x * 4];
+    part_s[threadIdx.x * pr + 1] = ml_s[threadIdx.x * 4 + 1];
+  }
+  __syncthreads();
+  for (int r2 = 0; r2 < n_ranks; ++r2) {
+    const AttItems it2 = att_items(G, dh, n_ranks, r2);
+    if (it2.t1 <= it2.t0) continue;
+    const int jlo2 = it2.t0 / dh, nh2 = (it2.t1 - 1) / dh + 1 - jlo2;
+    for (int t = threadIdx.x; t < nh2 * (pr / 4); t += blockDim.x) {
+      const int jj = t / (pr / 4), q4 = t - jj * (pr / 4);
+      const float4 v = *reinterpret_cast<const float4 *>(part_s + (jlo2 + jj) * pr + 4 * q4);
+      const uint32_t dst = cluster_map(recv_s + ((size_t)jj * kAttCluster + rank) * pr + 4 * q4, (uint32_t)r2);
+      asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v.x), "f"(v.y), "f"(v.z),
+                   "f"(v.w)
+                   : "memory");
+    }
+  }
+  cluster_sync();  // every partial is in place; no distributed access follows
   // Merge weights of the heads this CTA finishes (warp per head; ranks = lanes).
-  for (int j = j_lo + wid; j < j_hi; j += kWarps) {
+  for (int jj = wid; jj < j_hi - j_lo; jj += kWarps) {
+    const int j = j_lo + jj;
     float mr = -INFINITY, lr = 0.f;
     if (lane < n_ranks) {
-      const uint32_t base = cluster_map(part_s + j * (rv + 2), (uint32_t)lane);
-      mr = ld_cluster_f32(base);
-      lr = ld_cluster_f32(base + 4);
+      mr = recv_s[((size_t)jj * kAttCluster + lane) * pr];
+      lr = recv_s[((size_t)jj * kAttCluster + lane) * pr + 1];
     }
     float M = mr;
     for (int tk = lane; tk < ns; tk += 32) M = fmaxf(M, sw_s[j * kAttMaxSinks + tk]);
@@ -368,36 +515,51 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
     for (int tk = lane; tk < ns; tk += 32) den += __expf(sw_s[j * kAttMaxSinks + tk] - M);
     den = warp_sum(den);
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    if (lane < n_ranks) f_s[j * kAttCluster + lane] = fr * inv;
+    if (lane < n_ranks) f_s[jj * kAttCluster + lane] = fr * inv;
     __syncwarp();
     for (int tk = lane; tk < ns; tk += 32)
       sw_s[j * kAttMaxSinks + tk] = __expf(sw_s[j * kAttMaxSinks + tk] - M) * inv;
   }
   __syncthreads();
-  // acc[j][k] = sum_r f[j][r] acc_r[j][k], read through distributed shared memory.
+  // acc[j][k] = sum_r f[j][r] acc_r[j][k]
   for (int t = threadIdx.x; t < (j_hi - j_lo) * rv; t += blockDim.x) {
-    const int j = j_lo + t / rv, k = t % rv;
-    float v[kAttCluster];
-#pragma unroll
-    for (int r = 0; r < kAttCluster; ++r)
-      v[r] = (r < n_ranks) ? ld_cluster_f32(cluster_map(part_s + j * (rv + 2) + 2 + k, (uint32_t)r)) : 0.f;
+    const int jj = t / rv, k = t % rv;
     float a = 0.f;
 #pragma unroll
     for (int r = 0; r < kAttCluster; ++r)
-      if (r < n_ranks) a = fmaf(f_s[j * kAttCluster + r], v[r], a);
-    acc_s[j * rv + k] = a;
+      if (r < n_ranks) a = fmaf(f_s[jj * kAttCluster + r], recv_s[((size_t)jj * kAttCluster + r) * pr + 4 + k], a);
+    acc_s[jj * rv + k] = a;
   }
   mbar_wait(&bv_bar, 0, nullptr);
   __syncthreads();
-  // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e].
-  for (int t = it.t0 + (int)threadIdx.x; t < it.t1; t += blockDim.x) {
-    const int j = t / dh, e = t - j * dh;
-    float o = dot_f32_store(acc_s + j * rv, bv_s + (size_t)(e - it.e_lo) * pv, rv);
-    for (int tk = 0; tk < ns; ++tk)
-      o = fmaf(sw_s[j * kAttMaxSinks + tk], sv_s[tk * (it.e_hi - it.e_lo) + (e - it.e_lo)], o);
-    out[((int64_t)b * s.n_heads_q + g * G + j) * dh + e] = o;
+  // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e], four
+  // threads per output (16-byte chunks c = part, part + 4, ...).
+  const int n_items = it.t1 - it.t0;
+  for (int base = 0; base < 4 * n_items; base += blockDim.x) {
+    const int t = base + (int)threadIdx.x, item = t >> 2, part = t & 3;
+    const bool act = t < 4 * n_items;
+    float o = 0.f;
+    int j = 0, e = 0;
+    if (act) {
+      j = (it.t0 + item) / dh;
+      e = (it.t0 + item) - j * dh;
+      const float *av = acc_s + (j - j_lo) * rv;
+      const T *br = bv_s + (size_t)(e - it.e_lo) * pv;
+      for (int c = part * V; c < rv; c += 4 * V) {
+        float xv[V];
+        load16(br + c, xv);
+#pragma unroll
+        for (int u = 0; u < V; ++u) o = fmaf(av[c + u], xv[u], o);
+      }
+    }
+    o += __shfl_xor_sync(0xffffffffu, o, 1);
+    o += __shfl_xor_sync(0xffffffffu, o, 2);
+    if (act && part == 0) {
+      for (int tk = 0; tk < ns; ++tk)
+        o = fmaf(sw_s[j * kAttMaxSinks + tk], sv_s[tk * (it.e_hi - it.e_lo) + (e - it.e_lo)], o);
+      out[((int64_t)b * s.n_heads_q + g * G + j) * dh + e] = o;
+    }
   }
-  cluster_sync();  // every CTA has read the partials it needs
 }
 
 // Rebuild rows explicitly: out[e][d] = sum_j C[rows[e]][j] B[d][j] (fp32).

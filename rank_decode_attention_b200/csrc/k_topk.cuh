@@ -427,7 +427,6 @@ __device__ __forceinline__ void cl_pick_digit(TopkClShared &sh, uint32_t remaini
 template <typename ValueFn>
 __device__ __forceinline__ void cl_radix_select(ValueFn value, int n, uint32_t need, uint32_t lo_all,
                                                 uint32_t hi_all, TopkClShared &sh, uint32_t *tau, uint32_t *take_eq) {
-  const int lane = threadIdx.x & 31;
   const uint32_t diff = lo_all ^ hi_all;
   int top = 31;
   while (top >= 0 && !((diff >> top) & 1u)) --top;
@@ -441,12 +440,11 @@ __device__ __forceinline__ void cl_radix_select(ValueFn value, int n, uint32_t n
     for (int shift = (top / 8) * 8; shift >= 0; shift -= 8) {
       for (int j = threadIdx.x; j < kTopkBins; j += blockDim.x) sh.hist[j] = 0;
       __syncthreads();
+      // The common high bits are already fixed, so the digits of these few
+      // keys spread over the bins and plain shared atomics rarely collide.
       for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const uint32_t v = value(i);
-        const bool in = (v & mask) == prefix;
-        const uint32_t bin = in ? (v >> shift) & 255u : 0xffffffffu;
-        const uint32_t peers = __match_any_sync(__activemask(), bin);
-        if (in && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
+        if ((v & mask) == prefix) atomicAdd(&sh.hist[(v >> shift) & 255u], 1u);
       }
       __syncthreads();
       if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
@@ -602,9 +600,11 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       }
       cluster_sync();
       // tau among the gathered keys, then every rank's keys > tau and == tau.
-      const uint32_t lo_b = prefix, hi_b = prefix | ~mask;
-      auto value = [&](int i) -> uint32_t { return sh.gbuf[i]; };
-      cl_radix_select(value, (int)in_bin, remaining, lo_b, hi_b, sh, &tau, &take_eq);
+      {
+        const uint32_t lo_b = prefix, hi_b = prefix | ~mask;
+        auto value = [&](int i) -> uint32_t { return sh.gbuf[i]; };
+        cl_radix_select(value, (int)in_bin, remaining, lo_b, hi_b, sh, &tau, &take_eq);
+      }
       uint32_t gt_c[kTopkCl], eq_c[kTopkCl];
 #pragma unroll
       for (int c = 0; c < kTopkCl; ++c) gt_c[c] = eq_c[c] = 0u;
