@@ -63,9 +63,17 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   __shared__ __align__(16) T qraw[kProjRowBlock][128];                  // per-head query rows, 128 of d_h
   __shared__ __align__(16) T braw[128][kProjColBlock + 16 / sizeof(T)];  // basis slice (padded rows)
   constexpr int V = Vec16<T>::n;
-  pdl_wait();      // the previous call's kernels may still read this workspace
-  pdl_trigger();
   const int rank = (int)blockIdx.x, n_rank = (int)gridDim.x, cb = blockIdx.y;
+  // Programmatic launch: this kernel may start while the previous decode
+  // call's attention kernel still runs.  That kernel reads qt (and, through
+  // its predecessors, the rest of this workspace had been released before
+  // it started), so only the writes of cq / cqs / qt wait for it.  A CTA that
+  // projects a single kv group computes before waiting; one with several
+  // waits first.  The next kernel (scoring) only reads caller inputs before
+  // its own wait, so it may be released right away.
+  const bool early = (s.n_heads_kv - rank + n_rank - 1) / n_rank <= 1;
+  pdl_trigger();
+  if (!early) pdl_wait();
   const int n_rb = (int)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
   const int rb = blockIdx.z % n_rb, b = blockIdx.z / n_rb;
   const int G = s.group, W = s.query_window, Hq = s.n_heads_q, dh = s.head_dim, r = s.rank_k;
@@ -139,6 +147,7 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
           for (int j = 0; j < 4; ++j) acc[i][j] += (double)pp[i][j];
       }
     }
+    if (early) pdl_wait();   // single group: computed; now the writes
     // Per-head results of group g: qt, and PER_HEAD rows finished right here.
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
