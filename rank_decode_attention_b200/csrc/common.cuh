@@ -93,4 +93,7 @@ __device__ __forceinline__ int64_t n_candidates(int64_t L, int32_t w) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Bins of the float-exponent histogram of the candidate scores (bits 30..23).
+constexpr int kExpBins = 256;
+
 }  // namespace s4r

@@ -74,7 +74,7 @@ template <int R>
 __global__ void __launch_bounds__(kStcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
                 const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
-                unsigned int *__restrict__ bar, uint32_t *__restrict__ status) {
+                uint32_t *__restrict__ ehist, unsigned int *__restrict__ bar, uint32_t *__restrict__ status) {
   static_assert(R == 32 || R == 64, "scoring rows per CTA");
   extern __shared__ __align__(1024) unsigned char stc_smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -282,6 +282,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       ctl->alpha[t][row] = (k == 0) ? inv : ldexpf(inv, k);
     }
   }
+  // Exponent histogram of this CTA's candidate scores (rows before the
+  // local window) for the top-k kernel, in the now idle reduction scratch.
+  uint32_t *hist = reinterpret_cast<uint32_t *>(red);
+  for (int i = threadIdx.x; i < kExpBins; i += blockDim.x) hist[i] = 0u;
+  const int64_t n_cand = L > s.local_window ? L - s.local_window : 0;
   __syncthreads();
   if (epi)
     for (int t = 0; t < n_tiles; ++t) {
@@ -297,7 +302,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
         for (int j = 0; j < 32; ++j) acc = fmaf(ctl->alpha[t][c * 32 + j], __uint_as_float(ev[j]), acc);
       }
       if (pos < L) scores[(int64_t)b * s.cache_rows + pos] = acc;
+      const bool cand = pos < n_cand;
+      const uint32_t bin = cand ? (__float_as_uint(acc) >> 23) & (kExpBins - 1) : 0xffffffffu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);   // neighbours mostly share a bin
+      if (cand && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kExpBins; i += blockDim.x)
+    if (hist[i]) atomicAdd(&ehist[(int64_t)b * kExpBins + i], hist[i]);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kStcTmemCols);

@@ -390,8 +390,9 @@ struct TopkClShared {
   uint32_t g_hist[2][kTopkCl][kTopkBins];   // every rank's histogram (stored by that rank), two passes in flight
   uint32_t gbuf[kTopkGather];               // gathered keys of the final bin, rank segments in rank order
   uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau so far / in the chosen bin
+  uint32_t g_gt0[kTopkCl];                  // every rank's keys above the chosen exponent (pushed)
   uint32_t warp_tot[32];
-  uint32_t total, digit, above, gcount;
+  uint32_t total, digit, above, gcount, my_gt0;
   // The threshold, how many keys equal to it are taken overall, and this
   // rank's output offset and equal keys before it.
   uint32_t tau, take_eq, out_before, eq_before;
@@ -460,7 +461,7 @@ __device__ __forceinline__ void cl_radix_select(ValueFn value, int n, uint32_t n
 
 __global__ void __cluster_dims__(kTopkCl, 1, 1) __launch_bounds__(kTopkClThreads, 1)
 topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restrict__ keys_all,
-                    int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
+                    const uint32_t *__restrict__ ehist, int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) uint32_t tcl_dyn[];
   __shared__ TopkClShared sh;
   uint32_t *keys_s = tcl_dyn;                                   // this rank's keys (padded)
@@ -494,7 +495,10 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
                  : "memory");
   for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
   if (threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] = 0u;
-  if (threadIdx.x == 0) sh.gcount = 0u;
+  if (threadIdx.x == 0) {
+    sh.gcount = 0u;
+    sh.my_gt0 = 0u;
+  }
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
@@ -525,13 +529,38 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
 
   uint32_t prefix = 0u, mask = 0x80000000u, remaining = (uint32_t)need;
   uint32_t tau = 0u, take_eq = 0u;
-  histogram_and_store(prefix, mask, 23, 0);
-  cluster_sync();
-  for (int pass = 0;; ++pass) {
+  int first_pass = 0;
+  if (ehist != nullptr) {
+    // Pass 0 (the exponent) from the histogram the scoring kernel left for
+    // these candidates; every rank then counts its own keys above that
+    // exponent and stores the count into every rank with its pass-1 histogram.
+    if (threadIdx.x < kTopkBins) sh.hist[threadIdx.x] = __ldcg(ehist + (int64_t)b * kExpBins + threadIdx.x);
+    __syncthreads();
+    if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
+    __syncthreads();
+    const uint32_t d0 = sh.digit;
+    remaining -= sh.above;
+    prefix = d0 << 23;
+    mask |= 255u << 23;
+    uint32_t mine_gt = 0;
+    for (int i = threadIdx.x; i < my_n; i += blockDim.x) mine_gt += ((keys_s[kpad(i)] >> 23) & 255u) > d0;
+    mine_gt = warp_sum_u32(mine_gt);
+    if (lane == 0 && mine_gt) atomicAdd(&sh.my_gt0, mine_gt);
+    __syncthreads();
+    if (threadIdx.x < kTopkCl)
+      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(&sh.g_gt0[rank], threadIdx.x)), "r"(sh.my_gt0)
+                   : "memory");
+    first_pass = 1;
+  } else {
+    histogram_and_store(prefix, mask, 23, 0);
+    cluster_sync();
+  }
+  for (int pass = first_pass;; ++pass) {
     const int buf = pass & 1, shift = pass < 3 ? 23 - 8 * pass : 0;   // 23, 15, 7, 0
     if (pass > 0) {
       histogram_and_store(prefix, mask, shift, buf);
       cluster_sync();
+      if (pass == first_pass && threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] += sh.g_gt0[threadIdx.x];
     }
     // Every rank holds every rank's histogram and takes the same decisions.
     if (threadIdx.x < kTopkBins) {

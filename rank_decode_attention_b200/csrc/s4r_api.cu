@@ -35,7 +35,7 @@ inline size_t esize(s4r_dtype dt) { return dt == S4R_BF16 ? 2 : 4; }
 
 // Byte offsets of the decode workspace regions.
 struct Layout {
-  size_t status, barrier, cq, cqs, qt, tstat, rstat, rowsum, scores, pooled, total;
+  size_t status, barrier, cq, cqs, qt, tstat, rstat, rowsum, ehist, scores, pooled, total;
 };
 
 Layout layout_for(const Shape &s) {
@@ -52,6 +52,7 @@ Layout layout_for(const Shape &s) {
   l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
   l.rstat = off; off += round_up(sizeof(double) * 2 * s.batch * (size_t)s.n_rows);
   l.rowsum = off; off += round_up(sizeof(double) * s.batch * (size_t)kStcSumSlots * s.n_rows);
+  l.ehist = off; off += round_up(sizeof(uint32_t) * s.batch * (size_t)kExpBins);
   l.scores = off; off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.pooled = off; if (s.pool_kernel > 1) off += round_up(sizeof(float) * s.batch * (size_t)s.cache_rows);
   l.total = off;
@@ -217,7 +218,8 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
 
 template <int R>
 s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s, const int32_t *lengths,
-                           const unsigned char *cqs, float *scores, double *rowsum, unsigned int *bar, uint32_t *status,
+                           const unsigned char *cqs, float *scores, double *rowsum, uint32_t *ehist, unsigned int *bar,
+                           uint32_t *status,
                            cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
@@ -230,7 +232,7 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
   attr[1] = pdl_attr();
   cfg.attrs = attr;
   cfg.numAttrs = g_coop_pdl == 0 ? 1 : 2;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status);
+  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
   if (cfg.numAttrs == 2 && g_coop_pdl < 0) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     cudaStreamIsCapturing(st, &cap);
@@ -240,7 +242,7 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
       cudaGetLastError();   // not supported together: launch without it from now on
       g_coop_pdl = 0;
       cfg.numAttrs = 1;
-      err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, bar, status);
+      err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
     }
   }
   return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (cooperative launch)", err);
@@ -255,6 +257,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   double *tstat = reinterpret_cast<double *>(ws + ly.tstat);
   double *rstat = reinterpret_cast<double *>(ws + ly.rstat);
   double *rowsum = reinterpret_cast<double *>(ws + ly.rowsum);
+  uint32_t *ehist = reinterpret_cast<uint32_t *>(ws + ly.ehist);
   unsigned char *cqs = ws + ly.cqs;
   unsigned int *bar = reinterpret_cast<unsigned int *>(ws + ly.barrier);
   float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
@@ -283,7 +286,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    const cudaError_t err = cudaLaunchKernelEx(&cfg, project_kernel<T>, s, q, bk, cq, cqs, qt, rowsum, bar);
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, project_kernel<T>, s, q, bk, cq, cqs, qt, rowsum, ehist, bar);
     if (err != cudaSuccess) return fail("project_kernel (cluster launch)", err);
     if (check_launch("project_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
@@ -299,8 +302,9 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed for the key-coefficient cache");
       return S4R_ERR_CUDA;
     }
-    const s4r_status rc = plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, bar, status, st)
-                                       : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, bar, status, st);
+    const s4r_status rc =
+        plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st)
+                     : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st);
     if (rc != S4R_OK) return rc;
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
@@ -331,7 +335,10 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       cudaLaunchAttribute attr[1] = {pdl_attr()};
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      const cudaError_t err = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, s, a->lengths, keys, a->idx, status);
+      // The tensor-core scoring kernel also leaves the exponent histogram of
+      // the candidates' scores (unpooled keys only).
+      const uint32_t *kh = (plan.tc && keys == scores) ? ehist : nullptr;
+      const cudaError_t err = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, s, a->lengths, keys, kh, a->idx, status);
       if (err != cudaSuccess) return fail("topk_cluster_kernel (cluster launch)", err);
     } else {
       const size_t smem = topk_smem_bytes(s.cache_rows);

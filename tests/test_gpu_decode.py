@@ -126,3 +126,16 @@ def test_three_distinct_rows_tie_across_ranks(top_k):
     pats = synth.store(torch.randn(3, batch.coeff_k.shape[2], generator=g, dtype=torch.float64) * 0.5, "bf16")
     batch.coeff_k[0, :9000] = pats[torch.arange(9000) % 3]
     _run_exact_idx(batch)
+
+
+@pytest.mark.parametrize("rank_k,rank_v", [(136, 200), (200, 136), (64, 72)])
+def test_ranks_off_the_tensor_core_tiles(rank_k, rank_v):
+    # Ranks that are not multiples of 16 take the CUDA-core logits / value-sum
+    # paths of the attention kernel (and odd 64-column blocks of the scoring).
+    _run(make_batch(W1, lengths=[3100, 1700], rank_k=rank_k, rank_v=rank_v, top_k=300, tag="oddrank"))
+
+
+def test_many_selected_rows_take_several_chunks():
+    # k + w large enough that a CTA of the attention cluster stages its rows
+    # in more than one pass (rank 256 shrinks the staging capacity).
+    _run(make_batch(W3, lengths=[40000], top_k=3000, local_window=512, tag="chunks"))
