@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -118,6 +119,30 @@ s4r_status check_launch(const char *what) {
 }
 s4r_status last_cuda() { return check_launch("kernel launch"); }
 
+// Per-device caches of launch set-up, so that a decode call costs only its
+// launches on the host.
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : -1;
+}
+
+// Raise Kernel's dynamic shared-memory limit to `bytes` unless an earlier
+// launch on this device already raised it at least that far.
+template <auto Kernel>
+cudaError_t ensure_smem(size_t bytes) {
+  static std::atomic<int> set_to[kMaxDevices];
+  const int dev = current_device();
+  if (dev >= 0 && set_to[dev].load(std::memory_order_relaxed) >= (int)bytes) return cudaSuccess;
+  const cudaError_t err = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (err == cudaSuccess && dev >= 0) {
+    int cur = set_to[dev].load(std::memory_order_relaxed);
+    while (cur < (int)bytes && !set_to[dev].compare_exchange_weak(cur, (int)bytes)) {
+    }
+  }
+  return err;
+}
+
 // Launch attribute that lets a kernel start while the previous kernel in the
 // stream drains (its CTAs wait in pdl_wait before reading that kernel's
 // output).  Every decode kernel launched with it calls pdl_wait first.
@@ -168,7 +193,7 @@ s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const vo
       !make_tmap_bf16(&mb, basis, (uint64_t)r, (uint64_t)d, (uint64_t)r * 2, 64, kEncBK))
     return S4R_ERR_CUDA;
   const size_t smem = enc_smem_bytes(r);
-  cudaFuncSetAttribute(encode_tc_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  ensure_smem<encode_tc_kernel<bf16>>(smem);
   encode_tc_kernel<bf16><<<(unsigned)ceil_div(n, kEncBM), 128, smem, st>>>(ms, mb, static_cast<bf16 *>(coeffs),
                                                                             ldc, n, d, r);
   return last_cuda();
@@ -182,18 +207,33 @@ struct ScorePlan {
   size_t smem = 0;
 };
 
+// CTAs of the tensor-core scoring kernel that fit on the device at once
+// (cached per device and rank; 0 if they cannot be launched).
+template <int R>
+int tc_capacity(int rank) {
+  static std::atomic<int> cache[kMaxDevices][S4R_MAX_RANK / 8 + 1];   // capacity + 1; 0 = unknown
+  const int dev = current_device();
+  const int slot = rank / 8;
+  if (dev >= 0) {
+    const int c = cache[dev][slot].load(std::memory_order_relaxed);
+    if (c > 0) return c - 1;
+  }
+  const size_t smem = (size_t)stc_smem_bytes(R, rank);
+  int sms = 0, per_sm = 0, d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess ||
+      ensure_smem<score_tc_kernel<R>>(smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, kStcThreads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0) cache[dev][slot].store(per_sm * sms + 1, std::memory_order_relaxed);
+  return per_sm * sms;
+}
+
 template <int R>
 bool tc_fits(int rank, int grid, size_t *smem_out) {
-  const size_t smem = (size_t)stc_smem_bytes(R, rank);
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-  if (cudaFuncSetAttribute(score_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return false;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, kStcThreads, smem) != cudaSuccess)
-    return false;
-  *smem_out = smem;
-  return grid <= per_sm * sms;
+  *smem_out = (size_t)stc_smem_bytes(R, rank);
+  return grid <= tc_capacity<R>(rank);
 }
 
 ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
@@ -308,8 +348,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     if (rc != S4R_OK) return rc;
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
-    cudaFuncSetAttribute(score_stats_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(score_final_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem<score_stats_simt<T>>(smem);
+    ensure_smem<score_final_simt<T>>(smem);
     score_stats_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, tstat);
     score_merge<<<dim3((unsigned)ceil_div(s.n_rows, 8), s.batch), 256, 0, st>>>(s, a->lengths, tstat, rstat);
     score_final_simt<T><<<dim3(n_tiles, s.batch), kScoreThreads, smem, st>>>(s, a->lengths, ck, cq, rstat, scores);
@@ -326,7 +366,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   if (s.top_k > 0) {
     if (s.cache_rows <= (int64_t)kTopkCl * kTopkClKeys) {
       const size_t smem = topk_cl_smem_bytes();
-      cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      ensure_smem<topk_cluster_kernel>(smem);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(kTopkCl, (unsigned)s.batch);
       cfg.blockDim = dim3(kTopkClThreads);
@@ -342,7 +382,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       if (err != cudaSuccess) return fail("topk_cluster_kernel (cluster launch)", err);
     } else {
       const size_t smem = topk_smem_bytes(s.cache_rows);
-      cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      ensure_smem<topk_kernel>(smem);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)s.batch);
       cfg.blockDim = dim3(kTopkThreads);
@@ -360,7 +400,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   {
     const AttPlan pl = att_plan(s, (int)sizeof(T));
     const size_t smem = att_smem_bytes(s, (int)sizeof(T), pl);
-    cudaFuncSetAttribute(attend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem<attend_kernel<T>>(smem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)kAttCluster, (unsigned)s.n_heads_kv, (unsigned)s.batch);
     cfg.blockDim = dim3(kAttThreads);
