@@ -54,6 +54,27 @@ __device__ __forceinline__ void proj_finish(double x, int b, int R, int r, int i
   *reinterpret_cast<bf16 *>(blk + sw128_offset(2 * R + i, kk)) = lo;
 }
 
+// Per-head results of group g: qt (current query, scaled by 1/sqrt(d_h)) and,
+// for PER_HEAD rows, the finished scoring rows.
+__device__ __forceinline__ void proj_head_writes(const Shape &s, const double (&acc)[2][4], int g, int b, int pr0,
+                                                 int c0, double scale, float *cq, unsigned char *blk, float *qt) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int G = s.group, W = s.query_window, Hq = s.n_heads_q, dh = s.head_dim, r = s.rank_k, R = s.n_rows;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int row = pr0 + ty + 8 * i;
+    if (row >= W * G) continue;
+    const int w = row / G, j = row - w * G, h = g * G + j;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int kk = tx + 16 * jj, c = c0 + kk;
+      const double v = acc[i][jj];
+      if (w == W - 1 && c < r) qt[((int64_t)b * Hq + h) * r + c] = (float)(v / sqrt((double)dh));
+      if (s.row_mode == S4R_ROWS_PER_HEAD) proj_finish(c < r ? v * scale : 0.0, b, R, r, w * Hq + h, c, kk, cq, blk);
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kProjThreads)
 project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, float *__restrict__ cq,
@@ -93,6 +114,8 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   const int n_prow = W * G;  // per-head rows (w, j) of one group
   const int pr0 = rb * kProjRowBlock;
   double gsum[2][4];          // sum over this CTA's groups (CONCAT rows)
+  double keep[2][4] = {};     // the single group's results (early CTAs)
+  int g_keep = rank;
 #pragma unroll
   for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -148,54 +171,69 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
           for (int j = 0; j < 4; ++j) acc[i][j] += (double)pp[i][j];
       }
     }
-    if (early) pdl_wait();   // single group: computed; now the writes
-    // Per-head results of group g: qt, and PER_HEAD rows finished right here.
+    if (early) {
+      // Single group: keep its results; the writes wait below.
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          keep[i][jj] = acc[i][jj];
+          gsum[i][jj] += acc[i][jj];
+        }
+      g_keep = g;
+    } else {
+      proj_head_writes(s, acc, g, b, pr0, c0, scale, cq, blk, qt);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) gsum[i][jj] += acc[i][jj];
+    }
+  }
+  // CONCAT: rank 0 sums the ranks' group sums (fixed rank order).  The
+  // exchange needs nothing from the previous call, so it runs before the
+  // wait; only the stores follow it.  The group sums reuse the basis staging
+  // buffer, which is no longer read.
+  double x[2][4] = {};
+  if (s.row_mode == S4R_ROWS_CONCAT) {
+    static_assert(sizeof(double) * kProjRowBlock * kProjColBlock <= sizeof(T) * 128 * (kProjColBlock + 16 / sizeof(T)),
+                  "group sums must fit the staging buffer");
+    double(*part)[kProjColBlock] = reinterpret_cast<double(*)[kProjColBlock]>(&braw[0][0]);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) part[ty + 8 * i][tx + 16 * jj] = gsum[i][jj];
+    cluster_sync();
+    if (rank == 0) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int kk = tx + 16 * jj;
+          for (int rr = 0; rr < n_rank; ++rr) {
+            const uint32_t a = cluster_map(&part[ty + 8 * i][kk], (uint32_t)rr);
+            double v;
+            asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(a) : "memory");
+            x[i][jj] += v;
+          }
+        }
+    }
+    cluster_sync();  // rank 0 has read every partial
+  }
+  if (early) {
+    pdl_wait();
+    proj_head_writes(s, keep, g_keep, b, pr0, c0, scale, cq, blk, qt);
+  }
+  if (s.row_mode == S4R_ROWS_CONCAT && rank == 0)
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int row = pr0 + ty + 8 * i;
-      if (row >= n_prow) continue;
-      const int w = row / G, j = row - w * G, h = g * G + j;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int kk = tx + 16 * jj, c = c0 + kk;
-        const double v = acc[i][jj];
-        if (w == W - 1 && c < r) qt[((int64_t)b * Hq + h) * r + c] = (float)(v / sqrt((double)dh));
-        if (s.row_mode == S4R_ROWS_PER_HEAD) proj_finish(c < r ? v * scale : 0.0, b, R, r, w * Hq + h, c, kk, cq, blk);
-        gsum[i][jj] += v;
+        if (row < W * G) proj_finish(c < r ? x[i][jj] * scale : 0.0, b, R, r, row, c, kk, cq, blk);
       }
     }
-  }
-  if (s.row_mode != S4R_ROWS_CONCAT) return;  // no cluster barrier is used in this mode
-  // CONCAT: rank 0 sums the ranks' group sums (fixed rank order) and finishes.
-  // The group sums reuse the basis staging buffer, which is no longer read.
-  static_assert(sizeof(double) * kProjRowBlock * kProjColBlock <= sizeof(T) * 128 * (kProjColBlock + 16 / sizeof(T)),
-                "group sums must fit the staging buffer");
-  double(*part)[kProjColBlock] = reinterpret_cast<double(*)[kProjColBlock]>(&braw[0][0]);
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) part[ty + 8 * i][tx + 16 * jj] = gsum[i][jj];
-  cluster_sync();
-  if (rank == 0) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int prow = ty + 8 * i, row = pr0 + prow;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int kk = tx + 16 * jj, c = c0 + kk;
-        double x = 0.0;
-        for (int rr = 0; rr < n_rank; ++rr) {
-          const uint32_t a = cluster_map(&part[prow][kk], (uint32_t)rr);
-          double v;
-          asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(a) : "memory");
-          x += v;
-        }
-        if (row < n_prow) proj_finish(c < r ? x * scale : 0.0, b, R, r, row, c, kk, cq, blk);
-      }
-    }
-  }
-  cluster_sync();  // rank 0 has read every partial
 }
 
 }  // namespace s4r
