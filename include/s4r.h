@@ -22,6 +22,14 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls only enqueue work; none synchronises, except
  *     s4r_read_device_status.
+ *   - The kernels of consecutive decode calls on one stream overlap their
+ *     start-up (programmatic dependent launch): a call's first kernel may
+ *     begin, and read the call's inputs (queries, coefficient caches, bases,
+ *     sinks, lengths), while the previous decode call's last kernel is still
+ *     running; it touches the workspace and the outputs only after that
+ *     kernel has completed.  So the inputs of a call must be complete when
+ *     it is enqueued: written by earlier calls or copies, or by kernels that
+ *     do not release their dependents early.
  *   - Argument errors are detected on the host before anything is enqueued
  *     and returned as S4R_ERR_INVALID_ARG / S4R_ERR_UNSUPPORTED /
  *     S4R_ERR_WORKSPACE.  A failed launch returns S4R_ERR_CUDA.  Conditions
