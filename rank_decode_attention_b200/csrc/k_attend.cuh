@@ -170,22 +170,25 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
   bf16 *pb_s = reinterpret_cast<bf16 *>(f_s + 2 * kAttCluster);  // [16][ppb]
   const int ppb = att_pitch(E, 2);
   __shared__ int64_t rows_s[kAttEntriesMax];
-  __shared__ __align__(8) uint64_t stage_bar, bv_bar;
+  __shared__ __align__(8) uint64_t stage_bar, bv_bar, recv_bar;
 
   // 0. This CTA's output items and their rows of B^V[g] (inputs: the copies
   // start before the wait for the top-k kernel).
   const AttItems it = att_items(G, dh, n_ranks, (int)rank);
   const T *Bv = basis_v + (int64_t)b * Dp * rv + (int64_t)g * dh * rv;
+  const int j_lo = it.t1 > it.t0 ? it.t0 / dh : 0, j_hi = it.t1 > it.t0 ? (it.t1 - 1) / dh + 1 : 0;
   if (threadIdx.x == 0) {
     mbar_init(&stage_bar, 1);
     mbar_init(&bv_bar, 1);
+    mbar_init(&recv_bar, 1);
     mbar_fence_init();
     mbar_arrive_expect_tx(&bv_bar, (uint32_t)((it.e_hi - it.e_lo) * rv * sizeof(T)));
+    // Every rank's partial of each head finished here arrives by bulk copy.
+    mbar_arrive_expect_tx(&recv_bar, (uint32_t)(n_ranks * (j_hi - j_lo) * pr * sizeof(float)));
   }
   __syncthreads();
   for (int e = threadIdx.x; e < it.e_hi - it.e_lo; e += blockDim.x)
     bulk_load(bv_s + (size_t)e * pv, Bv + (int64_t)(it.e_lo + e) * rv, (uint32_t)(rv * sizeof(T)), &bv_bar);
-  const int j_lo = it.t1 > it.t0 ? it.t0 / dh : 0, j_hi = it.t1 > it.t0 ? (it.t1 - 1) / dh + 1 : 0;
   // The latent query (written by the projection kernel, which completed
   // before the top-k kernel started), the sink values of this CTA's output
   // columns and the sink logits of its heads: none of it depends on the
@@ -223,6 +226,8 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
       if (lane == 0) sw_s[j * kAttMaxSinks + tk] = d * qscale;
     }
   }
+  // Every rank's barriers are initialised before any rank copies into them.
+  cluster_sync();
   pdl_wait();      // idx comes from the preceding kernel
   pdl_trigger();
 
@@ -484,21 +489,26 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
     part_s[threadIdx.x * pr] = ml_s[threadIdx.x * 4];
     part_s[threadIdx.x * pr + 1] = ml_s[threadIdx.x * 4 + 1];
   }
+  // Bulk copies (the async proxy) read what the threads just wrote.
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
-  for (int r2 = 0; r2 < n_ranks; ++r2) {
+  // One copy per (rank finishing head j, head j) of this CTA's partial row.
+  if (threadIdx.x < n_ranks * 2) {
+    const int r2 = threadIdx.x >> 1, jj = threadIdx.x & 1;
     const AttItems it2 = att_items(G, dh, n_ranks, r2);
-    if (it2.t1 <= it2.t0) continue;
-    const int jlo2 = it2.t0 / dh, nh2 = (it2.t1 - 1) / dh + 1 - jlo2;
-    for (int t = threadIdx.x; t < nh2 * (pr / 4); t += blockDim.x) {
-      const int jj = t / (pr / 4), q4 = t - jj * (pr / 4);
-      const float4 v = *reinterpret_cast<const float4 *>(part_s + (jlo2 + jj) * pr + 4 * q4);
-      const uint32_t dst = cluster_map(recv_s + ((size_t)jj * kAttCluster + rank) * pr + 4 * q4, (uint32_t)r2);
-      asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v.x), "f"(v.y), "f"(v.z),
-                   "f"(v.w)
-                   : "memory");
+    if (it2.t1 > it2.t0) {
+      const int jlo2 = it2.t0 / dh, nh2 = (it2.t1 - 1) / dh + 1 - jlo2;
+      if (jj < nh2)
+        bulk_copy_to_peer(cluster_map(recv_s + ((size_t)jj * kAttCluster + rank) * pr, (uint32_t)r2),
+                          part_s + (size_t)(jlo2 + jj) * pr, (uint32_t)(pr * sizeof(float)),
+                          cluster_map(&recv_bar, (uint32_t)r2));
     }
   }
-  cluster_sync();  // every partial is in place; no distributed access follows
+  mbar_wait(&recv_bar, 0, nullptr);   // every partial of the heads finished here has arrived
+  // Every copy into this CTA is done.  A sender learns that its own copies
+  // have been read only from the receivers, so no CTA leaves before all have
+  // arrived here (the wait is at the end, after the merge and the output).
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   // Merge weights of the heads this CTA finishes (warp per head; ranks = lanes).
   for (int jj = wid; jj < j_hi - j_lo; jj += kWarps) {
     const int j = j_lo + jj;
@@ -560,6 +570,7 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
       out[((int64_t)b * s.n_heads_q + g * G + j) * dh + e] = o;
     }
   }
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Rebuild rows explicitly: out[e][d] = sum_j C[rows[e]][j] B[d][j] (fp32).
