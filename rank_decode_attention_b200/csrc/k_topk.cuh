@@ -382,15 +382,20 @@ constexpr int kTopkClThreads = 512;
 constexpr int kTopkClWarps = kTopkClThreads / 32;
 constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
 constexpr int kTopkGather = 1024;                // keys of the final bin gathered into every rank
+constexpr int kTopkHistRow = kTopkBins + 4;      // histogram row as copied: 256 bins, one count, padding
 __host__ inline size_t topk_cl_smem_bytes() { return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1); }
 
-struct TopkClShared {
+struct __align__(16) TopkClShared {
   uint32_t hist[kTopkBins];                 // summed histogram of the current pass
   uint32_t lhist[4][kTopkBins];             // this rank's histogram (warp w adds into copy w % 4)
-  uint32_t g_hist[2][kTopkCl][kTopkBins];   // every rank's histogram (stored by that rank), two passes in flight
+  uint32_t out_hist[2][kTopkHistRow];       // the summed copy sent to every rank, two passes in flight
+  uint64_t hbar[4];                         // per pass: every rank's histogram has arrived
+  // Every rank's histogram (copied in by that rank), two passes in flight.
+  // Word kTopkBins carries the sender's count of keys above the exponent
+  // chosen from the scoring kernel's histogram (pass 1 only).
+  uint32_t g_hist[2][kTopkCl][kTopkHistRow];
   uint32_t gbuf[kTopkGather];               // gathered keys of the final bin, rank segments in rank order
   uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau so far / in the chosen bin
-  uint32_t g_gt0[kTopkCl];                  // every rank's keys above the chosen exponent (pushed)
   uint32_t warp_tot[32];
   uint32_t total, digit, above, gcount, my_gt0;
   // The threshold, how many keys equal to it are taken overall, and this
@@ -465,6 +470,17 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   extern __shared__ __align__(16) uint32_t tcl_dyn[];
   __shared__ TopkClShared sh;
   uint32_t *keys_s = tcl_dyn;                                   // this rank's keys (padded)
+  // The ranks exchange histograms by bulk copies completing on per-pass
+  // mbarriers; they are initialised, and the cluster synchronised once,
+  // before waiting for the scoring kernel.
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&sh.hbar[q], 1);
+      mbar_arrive_expect_tx(&sh.hbar[q], (uint32_t)(kTopkCl * kTopkHistRow * sizeof(uint32_t)));
+    }
+    mbar_fence_init();
+  }
+  cluster_sync();
   pdl_wait();      // scores come from the preceding kernel
   pdl_trigger();
   const uint32_t rank = cluster_ctarank();
@@ -503,27 +519,28 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   __syncthreads();
 
   // This rank's histogram of the keys matching (prefix, mask) at digit
-  // `shift`, stored into slot `buf` of every rank.  Scores are >= 0, so
-  // their bit patterns order like the values and bit 31 is clear.
-  auto histogram_and_store = [&](uint32_t prefix, uint32_t mask, int shift, int buf) {
+  // `shift`, copied into slot `pass & 1` of every rank (completing on their
+  // hbar[pass]).  Scores are >= 0, so their bit patterns order like the
+  // values and bit 31 is clear.  A slot is refilled two passes later, after
+  // this rank has received the pass in between from every rank, which each
+  // rank sent only after reading the slot.
+  auto histogram_and_store = [&](uint32_t prefix, uint32_t mask, int shift, int pass) {
+    const int buf = pass & 1;
     for (int i = threadIdx.x; i < my_n; i += blockDim.x) {
       const uint32_t v = keys_s[kpad(i)];
       if ((v & mask) == prefix) atomicAdd(&sh.lhist[wid & 3][(v >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (threadIdx.x < kTopkBins) {
-      const uint32_t h = sh.lhist[0][threadIdx.x] + sh.lhist[1][threadIdx.x] + sh.lhist[2][threadIdx.x] +
-                         sh.lhist[3][threadIdx.x];
-      sh.lhist[0][threadIdx.x] = h;
-    }
+    if (threadIdx.x < kTopkBins)
+      sh.out_hist[buf][threadIdx.x] = sh.lhist[0][threadIdx.x] + sh.lhist[1][threadIdx.x] + sh.lhist[2][threadIdx.x] +
+                                      sh.lhist[3][threadIdx.x];
+    else if (threadIdx.x < kTopkHistRow)
+      sh.out_hist[buf][threadIdx.x] = threadIdx.x == kTopkBins ? sh.my_gt0 : 0u;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the copies read it through the async proxy
     __syncthreads();
-    for (int t = threadIdx.x; t < kTopkBins * kTopkCl; t += blockDim.x) {
-      const int bin = t & (kTopkBins - 1), dst = t / kTopkBins;
-      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(&sh.g_hist[buf][rank][bin], (uint32_t)dst)),
-                   "r"(sh.lhist[0][bin])
-                   : "memory");
-    }
-    __syncthreads();
+    if (threadIdx.x < kTopkCl)
+      bulk_copy_to_peer(cluster_map(&sh.g_hist[buf][rank][0], threadIdx.x), &sh.out_hist[buf][0],
+                        (uint32_t)(kTopkHistRow * sizeof(uint32_t)), cluster_map(&sh.hbar[pass], threadIdx.x));
     for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
   };
 
@@ -533,7 +550,7 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   if (ehist != nullptr) {
     // Pass 0 (the exponent) from the histogram the scoring kernel left for
     // these candidates; every rank then counts its own keys above that
-    // exponent and stores the count into every rank with its pass-1 histogram.
+    // exponent and sends the count to every rank with its pass-1 histogram.
     if (threadIdx.x < kTopkBins) sh.hist[threadIdx.x] = __ldcg(ehist + (int64_t)b * kExpBins + threadIdx.x);
     __syncthreads();
     if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
@@ -547,20 +564,17 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
     mine_gt = warp_sum_u32(mine_gt);
     if (lane == 0 && mine_gt) atomicAdd(&sh.my_gt0, mine_gt);
     __syncthreads();
-    if (threadIdx.x < kTopkCl)
-      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(&sh.g_gt0[rank], threadIdx.x)), "r"(sh.my_gt0)
-                   : "memory");
     first_pass = 1;
   } else {
     histogram_and_store(prefix, mask, 23, 0);
-    cluster_sync();
+    mbar_wait(&sh.hbar[0], 0, status);
   }
   for (int pass = first_pass;; ++pass) {
     const int buf = pass & 1, shift = pass < 3 ? 23 - 8 * pass : 0;   // 23, 15, 7, 0
     if (pass > 0) {
-      histogram_and_store(prefix, mask, shift, buf);
-      cluster_sync();
-      if (pass == first_pass && threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] += sh.g_gt0[threadIdx.x];
+      histogram_and_store(prefix, mask, shift, pass);
+      mbar_wait(&sh.hbar[pass], 0, status);
+      if (pass == first_pass && threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] += sh.g_hist[buf][threadIdx.x][kTopkBins];
     }
     // Every rank holds every rank's histogram and takes the same decisions.
     if (threadIdx.x < kTopkBins) {
@@ -660,6 +674,9 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       break;
     }
   }
+  // Every histogram copy into this rank has landed; the senders learn that
+  // theirs have been read only here, so no rank leaves before all arrive.
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   __syncthreads();
   if (threadIdx.x == 0) {
     uint32_t out_before = 0, eq_before = 0;
@@ -698,8 +715,7 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
     if (key == tau) { take = eq_seen < eq_take; ++eq_seen; }
     if (take && pos < (uint32_t)k) out[pos++] = (int32_t)(s.n_sink + i_begin + i);
   }
-  // Each rank's distributed accesses ended at its last cluster barrier, so
-  // no rank waits for the others before leaving.
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 }  // namespace s4r
