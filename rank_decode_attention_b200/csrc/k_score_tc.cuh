@@ -70,7 +70,13 @@ static_assert(stc_smem_bytes(64, 256) <= kStcMaxSmem && stc_smem_bytes(32, 256) 
 
 constexpr int kStcThreads = 160;  // warps 0-3: epilogue (one TMEM lane each); warp 4: TMA + MMA issue
 
-template <int R>
+// kMode 0: the fused single pass above (cooperative launch, grid barrier).
+// When the grid cannot be resident at once (many problems in one call), the
+// same work runs as two launches: kMode 1 adds every CTA's row sums and
+// stops; kMode 2 recomputes its tiles (identically: same operands, same
+// arithmetic, same per-tile offsets), reads the finished row sums and writes
+// the scores.  The cache is then read twice.
+template <int R, int kMode = 0>
 __global__ void __launch_bounds__(kStcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
                 const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
@@ -251,7 +257,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     __syncthreads();
   }
   // One fp64 atomic per row and CTA (both tiles belong to the same problem).
-  if (threadIdx.x < R && threadIdx.x < s.n_rows && n_tiles > 0) {
+  if (kMode != 2 && threadIdx.x < R && threadIdx.x < s.n_rows && n_tiles > 0) {
     const int row = threadIdx.x;
     double l = 0.0;
     for (int t = 0; t < n_tiles; ++t) {
@@ -261,8 +267,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + blockIdx.x % kStcSumSlots) * s.n_rows + row], l);
   }
 
-  // C: every tile of every problem has added its row sums.
-  const bool bar_ok = grid_barrier(bar, status, &ctl->flag);
+  // C: every tile of every problem has added its row sums (in kMode 2 the
+  // previous launch has).
+  bool bar_ok = true;
+  if (kMode == 0) bar_ok = grid_barrier(bar, status, &ctl->flag);
+  if (kMode != 1) {
 
   // D: scores.  l_row = sum of the row's slots (fixed order), then its
   // fp32 reciprocal.
@@ -310,6 +319,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   __syncthreads();
   for (int i = threadIdx.x; i < kExpBins; i += blockDim.x)
     if (hist[i]) atomicAdd(&ehist[(int64_t)b * kExpBins + i], hist[i]);
+  }  // kMode != 1
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kStcTmemCols);

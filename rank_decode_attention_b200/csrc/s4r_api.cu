@@ -201,7 +201,8 @@ s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const vo
 
 // Which latent-scoring kernel a decode call uses.
 struct ScorePlan {
-  bool tc = false;   // tensor-core single-pass kernel (else fp64 CUDA-core passes)
+  bool tc = false;   // tensor-core kernel (else fp64 CUDA-core passes)
+  bool two_pass = false;  // grid larger than what is resident at once: row sums, then scores
   int R = 0;         // rows per problem (template argument of the TC kernel)
   int grid = 0;
   size_t smem = 0;
@@ -230,10 +231,18 @@ int tc_capacity(int rank) {
   return per_sm * sms;
 }
 
+// 1: the fused single pass fits; 2: only the two-pass form does; 0: neither.
 template <int R>
-bool tc_fits(int rank, int grid, size_t *smem_out) {
+int tc_fits(int rank, int grid, size_t *smem_out) {
   *smem_out = (size_t)stc_smem_bytes(R, rank);
-  return grid <= tc_capacity<R>(rank);
+  const int cap = tc_capacity<R>(rank);
+  if (cap <= 0) return 0;
+  if (ensure_smem<score_tc_kernel<R, 1>>(*smem_out) != cudaSuccess ||
+      ensure_smem<score_tc_kernel<R, 2>>(*smem_out) != cudaSuccess) {
+    cudaGetLastError();
+    return grid <= cap ? 1 : 0;
+  }
+  return grid <= cap ? 1 : 2;
 }
 
 ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
@@ -242,18 +251,37 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   if (s.n_rows != 32 && s.n_rows != 64) return p;
   if ((int64_t)s.batch * s.cache_rows >= INT32_MAX) return p;
   const int64_t grid = (int64_t)s.batch * ceil_div(ceil_div(s.cache_rows, kStcTile), kStcTiles);
-  if (grid > 4096) return p;
+  if (grid > (int64_t)1 << 30) return p;
   size_t smem = 0;
-  const bool fits = s.n_rows == 64 ? tc_fits<64>(s.rank_k, (int)grid, &smem) : tc_fits<32>(s.rank_k, (int)grid, &smem);
+  const int fits = s.n_rows == 64 ? tc_fits<64>(s.rank_k, (int)grid, &smem) : tc_fits<32>(s.rank_k, (int)grid, &smem);
   if (!fits) {
     cudaGetLastError();
     return p;
   }
   p.tc = true;
+  p.two_pass = fits == 2;
   p.R = s.n_rows;
   p.grid = (int)grid;
   p.smem = smem;
   return p;
+}
+
+template <int R>
+s4r_status launch_score_tc_two_pass(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s,
+                                    const int32_t *lengths, const unsigned char *cqs, float *scores, double *rowsum,
+                                    uint32_t *ehist, unsigned int *bar, uint32_t *status, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3(kStcThreads);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R, 1>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
+  if (err != cudaSuccess) return fail("score_tc_kernel (row sums)", err);
+  err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R, 2>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
+  return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (scores)", err);
 }
 
 template <int R>
@@ -343,8 +371,11 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       return S4R_ERR_CUDA;
     }
     const s4r_status rc =
-        plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st)
-                     : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st);
+        plan.two_pass
+            ? (plan.R == 64 ? launch_score_tc_two_pass<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st)
+                            : launch_score_tc_two_pass<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st))
+            : (plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st)
+                            : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st));
     if (rc != S4R_OK) return rc;
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
@@ -437,7 +468,8 @@ int32_t s4r_decode_kernel_launches(const s4r_decode_args *args) {
   if (make_shape(args, &s) != S4R_OK) return 0;
   if (s.batch == 0) return 0;
   int32_t n = 1;                                  // projection
-  if (plan_scoring(s, args->dtype).tc) n += 1;    // scoring: one tensor-core pass
+  const ScorePlan plan = plan_scoring(s, args->dtype);
+  if (plan.tc) n += plan.two_pass ? 2 : 1;        // scoring: tensor cores, fused or row sums + scores
   else if (s.cache_rows > 0) n += 3;              // scoring: stats, merge, final
   if (s.pool_kernel > 1 && s.cache_rows > 0) n += 1;
   if (s.top_k > 0) n += 1;

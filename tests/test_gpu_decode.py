@@ -139,3 +139,38 @@ def test_many_selected_rows_take_several_chunks():
     # k + w large enough that a CTA of the attention cluster stages its rows
     # in more than one pass (rank 256 shrinks the staging capacity).
     _run(make_batch(W3, lengths=[40000], top_k=3000, local_window=512, tag="chunks"))
+
+
+def test_ragged_append_then_decode_steps():
+    """The ragged append workload over several steps: each step first appends
+    one encoded token per sequence (s4r_append on the device caches), then
+    decodes.  Appended rows match the fp64 encode within one bf16 ulp; each
+    decode is judged against the oracle run on the GPU's appended cache."""
+    import dataclasses
+    import rank_decode_attention_b200 as s4r
+    from test_gpu_encode import check_encode
+    lens = [L - 4 for L in synth.lengths(W4)]
+    batch = make_batch(W4, lengths=lens, cache_rows=max(lens) + 8, tag="append")
+    B, D = batch.batch, batch.basis_k.shape[1]
+    ck, cv = batch.coeff_k.cuda(), batch.coeff_v.cuda()
+    bk, bv = batch.basis_k.cuda(), batch.basis_v.cuda()
+    lengths = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    s4r.s4r_workspace_init(ws)
+    g = torch.Generator().manual_seed(21)
+    for step in range(3):
+        new_k = synth.store(torch.randn(B, D, generator=g, dtype=torch.float64), "bf16")
+        new_v = synth.store(torch.randn(B, D, generator=g, dtype=torch.float64), "bf16")
+        s4r.s4r_append(state_k=new_k.cuda(), state_v=new_v.cuda(), basis_k=bk, basis_v=bv,
+                       coeff_k=ck, coeff_v=cv, lengths=lengths, status_workspace=ws)
+        assert s4r.s4r_read_device_status(ws) == s4r.S4R_OK
+        Ls = lengths.cpu().tolist()
+        assert Ls == [L + step + 1 for L in lens]
+        ck_h, cv_h = ck.cpu(), cv.cpu()
+        for b in range(B):
+            row = Ls[b] - 1
+            check_encode(new_k[b:b + 1], batch.basis_k[b], ck_h[b, row:row + 1], "bf16")
+            check_encode(new_v[b:b + 1], batch.basis_v[b], cv_h[b, row:row + 1], "bf16")
+        q = synth.store(torch.randn(batch.q.shape, generator=g, dtype=torch.float64), "bf16")
+        step_batch = dataclasses.replace(batch, q=q, coeff_k=ck_h, coeff_v=cv_h, lengths=Ls)
+        _run(step_batch)
