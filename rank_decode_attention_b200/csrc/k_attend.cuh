@@ -78,9 +78,10 @@ __host__ __device__ inline AttItems att_items(int G, int dh, int n_ranks, int ra
 // so every region starts 16-byte aligned.
 __host__ __device__ inline size_t att_round4(size_t n) { return (n + 3) / 4 * 4; }
 
-// Launch plan: rows staged per pass (a multiple of 32) and B^V rows staged.
+// Launch plan: CTAs per cluster, rows staged per pass (a multiple of 32) and
+// B^V rows staged.
 struct AttPlan {
-  int e_cap, bv_rows;
+  int n_ranks, e_cap, bv_rows;
 };
 __host__ __device__ inline size_t att_float_words(const Shape &s, int e_cap, int bv_rows) {
   return (size_t)kAttMaxGroup * s.rank_k          // q_s
@@ -100,14 +101,26 @@ __host__ __device__ inline size_t att_smem_bytes(const Shape &s, int esize, cons
   const size_t bv = (size_t)pl.bv_rows * att_pitch(s.rank_v, esize) * esize;
   return rows + bv + sizeof(float) * att_float_words(s, pl.e_cap, pl.bv_rows);
 }
-__host__ inline AttPlan att_plan(const Shape &s, int esize) {
+// CTAs per (kv group, problem): enough clusters to cover about two CTAs per
+// SM, at most kAttCluster (a power of two), and at least G so that a CTA's
+// output slice spans at most two heads (its receive buffers hold two).
+__host__ inline int att_ranks(const Shape &s, int n_sms) {
+  const int64_t units = (int64_t)s.n_heads_kv * s.batch;
+  int lo = 1;
+  while (lo < s.group) lo <<= 1;
+  int n = kAttCluster;
+  while (n > lo && units * n > 2 * (int64_t)n_sms) n >>= 1;
+  return n;
+}
+__host__ inline AttPlan att_plan(const Shape &s, int esize, int n_ranks = kAttCluster) {
   AttPlan pl;
+  pl.n_ranks = n_ranks;
   pl.bv_rows = 0;
-  for (int c = 0; c < kAttCluster; ++c) {
-    const AttItems it = att_items(s.group, s.head_dim, kAttCluster, c);
+  for (int c = 0; c < n_ranks; ++c) {
+    const AttItems it = att_items(s.group, s.head_dim, n_ranks, c);
     pl.bv_rows = it.e_hi - it.e_lo > pl.bv_rows ? it.e_hi - it.e_lo : pl.bv_rows;
   }
-  const int64_t per = ceil_div((int64_t)s.top_k + s.local_window, kAttCluster);
+  const int64_t per = ceil_div((int64_t)s.top_k + s.local_window, n_ranks);
   int e = (int)smin<int64_t>(kAttEntriesMax, smax<int64_t>(32, (per + 31) / 32 * 32));
   pl.e_cap = e;
   while (pl.e_cap > 32 && att_smem_bytes(s, esize, pl) > kAttSmemBudget) pl.e_cap -= 32;

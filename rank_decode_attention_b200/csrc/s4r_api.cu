@@ -127,6 +127,23 @@ inline int current_device() {
   return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : -1;
 }
 
+// Multiprocessors of the current device (cached).
+inline int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  if (dev >= 0) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int d = 0, n = 148;
+  if (cudaGetDevice(&d) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) {
+    cudaGetLastError();
+    n = 148;
+  }
+  if (dev >= 0) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 // Raise Kernel's dynamic shared-memory limit to `bytes` unless an earlier
 // launch on this device already raised it at least that far.
 template <auto Kernel>
@@ -429,17 +446,18 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   }
   // 4. rebuild + exact attention (one cluster of CTAs per kv group)
   {
-    const AttPlan pl = att_plan(s, (int)sizeof(T));
+    AttPlan pl = att_plan(s, (int)sizeof(T), att_ranks(s, sm_count()));
+    if (att_smem_bytes(s, (int)sizeof(T), pl) > kAttSmemBudget) pl = att_plan(s, (int)sizeof(T));   // the checked plan
     const size_t smem = att_smem_bytes(s, (int)sizeof(T), pl);
     ensure_smem<attend_kernel<T>>(smem);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)kAttCluster, (unsigned)s.n_heads_kv, (unsigned)s.batch);
+    cfg.gridDim = dim3((unsigned)pl.n_ranks, (unsigned)s.n_heads_kv, (unsigned)s.batch);
     cfg.blockDim = dim3(kAttThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)kAttCluster;
+    attr[0].val.clusterDim.x = (unsigned)pl.n_ranks;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1] = pdl_attr();

@@ -174,3 +174,10 @@ def test_ragged_append_then_decode_steps():
         q = synth.store(torch.randn(batch.q.shape, generator=g, dtype=torch.float64), "bf16")
         step_batch = dataclasses.replace(batch, q=q, coeff_k=ck_h, coeff_v=cv_h, lengths=Ls)
         _run(step_batch)
+
+
+def test_many_small_problems_single_cta_clusters():
+    # G = 1 (as many query heads as kv heads) and 40 problems: the attention
+    # launch shrinks its clusters to a single CTA per (kv group, problem).
+    w = synth.Workload(**{**W1.__dict__, "n_heads_q": 8})
+    _run(make_batch(w, lengths=[600 + 37 * i for i in range(40)], top_k=64, local_window=32, tag="g1"))
