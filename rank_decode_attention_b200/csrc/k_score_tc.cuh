@@ -190,7 +190,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
           amax = valid ? fmaxf(amax, fabsf(y)) : amax;
           const float e = valid ? ex2_approx(y) : 0.f;
           ev[j] = __float_as_uint(e);
-          red[p * (R + 1) + c * 32 + j] = e;
+          if (kMode != 2) red[p * (R + 1) + c * 32 + j] = e;
         }
         tmem_st32(col0 + c * 32, hi);      // y
         tmem_st32(col0 + R + c * 32, ev);  // e
@@ -234,8 +234,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     }
     __syncthreads();
     // Row sums over the tile's 128 positions: TPR threads per row, four
-    // independent fp32 partial sums each, combined in a fixed order.
-    {
+    // independent fp32 partial sums each, combined in a fixed order (not
+    // needed when the finished sums come from the previous launch).
+    if (kMode != 2) {
       const int row = threadIdx.x % R, part = threadIdx.x / R;
       constexpr int kPer = kStcTile / TPR;
       float mine = 0.f;
