@@ -521,7 +521,8 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
   // Every copy into this CTA is done.  A sender learns that its own copies
   // have been read only from the receivers, so no CTA leaves before all have
   // arrived here (the wait is at the end, after the merge and the output).
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  // The arrive publishes no data, hence relaxed.
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   // Merge weights of the heads this CTA finishes (warp per head; ranks = lanes).
   for (int jj = wid; jj < j_hi - j_lo; jj += kWarps) {
     const int j = j_lo + jj;

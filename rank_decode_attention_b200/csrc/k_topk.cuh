@@ -364,16 +364,16 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
 // Cluster variant: the kTopkCl CTAs of a cluster split one problem's
 // candidates into contiguous shares held in shared memory.  The threshold
 // key tau is found by a radix select on the float bit patterns, one 8-bit
-// digit per pass from the exponent down:
+// digit per pass from the exponent down (bits 30-23, 22-15, 14-7, 7-0):
 //   * every rank histograms its keys that match the digits chosen so far and
-//     stores the histogram into every rank (distributed shared memory); after
-//     a cluster barrier each rank sums the ranks' histograms and takes the
-//     same decision: the digit of tau, and every rank's keys in higher bins
-//     (which are > tau);
-//   * once the chosen bin holds at most kTopkGather keys, the ranks store
-//     those keys into every rank instead (rank by rank, so each key's rank is
-//     known from its position) and each rank resolves tau among them alone;
-//   * a bin that is taken whole ends the search (tau = its lower bound - 1).
+//     copies the histogram into every rank (distributed shared memory, one
+//     bulk copy per destination completing on that pass's mbarrier); each
+//     rank then sums the ranks' histograms and takes the same decision: the
+//     digit of tau, and every rank's keys in higher bins (which are > tau);
+//   * a bin that is taken whole ends the search (tau = its lower bound - 1);
+//     otherwise the fourth pass resolves every bit of tau.
+// With the scoring kernel's exponent histogram the first pass is read, not
+// computed.  Passes cost one exchange each; no keys move between ranks.
 // Every rank then knows every rank's counts of keys > tau and == tau, hence
 // its own output offset; a stable compaction in index order writes the
 // rank's keys > tau and its share of the keys == tau (lower positions first).
@@ -381,7 +381,6 @@ constexpr int kTopkCl = 8;                       // CTAs per problem
 constexpr int kTopkClThreads = 512;
 constexpr int kTopkClWarps = kTopkClThreads / 32;
 constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
-constexpr int kTopkGather = 1024;                // keys of the final bin gathered into every rank
 constexpr int kTopkHistRow = kTopkBins + 4;      // histogram row as copied: 256 bins, one count, padding
 __host__ inline size_t topk_cl_smem_bytes() { return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1); }
 
@@ -394,10 +393,9 @@ struct __align__(16) TopkClShared {
   // Word kTopkBins carries the sender's count of keys above the exponent
   // chosen from the scoring kernel's histogram (pass 1 only).
   uint32_t g_hist[2][kTopkCl][kTopkHistRow];
-  uint32_t gbuf[kTopkGather];               // gathered keys of the final bin, rank segments in rank order
   uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau so far / in the chosen bin
   uint32_t warp_tot[32];
-  uint32_t total, digit, above, gcount, my_gt0;
+  uint32_t total, digit, above, my_gt0;
   // The threshold, how many keys equal to it are taken overall, and this
   // rank's output offset and equal keys before it.
   uint32_t tau, take_eq, out_before, eq_before;
@@ -425,43 +423,6 @@ __device__ __forceinline__ void cl_pick_digit(TopkClShared &sh, uint32_t remaini
     }
     run += cnt[j];
   }
-}
-
-// Block-wide radix select over n values of this CTA (value(i)): tau is the
-// need-th largest and take_eq how many keys equal to it are among the need
-// largest.  lo_all / hi_all bound the values (their common bits are skipped).
-template <typename ValueFn>
-__device__ __forceinline__ void cl_radix_select(ValueFn value, int n, uint32_t need, uint32_t lo_all,
-                                                uint32_t hi_all, TopkClShared &sh, uint32_t *tau, uint32_t *take_eq) {
-  const uint32_t diff = lo_all ^ hi_all;
-  int top = 31;
-  while (top >= 0 && !((diff >> top) & 1u)) --top;
-  uint32_t prefix = 0, mask = 0, remaining = need;
-  if (top < 31) {
-    const uint32_t common = (top < 0) ? 0xffffffffu : ~((2u << top) - 1u);
-    prefix = lo_all & common;
-    mask = common;
-  }
-  if (top >= 0)
-    for (int shift = (top / 8) * 8; shift >= 0; shift -= 8) {
-      for (int j = threadIdx.x; j < kTopkBins; j += blockDim.x) sh.hist[j] = 0;
-      __syncthreads();
-      // The common high bits are already fixed, so the digits of these few
-      // keys spread over the bins and plain shared atomics rarely collide.
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint32_t v = value(i);
-        if ((v & mask) == prefix) atomicAdd(&sh.hist[(v >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
-      __syncthreads();
-      remaining -= sh.above;
-      prefix |= sh.digit << shift;
-      mask |= 255u << shift;
-      __syncthreads();   // digit / above are rewritten by the next pass
-    }
-  *tau = prefix;
-  *take_eq = remaining;
 }
 
 __global__ void __cluster_dims__(kTopkCl, 1, 1) __launch_bounds__(kTopkClThreads, 1)
@@ -504,6 +465,9 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   const int chunk = (nc + kTopkCl - 1) / kTopkCl;
   const int i_begin = min(nc, (int)rank * chunk), i_end = min(nc, i_begin + chunk);
   const int my_n = i_end - i_begin;
+  // The scoring kernel's exponent histogram is read while the keys stage.
+  uint32_t eh = 0u;
+  if (ehist != nullptr && threadIdx.x < kTopkBins) eh = __ldcg(ehist + (int64_t)b * kExpBins + threadIdx.x);
   // Asynchronous 4-byte copies: every load of the share is in flight at once.
   for (int i = threadIdx.x; i < my_n; i += blockDim.x)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(keys_s + kpad(i))),
@@ -512,7 +476,6 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
   if (threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
-    sh.gcount = 0u;
     sh.my_gt0 = 0u;
   }
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -524,11 +487,19 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   // values and bit 31 is clear.  A slot is refilled two passes later, after
   // this rank has received the pass in between from every rank, which each
   // rank sent only after reading the slot.
-  auto histogram_and_store = [&](uint32_t prefix, uint32_t mask, int shift, int pass) {
+  // With exp_above < 256 the same loop also counts the keys whose exponent
+  // lies above it (into my_gt0, copied with the histogram).
+  auto histogram_and_store = [&](uint32_t prefix, uint32_t mask, int shift, int pass, uint32_t exp_above) {
     const int buf = pass & 1;
+    uint32_t above = 0u;
     for (int i = threadIdx.x; i < my_n; i += blockDim.x) {
       const uint32_t v = keys_s[kpad(i)];
       if ((v & mask) == prefix) atomicAdd(&sh.lhist[wid & 3][(v >> shift) & 255u], 1u);
+      above += ((v >> 23) & 255u) > exp_above;
+    }
+    if (exp_above < 256u) {
+      above = warp_sum_u32(above);
+      if (lane == 0 && above) atomicAdd(&sh.my_gt0, above);
     }
     __syncthreads();
     if (threadIdx.x < kTopkBins)
@@ -545,34 +516,29 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   };
 
   uint32_t prefix = 0u, mask = 0x80000000u, remaining = (uint32_t)need;
-  uint32_t tau = 0u, take_eq = 0u;
+  uint32_t tau = 0u, take_eq = 0u, exp_above = 256u;
   int first_pass = 0;
   if (ehist != nullptr) {
     // Pass 0 (the exponent) from the histogram the scoring kernel left for
-    // these candidates; every rank then counts its own keys above that
-    // exponent and sends the count to every rank with its pass-1 histogram.
-    if (threadIdx.x < kTopkBins) sh.hist[threadIdx.x] = __ldcg(ehist + (int64_t)b * kExpBins + threadIdx.x);
+    // these candidates; every rank counts its own keys above that exponent
+    // in its pass-1 histogram loop and sends the count along with it.
+    if (threadIdx.x < kTopkBins) sh.hist[threadIdx.x] = eh;
     __syncthreads();
     if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
     __syncthreads();
-    const uint32_t d0 = sh.digit;
+    exp_above = sh.digit;
     remaining -= sh.above;
-    prefix = d0 << 23;
+    prefix = exp_above << 23;
     mask |= 255u << 23;
-    uint32_t mine_gt = 0;
-    for (int i = threadIdx.x; i < my_n; i += blockDim.x) mine_gt += ((keys_s[kpad(i)] >> 23) & 255u) > d0;
-    mine_gt = warp_sum_u32(mine_gt);
-    if (lane == 0 && mine_gt) atomicAdd(&sh.my_gt0, mine_gt);
-    __syncthreads();
     first_pass = 1;
   } else {
-    histogram_and_store(prefix, mask, 23, 0);
+    histogram_and_store(prefix, mask, 23, 0, 256u);
     mbar_wait(&sh.hbar[0], 0, status);
   }
   for (int pass = first_pass;; ++pass) {
     const int buf = pass & 1, shift = pass < 3 ? 23 - 8 * pass : 0;   // 23, 15, 7, 0
     if (pass > 0) {
-      histogram_and_store(prefix, mask, shift, pass);
+      histogram_and_store(prefix, mask, shift, pass, pass == first_pass ? exp_above : 256u);
       mbar_wait(&sh.hbar[pass], 0, status);
       if (pass == first_pass && threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] += sh.g_hist[buf][threadIdx.x][kTopkBins];
     }
@@ -615,68 +581,11 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       take_eq = remaining;
       break;
     }
-    if (in_bin <= (uint32_t)kTopkGather) {
-      // Gather the bin's keys into every rank, rank by rank.
-      uint32_t seg[kTopkCl + 1];
-      seg[0] = 0u;
-#pragma unroll
-      for (int c = 0; c < kTopkCl; ++c) seg[c + 1] = seg[c] + sh.eq_acc[c];
-      uint32_t my_off = 0u;
-#pragma unroll
-      for (int c = 0; c < kTopkCl; ++c) my_off = (uint32_t)c == rank ? seg[c] : my_off;
-      for (int i0 = 0; i0 < my_n; i0 += blockDim.x) {
-        const int i = i0 + threadIdx.x;
-        const uint32_t v = i < my_n ? keys_s[kpad(i)] : 0u;
-        const bool in = i < my_n && (v & mask) == prefix;
-        const uint32_t ball = __ballot_sync(0xffffffffu, in);
-        if (ball == 0u) continue;
-        uint32_t base = 0u;
-        if (lane == 0) base = atomicAdd(&sh.gcount, (uint32_t)__popc(ball));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (in) {
-          const uint32_t pos = my_off + base + __popc(ball & ((1u << lane) - 1u));
-#pragma unroll
-          for (int dst = 0; dst < kTopkCl; ++dst)
-            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(&sh.gbuf[pos], (uint32_t)dst)), "r"(v)
-                         : "memory");
-        }
-      }
-      cluster_sync();
-      // tau among the gathered keys, then every rank's keys > tau and == tau.
-      {
-        const uint32_t lo_b = prefix, hi_b = prefix | ~mask;
-        auto value = [&](int i) -> uint32_t { return sh.gbuf[i]; };
-        cl_radix_select(value, (int)in_bin, remaining, lo_b, hi_b, sh, &tau, &take_eq);
-      }
-      uint32_t gt_c[kTopkCl], eq_c[kTopkCl];
-#pragma unroll
-      for (int c = 0; c < kTopkCl; ++c) gt_c[c] = eq_c[c] = 0u;
-      for (uint32_t i = threadIdx.x; i < in_bin; i += blockDim.x) {
-        const uint32_t v = sh.gbuf[i];
-#pragma unroll
-        for (int c = 0; c < kTopkCl; ++c) {
-          const bool mine_c = i >= seg[c] && i < seg[c + 1];
-          gt_c[c] += mine_c && v > tau;
-          eq_c[c] += mine_c && v == tau;
-        }
-      }
-      if (threadIdx.x < kTopkCl) sh.eq_acc[threadIdx.x] = 0u;
-      __syncthreads();
-#pragma unroll
-      for (int c = 0; c < kTopkCl; ++c) {
-        const uint32_t g = __reduce_add_sync(0xffffffffu, gt_c[c]);
-        const uint32_t e = __reduce_add_sync(0xffffffffu, eq_c[c]);
-        if (lane == 0) {
-          if (g) atomicAdd(&sh.gt_acc[c], g);
-          if (e) atomicAdd(&sh.eq_acc[c], e);
-        }
-      }
-      break;
-    }
   }
   // Every histogram copy into this rank has landed; the senders learn that
   // theirs have been read only here, so no rank leaves before all arrive.
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  // The arrive publishes no data, hence relaxed.
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   __syncthreads();
   if (threadIdx.x == 0) {
     uint32_t out_before = 0, eq_before = 0;
