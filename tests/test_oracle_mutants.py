@@ -82,3 +82,45 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new):
     assert src.count(old) == 1, f"mutation site of '{name}' not unique"
     res = _run_pins(_build(tmp_path, src.replace(old, new)))
     assert res.returncode == 1, f"pins did not catch: {name}\n{res.stdout[-2000:]}"
+
+
+# The basis oracle (oracle/basis.py, NumPy): mistakes planted in a copy of the
+# module, which tests/test_oracle_basis_pins.py then loads instead.
+BASIS_SRC = os.path.join(ROOT, "oracle", "basis.py")
+BASIS_MUTANTS = [
+    ("3:7 instead of 7:3", "n_recent = (7 * n + 5) // 10", "n_recent = (3 * n + 5) // 10"),
+    ("recent share rounded down", "n_recent = (7 * n + 5) // 10", "n_recent = (7 * n) // 10"),
+    ("uniform rows reach into the sinks", "uniform = [n_sink + (j * span) // n_uniform",
+     "uniform = [(j * (span + n_sink)) // n_uniform"),
+    ("recent share one row short", "recent = list(range(L - n_recent, L))", "recent = list(range(L - n_recent, L - 1))"),
+    ("normalisation dropped", "out[nz] = A[nz] / norms[nz, None]", "out[nz] = A[nz]"),
+    ("normalised by the squared norm", "out[nz] = A[nz] / norms[nz, None]", "out[nz] = A[nz] / (norms[nz, None] ** 2)"),
+    ("smallest singular directions kept", "B = sign_convention(vt[:rank].T)", "B = sign_convention(vt[-rank:].T)"),
+    ("sample transposed (left singular vectors)", "_, s, vt = np.linalg.svd(A, full_matrices=False)",
+     "_, s, vt = np.linalg.svd(A.T, full_matrices=False)"),
+    ("no sign convention", "        if B[d, k] < 0:\n", "        if False:\n"),
+]
+
+
+def _run_basis_pins(path):
+    env = dict(os.environ, S4R_BASIS_ORACLE=path)
+    return subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle_basis_pins.py"),
+                           "-x", "-q", "-p", "no:cacheprovider", "-m", "not gpu"],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+def test_basis_unmodified_copy_passes(tmp_path):
+    p = tmp_path / "basis.py"
+    p.write_text(open(BASIS_SRC).read())
+    res = _run_basis_pins(str(p))
+    assert res.returncode == 0, res.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name,old,new", BASIS_MUTANTS, ids=[m[0] for m in BASIS_MUTANTS])
+def test_basis_pins_catch_planted_mistake(tmp_path, name, old, new):
+    src = open(BASIS_SRC).read()
+    assert src.count(old) == 1, f"mutation site of '{name}' not unique"
+    p = tmp_path / "basis.py"
+    p.write_text(src.replace(old, new))
+    res = _run_basis_pins(str(p))
+    assert res.returncode == 1, f"pins did not catch: {name}\n{res.stdout[-2000:]}"
