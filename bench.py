@@ -2,7 +2,7 @@
 """S4R compressed-KV decode benchmark on B200.  Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl s4r|reference]
-                    [--workload 1] [--no-encode]
+                    [--workload 1] [--no-encode] [--no-basis]
 
 Workload (default 1): Llama-3-8B-shaped attention, 32 layers with their own
 bases, batch 1, prompt L = 32768 (4 sinks + 32764 coefficient rows), rank 192,
@@ -326,6 +326,41 @@ def run_encode_bench(w, device, reps=5):
             "peaks": src}
 
 
+def run_basis_bench(w, device, reps=3):
+    """Prefill bases for every (layer, K or V) problem of one sequence of the
+    workload: 7:3 sample of n_sample non-sink rows, unit-norm rows, top-r
+    right singular vectors in fp64 (s4r_build_basis, Eqs. 1-2)."""
+    import rank_decode_attention_b200 as s4r
+    P, L, D, r = 2 * w.layers, w.prompt_len, w.d_model, w.rank
+    states = torch.empty(P, L, D, dtype=synth.storage_dtype(w.dtype), device=device)
+    for p in range(P):
+        states[p] = synth.states(L, D, w.true_rank, w.n_sink, w.n_needles, w.needle_middle,
+                                 synth.seed_of(w.name, "basis", p), device).to(torch.float32).to(states.dtype)
+    lengths = torch.full((P,), L, dtype=torch.int32, device=device)
+    out = torch.empty(P, D, r, dtype=states.dtype, device=device)
+    a = s4r.basis_args(states=states, lengths=lengths, rank=r, n_sink=w.n_sink, n_sample=w.n_sample)
+    ws = torch.empty(s4r.s4r_basis_workspace_bytes(a), dtype=torch.uint8, device=device)
+    s4r.s4r_workspace_init(ws)
+    a = s4r.basis_args(states=states, lengths=lengths, rank=r, n_sink=w.n_sink, n_sample=w.n_sample,
+                       basis_out=out, workspace=ws)
+    s4r.s4r_build_basis(a)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        s4r.s4r_build_basis(a)
+    e1.record()
+    torch.cuda.synchronize()
+    status = s4r.s4r_read_device_status(ws)
+    t = e0.elapsed_time(e1) / reps / 1e3
+    m = min(w.n_sample, D)
+    del states
+    return {"problems": P, "n_sample": w.n_sample, "rank": r, "gram_dim": m, "ms_all_problems": t * 1e3,
+            "us_per_basis": t / P * 1e6, "status": s4r.s4r_status_string(status),
+            "timing": "CUDA events around the whole call (6 kernels: sample norms, Gram, "
+                      "cooperative Jacobi sweeps, order, columns, sign and output)"}
+
+
 def run_s4r(args, w, rank, world, local_rank):
     import rank_decode_attention_b200 as s4r
     s4r.lib()
@@ -465,6 +500,8 @@ def run_s4r(args, w, rank, world, local_rank):
     }
     if not args.no_encode:
         line["encode"] = run_encode_bench(w, device)
+    if not args.no_basis and world == 1:
+        line["basis"] = run_basis_bench(w, device)
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
@@ -481,6 +518,7 @@ def main():
     ap.add_argument("--impl", default="s4r", choices=["s4r", "reference"])
     ap.add_argument("--workload", type=int, default=1)
     ap.add_argument("--no-encode", action="store_true")
+    ap.add_argument("--no-basis", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]

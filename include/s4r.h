@@ -82,6 +82,7 @@ typedef enum { S4R_ROWS_CONCAT = 0, S4R_ROWS_PER_HEAD = 1 } s4r_row_mode;
 #define S4R_MAX_GROUP 8         /* G = n_heads_q / n_heads_kv */
 #define S4R_MAX_SINKS 16        /* n_sink */
 #define S4R_MAX_SELECTED 8192   /* top_k + local_window */
+#define S4R_MAX_BASIS_SAMPLE 1048576  /* n_sample T' of s4r_build_basis */
 
 /* ------------------------------------------------------------------ encode */
 
@@ -116,6 +117,58 @@ typedef struct {
 } s4r_append_args;
 
 s4r_status s4r_append(const s4r_append_args *args, void *stream);
+
+/* ------------------------------------------------------------------ bases */
+
+/* Build the low-rank bases at prefill ("What carries the argument" and the
+ * Referee Report's summary, Eqs. 1-2; "Core claim" for the sample): for each
+ * problem, the top-r right singular vectors of a sampled, token-wise
+ * normalised set of its non-sink states.  With L = lengths[p] (read on the
+ * device) and n = min(n_sample, L - n_sink) sample rows:
+ *   - the last (7n + 5) div 10 rows L-1, L-2, ... (0.7 n rounded half up)
+ *     and n_u = n - that many rows s + floor(j * span / n_u), j < n_u,
+ *     spread over the older non-sink rows (span = L - s - recent rows);
+ *   - every sampled row scaled to unit Euclidean norm (zero rows stay zero);
+ *   - basis column k = right singular vector of the k-th largest singular
+ *     value sigma[k], signed so that its largest-magnitude entry (lowest
+ *     index on ties) is positive.
+ * Arithmetic is fp64 throughout (the Gram matrix of the smaller side of the
+ * sample and its eigenvectors by parallel cyclic Jacobi rotations); the
+ * library owns no memory, so the caller passes a workspace of
+ * s4r_basis_workspace_bytes() bytes whose first word is the sticky device
+ * status (zero it once with s4r_workspace_init; read it with
+ * s4r_read_device_status).  The status is set (S4R_ERR_DEVICE) when a
+ * length lies outside [0, state_rows], when a sample has fewer than r rows
+ * or rank below r (a kept sigma^2 at or below 1e-13 of the largest), or when
+ * the rotations do not settle within 30 sweeps; S4R_ERR_TIMEOUT when a
+ * grid-wide wait gave up.  The outputs of such a problem are then not a
+ * basis. */
+typedef struct {
+  int32_t n_problems;     /* independent (sequence, layer, K or V) problems */
+  int32_t d_model;        /* D' (<= S4R_MAX_D_MODEL) */
+  int32_t rank;           /* r (<= min(n_sample, D', S4R_MAX_RANK)) */
+  int32_t n_sink;         /* s: leading rows never sampled */
+  int32_t n_sample;       /* T' (<= S4R_MAX_BASIS_SAMPLE) */
+  s4r_dtype dtype;        /* type of states and basis_out */
+  int64_t state_rows;     /* rows per problem in states (>= every length) */
+  const int32_t *lengths; /* [n_problems] prompt length L of each problem */
+  const void *states;     /* [n_problems][state_rows][D'] token states */
+  void *basis_out;        /* [n_problems][D'][r] in dtype (fp64 -> fp32 -> dtype,
+                             nearest even), or NULL */
+  double *basis_f64;      /* [n_problems][D'][r] fp64, or NULL (not both NULL) */
+  double *sigma;          /* [n_problems][r] singular values, or NULL */
+  void *workspace;        /* s4r_basis_workspace_bytes(args) bytes */
+  size_t workspace_bytes;
+} s4r_basis_args;
+
+/* Workspace bytes for these arguments (0 if they are invalid). */
+size_t s4r_basis_workspace_bytes(const s4r_basis_args *args);
+
+/* Enqueue the basis build (six kernels, one of them a cooperative launch).
+ * Host-side argument errors: S4R_ERR_INVALID_ARG (null or misaligned
+ * pointers, rank above n_sample or D'), S4R_ERR_UNSUPPORTED (sizes above the
+ * limits), S4R_ERR_WORKSPACE. */
+s4r_status s4r_build_basis(const s4r_basis_args *args, void *stream);
 
 /* ------------------------------------------------------------------ decode */
 

@@ -63,6 +63,17 @@ class AppendArgs(ctypes.Structure):
     ]
 
 
+class BasisArgs(ctypes.Structure):
+    _fields_ = [
+        ("n_problems", ctypes.c_int32), ("d_model", ctypes.c_int32), ("rank", ctypes.c_int32),
+        ("n_sink", ctypes.c_int32), ("n_sample", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("state_rows", ctypes.c_int64),
+        ("lengths", ctypes.c_void_p), ("states", ctypes.c_void_p), ("basis_out", ctypes.c_void_p),
+        ("basis_f64", ctypes.c_void_p), ("sigma", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 # Exported symbols and their C signatures (restype, argtypes).
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 SIGNATURES = {
@@ -73,6 +84,8 @@ SIGNATURES = {
     "s4r_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "s4r_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeArgs), _vp]),
     "s4r_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(DecodeArgs), _vp]),
+    "s4r_basis_workspace_bytes": (_sz, [ctypes.POINTER(BasisArgs)]),
+    "s4r_build_basis": (ctypes.c_int, [ctypes.POINTER(BasisArgs), _vp]),
     "s4r_reconstruct": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i32, _vp, _i64, _vp, ctypes.c_int, _vp]),
     "s4r_read_device_status": (ctypes.c_int, [_vp, _vp]),
     "s4r_clear_device_status": (ctypes.c_int, [_vp, _vp]),
@@ -204,6 +217,29 @@ def s4r_decode_step_noalloc(args: DecodeArgs, stream=None) -> int:
     workspace, nothing allocated; see include/s4r.h for its limits)."""
     return _check(lib().s4r_decode_step_noalloc(ctypes.byref(args), _stream(stream)),
                   "s4r_decode_step_noalloc")
+
+
+def basis_args(*, states, lengths, rank, n_sink, n_sample, basis_out=None, basis_f64=None, sigma=None,
+               workspace=None, workspace_bytes=None) -> BasisArgs:
+    """Fill s4r_basis_args: states [P][state_rows][D'] (bf16 or fp32), lengths
+    [P] int32 (device), outputs basis_out [P][D'][r] (states' dtype),
+    basis_f64 [P][D'][r] float64, sigma [P][r] float64."""
+    P, state_rows, d = states.shape
+    if workspace is not None and workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return BasisArgs(P, d, rank, n_sink, n_sample, _DTYPE[states.dtype], state_rows, _ptr(lengths),
+                     _ptr(states), _ptr(basis_out), _ptr(basis_f64), _ptr(sigma), _ptr(workspace),
+                     workspace_bytes or 0)
+
+
+def s4r_basis_workspace_bytes(args: BasisArgs) -> int:
+    return int(lib().s4r_basis_workspace_bytes(ctypes.byref(args)))
+
+
+def s4r_build_basis(args: BasisArgs, stream=None) -> int:
+    """Prefill bases: 7:3 sample, unit-norm rows, top-r right singular
+    vectors in fp64 (Eqs. 1-2; see include/s4r.h)."""
+    return _check(lib().s4r_build_basis(ctypes.byref(args), _stream(stream)), "s4r_build_basis")
 
 
 def s4r_reconstruct(coeffs: torch.Tensor, basis: torch.Tensor, rows: torch.Tensor,

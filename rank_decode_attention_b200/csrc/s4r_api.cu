@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "k_attend.cuh"
+#include "k_basis.cuh"
 #include "k_encode_simt.cuh"
 #include "k_encode_tc.cuh"
 #include "k_project.cuh"
@@ -471,6 +472,94 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   return last_cuda();
 }
 
+// ---- prefill bases
+struct BasisLayout {
+  size_t ctl, rows, inv, M, V, order, sig, Bw, total;
+};
+
+s4r_status basis_shape(const s4r_basis_args *a, BasisShape *bs) {
+  if (!a) return S4R_ERR_INVALID_ARG;
+  if (a->dtype != S4R_F32 && a->dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
+  if (a->n_problems < 0 || a->d_model <= 0 || a->rank <= 0 || a->n_sink < 0 || a->n_sample <= 0 ||
+      a->state_rows < 0)
+    return S4R_ERR_INVALID_ARG;
+  if (a->rank > a->n_sample || a->rank > a->d_model) return S4R_ERR_INVALID_ARG;
+  if (a->d_model > S4R_MAX_D_MODEL || a->rank > S4R_MAX_RANK || a->n_sample > S4R_MAX_BASIS_SAMPLE)
+    return S4R_ERR_UNSUPPORTED;
+  bs->P = a->n_problems;
+  bs->D = a->d_model;
+  bs->r = a->rank;
+  bs->s = a->n_sink;
+  bs->T = a->n_sample;
+  bs->t_side = a->n_sample <= a->d_model ? 1 : 0;
+  const int mm = bs->t_side ? a->n_sample : a->d_model;
+  bs->m = (mm + 1) & ~1;
+  bs->state_rows = a->state_rows;
+  return S4R_OK;
+}
+
+BasisLayout basis_layout(const BasisShape &bs) {
+  BasisLayout l;
+  const size_t P = (size_t)bs.P, m = (size_t)bs.m;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += round_up(bytes); return o; };
+  l.ctl = take(sizeof(BasisCtl));
+  l.rows = take(P * bs.T * sizeof(int64_t));
+  l.inv = take(P * bs.T * sizeof(double));
+  l.M = take(P * 2 * m * m * sizeof(double));
+  l.V = take(P * m * m * sizeof(double));
+  l.order = take(P * bs.r * sizeof(int32_t));
+  l.sig = take(P * bs.r * sizeof(double));
+  l.Bw = take(P * bs.D * bs.r * sizeof(double));
+  l.total = off;
+  return l;
+}
+
+template <typename T>
+s4r_status basis_launch(const s4r_basis_args *a, const BasisShape &bs, const BasisLayout &ly, cudaStream_t st) {
+  unsigned char *ws = static_cast<unsigned char *>(a->workspace);
+  BasisCtl *ctl = reinterpret_cast<BasisCtl *>(ws + ly.ctl);
+  int64_t *rows = reinterpret_cast<int64_t *>(ws + ly.rows);
+  double *inv = reinterpret_cast<double *>(ws + ly.inv);
+  double *M = reinterpret_cast<double *>(ws + ly.M);
+  double *V = reinterpret_cast<double *>(ws + ly.V);
+  int32_t *order = reinterpret_cast<int32_t *>(ws + ly.order);
+  double *sig = reinterpret_cast<double *>(ws + ly.sig);
+  double *Bw = reinterpret_cast<double *>(ws + ly.Bw);
+  const T *states = static_cast<const T *>(a->states);
+  const unsigned P = (unsigned)bs.P;
+  basis_prep_kernel<T><<<dim3((unsigned)ceil_div(bs.T, 8), P), 256, 0, st>>>(bs, a->lengths, states, rows, inv, ctl);
+  if (check_launch("basis_prep_kernel") != S4R_OK) return S4R_ERR_CUDA;
+  const unsigned mt = (unsigned)ceil_div(bs.m, 32);
+  basis_gram_kernel<T><<<dim3(mt, mt, P), 256, 0, st>>>(bs, states, rows, inv, M, V);
+  if (check_launch("basis_gram_kernel") != S4R_OK) return S4R_ERR_CUDA;
+  {
+    // One cooperative grid for the Jacobi rounds of every problem.
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, basis_jacobi_kernel, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+      return fail("basis_jacobi_kernel occupancy", cudaGetLastError());
+    const int64_t h = bs.m / 2;
+    const int64_t work = (int64_t)bs.P * (h * h + (int64_t)bs.m * h);
+    const int64_t want = ceil_div(work, (int64_t)256);
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
+    BasisShape bsv = bs;
+    void *kargs[] = {&bsv, &M, &V, &ctl};
+    const cudaError_t err = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(basis_jacobi_kernel),
+                                                        dim3(grid), dim3(256), kargs, 0, st);
+    if (err != cudaSuccess) return fail("basis_jacobi_kernel (cooperative launch)", err);
+  }
+  basis_order_kernel<<<P, 1024, 0, st>>>(bs, M, order, sig, a->sigma, ctl);
+  if (check_launch("basis_order_kernel") != S4R_OK) return S4R_ERR_CUDA;
+  basis_columns_kernel<T><<<dim3((unsigned)ceil_div(bs.r, 32), (unsigned)ceil_div(bs.D, 32), P), 256, 0, st>>>(
+      bs, states, rows, inv, V, order, sig, Bw);
+  if (check_launch("basis_columns_kernel") != S4R_OK) return S4R_ERR_CUDA;
+  basis_output_kernel<T><<<dim3((unsigned)bs.r, P), 256, 0, st>>>(bs, Bw, a->basis_f64,
+                                                                   static_cast<T *>(a->basis_out));
+  return check_launch("basis_output_kernel");
+}
+
 }  // namespace
 
 extern "C" {
@@ -601,6 +690,28 @@ s4r_status s4r_reconstruct(const void *coeffs, int64_t n_rows_total, const void 
                                                     static_cast<const float *>(basis), d_model, rank,
                                                     rows, n, out);
   return last_cuda();
+}
+
+size_t s4r_basis_workspace_bytes(const s4r_basis_args *args) {
+  BasisShape bs;
+  if (basis_shape(args, &bs) != S4R_OK) return 0;
+  return basis_layout(bs).total;
+}
+
+s4r_status s4r_build_basis(const s4r_basis_args *a, void *stream) {
+  BasisShape bs;
+  const s4r_status rc = basis_shape(a, &bs);
+  if (rc != S4R_OK) return rc;
+  if (bs.P == 0) return S4R_OK;
+  if (!a->lengths || !a->states || !aligned16(a->lengths) || !aligned16(a->states)) return S4R_ERR_INVALID_ARG;
+  if (!a->basis_out && !a->basis_f64) return S4R_ERR_INVALID_ARG;
+  if ((a->basis_out && !aligned16(a->basis_out)) || (a->basis_f64 && !aligned16(a->basis_f64)) ||
+      (a->sigma && !aligned16(a->sigma)))
+    return S4R_ERR_INVALID_ARG;
+  const BasisLayout ly = basis_layout(bs);
+  if (!a->workspace || !aligned16(a->workspace) || a->workspace_bytes < ly.total) return S4R_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return a->dtype == S4R_BF16 ? basis_launch<bf16>(a, bs, ly, st) : basis_launch<float>(a, bs, ly, st);
 }
 
 s4r_status s4r_read_device_status(const void *workspace, void *stream) {

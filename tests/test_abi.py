@@ -59,6 +59,9 @@ int main(void) {
   F(s4r_decode_args, cache_rows) F(s4r_decode_args, lengths) F(s4r_decode_args, out)
   F(s4r_decode_args, workspace) F(s4r_decode_args, workspace_bytes) F(s4r_decode_args, dtype)
   F(s4r_append_args, cache_rows) F(s4r_append_args, lengths) F(s4r_append_args, status_workspace)
+  printf("s4r_basis_args size %zu\n", sizeof(s4r_basis_args));
+  F(s4r_basis_args, dtype) F(s4r_basis_args, state_rows) F(s4r_basis_args, lengths) F(s4r_basis_args, sigma)
+  F(s4r_basis_args, workspace) F(s4r_basis_args, workspace_bytes)
   return 0;
 }
 '''
@@ -70,10 +73,12 @@ int main(void) {
     c = {tuple(l.split()[:2]): int(l.split()[2]) for l in lines if l}
     assert c[("s4r_decode_args", "size")] == ctypes.sizeof(s4r.DecodeArgs)
     assert c[("s4r_append_args", "size")] == ctypes.sizeof(s4r.AppendArgs)
+    assert c[("s4r_basis_args", "size")] == ctypes.sizeof(s4r.BasisArgs)
     for (T, m), off in c.items():
         if m == "size":
             continue
-        cls = s4r.DecodeArgs if T == "s4r_decode_args" else s4r.AppendArgs
+        cls = {"s4r_decode_args": s4r.DecodeArgs, "s4r_append_args": s4r.AppendArgs,
+               "s4r_basis_args": s4r.BasisArgs}[T]
         assert getattr(cls, m).offset == off, (T, m)
 
 
@@ -136,3 +141,34 @@ def test_status_strings():
     assert len(names) == 7
     assert s4r.s4r_status_string(99) == "unknown status"
     assert s4r.s4r_version() >= 100
+
+
+def basis_good(**over):
+    kw = dict(n_problems=4, d_model=1024, rank=192, n_sink=4, n_sample=256, dtype=1, state_rows=32768,
+              lengths=0x1000, states=0x2000, basis_out=0x3000, basis_f64=None, sigma=None,
+              workspace=0x4000, workspace_bytes=0)
+    kw.update(over)
+    a = s4r.BasisArgs()
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_basis_workspace_bytes_and_validation():
+    n = s4r.s4r_basis_workspace_bytes(basis_good())
+    # Gram of the 256 sampled rows: two 256 x 256 buffers and the eigenvectors per problem, plus the
+    # fp64 columns, in fp64
+    assert n >= 4 * (3 * 256 * 256 + 1024 * 192) * 8 and n % 256 == 0
+    # more samples than D': the Gram of the 1024 columns instead
+    assert s4r.s4r_basis_workspace_bytes(basis_good(n_sample=2048)) >= 4 * 3 * 1024 * 1024 * 8
+    for bad in (dict(rank=0), dict(rank=257, n_sample=300), dict(rank=300, n_sample=200), dict(dtype=7),
+                dict(d_model=0), dict(n_sample=0), dict(n_problems=-1), dict(d_model=2048),
+                dict(n_sink=-1), dict(state_rows=-5)):
+        assert s4r.s4r_basis_workspace_bytes(basis_good(**bad)) == 0, bad
+    lib = s4r.lib()
+    assert lib.s4r_build_basis(ctypes.byref(basis_good(rank=300, n_sample=200)), None) == s4r.S4R_ERR_INVALID_ARG
+    assert lib.s4r_build_basis(ctypes.byref(basis_good(d_model=2048)), None) == s4r.S4R_ERR_UNSUPPORTED
+    assert lib.s4r_build_basis(ctypes.byref(basis_good(states=0x2008)), None) == s4r.S4R_ERR_INVALID_ARG
+    assert lib.s4r_build_basis(ctypes.byref(basis_good(basis_out=None)), None) == s4r.S4R_ERR_INVALID_ARG
+    assert lib.s4r_build_basis(ctypes.byref(basis_good(workspace_bytes=64)), None) == s4r.S4R_ERR_WORKSPACE
+    assert lib.s4r_build_basis(ctypes.byref(basis_good(n_problems=0)), None) == s4r.S4R_OK
