@@ -21,9 +21,15 @@
 // eigenvectors).  Its eigenvectors come from a two-sided cyclic Jacobi
 // method in parallel rounds: the m/2 disjoint pairs of a round (round-robin
 // order, every pair once per sweep) rotate together, so M' = J^T M J splits
-// into independent 2x2 blocks R_a^T M[a][b] R_b; M is double-buffered and the
-// rounds of all problems are separated by a grid-wide barrier of one
-// cooperative launch.  A sweep without a rotation ends the iteration.
+// into independent 2x2 blocks R_a^T M[a][b] R_b.  The matrix is stored in
+// the round's slot order (pair a in slots 2a, 2a+1), so a block is two
+// 16-byte loads; each round writes its result into the other buffer already
+// in the next round's slot order, and keeps only the upper blocks' work
+// (the lower ones are their transposes).  The eigenvectors are kept as the
+// rows of V^T in the same slot order, so their rotation is a pair of
+// contiguous rows.  The rounds of all problems are separated by a grid-wide
+// barrier of one cooperative launch; a sweep without a rotation ends the
+// iteration.
 // Near the rank cut the eigenvalues of the workloads' samples differ by
 // 1e-5 .. 1e-3 of the largest, so single precision would mix kept and
 // dropped directions; fp64 keeps them apart to ~1e-10.
@@ -51,7 +57,7 @@ struct BasisShape {
 struct BasisCtl {
   uint32_t status;
   uint32_t bar;                   // grid barrier arrivals (monotone)
-  uint32_t final_buf;             // M buffer holding the converged matrix
+  uint32_t final_buf;             // buffer of M and V^T holding the converged result
   uint32_t pad;
   uint32_t rot[kBasisMaxSweeps];  // CTAs that rotated in sweep i
 };
@@ -67,20 +73,22 @@ __host__ __device__ __forceinline__ int64_t basis_sample_row(int64_t L, int64_t 
   return L - n_recent + (j - n_uniform);
 }
 
-// Pair a (< m/2) of round k (< m-1): player m-1 is fixed, the others sit on
-// a circle of m-1 places; returns p < q.
-__host__ __device__ __forceinline__ void jacobi_pair(int m, int k, int a, int &p, int &q) {
-  const int n1 = m - 1;
-  int x, y;
-  if (a == 0) {
-    x = m - 1;
-    y = k % n1;
-  } else {
-    x = (k + a) % n1;
-    y = (k - a + n1) % n1;
-  }
-  p = x < y ? x : y;
-  q = x < y ? y : x;
+// Round-robin schedule (circle method): player m-1 is fixed, the others sit
+// on a circle of n1 = m-1 places; in round k (< n1) pair 0 is (m-1, k) and
+// pair a >= 1 is ((k+a) mod n1, (k-a) mod n1).  Every pair meets once in n1
+// rounds.  Pair a occupies slots 2a (first) and 2a+1 (second).
+__host__ __device__ __forceinline__ int jac_player(int m, int k, int u) {
+  const int n1 = m - 1, a = u >> 1;
+  if ((u & 1) == 0) return a == 0 ? m - 1 : (k + a) % n1;
+  return a == 0 ? k % n1 : (k - a + n1) % n1;
+}
+__host__ __device__ __forceinline__ int jac_slot(int m, int k, int x) {
+  const int n1 = m - 1, h = m / 2;
+  if (x == m - 1) return 0;
+  const int d = ((x - k) % n1 + n1) % n1;
+  if (d == 0) return 1;
+  if (d <= h - 1) return 2 * d;
+  return 2 * (n1 - d) + 1;
 }
 
 __device__ __forceinline__ int64_t basis_n(const BasisShape &bs, const int32_t *lengths, int p) {
@@ -138,7 +146,7 @@ __device__ __forceinline__ double basis_a(const BasisShape &bs, const T *states,
   return (double)to_f(states[((int64_t)p * bs.state_rows + row) * bs.D + d]) * inv_p[j];
 }
 
-// 2. Gram matrix M (buffer 0) and V = I.  32 x 32 output tile per CTA, four
+// 2. Gram matrix M (buffer 0, slot order of round 0) and V^T = I.  32 x 32 output tile per CTA, four
 // outputs per thread, inner dimension in chunks of 32 staged in shared
 // memory.  Gram of the rows: M[i][j] = sum_d a[i][d] a[j][d]; of the
 // columns: M[i][j] = sum_t a[t][i] a[t][j].
@@ -177,14 +185,17 @@ __global__ void __launch_bounds__(256) basis_gram_kernel(BasisShape bs, const T 
     }
     __syncthreads();
   }
+  // Round 0's slot order; row slot(i) of V^T starts as e_i.
   double *Mp = M + (int64_t)p * 2 * m * m;
-  double *Vp = V + (int64_t)p * m * m;
+  double *Vp = V + (int64_t)p * 2 * m * m;
+  const int sj = (j0 + tx < m) ? jac_slot(m, 0, j0 + tx) : 0;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int i = i0 + ty + 8 * u, j = j0 + tx;
     if (i < m && j < m) {
-      Mp[(int64_t)i * m + j] = acc[u];
-      Vp[(int64_t)i * m + j] = (i == j) ? 1.0 : 0.0;
+      const int si = jac_slot(m, 0, i);
+      Mp[(int64_t)si * m + sj] = acc[u];
+      Vp[(int64_t)si * m + j] = (i == j) ? 1.0 : 0.0;
     }
   }
 }
@@ -234,73 +245,111 @@ __device__ __forceinline__ double jacobi_angle(const double *Mc, int m, int p, i
   return t;
 }
 
-// 3. Jacobi sweeps for every problem (cooperative launch).
+// Upper-triangle block t (< h(h+1)/2, row-major over a <= b) -> (a, b): a
+// single-precision root (exact operands below 2^24), then integer steps.
+__device__ __forceinline__ void upper_block(int h, int t, int &a, int &b) {
+  const float w = 2.0f * (float)h + 1.0f;
+  int x = (int)floorf((w - sqrtf(w * w - 8.0f * (float)t)) * 0.5f);
+  x = x < 0 ? 0 : (x >= h ? h - 1 : x);
+  auto start = [h](int r) { return r * h - r * (r - 1) / 2; };
+  while (x > 0 && start(x) > t) --x;
+  while (x + 1 < h && start(x + 1) <= t) ++x;
+  a = x;
+  b = x + (t - start(x));
+}
+
+// 3. Jacobi sweeps for every problem (cooperative launch).  M and V^T are
+// [P][2][m][m]; round g reads buffer g & 1 and writes the other one.  CTA c
+// owns the items [c N / G, (c+1) N / G) of the N = P (h(h+1)/2 + h m) items
+// of a round (upper blocks of M, then the rotated row pairs of V^T, problem
+// by problem), so it meets one or two problems per round and computes their
+// h rotations once, into shared memory.
 __global__ void __launch_bounds__(256) basis_jacobi_kernel(BasisShape bs, double *__restrict__ M,
                                                            double *__restrict__ V, BasisCtl *ctl) {
   __shared__ int flag_s, rot_s;
-  const int m = bs.m, h = m / 2;
+  __shared__ int ns_s[S4R_MAX_D_MODEL];            // next-round slot of the player in slot u
+  __shared__ double c_s[S4R_MAX_D_MODEL / 2], s_s[S4R_MAX_D_MODEL / 2], t_s[S4R_MAX_D_MODEL / 2];
+  const int m = bs.m, h = m / 2, n1 = m - 1;
   const int64_t mm = (int64_t)m * m;
-  const int64_t nM = (int64_t)bs.P * h * h, nV = (int64_t)bs.P * m * h;
-  const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t gstride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t nMp = (int64_t)h * (h + 1) / 2, nUp = nMp + (int64_t)h * m;   // items per problem
+  const int64_t N = (int64_t)bs.P * nUp;
+  const int64_t i_begin = N * blockIdx.x / gridDim.x, i_end = N * (blockIdx.x + 1) / gridDim.x;
   if (threadIdx.x == 0) rot_s = 0;
   uint32_t gen = 0, round = 0;
   bool converged = false;
   for (int sweep = 0; sweep < kBasisMaxSweeps && !converged; ++sweep) {
-    for (int k = 0; k < m - 1; ++k, ++round) {
+    for (int k = 0; k < n1; ++k, ++round) {
       const int cur = (int)(round & 1u);
-      for (int64_t u = gtid; u < nM + nV; u += gstride) {
-        if (u < nM) {
-          const int p = (int)(u / ((int64_t)h * h));
-          const int64_t rem = u - (int64_t)p * h * h;
-          const int a = (int)(rem / h), b = (int)(rem - (int64_t)a * h);
-          const double *Mc = M + ((int64_t)p * 2 + cur) * mm;
-          double *Mn = M + ((int64_t)p * 2 + (cur ^ 1)) * mm;
-          int pa, qa, pb, qb;
-          jacobi_pair(m, k, a, pa, qa);
-          jacobi_pair(m, k, b, pb, qb);
-          double ca, sa, app, aqq, apq;
-          const double ta = jacobi_angle(Mc, m, pa, qa, ca, sa, app, aqq, apq);
-          if (a == b) {
-            if (ta != 0.0) {
-              Mn[(int64_t)pa * m + pa] = app - ta * apq;
-              Mn[(int64_t)qa * m + qa] = aqq + ta * apq;
-              Mn[(int64_t)pa * m + qa] = 0.0;
-              Mn[(int64_t)qa * m + pa] = 0.0;
-              rot_s = 1;
+      const int kn = (k + 1) % n1;
+      for (int u = threadIdx.x; u < m; u += blockDim.x) ns_s[u] = jac_slot(m, kn, jac_player(m, k, u));
+      for (int64_t p0 = i_begin / nUp; p0 * nUp < i_end; ++p0) {
+        const int p = (int)p0;
+        const double *Mc = M + ((int64_t)p * 2 + cur) * mm;
+        double *Mn = M + ((int64_t)p * 2 + (cur ^ 1)) * mm;
+        const double *Vc = V + ((int64_t)p * 2 + cur) * mm;
+        double *Vn = V + ((int64_t)p * 2 + (cur ^ 1)) * mm;
+        __syncthreads();   // ns_s written; the previous problem's rotations consumed
+        for (int a = threadIdx.x; a < h; a += blockDim.x) {
+          double c, sn, app, aqq, apq;
+          const double t = jacobi_angle(Mc, m, 2 * a, 2 * a + 1, c, sn, app, aqq, apq);
+          c_s[a] = c;
+          s_s[a] = sn;
+          t_s[a] = t;
+          if (t != 0.0) rot_s = 1;
+        }
+        __syncthreads();
+        // Item indices within one problem stay below 2^31 (32-bit arithmetic).
+        const int lo = (int)(i_begin > p0 * nUp ? i_begin - p0 * nUp : 0);
+        const int hi = (int)(i_end < (p0 + 1) * nUp ? i_end - p0 * nUp : nUp);
+        const int nM32 = (int)nMp;
+        for (int it = lo + (int)threadIdx.x; it < hi; it += blockDim.x) {
+          if (it < nM32) {
+            int a, b;
+            upper_block(h, it, a, b);
+            const int r0 = ns_s[2 * a], r1 = ns_s[2 * a + 1];
+            const double ca = c_s[a], sa = s_s[a], ta = t_s[a];
+            if (a == b) {
+              const double app = Mc[(int64_t)(2 * a) * m + 2 * a], aqq = Mc[(int64_t)(2 * a + 1) * m + 2 * a + 1];
+              const double apq = Mc[(int64_t)(2 * a) * m + 2 * a + 1];
+              double z00 = app, z01 = apq, z10 = Mc[(int64_t)(2 * a + 1) * m + 2 * a], z11 = aqq;
+              if (ta != 0.0) {
+                z00 = app - ta * apq;
+                z11 = aqq + ta * apq;
+                z01 = z10 = 0.0;
+              }
+              Mn[(int64_t)r0 * m + r0] = z00;
+              Mn[(int64_t)r0 * m + r1] = z01;
+              Mn[(int64_t)r1 * m + r0] = z10;
+              Mn[(int64_t)r1 * m + r1] = z11;
             } else {
-              Mn[(int64_t)pa * m + pa] = app;
-              Mn[(int64_t)qa * m + qa] = aqq;
-              Mn[(int64_t)pa * m + qa] = apq;
-              Mn[(int64_t)qa * m + pa] = Mc[(int64_t)qa * m + pa];
+              const double cb = c_s[b], sb = s_s[b];
+              const double2 x0 = *reinterpret_cast<const double2 *>(Mc + (int64_t)(2 * a) * m + 2 * b);
+              const double2 x1 = *reinterpret_cast<const double2 *>(Mc + (int64_t)(2 * a + 1) * m + 2 * b);
+              // y = R_a^T x, then z = y R_b, R = [[c, s], [-s, c]].
+              const double y00 = ca * x0.x - sa * x1.x, y01 = ca * x0.y - sa * x1.y;
+              const double y10 = sa * x0.x + ca * x1.x, y11 = sa * x0.y + ca * x1.y;
+              const double z00 = y00 * cb - y01 * sb, z01 = y00 * sb + y01 * cb;
+              const double z10 = y10 * cb - y11 * sb, z11 = y10 * sb + y11 * cb;
+              const int c0 = ns_s[2 * b], c1 = ns_s[2 * b + 1];
+              Mn[(int64_t)r0 * m + c0] = z00;
+              Mn[(int64_t)r0 * m + c1] = z01;
+              Mn[(int64_t)r1 * m + c0] = z10;
+              Mn[(int64_t)r1 * m + c1] = z11;
+              Mn[(int64_t)c0 * m + r0] = z00;
+              Mn[(int64_t)c1 * m + r0] = z01;
+              Mn[(int64_t)c0 * m + r1] = z10;
+              Mn[(int64_t)c1 * m + r1] = z11;
             }
           } else {
-            double cb, sb, bpp, bqq, bpq;
-            jacobi_angle(Mc, m, pb, qb, cb, sb, bpp, bqq, bpq);
-            const double x00 = Mc[(int64_t)pa * m + pb], x01 = Mc[(int64_t)pa * m + qb];
-            const double x10 = Mc[(int64_t)qa * m + pb], x11 = Mc[(int64_t)qa * m + qb];
-            // y = R_a^T x, then z = y R_b, R = [[c, s], [-s, c]].
-            const double y00 = ca * x00 - sa * x10, y01 = ca * x01 - sa * x11;
-            const double y10 = sa * x00 + ca * x10, y11 = sa * x01 + ca * x11;
-            Mn[(int64_t)pa * m + pb] = y00 * cb - y01 * sb;
-            Mn[(int64_t)pa * m + qb] = y00 * sb + y01 * cb;
-            Mn[(int64_t)qa * m + pb] = y10 * cb - y11 * sb;
-            Mn[(int64_t)qa * m + qb] = y10 * sb + y11 * cb;
-          }
-        } else {
-          const int64_t v = u - nM;
-          const int p = (int)(v / ((int64_t)m * h));
-          const int64_t rem = v - (int64_t)p * m * h;
-          const int i = (int)(rem / h), a = (int)(rem - (int64_t)i * h);
-          const double *Mc = M + ((int64_t)p * 2 + cur) * mm;
-          int pa, qa;
-          jacobi_pair(m, k, a, pa, qa);
-          double c, s, app, aqq, apq;
-          if (jacobi_angle(Mc, m, pa, qa, c, s, app, aqq, apq) != 0.0) {
-            double *Vr = V + (int64_t)p * mm + (int64_t)i * m;
-            const double vp = Vr[pa], vq = Vr[qa];
-            Vr[pa] = c * vp - s * vq;
-            Vr[qa] = s * vp + c * vq;
+            // V' = V J on the rows of V^T: rows 2a, 2a+1 (column i) into the
+            // rows of their next slots.
+            const int v = it - nM32;
+            const int a = v / m, i = v - a * m;
+            const double c = c_s[a], sn = s_s[a];
+            const bool rot = t_s[a] != 0.0;
+            const double v0 = Vc[(int64_t)(2 * a) * m + i], v1 = Vc[(int64_t)(2 * a + 1) * m + i];
+            Vn[(int64_t)ns_s[2 * a] * m + i] = rot ? c * v0 - sn * v1 : v0;
+            Vn[(int64_t)ns_s[2 * a + 1] * m + i] = rot ? sn * v0 + c * v1 : v1;
           }
         }
       }
@@ -354,21 +403,22 @@ __global__ void __launch_bounds__(1024) basis_order_kernel(BasisShape bs, const 
 
 // 5. Unsigned basis columns Bw[d][k].  Gram of the rows: B = A^T U / sigma,
 // a 32 x 32 tile of (d, k) per CTA over the sample rows in chunks of 32;
-// Gram of the columns: B[d][k] = V[d][order[k]].
+// Gram of the columns: B[d][k] = V^T[order[k]][d].
 template <typename T>
 __global__ void __launch_bounds__(256) basis_columns_kernel(BasisShape bs, const T *__restrict__ states,
                                                             const int64_t *__restrict__ rows,
                                                             const double *__restrict__ inv,
                                                             const double *__restrict__ V,
                                                             const int32_t *__restrict__ order,
-                                                            const double *__restrict__ sig, double *__restrict__ Bw) {
+                                                            const double *__restrict__ sig, const BasisCtl *ctl,
+                                                            double *__restrict__ Bw) {
   __shared__ double a_s[32][33], u_s[32][33];
   __shared__ int ord_s[32];
   const int p = blockIdx.z;
   const int d0 = blockIdx.y * 32, k0 = blockIdx.x * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int m = bs.m;
-  const double *Vp = V + (int64_t)p * m * m;
+  const double *Vp = V + ((int64_t)p * 2 + ctl->final_buf) * m * m;   // V^T, rows in slot order
   if (threadIdx.x < 32) ord_s[threadIdx.x] = (k0 + threadIdx.x < bs.r) ? order[(int64_t)p * bs.r + k0 + threadIdx.x] : 0;
   __syncthreads();
   double *Bp = Bw + (int64_t)p * bs.D * bs.r;
@@ -376,7 +426,7 @@ __global__ void __launch_bounds__(256) basis_columns_kernel(BasisShape bs, const
     for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
       const int dd = e >> 5, kk = e & 31;
       const int d = d0 + dd, k = k0 + kk;
-      if (d < bs.D && k < bs.r) Bp[(int64_t)d * bs.r + k] = Vp[(int64_t)d * m + ord_s[kk]];
+      if (d < bs.D && k < bs.r) Bp[(int64_t)d * bs.r + k] = Vp[(int64_t)ord_s[kk] * m + d];
     }
     return;
   }
@@ -385,9 +435,9 @@ __global__ void __launch_bounds__(256) basis_columns_kernel(BasisShape bs, const
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int j0 = 0; j0 < bs.T; j0 += 32) {
     for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
-      const int jj = e >> 5, x = e & 31;
-      a_s[x][jj] = basis_a(bs, states, rows_p, inv_p, p, j0 + jj, d0 + x);      // consecutive threads walk d
-      u_s[jj][x] = (j0 + jj < m && k0 + x < bs.r) ? Vp[(int64_t)(j0 + jj) * m + ord_s[x]] : 0.0;
+      const int hi = e >> 5, lo = e & 31;
+      a_s[lo][hi] = basis_a(bs, states, rows_p, inv_p, p, j0 + hi, d0 + lo);     // consecutive threads walk d
+      u_s[lo][hi] = (j0 + lo < m && k0 + hi < bs.r) ? Vp[(int64_t)ord_s[hi] * m + j0 + lo] : 0.0;   // ... and j
     }
     __syncthreads();
 #pragma unroll 8

@@ -507,7 +507,7 @@ BasisLayout basis_layout(const BasisShape &bs) {
   l.rows = take(P * bs.T * sizeof(int64_t));
   l.inv = take(P * bs.T * sizeof(double));
   l.M = take(P * 2 * m * m * sizeof(double));
-  l.V = take(P * m * m * sizeof(double));
+  l.V = take(P * 2 * m * m * sizeof(double));
   l.order = take(P * bs.r * sizeof(int32_t));
   l.sig = take(P * bs.r * sizeof(double));
   l.Bw = take(P * bs.D * bs.r * sizeof(double));
@@ -540,7 +540,7 @@ s4r_status basis_launch(const s4r_basis_args *a, const BasisShape &bs, const Bas
         per_sm < 1)
       return fail("basis_jacobi_kernel occupancy", cudaGetLastError());
     const int64_t h = bs.m / 2;
-    const int64_t work = (int64_t)bs.P * (h * h + (int64_t)bs.m * h);
+    const int64_t work = (int64_t)bs.P * (h * (h + 1) / 2 + (int64_t)bs.m * h);
     const int64_t want = ceil_div(work, (int64_t)256);
     const int64_t cap = (int64_t)per_sm * sm_count();
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
@@ -553,7 +553,7 @@ s4r_status basis_launch(const s4r_basis_args *a, const BasisShape &bs, const Bas
   basis_order_kernel<<<P, 1024, 0, st>>>(bs, M, order, sig, a->sigma, ctl);
   if (check_launch("basis_order_kernel") != S4R_OK) return S4R_ERR_CUDA;
   basis_columns_kernel<T><<<dim3((unsigned)ceil_div(bs.r, 32), (unsigned)ceil_div(bs.D, 32), P), 256, 0, st>>>(
-      bs, states, rows, inv, V, order, sig, Bw);
+      bs, states, rows, inv, V, order, sig, ctl, Bw);
   if (check_launch("basis_columns_kernel") != S4R_OK) return S4R_ERR_CUDA;
   basis_output_kernel<T><<<dim3((unsigned)bs.r, P), 256, 0, st>>>(bs, Bw, a->basis_f64,
                                                                    static_cast<T *>(a->basis_out));
