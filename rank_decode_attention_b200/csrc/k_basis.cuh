@@ -28,8 +28,9 @@
 // (the lower ones are their transposes).  The eigenvectors are kept as the
 // rows of V^T in the same slot order, so their rotation is a pair of
 // contiguous rows.  The rounds of all problems are separated by a grid-wide
-// barrier of one cooperative launch; a sweep without a rotation ends the
-// iteration.
+// barrier of one cooperative launch.  The sweep in which every pair meets
+// an off-diagonal entry below 1e-8 of its diagonal scale is the last one:
+// its rotations leave them near their squares.
 // Near the rank cut the eigenvalues of the workloads' samples differ by
 // 1e-5 .. 1e-3 of the largest, so single precision would mix kept and
 // dropped directions; fp64 keeps them apart to ~1e-10.
@@ -41,6 +42,9 @@ namespace s4r {
 
 constexpr int kBasisMaxSweeps = 30;
 constexpr double kJacobiTol = 1e-12;   // rotate while |a_pq| > tol * sqrt(a_pp a_qq)
+// A sweep in which no pair starts above this relative size leaves every
+// off-diagonal entry near its square (quadratic convergence): the last sweep.
+constexpr double kJacobiLastSweep = 1e-8;
 
 struct BasisShape {
   int32_t P;         // problems
@@ -59,7 +63,7 @@ struct BasisCtl {
   uint32_t bar;                   // grid barrier arrivals (monotone)
   uint32_t final_buf;             // buffer of M and V^T holding the converged result
   uint32_t pad;
-  uint32_t rot[kBasisMaxSweeps];  // CTAs that rotated in sweep i
+  uint32_t rot[kBasisMaxSweeps];  // CTAs that met a pair above kJacobiLastSweep in sweep i
 };
 
 // Row of sample j (< n) of a problem with L rows ("Core claim", 7:3 split).
@@ -219,6 +223,7 @@ __device__ __forceinline__ bool basis_grid_sync(BasisCtl *ctl, uint32_t gen, int
         ok = 0;
         break;
       }
+      __nanosleep(64);   // fewer polls on the counter line while the arrivals land
     }
     *flag_smem = ok;
   }
@@ -295,7 +300,7 @@ __global__ void __launch_bounds__(256) basis_jacobi_kernel(BasisShape bs, double
           c_s[a] = c;
           s_s[a] = sn;
           t_s[a] = t;
-          if (t != 0.0) rot_s = 1;
+          if (t != 0.0 && fabs(apq) > kJacobiLastSweep * sqrt(fabs(app) * fabs(aqq))) rot_s = 1;
         }
         __syncthreads();
         // Item indices within one problem stay below 2^31 (32-bit arithmetic).
