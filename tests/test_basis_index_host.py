@@ -1,0 +1,85 @@
+"""Index arithmetic of the GPU basis build, checked on the CPU.
+
+The sample-row formula, the round-robin (circle) schedule of the Jacobi
+rounds and the slot maps of k_basis.cuh are __host__ __device__ functions.
+This test compiles them into a host-only program with nvcc (no GPU needed)
+and checks them bit-exactly: the sampled rows against the basis oracle
+(oracle/basis.py, an independent implementation of the 7:3 rule), and the
+schedule against its definition (every pair of m players meets exactly once
+in m - 1 rounds, the pairs of a round are disjoint, and the slot map of a
+round inverts its player map).
+"""
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import basis as obasis
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "rank_decode_attention_b200", "csrc")
+
+PROG = r'''
+#include <cstdio>
+#include <cstdlib>
+#include "umma.cuh"
+#include "k_basis.cuh"
+using namespace s4r;
+int main(int argc, char **argv) {
+  if (argv[1][0] == 'r') {            // r L s T: the sampled rows
+    const long long L = atoll(argv[2]), s = atoll(argv[3]), T = atoll(argv[4]);
+    const long long avail = L - s > 0 ? L - s : 0, n = avail < T ? avail : T;
+    for (long long j = 0; j < n; ++j) printf("%lld\n", (long long)basis_sample_row(L, s, n, j));
+    return 0;
+  }
+  const int m = atoi(argv[2]);        // p m: players of every slot of every round, then slots
+  for (int k = 0; k < m - 1; ++k)
+    for (int u = 0; u < m; ++u) {
+      const int x = jac_player(m, k, u);
+      printf("%d %d %d %d\n", k, u, x, jac_slot(m, k, x));
+    }
+  return 0;
+}
+'''
+
+
+@pytest.fixture(scope="module")
+def exe(tmp_path_factory):
+    if shutil.which("nvcc") is None:
+        pytest.skip("nvcc not available")
+    d = tmp_path_factory.mktemp("basis_host")
+    src, out = d / "idx.cu", d / "idx"
+    src.write_text(PROG)
+    subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-std=c++17", "-O1",
+                    "-I", os.path.join(ROOT, "include"), "-I", CSRC,
+                    "-o", str(out), str(src)], check=True, capture_output=True)
+    return str(out)
+
+
+@pytest.mark.parametrize("L,s,T", [(20, 4, 10), (14, 4, 10), (100, 0, 5), (9, 4, 10), (50, 4, 1), (50, 4, 2),
+                                   (50, 4, 3), (4, 4, 8), (1000, 4, 20), (32768, 4, 256), (8192, 4, 512),
+                                   (700, 4, 512), (131072, 4, 256), (2048, 4, 256), (5, 4, 3)])
+def test_sample_rows_match_the_oracle(exe, L, s, T):
+    out = subprocess.run([exe, "r", str(L), str(s), str(T)], capture_output=True, text=True, check=True).stdout
+    gpu_rows = [int(v) for v in out.split()]
+    assert gpu_rows == obasis.sample_rows(L, s, T).tolist()
+
+
+@pytest.mark.parametrize("m", [2, 4, 6, 38, 256, 1024])
+def test_round_robin_schedule_and_slot_maps(exe, m):
+    out = subprocess.run([exe, "p", str(m)], capture_output=True, text=True, check=True).stdout
+    rec = np.array([[int(v) for v in line.split()] for line in out.splitlines()])
+    assert rec.shape == ((m - 1) * m, 4)
+    seen = set()
+    for k in range(m - 1):
+        r = rec[rec[:, 0] == k]
+        players = r[np.argsort(r[:, 1]), 2]
+        assert sorted(players.tolist()) == list(range(m))                  # a permutation of the players
+        assert (r[:, 3] == r[:, 1]).all()                                   # slot map inverts player map
+        for a in range(m // 2):
+            pair = tuple(sorted((int(players[2 * a]), int(players[2 * a + 1]))))
+            assert pair not in seen
+            seen.add(pair)
+    assert len(seen) == m * (m - 1) // 2                                    # every pair once per sweep
