@@ -145,7 +145,7 @@ def test_ragged_append_then_decode_steps():
     """The ragged append workload over several steps: each step first appends
     one encoded token per sequence (s4r_append on the device caches), then
     decodes.  Appended rows match the fp64 encode within one bf16 ulp; each
-    decode is judged against the oracle run on the GPU's appended cache."""
+    decode is compared with the oracle run on the GPU's appended cache."""
     import dataclasses
     import rank_decode_attention_b200 as s4r
     from test_gpu_encode import check_encode
