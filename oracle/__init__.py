@@ -26,6 +26,8 @@ _LIB = os.path.join(_HERE, "_build", "libs4r_oracle.so")
 
 ROWS_CONCAT = 0
 ROWS_PER_HEAD = 1
+POOL_MAX = 0
+POOL_AVG = 1
 
 
 def build(force: bool = False) -> str:
@@ -50,7 +52,7 @@ class _Problem(ctypes.Structure):
         ("rank_k", ctypes.c_int32), ("rank_v", ctypes.c_int32),
         ("n_sink", ctypes.c_int32), ("local_window", ctypes.c_int32), ("top_k", ctypes.c_int32),
         ("query_window", ctypes.c_int32), ("pool_kernel", ctypes.c_int32),
-        ("row_mode", ctypes.c_int32),
+        ("row_mode", ctypes.c_int32), ("pool_mode", ctypes.c_int32),
         ("n_coeff", ctypes.c_int64),
         ("q", ctypes.c_void_p), ("coeff_k", ctypes.c_void_p), ("coeff_v", ctypes.c_void_p),
         ("basis_k", ctypes.c_void_p), ("basis_v", ctypes.c_void_p),
@@ -74,7 +76,7 @@ def _load():
         lib.s4r_oracle_reconstruct.argtypes = [dp, ctypes.c_int64, ctypes.c_int32, dp, ctypes.c_int32, dp]
         lib.s4r_oracle_reconstruct.restype = None
         lib.s4r_oracle_scores.argtypes = [P, dp]
-        lib.s4r_oracle_pool.argtypes = [dp, ctypes.c_int64, ctypes.c_int32, dp]
+        lib.s4r_oracle_pool.argtypes = [dp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, dp]
         lib.s4r_oracle_select.argtypes = [P, dp, dp]
         lib.s4r_oracle_decode_given_idx.argtypes = [P, dp, ctypes.c_int64, dp]
         lib.s4r_oracle_decode_step.argtypes = [P, dp, dp, dp]
@@ -113,6 +115,7 @@ class Problem:
     top_k: int
     pool_kernel: int = 1
     row_mode: int = ROWS_CONCAT
+    pool_mode: int = POOL_MAX
 
     def __post_init__(self):
         for name in ("q", "coeff_k", "coeff_v", "basis_k", "basis_v", "sink_k", "sink_v"):
@@ -133,7 +136,7 @@ class Problem:
     def _c(self) -> _Problem:
         return _Problem(self.n_heads_q, self.n_heads_kv, self.head_dim, self.rank_k, self.rank_v,
                         self.n_sink, self.local_window, self.top_k, self.query_window,
-                        self.pool_kernel, self.row_mode, self.n_coeff,
+                        self.pool_kernel, self.row_mode, self.pool_mode, self.n_coeff,
                         _ptr(self.q), _ptr(self.coeff_k), _ptr(self.coeff_v), _ptr(self.basis_k),
                         _ptr(self.basis_v), _ptr(self.sink_k), _ptr(self.sink_v))
 
@@ -171,10 +174,11 @@ def scores(p: Problem) -> np.ndarray:
     return out[: p.n_coeff]
 
 
-def pool(score_vec, n_cand: int, kernel: int) -> np.ndarray:
+def pool(score_vec, n_cand: int, kernel: int, mode: int = POOL_MAX) -> np.ndarray:
+    """Pooled candidate scores: max or mean over the in-range neighbours."""
     s = _f64(score_vec)
     out = np.empty(max(n_cand, 1), dtype=np.float64)
-    _check(_load().s4r_oracle_pool(_ptr(s), n_cand, kernel, _ptr(out)), "pool")
+    _check(_load().s4r_oracle_pool(_ptr(s), n_cand, kernel, mode, _ptr(out)), "pool")
     return out[:n_cand]
 
 

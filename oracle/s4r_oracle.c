@@ -62,6 +62,7 @@ static int check_problem(const s4r_oracle_problem *p) {
   if (p->rank_k <= 0 || p->rank_v <= 0 || p->query_window <= 0) return -1;
   if (p->n_sink < 0 || p->local_window < 0 || p->top_k < 0 || p->n_coeff < 0) return -1;
   if (p->pool_kernel < 1 || (p->pool_kernel > 1 && p->pool_kernel % 2 == 0)) return -1;
+  if (p->pool_mode != S4R_ORACLE_POOL_MAX && p->pool_mode != S4R_ORACLE_POOL_AVG) return -1;
   if (p->row_mode != S4R_ORACLE_ROWS_CONCAT && p->row_mode != S4R_ORACLE_ROWS_PER_HEAD) return -1;
   return 0;
 }
@@ -153,16 +154,27 @@ int s4r_oracle_scores(const s4r_oracle_problem *p, double *scores) {
 }
 
 /* Score pooling with kernel kappa ("free parameters": pooling kernel 7, taken
- * from SnapKV).  READING: max-pool, stride 1, same padding, over the
- * candidate positions only; kappa must be odd. */
-int s4r_oracle_pool(const double *scores, int64_t n_cand, int32_t pool_kernel, double *pooled) {
+ * from SnapKV; the referee report lists the pooling/aggregation choices as
+ * open).  READING: stride 1, same padding, over the candidate positions only;
+ * kappa must be odd.  The window of position i is j = i - kappa/2 ..
+ * i + kappa/2; neighbours outside [0, n_cand) are left out, so
+ *   POOL_MAX: pooled[i] = max of scores[j] over the in-range j,
+ *   POOL_AVG: pooled[i] = (sum of scores[j] over the in-range j) / (their count). */
+int s4r_oracle_pool(const double *scores, int64_t n_cand, int32_t pool_kernel, int32_t pool_mode,
+                    double *pooled) {
   if (pool_kernel < 1 || pool_kernel % 2 == 0) return -1;
+  if (pool_mode != S4R_ORACLE_POOL_MAX && pool_mode != S4R_ORACLE_POOL_AVG) return -1;
   const int64_t half = pool_kernel / 2;
   for (int64_t i = 0; i < n_cand; ++i) {
-    double m = -INFINITY;
+    double m = -INFINITY, sum = 0.0;
+    int64_t count = 0;
     for (int64_t j = i - half; j <= i + half; ++j)
-      if (j >= 0 && j < n_cand) m = fmax(m, scores[j]);
-    pooled[i] = m;
+      if (j >= 0 && j < n_cand) {
+        m = fmax(m, scores[j]);
+        sum += scores[j];
+        count += 1;
+      }
+    pooled[i] = (pool_mode == S4R_ORACLE_POOL_MAX) ? m : sum / (double)count;
   }
   return 0;
 }
@@ -203,7 +215,7 @@ int s4r_oracle_select(const s4r_oracle_problem *p, const double *scores, int32_t
   if (p->pool_kernel > 1) {
     pooled = (double *)malloc(sizeof(double) * n_cand);
     if (!pooled) return -3;
-    s4r_oracle_pool(scores, n_cand, p->pool_kernel, pooled);
+    s4r_oracle_pool(scores, n_cand, p->pool_kernel, p->pool_mode, pooled);
     rank_by = pooled;
   }
   keyed *all = (keyed *)malloc(sizeof(keyed) * n_cand);

@@ -28,6 +28,11 @@ extern "C" {
 #endif
 
 enum {
+  S4R_ORACLE_POOL_MAX = 0,      /* pooled score = largest neighbour score */
+  S4R_ORACLE_POOL_AVG = 1       /* pooled score = mean of the in-range neighbour scores */
+};
+
+enum {
   S4R_ORACLE_ROWS_CONCAT = 0,   /* W*G rows, heads of one GQA slot concatenated to D' */
   S4R_ORACLE_ROWS_PER_HEAD = 1  /* W*H_q rows, each head projected with its own slice */
 };
@@ -37,6 +42,7 @@ typedef struct {
   int32_t rank_k, rank_v;
   int32_t n_sink, local_window, top_k, query_window, pool_kernel;
   int32_t row_mode;             /* S4R_ORACLE_ROWS_* */
+  int32_t pool_mode;            /* S4R_ORACLE_POOL_* (used when pool_kernel > 1) */
   int64_t n_coeff;              /* L_c */
   const double *q;              /* [W][H_q][d_h]; row W-1 is the current query */
   const double *coeff_k;        /* [L_c][rank_k] */
@@ -59,10 +65,11 @@ void s4r_oracle_reconstruct(const double *C, int64_t n, int32_t r,
  * Returns 0, or -1 on invalid shapes. */
 int s4r_oracle_scores(const s4r_oracle_problem *p, double *scores);
 
-/* Max-pool of candidate scores with an odd window pool_kernel (stride 1,
- * same padding, candidates only); pooled[n_cand]. */
+/* Pooling of candidate scores with an odd window pool_kernel (stride 1,
+ * same padding, candidates only): the largest (POOL_MAX) or the mean
+ * (POOL_AVG) of the neighbours that lie inside [0, n_cand); pooled[n_cand]. */
 int s4r_oracle_pool(const double *scores, int64_t n_cand, int32_t pool_kernel,
-                    double *pooled);
+                    int32_t pool_mode, double *pooled);
 
 /* Top-k global positions (Eqs. 13-15): idx[top_k] = absolute positions,
  * ascending, -1 padded.  Ranking uses the pooled scores when pool_kernel > 1. */

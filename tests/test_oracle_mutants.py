@@ -45,6 +45,11 @@ MUTANTS = [
     ("attention uses the oldest window slot", "const double *q = p->q + ((int64_t)(W - 1) * Hq + h) * dh;",
      "const double *q = p->q + ((int64_t)0 * Hq + h) * dh;"),
     ("pool window one wider", "const int64_t half = pool_kernel / 2;", "const int64_t half = pool_kernel / 2 + 1;"),
+    ("average pool counts the padding", "sum / (double)count;", "sum / (double)pool_kernel;"),
+    ("average pool takes the maximum", "(pool_mode == S4R_ORACLE_POOL_MAX) ? m : sum / (double)count;",
+     "m;"),
+    ("average pool leaves out the right neighbours", "for (int64_t j = i - half; j <= i + half; ++j)",
+     "for (int64_t j = i - half; j <= i + (pool_mode == S4R_ORACLE_POOL_MAX ? half : 0); ++j)"),
     ("per-head rows use group 0's basis slice",
      "acc += p->q[((int64_t)w * Hq + h) * dh + t] * p->basis_k[(int64_t)(g * dh + t) * r + k];",
      "acc += p->q[((int64_t)w * Hq + h) * dh + t] * p->basis_k[(int64_t)(t) * r + k];"),

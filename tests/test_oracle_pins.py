@@ -10,7 +10,8 @@ Long-Context KV Caching", arXiv 2608.00528) fix:
   scoring (Eqs. 8-10)      -> torch SDPA weights (value = identity) when the
                               basis is a full rotation; conservation; rotation
                               invariance; single-row monotone reduction
-  pooling                  -> torch max_pool1d
+  pooling                  -> torch max_pool1d / avg_pool1d (padding left out of
+                              the count); a hand-worked average
   selection (Eqs. 13-15)   -> numpy stable lexsort brute force, forced ties
   attention (Eqs. 16-18)   -> torch SDPA (GQA) over all keys when nothing is
                               dropped; sinks-only case; convexity
@@ -36,7 +37,7 @@ def rand_orthonormal(rng, rows, cols):
 
 
 def make_problem(rng, *, W=3, Hq=4, Hkv=2, dh=8, r=None, L=40, s=2, w=5, k=6, pool=1,
-                 row_mode=oracle.ROWS_CONCAT, full_rank=False):
+                 row_mode=oracle.ROWS_CONCAT, full_rank=False, pool_mode=oracle.POOL_MAX):
     Dp = Hkv * dh
     r = Dp if full_rank else (r or 6)
     K = rng.standard_normal((L, Dp))
@@ -48,7 +49,7 @@ def make_problem(rng, *, W=3, Hq=4, Hkv=2, dh=8, r=None, L=40, s=2, w=5, k=6, po
     p = oracle.Problem(q=rng.standard_normal((W, Hq, dh)), coeff_k=K @ Bk, coeff_v=V @ Bv,
                        basis_k=Bk, basis_v=Bv, sink_k=rng.standard_normal((s, Dp)),
                        sink_v=rng.standard_normal((s, Dp)), n_heads_kv=Hkv, local_window=w,
-                       top_k=k, pool_kernel=pool, row_mode=row_mode)
+                       top_k=k, pool_kernel=pool, row_mode=row_mode, pool_mode=pool_mode)
     return p, K, V
 
 
@@ -150,6 +151,25 @@ def test_pool_matches_torch_max_pool(kernel):
     np.testing.assert_array_equal(oracle.pool(s, s.size, kernel), want)
 
 
+@pytest.mark.parametrize("kernel", [3, 7])
+def test_avg_pool_matches_torch_avg_pool_without_padding_in_the_count(kernel):
+    rng = np.random.default_rng(18)
+    s = rng.random(41)
+    want = F.avg_pool1d(torch.from_numpy(s)[None, None], kernel, stride=1, padding=kernel // 2,
+                        count_include_pad=False)[0, 0].numpy()
+    np.testing.assert_allclose(oracle.pool(s, s.size, kernel, oracle.POOL_AVG), want, rtol=1e-15, atol=0)
+
+
+def test_avg_pool_hand_worked():
+    # kappa = 3 over [1, 2, 3, 4, 5]: the ends average two in-range neighbours,
+    # (1 + 2) / 2 and (4 + 5) / 2; the middle ones three.
+    got = oracle.pool(np.array([1.0, 2.0, 3.0, 4.0, 5.0]), 5, 3, oracle.POOL_AVG)
+    np.testing.assert_array_equal(got, [1.5, 2.0, 3.0, 4.0, 4.5])
+    # kappa = 7 over three candidates: every window covers all of them.
+    got = oracle.pool(np.array([3.0, 0.0, 6.0]), 3, 7, oracle.POOL_AVG)
+    np.testing.assert_array_equal(got, [3.0, 3.0, 3.0])
+
+
 def brute_topk(scores, n_cand, k, s):
     # stable lexsort: primary key -score, secondary key position
     order = np.lexsort((np.arange(n_cand), -scores[:n_cand]))
@@ -172,6 +192,17 @@ def test_select_with_pooling_uses_pooled_ranking():
     p, _, _ = make_problem(rng, L=L, w=w, k=k, s=s, pool=5)
     scores = rng.random(L)
     pooled = F.max_pool1d(torch.from_numpy(scores[:L - w])[None, None], 5, 1, 2)[0, 0].numpy()
+    want = brute_topk(np.concatenate([pooled, scores[L - w:]]), L - w, k, s)
+    np.testing.assert_array_equal(oracle.select(p, scores), want)
+
+
+def test_select_with_avg_pooling_uses_pooled_ranking():
+    rng = np.random.default_rng(19)
+    L, w, k, s = 64, 8, 10, 4
+    p, _, _ = make_problem(rng, L=L, w=w, k=k, s=s, pool=7, pool_mode=oracle.POOL_AVG)
+    scores = rng.random(L)
+    pooled = F.avg_pool1d(torch.from_numpy(scores[:L - w])[None, None], 7, 1, 3,
+                          count_include_pad=False)[0, 0].numpy()
     want = brute_topk(np.concatenate([pooled, scores[L - w:]]), L - w, k, s)
     np.testing.assert_array_equal(oracle.select(p, scores), want)
 
