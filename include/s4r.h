@@ -73,6 +73,14 @@ typedef enum { S4R_F32 = 0, S4R_BF16 = 1 } s4r_dtype;
  *   rows of the key basis that belong to its kv group. */
 typedef enum { S4R_ROWS_CONCAT = 0, S4R_ROWS_PER_HEAD = 1 } s4r_row_mode;
 
+/* Pooling of the candidate scores before selection (pool_kernel = odd kappa
+ * > 1; "free parameters": kernel 7, from SnapKV).  Stride 1, same padding,
+ * over the candidates only; neighbours outside the candidates are left out.
+ * MAX: the largest neighbour score.  AVG: the mean of the in-range
+ * neighbour scores (their sum in fp32, in position order, divided by their
+ * count). */
+typedef enum { S4R_POOL_MAX = 0, S4R_POOL_AVG = 1 } s4r_pool_mode;
+
 /* Supported range (S4R_ERR_UNSUPPORTED outside it). */
 #define S4R_MAX_D_MODEL 1024    /* D' */
 #define S4R_MAX_RANK 256        /* rank_k, rank_v; multiples of 8 */
@@ -180,7 +188,8 @@ typedef struct {
   int32_t local_window;               /* w: newest coefficient rows always kept */
   int32_t top_k;                      /* k: global positions chosen before the window */
   int32_t query_window;               /* W: query rows scored per step */
-  int32_t pool_kernel;                /* 1 = off; odd kappa = max-pool of candidate scores */
+  int32_t pool_kernel;                /* 1 = off; odd kappa = pool candidate scores */
+  int32_t pool_mode;                  /* s4r_pool_mode (read when pool_kernel > 1) */
   int32_t row_mode;                   /* s4r_row_mode */
   s4r_dtype dtype;                    /* storage type of q, coefficients, bases, sinks */
   int64_t cache_rows;                 /* row capacity (stride) of the coefficient caches */
@@ -219,8 +228,9 @@ s4r_status s4r_workspace_init(void *workspace, size_t workspace_bytes, void *str
  *   1. C_Q = Q' . B^K for the query window (rows per row_mode);
  *   2. Z = C_Q . C_K^T / sqrt(rank_k), softmax of every row over the L_c
  *      coefficient rows, score[i] = sum of the rows' probabilities (Eqs. 8-10);
- *   3. idx = the top_k rows among 0 .. L_c-w-1 by score (max-pooled when
- *      pool_kernel > 1), equal scores -> lower position (Eqs. 13-15);
+ *   3. idx = the top_k rows among 0 .. L_c-w-1 by score (pooled by
+ *      pool_mode when pool_kernel > 1), equal scores -> lower position
+ *      (Eqs. 13-15);
  *   4. for every query head h, exact attention of q[W-1][h] over the sinks,
  *      the chosen rows and the last w rows, with keys c_K . B^K^T and values
  *      c_V . B^V^T restricted to the head's kv group, logits scaled by
@@ -277,6 +287,21 @@ s4r_status s4r_read_device_status(const void *workspace, void *stream);
  * library-wide word of the current device when workspace == NULL (this
  * form synchronises `stream`). */
 s4r_status s4r_clear_device_status(void *workspace, void *stream);
+
+/* Testing hook for the device-side bounded waits; the S4R paper has no
+ * counterpart.  Every spin-wait of the kernels (mbarrier waits, grid-wide
+ * barriers) gives up after a limit, sets S4R_ERR_TIMEOUT in the device
+ * status and lets the kernel finish without it (the call's results are then
+ * not defined, but nothing hangs and the context stays usable).  This call
+ * sets, for the current device:
+ *   - limit_cycles: the limit in SM clock cycles (<= 0: the default, about
+ *     2 s);
+ *   - unreachable_barrier: when non-zero, the grid-wide barrier of the
+ *     latent-scoring kernel waits for one arrival more than its grid has,
+ *     so it always runs out after the limit.
+ * It synchronises the device (cudaMemcpyToSymbol); do not call it while
+ * other work of this library runs.  S4R_ERR_CUDA if the copy fails. */
+s4r_status s4r_debug_waits(int64_t limit_cycles, int32_t unreachable_barrier);
 
 /* Static description of a status code. */
 const char *s4r_status_string(s4r_status status);

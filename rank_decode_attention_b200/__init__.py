@@ -22,6 +22,7 @@ S4R_OK, S4R_ERR_INVALID_ARG, S4R_ERR_UNSUPPORTED, S4R_ERR_CUDA, S4R_ERR_TIMEOUT,
     S4R_ERR_DEVICE, S4R_ERR_WORKSPACE = range(7)
 S4R_F32, S4R_BF16 = 0, 1
 S4R_ROWS_CONCAT, S4R_ROWS_PER_HEAD = 0, 1
+S4R_POOL_MAX, S4R_POOL_AVG = 0, 1
 
 _DTYPE = {torch.float32: S4R_F32, torch.bfloat16: S4R_BF16}
 
@@ -40,7 +41,7 @@ class DecodeArgs(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("rank_k", ctypes.c_int32), ("rank_v", ctypes.c_int32),
         ("n_sink", ctypes.c_int32), ("local_window", ctypes.c_int32), ("top_k", ctypes.c_int32),
         ("query_window", ctypes.c_int32), ("pool_kernel", ctypes.c_int32),
-        ("row_mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("pool_mode", ctypes.c_int32), ("row_mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("cache_rows", ctypes.c_int64),
         ("lengths", ctypes.c_void_p), ("q", ctypes.c_void_p),
         ("coeff_k", ctypes.c_void_p), ("coeff_v", ctypes.c_void_p),
@@ -89,6 +90,7 @@ SIGNATURES = {
     "s4r_reconstruct": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i32, _vp, _i64, _vp, ctypes.c_int, _vp]),
     "s4r_read_device_status": (ctypes.c_int, [_vp, _vp]),
     "s4r_clear_device_status": (ctypes.c_int, [_vp, _vp]),
+    "s4r_debug_waits": (ctypes.c_int, [_i64, _i32]),
     "s4r_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "s4r_version": (_i32, []),
     "s4r_last_error": (ctypes.c_char_p, []),
@@ -172,8 +174,8 @@ def s4r_append(stream=None, **kw) -> int:
 
 def decode_args(*, q, coeff_k, coeff_v, basis_k, basis_v, sink_k, sink_v, lengths, n_heads_kv,
                 local_window, top_k, out=None, idx=None, scores=None, workspace=None,
-                workspace_bytes=None, pool_kernel=1, row_mode=S4R_ROWS_CONCAT,
-                profile_events=None) -> DecodeArgs:
+                workspace_bytes=None, pool_kernel=1, pool_mode=S4R_POOL_MAX,
+                row_mode=S4R_ROWS_CONCAT, profile_events=None) -> DecodeArgs:
     """Fill s4r_decode_args from tensors: q [B][W][H_q][d_h], coeff_k/v
     [B][cache_rows][r], basis_k/v [B][D'][r], sink_k/v [B][s][D'],
     lengths [B] int32 (device)."""
@@ -183,7 +185,8 @@ def decode_args(*, q, coeff_k, coeff_v, basis_k, basis_v, sink_k, sink_v, length
     if workspace is not None and workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size()
     a = DecodeArgs(B, Hq, n_heads_kv, dh, coeff_k.shape[2], coeff_v.shape[2], n_sink,
-                   local_window, top_k, W, pool_kernel, row_mode, _DTYPE[q.dtype], cache_rows,
+                   local_window, top_k, W, pool_kernel, pool_mode, row_mode, _DTYPE[q.dtype],
+                   cache_rows,
                    _ptr(lengths), _ptr(q), _ptr(coeff_k), _ptr(coeff_v), _ptr(basis_k),
                    _ptr(basis_v), _ptr(sink_k), _ptr(sink_v), _ptr(out), _ptr(idx),
                    _ptr(scores), _ptr(workspace), workspace_bytes or 0)
@@ -254,6 +257,14 @@ def s4r_reconstruct(coeffs: torch.Tensor, basis: torch.Tensor, rows: torch.Tenso
 def s4r_read_device_status(workspace, stream=None) -> int:
     """Synchronise the stream and return the sticky device status code."""
     return int(lib().s4r_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def s4r_debug_waits(limit_cycles: int = 0, unreachable_barrier: bool = False) -> int:
+    """Testing hook: limit of the device-side bounded waits (SM cycles, 0 =
+    default) and the switch that makes the scoring kernel's grid barrier
+    unreachable (see include/s4r.h)."""
+    return _check(lib().s4r_debug_waits(int(limit_cycles), 1 if unreachable_barrier else 0),
+                  "s4r_debug_waits")
 
 
 def s4r_clear_device_status(workspace, stream=None) -> int:

@@ -68,7 +68,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // Decode-step shape shared by the kernels (plain values, passed by value).
 struct Shape {
   int32_t batch, n_heads_q, n_heads_kv, head_dim, rank_k, rank_v;
-  int32_t n_sink, local_window, top_k, query_window, pool_kernel, row_mode;
+  int32_t n_sink, local_window, top_k, query_window, pool_kernel, pool_mode, row_mode;
   int32_t d_model, group, n_rows;  // D', G, scoring rows R
   int64_t cache_rows;
 };

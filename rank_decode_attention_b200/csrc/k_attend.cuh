@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const int32_t *__restrict__ idx,
               const T *__restrict__ coeff_k, const T *__restrict__ coeff_v, const float *__restrict__ qt_all,
               const T *__restrict__ q, const T *__restrict__ basis_v, const T *__restrict__ sink_k,
-              const T *__restrict__ sink_v, float *__restrict__ out) {
+              const T *__restrict__ sink_v, float *__restrict__ out, uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) unsigned char att_smem[];
   constexpr int V = Vec16<T>::n;
   constexpr int kWarps = kAttThreads / 32;
@@ -276,7 +276,8 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
       for (int d = 0; d < 4; ++d) accf[a][c][d] = 0.f;
 
   uint32_t phase = 0;
-  for (int64_t c0 = e_begin; c0 < e_end; c0 += E) {
+  bool staged_ok = true;   // false once a wait for staged rows gave up: no further chunks are staged
+  for (int64_t c0 = e_begin; c0 < e_end && staged_ok; c0 += E) {
     const int n_e = (int)smin<int64_t>(E, e_end - c0);
     __syncthreads();  // previous chunk fully consumed
     int live = 0;     // E <= blockDim.x: at most one entry per thread
@@ -306,9 +307,10 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
         for (int c = 0; c < n; c += V) *reinterpret_cast<uint4 *>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    mbar_wait(&stage_bar, phase, nullptr);
+    // Every thread waits (bounded) and sees the same outcome unless the copies
+    // land right at the limit; the vote makes the decision uniform.
+    staged_ok = __syncthreads_and(mbar_wait(&stage_bar, phase, status)) != 0;
     phase ^= 1u;
-    __syncthreads();
     if (sizeof(T) == 2 && rk % 16 == 0) {
       // logits on the tensor cores: per warp, 16-entry tiles of
       // C_K[16 x rk] . Qsplit[rk x 8] (mma m16n8k16, bf16 in, fp32 out); the
@@ -517,7 +519,7 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
                           cluster_map(&recv_bar, (uint32_t)r2));
     }
   }
-  mbar_wait(&recv_bar, 0, nullptr);   // every partial of the heads finished here has arrived
+  mbar_wait(&recv_bar, 0, status);    // every partial of the heads finished here has arrived
   // Every copy into this CTA is done.  A sender learns that its own copies
   // have been read only from the receivers, so no CTA leaves before all have
   // arrived here (the wait is at the end, after the merge and the output).
@@ -554,7 +556,7 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
       if (r < n_ranks) a = fmaf(f_s[jj * kAttCluster + r], recv_s[((size_t)jj * kAttCluster + r) * pr + 4 + k], a);
     acc_s[jj * rv + k] = a;
   }
-  mbar_wait(&bv_bar, 0, nullptr);
+  mbar_wait(&bv_bar, 0, status);
   __syncthreads();
   // out[h][e] = acc[j] . B^V[g*dh + e] + sum_t w_t sink_v[t][g*dh + e], four
   // threads per output (16-byte chunks c = part, part + 4, ...).

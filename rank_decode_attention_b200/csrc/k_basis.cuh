@@ -37,6 +37,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "umma.cuh"
 
 namespace s4r {
 
@@ -213,12 +214,13 @@ __device__ __forceinline__ bool basis_grid_sync(BasisCtl *ctl, uint32_t gen, int
     __threadfence();
     atomicAdd(&ctl->bar, 1u);
     const uint32_t target = gen * gridDim.x;
+    const long long limit = wait_limit();
     const long long t0 = clock64();
     while (true) {
       uint32_t v;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&ctl->bar) : "memory");
       if (v >= target) break;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         set_status(&ctl->status, kDevStatusTimeout);
         ok = 0;
         break;

@@ -286,11 +286,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
 #pragma unroll
       for (int q = 0; q < kStcSumSlots; ++q) l += part[q];
     }
-    const float inv = (l > 0.0) ? 1.f / (float)l : 0.f;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int k = ctl->kofs[t][row];
-      ctl->alpha[t][row] = (k == 0) ? inv : ldexpf(inv, k);
-    }
+    // alpha = 2^k / l in fp64 first: l itself may lie outside the fp32 range
+    // when a row's logits are far from 0 (the tiles then carry offsets k).
+    const double inv = (l > 0.0) ? 1.0 / l : 0.0;
+    for (int t = 0; t < n_tiles; ++t) ctl->alpha[t][row] = (float)ldexp(inv, ctl->kofs[t][row]);
   }
   // Exponent histogram of this CTA's candidate scores (rows before the
   // local window) for the top-k kernel, in the now idle reduction scratch.

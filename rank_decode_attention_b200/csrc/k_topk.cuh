@@ -22,20 +22,30 @@ __device__ __forceinline__ int64_t valid_length(int64_t L, int64_t cap) {
   return (L >= 0 && L <= cap) ? L : 0;
 }
 
-// Max-pool of candidate scores, stride 1, same padding, odd kernel.
+// Pooling of candidate scores, stride 1, same padding, odd kernel: the
+// largest (S4R_POOL_MAX) or the mean (S4R_POOL_AVG) of the neighbours inside
+// the candidates.  The mean sums in position order in fp32 and divides by the
+// count of in-range neighbours.
 __global__ void pool_kernel(Shape s, const int32_t *__restrict__ lengths,
                             const float *__restrict__ scores, float *__restrict__ pooled) {
+  pdl_wait();      // scores come from the preceding kernel
+  pdl_trigger();
   const int b = blockIdx.y;
   const int64_t L = valid_length(lengths[b], s.cache_rows);
   const int64_t nc = n_candidates(L, s.local_window);
   const int half = s.pool_kernel / 2;
+  const bool avg = s.pool_mode == S4R_POOL_AVG;
   const float *sb = scores + (int64_t)b * s.cache_rows;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nc;
        i += (int64_t)gridDim.x * blockDim.x) {
-    float m = sb[i];
-    for (int64_t j = smax<int64_t>(0, i - half); j <= smin<int64_t>(nc - 1, i + half); ++j)
-      m = fmaxf(m, sb[j]);
-    pooled[(int64_t)b * s.cache_rows + i] = m;
+    const int64_t j0 = smax<int64_t>(0, i - half), j1 = smin<int64_t>(nc - 1, i + half);
+    float m = sb[i], sum = 0.f;
+    for (int64_t j = j0; j <= j1; ++j) {
+      const float v = sb[j];
+      m = fmaxf(m, v);
+      sum += v;
+    }
+    pooled[(int64_t)b * s.cache_rows + i] = avg ? sum / (float)(j1 - j0 + 1) : m;
   }
 }
 

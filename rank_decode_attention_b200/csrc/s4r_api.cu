@@ -72,6 +72,7 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
   if (a->dtype != S4R_F32 && a->dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
   if (a->row_mode != S4R_ROWS_CONCAT && a->row_mode != S4R_ROWS_PER_HEAD) return S4R_ERR_INVALID_ARG;
   if (a->pool_kernel % 2 == 0) return S4R_ERR_INVALID_ARG;
+  if (a->pool_mode != S4R_POOL_MAX && a->pool_mode != S4R_POOL_AVG) return S4R_ERR_INVALID_ARG;
   const int64_t G = a->n_heads_q / a->n_heads_kv;
   const int64_t Dp = (int64_t)a->n_heads_kv * a->head_dim;
   const int64_t R = (a->row_mode == S4R_ROWS_CONCAT) ? (int64_t)a->query_window * G
@@ -94,6 +95,7 @@ s4r_status make_shape(const s4r_decode_args *a, Shape *s) {
   s->top_k = a->top_k;
   s->query_window = a->query_window;
   s->pool_kernel = a->pool_kernel;
+  s->pool_mode = a->pool_mode;
   s->row_mode = a->row_mode;
   s->d_model = (int32_t)Dp;
   s->group = (int32_t)G;
@@ -465,7 +467,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     const cudaError_t err = cudaLaunchKernelEx(&cfg, attend_kernel<T>, s, pl, a->lengths, a->idx, ck, cv, qt, q, bv, sk,
-                                               sv, a->out);
+                                               sv, a->out, status);
     if (err != cudaSuccess) return fail("attend_kernel (cluster launch)", err);
     if (check_launch("attend_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
@@ -744,6 +746,14 @@ s4r_status s4r_clear_device_status(void *workspace, void *stream) {
     if (cudaStreamSynchronize(st) != cudaSuccess) return S4R_ERR_CUDA;
   }
   return S4R_OK;
+}
+
+s4r_status s4r_debug_waits(int64_t limit_cycles, int32_t unreachable_barrier) {
+  const long long limit = limit_cycles > 0 ? (long long)limit_cycles : kWaitCycles;
+  const uint32_t unreach = unreachable_barrier ? 1u : 0u;
+  cudaError_t err = cudaMemcpyToSymbol(g_wait_limit, &limit, sizeof(limit));
+  if (err == cudaSuccess) err = cudaMemcpyToSymbol(g_barrier_unreachable, &unreach, sizeof(unreach));
+  return err == cudaSuccess ? S4R_OK : fail("s4r_debug_waits", err);
 }
 
 const char *s4r_status_string(s4r_status status) {

@@ -16,6 +16,17 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 // Library-wide status word for kernels that have no workspace (encode).
 __device__ uint32_t g_device_status;
 
+// Limit of every bounded wait in SM cycles, and a switch that makes the
+// latent-scoring kernel's grid barrier wait for one arrival more than its grid
+// has.  Only s4r_debug_waits changes them (so that tests can make a wait run
+// out); they are read once per wait, on its slow path.
+__device__ long long g_wait_limit = kWaitCycles;
+__device__ uint32_t g_barrier_unreachable = 0u;
+__device__ __forceinline__ long long wait_limit() {
+  const long long v = *reinterpret_cast<volatile long long *>(&g_wait_limit);
+  return v > 0 ? v : kWaitCycles;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -48,9 +59,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
+  const long long limit = wait_limit();
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       set_status(status ? status : &g_device_status, kDevStatusTimeout);
       return false;
     }
@@ -184,12 +196,14 @@ __device__ __forceinline__ bool grid_barrier(unsigned int *bar, uint32_t *status
     int ok = 1;
     __threadfence();
     atomicAdd(bar, 1u);
+    const unsigned int target = gridDim.x + (*reinterpret_cast<volatile uint32_t *>(&g_barrier_unreachable) ? 1u : 0u);
+    const long long limit = wait_limit();
     const long long t0 = clock64();
     while (true) {
       unsigned int v;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-      if (v >= gridDim.x) break;
-      if (clock64() - t0 > kWaitCycles) {
+      if (v >= target) break;
+      if (clock64() - t0 > limit) {
         set_status(status, kDevStatusTimeout);
         ok = 0;
         break;

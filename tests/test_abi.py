@@ -58,6 +58,7 @@ int main(void) {
   printf("s4r_append_args size %zu\n", sizeof(s4r_append_args));
   F(s4r_decode_args, cache_rows) F(s4r_decode_args, lengths) F(s4r_decode_args, out)
   F(s4r_decode_args, workspace) F(s4r_decode_args, workspace_bytes) F(s4r_decode_args, dtype)
+  F(s4r_decode_args, pool_mode) F(s4r_decode_args, row_mode)
   F(s4r_append_args, cache_rows) F(s4r_append_args, lengths) F(s4r_append_args, status_workspace)
   printf("s4r_basis_args size %zu\n", sizeof(s4r_basis_args));
   F(s4r_basis_args, dtype) F(s4r_basis_args, state_rows) F(s4r_basis_args, lengths) F(s4r_basis_args, sigma)
@@ -102,7 +103,7 @@ def test_workspace_bytes_and_shape_validation():
     assert s4r.s4r_decode_workspace_bytes(good_args(pool_kernel=7)) > n
     for bad in (dict(n_heads_q=30), dict(rank_k=0), dict(pool_kernel=4), dict(dtype=9),
                 dict(row_mode=3), dict(query_window=0), dict(top_k=-1), dict(head_dim=100),
-                dict(rank_v=264), dict(n_heads_kv=16, head_dim=128)):
+                dict(rank_v=264), dict(n_heads_kv=16, head_dim=128), dict(pool_mode=2)):
         assert s4r.s4r_decode_workspace_bytes(good_args(**bad)) == 0, bad
 
 
