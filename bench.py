@@ -2,25 +2,39 @@
 """S4R compressed-KV decode benchmark on B200.  Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl s4r|reference]
-                    [--workload 1] [--no-encode] [--no-basis]
+                    [--workload 1] [--extra 0,2,3,4,1b,3b | none]
+                    [--no-encode] [--no-basis] [--no-cpu-baseline]
 
-Workload (default 1): Llama-3-8B-shaped attention, 32 layers with their own
-bases, batch 1, prompt L = 32768 (4 sinks + 32764 coefficient rows), rank 192,
-top-k 1024, local window 128, query window 16.  One step = one decode step of
-all 32 layers, issued as 32 sequential per-layer s4r_decode_step calls (the
-layers of a real model run one after another); each step's calls are captured
-once in a CUDA graph and replayed.  Step t uses query rows t .. t+15.
+Headline (the line's top-level keys): Llama-3-8B-shaped attention, 32 layers
+with their own bases, batch 1, prompt L = 32768 (4 sinks + 32764 coefficient
+rows), rank 192, top-k 1024, local window 128, query window 16.  One step =
+one decode step of all 32 layers, issued as 32 sequential per-layer
+s4r_decode_step calls (the layers of a real model run one after another);
+each step's calls are captured once in a CUDA graph and replayed.  Step t
+uses query rows t .. t+15.
+
+`workloads` (one GPU only) times the other configurations in the same run,
+each with its own roofline, end-to-end figure and oracle sample:
+  0   tiny fp32 single layer (L = 2048, r = 32);
+  2   batched decode, 16 sequences x 32 layers, L = 8192, r = 128;
+  3   long context, 32 layers, L = 131072, r = 256;
+  4   ragged encode + decode: 8 sequences, L ~ U[4096, 65536], r = 256; each
+      step appends one encoded token per sequence, then decodes;
+  1b  the headline's 32 layers in ONE call (batch of 32 problems);
+  3b  the long-context 32 layers in ONE call.
+The layers-in-one-call variants are labelled as such: a real model cannot
+batch its layers, whose queries depend on the previous layer's output.
 
 Everything is synthetic (seeded generator, see synth/); the coefficient
 caches are made on the GPU by the library's own encode kernel before timing.
-The caches (805 MB) exceed L2 (126 MB) and each step streams 460.8 MB, so no
-L2 flush is needed between steps.
+Every workload's per-step reads exceed L2 (126 MB) except the tiny one,
+which is latency-bound (stated in its entry); no L2 flush is used.
 
 With --gpus N > 1 (torchrun), every rank runs an independent replica of the
-workload: the problems shard with no exchange, so there is no collective on
+headline: the problems shard with no exchange, so there is no collective on
 the data path; the timed region is bracketed by barriers and the time is the
 max over ranks.  `--impl reference` times the fp64 CPU oracle on the host
-cores instead (rank 0 only).
+cores instead (rank 0 only), on the same workload and config.
 """
 from __future__ import annotations
 
@@ -28,7 +42,6 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
 import statistics
 import sys
@@ -44,11 +57,14 @@ import synth  # noqa: E402
 
 METRIC = "compressed-KV decode steps/s and achieved HBM GB/s (% of roofline) at L=32K"
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+EXTRA_DEFAULT = "0,2,3,4,1b,3b"
+MAX_WINDOWS = 32          # distinct query windows per workload (steps cycle through them)
 
 
 # ----------------------------------------------------------------- helpers
 
 def peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s burst, source)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
@@ -127,87 +143,158 @@ def source_sha(paths) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key: str):
-    """DRAM bytes per launch from a committed ncu summary, only while the
-    kernel source is unchanged since the capture."""
+def profiled(kernel: str, workload: str):
+    """ncu figures of one kernel on one workload from the committed summary
+    (profiles/traffic.json): DRAM bytes per launch and the serialised launch
+    duration, each only while the kernel's sources are unchanged since the
+    capture (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
-        return None
-    d = json.load(open(p)).get(kernel_key)
+        return None, None
+    d = json.load(open(p)).get(f"{kernel}/{workload}")
     if not d or d.get("source_sha") != source_sha(d["sources"]):
-        return None
-    return d["dram_bytes_per_launch"]
+        return None, None
+    return d.get("dram_bytes_per_launch"), d.get("ncu_duration_us")
+
+
+def workload_config(w: synth.Workload, calls: str) -> dict:
+    """The `config` object of a workload."""
+    L = synth.lengths(w)
+    return {"workload": w.name, "layers": w.layers, "batch": w.batch,
+            "prompt_len": L[0] if not w.ragged else f"U[{w.ragged[0]}, {w.ragged[1]}] (drawn: {L})",
+            "rank": w.rank, "top_k": w.top_k, "local_window": w.local_window,
+            "query_window": w.query_window, "n_heads_q": w.n_heads_q, "n_heads_kv": w.n_heads_kv,
+            "head_dim": w.head_dim, "n_sink": w.n_sink, "storage": w.dtype,
+            "append_per_step": w.append, "calls": calls}
+
+
+def headline_config(w: synth.Workload, world: int) -> dict:
+    """The headline line's `config`, identical in the GPU arm and the
+    reference arm."""
+    Lc = [L - w.n_sink for L in synth.lengths(w)]
+    step_bytes = algorithmic_bytes(w, Lc)[0] * w.layers
+    cfg = workload_config(w, HEADLINE_CALLS)
+    cfg["l2"] = f"inputs larger than L2: {step_bytes / 1e6:.1f} MB read per step"
+    cfg["parallelism"] = f"replicas x{world}"
+    return cfg
+
+
+HEADLINE_CALLS = "32 sequential per-layer calls per step, CUDA graph per step"
 
 
 # ----------------------------------------------------------------- workload on the GPU
 
 class GpuWorkload:
-    """All layers of one replica, resident in HBM."""
+    """Every (layer, sequence) problem of one replica, resident in HBM.
+    Problem p = layer * batch + sequence; the problems of one layer are a
+    contiguous slice, so the per-layer calls and the all-layers call read the
+    same memory."""
 
-    def __init__(self, w: synth.Workload, replica: int, device, n_windows: int):
+    def __init__(self, w: synth.Workload, replica: int, device, n_windows: int, append_rows: int = 0):
         import rank_decode_attention_b200 as s4r
         self.w, self.dev = w, device
-        B, s = w.batch, w.n_sink
-        self.Lc = [L - s for L in synth.lengths(w)]
-        self.cap = max(self.Lc)
+        B, s, Ly, W = w.batch, w.n_sink, w.layers, w.query_window
+        self.P = P = B * Ly
+        self.L_seq = synth.lengths(w)
+        self.Lc = [L - s for L in self.L_seq] * Ly
+        self.cap = max(self.Lc) + append_rows
         self.n_windows = n_windows
         sdt = synth.storage_dtype(w.dtype)
-        self.layers = []
-        for layer in range(w.layers):
-            ck = torch.zeros(B, self.cap, w.rank, dtype=sdt, device=device)
-            cv = torch.zeros_like(ck)
-            bk = torch.empty(B, w.d_model, w.rank, dtype=sdt, device=device)
-            bv = torch.empty_like(bk)
-            sk = torch.empty(B, s, w.d_model, dtype=sdt, device=device)
-            sv = torch.empty_like(sk)
-            qs = torch.empty(n_windows, B, w.query_window, w.n_heads_q, w.head_dim, dtype=sdt,
-                             device=device)
+        D, r = w.d_model, w.rank
+        self.ck = torch.zeros(P, self.cap, r, dtype=sdt, device=device)
+        self.cv = torch.zeros_like(self.ck)
+        self.bk = torch.empty(P, D, r, dtype=sdt, device=device)
+        self.bv = torch.empty_like(self.bk)
+        self.sk = torch.empty(P, s, D, dtype=sdt, device=device)
+        self.sv = torch.empty_like(self.sk)
+        self.q = torch.empty(n_windows, P, W, w.n_heads_q, w.head_dim, dtype=sdt, device=device)
+        for layer in range(Ly):
             for b in range(B):
-                pin = synth.problem_inputs(w, layer, b, device=device, L=self.Lc[b] + s,
-                                           n_query_rows=n_windows + w.query_window - 1,
-                                           tag=f"replica{replica}")
-                bk[b], bv[b] = pin.basis_k, pin.basis_v
-                sk[b], sv[b] = pin.states_k[:s], pin.states_v[:s]
+                p = layer * B + b
+                pin = synth.problem_inputs(w, layer, b, device=device, L=self.L_seq[b],
+                                           n_query_rows=n_windows + W - 1, tag=f"replica{replica}")
+                self.bk[p], self.bv[p] = pin.basis_k, pin.basis_v
+                self.sk[p], self.sv[p] = pin.states_k[:s], pin.states_v[:s]
                 # prefill encode through the library (C = S . B)
-                s4r.s4r_encode(pin.states_k[s:], pin.basis_k, ck[b, :self.Lc[b]])
-                s4r.s4r_encode(pin.states_v[s:], pin.basis_v, cv[b, :self.Lc[b]])
+                s4r.s4r_encode(pin.states_k[s:], pin.basis_k, self.ck[p, :self.Lc[p]])
+                s4r.s4r_encode(pin.states_v[s:], pin.basis_v, self.cv[p, :self.Lc[p]])
                 for t in range(n_windows):
-                    qs[t, b] = pin.window(t, w.query_window)
+                    self.q[t, p] = pin.window(t, W)
                 del pin
-            lengths = torch.tensor(self.Lc, dtype=torch.int32, device=device)
-            self.layers.append(dict(ck=ck, cv=cv, bk=bk, bv=bv, sk=sk, sv=sv, q=qs, lengths=lengths))
+        # lengths: one tensor per layer (each 16-byte aligned) and one for all problems
+        self.lengths0 = torch.tensor(self.Lc, dtype=torch.int32, device=device)
+        self.len_layer = [self.lengths0[l * B:(l + 1) * B].clone() for l in range(Ly)]
+        self.len_all = self.lengths0.clone()
+        self.out = torch.empty(P, w.n_heads_q, w.head_dim, device=device)
+        self.idx = torch.empty(P, w.top_k, dtype=torch.int32, device=device)
+        if w.append:
+            g = torch.Generator(device=device).manual_seed(synth.seed_of(w.name, "append", replica))
+            self.new_k = synth.store(torch.randn(n_windows, P, D, generator=g, device=device,
+                                                 dtype=torch.float64), w.dtype)
+            self.new_v = synth.store(torch.randn(n_windows, P, D, generator=g, device=device,
+                                                 dtype=torch.float64), w.dtype)
         torch.cuda.synchronize()
-        L0 = self.layers[0]
-        self.out = torch.empty(w.layers, B, w.n_heads_q, w.head_dim, device=device)
-        self.idx = torch.empty(w.layers, B, w.top_k, dtype=torch.int32, device=device)
-        a = self.args(0, 0)
-        self.ws_bytes = s4r.s4r_decode_workspace_bytes(a)
+        big = self.args(None, 0)
+        self.ws_bytes = max(s4r.s4r_decode_workspace_bytes(big),
+                            max(s4r.s4r_decode_workspace_bytes(self.args(l, 0)) for l in range(Ly)))
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
         s4r.s4r_workspace_init(self.ws)
-        self.launches_per_call = s4r.s4r_decode_kernel_launches(a)
+        self.launches_layer = s4r.s4r_decode_kernel_launches(self.args(0, 0))
+        self.launches_all = s4r.s4r_decode_kernel_launches(big)
+
+    def reset_lengths(self):
+        """Undo the appends of a timed pass (append workloads)."""
+        self.len_all.copy_(self.lengths0)
+        for l, t in enumerate(self.len_layer):
+            t.copy_(self.lengths0[l * self.w.batch:(l + 1) * self.w.batch])
+
+    def _slice(self, layer):
+        B = self.w.batch
+        return slice(0, self.P) if layer is None else slice(layer * B, (layer + 1) * B)
 
     def args(self, layer, window, events=None):
+        """Decode arguments of one layer's problems, or of every problem
+        (layer None, the all-layers call)."""
         import rank_decode_attention_b200 as s4r
-        L = self.layers[layer]
-        return s4r.decode_args(q=L["q"][window], coeff_k=L["ck"], coeff_v=L["cv"], basis_k=L["bk"],
-                               basis_v=L["bv"], sink_k=L["sk"], sink_v=L["sv"],
-                               lengths=L["lengths"], n_heads_kv=self.w.n_heads_kv,
+        sl = self._slice(layer)
+        lengths = self.len_all if layer is None else self.len_layer[layer]
+        return s4r.decode_args(q=self.q[window, sl], coeff_k=self.ck[sl], coeff_v=self.cv[sl],
+                               basis_k=self.bk[sl], basis_v=self.bv[sl], sink_k=self.sk[sl],
+                               sink_v=self.sv[sl], lengths=lengths, n_heads_kv=self.w.n_heads_kv,
                                local_window=self.w.local_window, top_k=self.w.top_k,
-                               out=self.out[layer], idx=self.idx[layer],
-                               workspace=getattr(self, "ws", None),
+                               out=self.out[sl], idx=self.idx[sl], workspace=getattr(self, "ws", None),
                                workspace_bytes=getattr(self, "ws_bytes", None),
                                pool_kernel=self.w.pool_kernel, profile_events=events)
 
-    def step_calls(self, window, events=None):
+    def append(self, layer, window):
         import rank_decode_attention_b200 as s4r
-        for layer in range(self.w.layers):
-            ev = events[layer] if events is not None else None
+        sl = self._slice(layer)
+        lengths = self.len_all if layer is None else self.len_layer[layer]
+        s4r.s4r_append(state_k=self.new_k[window, sl], state_v=self.new_v[window, sl],
+                       basis_k=self.bk[sl], basis_v=self.bv[sl], coeff_k=self.ck[sl], coeff_v=self.cv[sl],
+                       lengths=lengths, status_workspace=self.ws)
+
+    def step_calls(self, window, batched=False, events=None):
+        """One decode step: the per-layer calls in layer order, or one call."""
+        import rank_decode_attention_b200 as s4r
+        layers = [None] if batched else list(range(self.w.layers))
+        for i, layer in enumerate(layers):
+            if self.w.append:
+                self.append(layer, window)
+            ev = events[i] if events is not None else None
             s4r.s4r_decode_step(self.args(layer, window, ev))
+
+    def calls_per_step(self, batched):
+        return 1 if batched else self.w.layers
+
+    def launches_per_step(self, batched):
+        per = self.launches_all if batched else self.launches_layer * self.w.layers
+        return per + (self.calls_per_step(batched) * 2 if self.w.append else 0)   # append: 2 kernels
 
 
 def algorithmic_bytes(w: synth.Workload, Lc: list):
-    """Per decode call (one layer, all problems): (whole step, scoring kernel).
-    Whole step per problem: L_c*r*e (C_K once) + 2(k+w)*r*e (selected C_K and
+    """Per decode call over the given problems: (whole path, scoring kernel).
+    Whole path per problem: L_c*r*e (C_K once) + 2(k+w)*r*e (selected C_K and
     C_V rows) + 2*D'*r*e (bases) + 2*s*D'*e (sinks) + W*H_q*d_h*e (queries).
     Scoring kernel per problem: L_c*r*e + R*r*4 (C_Q) + L_c*4 (scores out)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -221,84 +308,229 @@ def algorithmic_bytes(w: synth.Workload, Lc: list):
     return step, score
 
 
+def time_decode(wl: GpuWorkload, steps: int, warmup: int, batched: bool, dist, device, world: int,
+                clocks: ClockSampler | None = None):
+    """Time `steps` decode steps of the workload (CUDA graphs of each step's
+    calls), then the same steps again with event pairs around every scoring
+    kernel, then end to end through the ABI from pinned host memory."""
+    import rank_decode_attention_b200 as s4r
+    w = wl.w
+    n_win = min(steps, wl.n_windows)
+    n_calls = wl.calls_per_step(batched)
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_calls)] for _ in range(n_win)]
+    for evs in events:
+        for a, b in evs:
+            a.record(); b.record()          # materialise the event handles
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device)
+    graphs, graphs_ev = [], []
+    with torch.cuda.stream(stream):
+        wl.step_calls(0, batched)           # warm the launch path before capture
+        torch.cuda.synchronize()
+        for t in range(n_win):
+            for evs, dst in ((None, graphs), (events[t], graphs_ev)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    wl.step_calls(t, batched, evs)
+                dst.append(g)
+    torch.cuda.synchronize()
+
+    def replay_pass(gs):
+        wl.reset_lengths()
+        for i in range(warmup):
+            gs[i % n_win].replay()
+        if w.append:
+            torch.cuda.synchronize()
+            wl.reset_lengths()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(steps):
+                gs[i % n_win].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        h1 = time.perf_counter()
+        if dist:
+            dist.barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device), h0, h1
+
+    torch.cuda.cudart().cudaProfilerStart()   # a profiler started with capture off sees this pass only
+    elapsed, h0, h1 = replay_pass(graphs)
+    torch.cuda.cudart().cudaProfilerStop()
+    clk = clocks.summary(h0, h1) if clocks is not None else None
+    elapsed_ev, _, _ = replay_pass(graphs_ev)
+    score_ms = []
+    for i in range(min(steps, n_win)):
+        score_ms += [a.elapsed_time(b) for a, b in events[i]]
+    del graphs, graphs_ev
+
+    # End to end through the public API from pinned host memory: every step
+    # copies the new query row of every problem (and, when appending, the new
+    # token states) host -> device, makes the decode calls directly (no
+    # graph) and reads out + idx back to pinned host memory.
+    W = w.query_window
+    host_q = wl.q.cpu().pin_memory()
+    host_out = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    host_idx = torch.empty(wl.idx.shape, dtype=wl.idx.dtype).pin_memory()
+    h2d = host_q[0, :, W - 1].numel() * host_q.element_size()
+    if w.append:
+        host_nk, host_nv = wl.new_k.cpu().pin_memory(), wl.new_v.cpu().pin_memory()
+        h2d += 2 * host_nk[0].numel() * host_nk.element_size()
+    d2h = host_out.numel() * 4 + host_idx.numel() * 4
+    layers = [None] if batched else list(range(w.layers))
+    call_args = [[wl.args(l, t) for l in layers] for t in range(n_win)]
+    wl.reset_lengths()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(steps):
+            t = i % n_win
+            wl.q[t, :, W - 1].copy_(host_q[t, :, W - 1], non_blocking=True)
+            if w.append:
+                wl.new_k[t].copy_(host_nk[t], non_blocking=True)
+                wl.new_v[t].copy_(host_nv[t], non_blocking=True)
+            for j, l in enumerate(layers):
+                if w.append:
+                    wl.append(l, t)
+                s4r.s4r_decode_step(call_args[t][j])
+            host_out.copy_(wl.out, non_blocking=True)
+            host_idx.copy_(wl.idx, non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_elapsed = max_over_ranks(f0.elapsed_time(f1) / 1e3, dist, device)
+    status = s4r.s4r_read_device_status(wl.ws)
+    if status != 0:
+        raise RuntimeError(f"{w.name}: device status {status} after the timed passes")
+    wl.reset_lengths()
+    return {"elapsed": elapsed, "elapsed_ev": elapsed_ev, "score_ms": score_ms, "clocks": clk,
+            "e2e": {"value": replica_value(world, steps, e2e_elapsed), "unit": "steps/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}}
+
+
+def roofline_entry(w, wl, batched, res, steps, hbm, src, label):
+    """Roofline of the latent-scoring kernel (the dominant byte mover) and the
+    whole path's achieved bandwidth for one timed workload."""
+    B = w.batch
+    per_call_Lc = wl.Lc if batched else wl.Lc[:B]
+    step_bytes_call, score_bytes = algorithmic_bytes(w, per_call_Lc)
+    n_calls = wl.calls_per_step(batched)
+    step_bytes = step_bytes_call * n_calls
+    avg_score_s = statistics.mean(res["score_ms"]) / 1e3
+    achieved = score_bytes / avg_score_s / 1e9
+    traffic, ncu_us = profiled("latent_scoring", label)
+    ms_per_step = res["elapsed"] / steps * 1e3
+    return step_bytes, {
+        "bound": "hbm", "kernel": "latent_scoring", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+        "frac": achieved / hbm, "peak_source": src, "traffic": traffic,
+        "algorithmic_bytes_per_launch": score_bytes, "avg_launch_us": avg_score_s * 1e6,
+        "launches_timed": len(res["score_ms"]), "ncu_launch_us": ncu_us,
+        "timing": "CUDA events on the launching stream around every scoring kernel, in a second timed "
+                  "pass of the same steps (the event nodes keep the kernel from overlapping its "
+                  "neighbours' launch); ncu_launch_us is ncu's serialised duration of the same launch",
+        "ms_per_step_with_events": res["elapsed_ev"] / steps * 1e3,
+        "whole_path_gbs": step_bytes / (ms_per_step / 1e3) / 1e9,
+        "whole_path_frac": step_bytes / (ms_per_step / 1e3) / 1e9 / hbm}
+
+
 # ----------------------------------------------------------------- oracle (CPU) leg
 
-def oracle_layer_sample(w: synth.Workload):
+def oracle_problem(w: synth.Workload, seq: int = 0, tag="cpu-sample"):
     """One (sequence, layer) problem of the workload at full length, on the CPU."""
     import oracle
-    L = synth.lengths(w)[0]
-    pin = synth.problem_inputs(w, 0, 0, L=L, n_query_rows=w.query_window, tag="cpu-sample")
+    L = synth.lengths(w)[seq]
+    pin = synth.problem_inputs(w, 0, seq, L=L, n_query_rows=w.query_window, tag=tag)
     s = w.n_sink
     enc = lambda S, Bm: synth.store(S.double() @ Bm.double(), w.dtype).double().numpy()
-    p = oracle.Problem(q=pin.window(0, w.query_window).double().numpy(),
-                       coeff_k=enc(pin.states_k[s:], pin.basis_k),
-                       coeff_v=enc(pin.states_v[s:], pin.basis_v),
-                       basis_k=pin.basis_k.double().numpy(), basis_v=pin.basis_v.double().numpy(),
-                       sink_k=pin.states_k[:s].double().numpy(), sink_v=pin.states_v[:s].double().numpy(),
-                       n_heads_kv=w.n_heads_kv, local_window=w.local_window, top_k=w.top_k,
-                       pool_kernel=w.pool_kernel)
-    return p
+    return oracle.Problem(q=pin.window(0, w.query_window).double().numpy(),
+                          coeff_k=enc(pin.states_k[s:], pin.basis_k),
+                          coeff_v=enc(pin.states_v[s:], pin.basis_v),
+                          basis_k=pin.basis_k.double().numpy(), basis_v=pin.basis_v.double().numpy(),
+                          sink_k=pin.states_k[:s].double().numpy(), sink_v=pin.states_v[:s].double().numpy(),
+                          n_heads_kv=w.n_heads_kv, local_window=w.local_window, top_k=w.top_k,
+                          pool_kernel=w.pool_kernel)
 
 
-def time_oracle(w, n_calls=None, budget_s=15.0, warmup=1):
+def time_oracle(w, budget_s=15.0, max_calls=50, min_calls=1, threads=None):
+    """The oracle timed on one full-length problem; steps/s extrapolated to
+    every (layer, sequence) problem of a step."""
     import oracle
-    p = oracle_layer_sample(w)
-    for _ in range(warmup):
-        oracle.decode_step(p)
-    times, t_begin = [], time.perf_counter()
-    while True:
-        t0 = time.perf_counter()
-        oracle.decode_step(p)
-        times.append(time.perf_counter() - t0)
-        if n_calls is not None and len(times) >= n_calls:
-            break
-        if n_calls is None and (time.perf_counter() - t_begin > budget_s or len(times) >= 50):
-            break
+    p = oracle_problem(w)
+    n_cores = oracle.threads() if threads is None else threads
+    if threads is not None:
+        oracle.set_threads(threads)
+    try:
+        oracle.decode_step(p)            # warm-up
+        times, t_begin = [], time.perf_counter()
+        while len(times) < max_calls and (len(times) < min_calls or time.perf_counter() - t_begin < budget_s):
+            t0 = time.perf_counter()
+            oracle.decode_step(p)
+            times.append(time.perf_counter() - t0)
+    finally:
+        if threads is not None:
+            oracle.set_threads(n_cores_all())
     t = statistics.mean(times)
-    problems_per_step = w.layers * w.batch
-    return {"value": 1.0 / (t * problems_per_step), "unit": "steps/s", "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": f"{len(times)} oracle decode calls of one (sequence, layer) problem at full "
-                      f"length (L={synth.lengths(w)[0]}, r={w.rank}); a step is {problems_per_step} "
-                      f"such problems, mean {t * 1e3:.1f} ms per problem"}, times
+    per_step = w.layers * w.batch
+    L = synth.lengths(w)[0]
+    return {"value": 1.0 / (t * per_step), "unit": "steps/s", "cores": n_cores, "kind": "oracle",
+            "sample": f"{len(times)} oracle decode calls of one (sequence, layer) problem at full length "
+                      f"(L={L}, r={w.rank}), mean {t * 1e3:.1f} ms; a step is {per_step} such problems"}
+
+
+def n_cores_all() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
 
 
 # ----------------------------------------------------------------- main legs
 
 def run_reference(args, w, rank):
+    """The reference arm: the fp64 oracle on the host cores.  One step is the
+    full step of the workload: one oracle decode call per (layer, sequence)
+    problem, on one full-length problem standing in for each of them."""
     if rank != 0:
         return
     import oracle
     oracle.build()
-    p = oracle_layer_sample(w)
+    p = oracle_problem(w)
+    per_step = w.layers * w.batch
+
+    def one_step():
+        for _ in range(per_step):
+            oracle.decode_step(p)
+
     for _ in range(args.warmup):
-        oracle.decode_step(p)
+        one_step()
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.decode_step(p)
+        one_step()
         times.append(time.perf_counter() - t0)
-    t = statistics.mean(times) * w.layers * w.batch
+    t = statistics.mean(times)
     value = 1.0 / t
+    cores = oracle.threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "layers": w.layers, "batch": w.batch,
-                       "prompt_len": synth.lengths(w)[0], "rank": w.rank, "top_k": w.top_k,
-                       "local_window": w.local_window, "query_window": w.query_window},
-            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": oracle.threads(),
-                             "kind": "oracle",
-                             "sample": f"each step = one oracle decode call of one (sequence, layer) "
-                                       f"problem at full length, scaled by {w.layers * w.batch} "
-                                       f"problems per step"},
+            "config": headline_config(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step = {per_step} oracle decode calls (one per layer) on one "
+                                       f"full-length (sequence, layer) problem (L={synth.lengths(w)[0]}, "
+                                       f"r={w.rank})"},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_encode_bench(w, device, reps=5):
+def run_encode_bench(device, reps=5):
     import rank_decode_attention_b200 as s4r
-    n, D, r = synth.BULK_ENCODE_TOKENS, w.d_model, 256
+    n, D, r = synth.BULK_ENCODE_TOKENS, 1024, 256
     g = torch.Generator(device=device).manual_seed(1234)
     S = [synth.store(torch.randn(n, D, generator=g, device=device, dtype=torch.float32), "bf16")
          for _ in range(2)]
@@ -323,7 +555,7 @@ def run_encode_bench(w, device, reps=5):
     return {"tokens": n, "rank": r, "tokens_per_s": n / t, "ms_k_plus_v": t * 1e3,
             "tflops": flops / t / 1e12, "hbm_gbs": nbytes / t / 1e9,
             "frac_hbm": nbytes / t / 1e9 / hbm, "frac_tensor": flops / t / 1e12 / bf16_tf,
-            "peaks": src}
+            "peaks": src, "timing": f"CUDA events around {reps} x (K + V) encode calls, inputs 268 MB"}
 
 
 def run_basis_bench(w, device, reps=3):
@@ -358,7 +590,39 @@ def run_basis_bench(w, device, reps=3):
     return {"problems": P, "n_sample": w.n_sample, "rank": r, "gram_dim": m, "ms_all_problems": t * 1e3,
             "us_per_basis": t / P * 1e6, "status": s4r.s4r_status_string(status),
             "timing": "CUDA events around the whole call (6 kernels: sample norms, Gram, "
-                      "cooperative Jacobi sweeps, order, columns, sign and output)"}
+                      "cooperative Jacobi sweeps, order, columns, sign and output), mean of "
+                      f"{reps} calls after one untimed call"}
+
+
+def run_extra(key, args, device):
+    """One entry of `workloads`: a configuration other than the headline."""
+    batched = key.endswith("b")
+    w = synth.WORKLOADS[int(key.rstrip("b"))]
+    steps = min(args.steps, w.steps) if w.append else args.steps
+    n_win = max(1, min(steps, w.steps, MAX_WINDOWS))
+    append_rows = (args.warmup + 3 * steps + 8) if w.append else 0
+    wl = GpuWorkload(w, 0, device, n_win, append_rows=append_rows)
+    res = time_decode(wl, steps, args.warmup, batched, None, device, 1)
+    hbm, _, src = peaks()
+    label = w.name + ("/layers-in-one-call" if batched else "")
+    step_bytes, roof = roofline_entry(w, wl, batched, res, steps, hbm, src, label)
+    calls = (f"all {w.layers * w.batch} (layer, sequence) problems in ONE call per step (layers batched, "
+             "not a model's sequential order), CUDA graph per step") if batched else \
+        (f"{w.layers} sequential per-layer calls per step" if w.layers > 1 else "1 call per step") + \
+        (", each preceded by s4r_append of one token per sequence" if w.append else "") + ", CUDA graph per step"
+    cfg = workload_config(w, calls)
+    l2 = ("per-step reads exceed L2" if step_bytes > 126e6 else
+          "per-step reads fit in L2 (latency-bound; no flush)")
+    cfg["l2"] = f"{l2}: {step_bytes / 1e6:.1f} MB read per step"
+    entry = {"value": replica_value(1, steps, res["elapsed"]), "unit": "steps/s", "steps": steps,
+             "warmup": args.warmup, "ms_per_step": res["elapsed"] / steps * 1e3, "config": cfg,
+             "roofline": roof, "e2e": res["e2e"], "gpu_launches": steps * wl.launches_per_step(batched),
+             "clocks": None}
+    if not args.no_cpu_baseline:
+        entry["cpu_baseline"] = time_oracle(w, budget_s=3.0, max_calls=3)
+    del wl
+    torch.cuda.empty_cache()
+    return label, entry
 
 
 def run_s4r(args, w, rank, world, local_rank):
@@ -367,145 +631,47 @@ def run_s4r(args, w, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     dist = torch.distributed if world > 1 else None
-    n_windows = max(1, min(args.steps, w.steps))
+    n_windows = max(1, min(args.steps, w.steps, 64))
     wl = GpuWorkload(w, rank, device, n_windows)
-    # One graph per distinct query window holding the 32 per-layer calls.  A
-    # second set carries an event pair around every layer's scoring kernel;
-    # it is timed in its own pass, because event nodes between kernels stop
-    # the kernels on either side from overlapping their launch.
-    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(w.layers)] for _ in range(n_windows)]
-    for evs in events:
-        for a, b in evs:
-            a.record(); b.record()          # materialise the event handles
-    torch.cuda.synchronize()
-    stream = torch.cuda.Stream(device)
-    graphs, graphs_ev = [], []
-    with torch.cuda.stream(stream):
-        wl.step_calls(0)                    # warm the launch path before capture
-        torch.cuda.synchronize()
-        for t in range(n_windows):
-            for evs, dst in ((None, graphs), (events[t], graphs_ev)):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    wl.step_calls(t, evs)
-                dst.append(g)
-    torch.cuda.synchronize()
-    for i in range(args.warmup):
-        graphs[i % n_windows].replay()
-    torch.cuda.synchronize()
-
     clocks = ClockSampler(device.index)
     clocks.start()
     time.sleep(0.05)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0 = time.perf_counter()
-    torch.cuda.cudart().cudaProfilerStart()   # a profiler started with capture off sees this region only
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(args.steps):
-            graphs[i % n_windows].replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    torch.cuda.cudart().cudaProfilerStop()
-    h1 = time.perf_counter()
-    if dist:
-        dist.barrier()
+    res = time_decode(wl, args.steps, args.warmup, False, dist, device, world, clocks)
     clocks.stop()
-    elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
-    value = replica_value(world, args.steps, elapsed)
-
-    # The same K steps again with the event pairs around the scoring kernels.
-    graphs_ev[0].replay()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(args.steps):
-            graphs_ev[i % n_windows].replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    elapsed_ev = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
-    score_ms = []
-    for i in range(min(args.steps, n_windows)):
-        score_ms += [a.elapsed_time(b) for a, b in events[i]]
-
-    # End to end through the public API from pinned host memory: every step
-    # copies its new query row of every layer host->device, makes the 32
-    # per-layer s4r_decode_step calls (no graph) and reads the outputs
-    # (out + idx) back to pinned host memory.
-    B, W = w.batch, w.query_window
-    call_args = [[wl.args(l, t) for l in range(w.layers)] for t in range(n_windows)]
-    host_q = [wl.layers[l]["q"].cpu().pin_memory() for l in range(w.layers)]
-    host_out = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-    host_idx = torch.empty(wl.idx.shape, dtype=wl.idx.dtype).pin_memory()
-    h2d = sum(hq[0, :, W - 1].numel() * hq.element_size() for hq in host_q)
-    d2h = host_out.numel() * 4 + host_idx.numel() * 4
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for i in range(args.steps):
-            t = i % n_windows
-            for l in range(w.layers):
-                wl.layers[l]["q"][t, :, W - 1].copy_(host_q[l][t, :, W - 1], non_blocking=True)
-            for l in range(w.layers):
-                s4r.s4r_decode_step(call_args[t][l])
-            host_out.copy_(wl.out, non_blocking=True)
-            host_idx.copy_(wl.idx, non_blocking=True)
-        f1.record(stream)
-    torch.cuda.synchronize()
-    e2e_elapsed = max_over_ranks(f0.elapsed_time(f1) / 1e3, dist, device)
-    e2e_value = replica_value(world, args.steps, e2e_elapsed)
-
-    status = s4r.s4r_read_device_status(wl.ws)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
-
+    value = replica_value(world, args.steps, res["elapsed"])
+    launches = wl.launches_per_step(False)
     if rank != 0:
         return
     hbm, bf16_tf, src = peaks()
-    step_bytes, score_bytes = algorithmic_bytes(w, wl.Lc)
-    avg_score_s = statistics.mean(score_ms) / 1e3
-    achieved = score_bytes / avg_score_s / 1e9
-    traffic = profiled_traffic("latent_scoring")
+    step_bytes, roof = roofline_entry(w, wl, False, res, args.steps, hbm, src, w.name)
+    del wl
+    torch.cuda.empty_cache()
+    cfg = headline_config(w, world)
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage": w.dtype,
-        "data": "synthetic",
-        "config": {"workload": w.name, "layers": w.layers, "batch": w.batch,
-                   "prompt_len": synth.lengths(w)[0], "rank": w.rank, "top_k": w.top_k,
-                   "local_window": w.local_window, "query_window": w.query_window,
-                   "n_heads_q": w.n_heads_q, "n_heads_kv": w.n_heads_kv, "head_dim": w.head_dim,
-                   "calls": "32 sequential per-layer calls per step, CUDA graph per step",
-                   "l2": f"inputs larger than L2: {step_bytes * w.layers / 1e6:.1f} MB read per step",
-                   "parallelism": f"replicas x{world}"},
-        "achieved_step_gbs": step_bytes * w.layers / (elapsed / args.steps) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "latent_scoring", "achieved": achieved,
-                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_source": src,
-                     "traffic": traffic, "algorithmic_bytes_per_launch": score_bytes,
-                     "avg_launch_us": avg_score_s * 1e6, "launches_timed": len(score_ms),
-                     "timing": "CUDA events on the launching stream around every layer's scoring kernel, "
-                               "in a second timed pass of the same steps",
-                     "ms_per_step_with_events": elapsed_ev / args.steps * 1e3},
-        "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * w.layers * wl.launches_per_call,
-        "clocks": clocks.summary(h0, h1),
+        "warmup": args.warmup, "ms_per_step": res["elapsed"] / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage": w.dtype, "data": "synthetic",
+        "config": cfg,
+        "achieved_step_gbs": roof["whole_path_gbs"],
+        "roofline": roof,
+        "e2e": res["e2e"],
+        "gpu_launches": args.steps * launches,
+        "clocks": res["clocks"],
     }
+    if world == 1 and args.extra != "none":
+        line["workloads"] = {}
+        for key in args.extra.split(","):
+            label, entry = run_extra(key.strip(), args, device)
+            line["workloads"][label] = entry
     if not args.no_encode:
-        line["encode"] = run_encode_bench(w, device)
+        line["encode"] = run_encode_bench(device)
     if not args.no_basis and world == 1:
         line["basis"] = run_basis_bench(w, device)
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        cpu, _ = time_oracle(w)
+        cpu = time_oracle(w)
+        cpu["single_thread"] = time_oracle(w, budget_s=4.0, max_calls=3, min_calls=2, threads=1)
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
 
@@ -513,10 +679,12 @@ def run_s4r(args, w, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="s4r", choices=["s4r", "reference"])
     ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--extra", default=EXTRA_DEFAULT,
+                    help="comma list of other workloads to time on one GPU (0,2,3,4,1b,3b) or 'none'")
     ap.add_argument("--no-encode", action="store_true")
     ap.add_argument("--no-basis", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

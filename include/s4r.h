@@ -85,7 +85,7 @@ typedef enum { S4R_POOL_MAX = 0, S4R_POOL_AVG = 1 } s4r_pool_mode;
 #define S4R_MAX_D_MODEL 1024    /* D' */
 #define S4R_MAX_RANK 256        /* rank_k, rank_v; multiples of 8 */
 #define S4R_MAX_HEAD_DIM 256    /* multiple of 8 */
-#define S4R_MAX_SCORE_ROWS 256  /* W*G (CONCAT) or W*H_q (PER_HEAD) */
+#define S4R_MAX_SCORE_ROWS 512  /* W*G (CONCAT) or W*H_q (PER_HEAD) */
 #define S4R_MAX_POOL_KERNEL 63  /* odd */
 #define S4R_MAX_GROUP 8         /* G = n_heads_q / n_heads_kv */
 #define S4R_MAX_SINKS 16        /* n_sink */

@@ -81,6 +81,7 @@ def _load():
         lib.s4r_oracle_decode_given_idx.argtypes = [P, dp, ctypes.c_int64, dp]
         lib.s4r_oracle_decode_step.argtypes = [P, dp, dp, dp]
         lib.s4r_oracle_threads.argtypes = []
+        lib.s4r_oracle_set_threads.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -88,6 +89,11 @@ def _load():
 def threads() -> int:
     """OpenMP threads the oracle uses (set OMP_NUM_THREADS before loading)."""
     return int(_load().s4r_oracle_threads())
+
+
+def set_threads(n: int) -> int:
+    """Use n OpenMP threads from now on (results do not depend on n)."""
+    return int(_load().s4r_oracle_set_threads(int(n)))
 
 
 def _f64(a) -> np.ndarray:

@@ -28,6 +28,13 @@ int s4r_oracle_threads(void) {
 #endif
 }
 
+int s4r_oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#endif
+  return s4r_oracle_threads();
+}
+
 /* Eq. 3 ("What carries the argument"): every non-sink token state s is stored
  * as its coefficients c = s . B in the rank-r basis B (D' x r). */
 void s4r_oracle_encode(const double *S, int64_t n, int32_t d, const double *B,

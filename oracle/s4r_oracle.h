@@ -90,6 +90,11 @@ int s4r_oracle_decode_step(const s4r_oracle_problem *p, double *out,
 /* Number of OpenMP threads the oracle runs on (1 when built without OpenMP). */
 int s4r_oracle_threads(void);
 
+/* Set the number of OpenMP threads for later calls (n >= 1); returns the
+ * number now in effect.  Results do not depend on it: every output is a
+ * sequential sum computed by one thread. */
+int s4r_oracle_set_threads(int n);
+
 #ifdef __cplusplus
 }
 #endif

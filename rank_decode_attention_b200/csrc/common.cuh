@@ -93,7 +93,10 @@ __device__ __forceinline__ int64_t n_candidates(int64_t L, int32_t w) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Bins of the float-exponent histogram of the candidate scores (bits 30..23).
-constexpr int kExpBins = 256;
+// Bins of the histogram of the candidate scores' leading bits: the IEEE bit
+// pattern of a non-negative float orders like its value, and bits 30..19
+// (exponent and the top 4 mantissa bits) index 4096 bins.
+constexpr int kExpBins = 4096;
+constexpr int kExpShift = 19;
 
 }  // namespace s4r

@@ -79,7 +79,7 @@ template <typename T>
 __global__ void __launch_bounds__(kProjThreads)
 project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, float *__restrict__ cq,
                unsigned char *__restrict__ cqs, float *__restrict__ qt, double *__restrict__ row_sum,
-               uint32_t *__restrict__ ehist, unsigned int *__restrict__ barrier) {
+               uint32_t *__restrict__ ehist, unsigned int *__restrict__ counters) {
   // Raw storage-type slices, copied with 16-byte cp.async (all in flight at once).
   __shared__ __align__(16) T qraw[kProjRowBlock][128];                  // per-head query rows, 128 of d_h
   __shared__ __align__(16) T braw[128][kProjColBlock + 16 / sizeof(T)];  // basis slice (padded rows)
@@ -109,7 +109,7 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   if (rank == 0 && cb == 0 && rb == 0) {
     for (int e = threadIdx.x; e < kStcSumSlots * R; e += blockDim.x) row_sum[(int64_t)b * kStcSumSlots * R + e] = 0.0;
     for (int e = threadIdx.x; e < kExpBins; e += blockDim.x) ehist[(int64_t)b * kExpBins + e] = 0u;
-    if (b == 0 && threadIdx.x < kBarWords) barrier[threadIdx.x] = 0u;
+    if (threadIdx.x == 0) counters[b] = 0u;
   }
   const int n_prow = W * G;  // per-head rows (w, j) of one group
   const int pr0 = rb * kProjRowBlock;

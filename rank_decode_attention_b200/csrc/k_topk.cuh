@@ -373,51 +373,79 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
 // ---------------------------------------------------------------------------
 // Cluster variant: the kTopkCl CTAs of a cluster split one problem's
 // candidates into contiguous shares held in shared memory.  The threshold
-// key tau is found by a radix select on the float bit patterns, one 8-bit
-// digit per pass from the exponent down (bits 30-23, 22-15, 14-7, 7-0):
-//   * every rank histograms its keys that match the digits chosen so far and
-//     copies the histogram into every rank (distributed shared memory, one
-//     bulk copy per destination completing on that pass's mbarrier); each
-//     rank then sums the ranks' histograms and takes the same decision: the
-//     digit of tau, and every rank's keys in higher bins (which are > tau);
-//   * a bin that is taken whole ends the search (tau = its lower bound - 1);
-//     otherwise the fourth pass resolves every bit of tau.
-// With the scoring kernel's exponent histogram the first pass is read, not
-// computed.  Passes cost one exchange each; no keys move between ranks.
-// Every rank then knows every rank's counts of keys > tau and == tau, hence
-// its own output offset; a stable compaction in index order writes the
-// rank's keys > tau and its share of the keys == tau (lower positions first).
+// key tau is found from histograms of the float bit patterns in up to three
+// levels of digits (bits 30-19 and 18-7 in 4096 bins, bits 6-0 in 128):
+//   * level 0 comes from the histogram the scoring kernel leaves for these
+//     candidates (or, without it, from every rank's histogram of its keys,
+//     exchanged through distributed shared memory); every rank takes the
+//     same decision: the bin holding the remaining-th largest key;
+//   * if that bin holds at most kTopkGather keys, every rank publishes its
+//     keys of the bin (with their positions, in position order) and its count
+//     of keys above the bin; after one cluster barrier every rank reads them
+//     all, finds tau among the gathered keys by a radix select and knows
+//     every rank's counts of keys > tau and == tau;
+//   * a bin taken whole needs only the ranks' counts; a fuller bin goes down
+//     one level; at the last level every bit of tau is fixed.
+// Usually that is one exchange.  No keys move except the threshold bin's.
+// A stable compaction in index order then writes the rank's keys > tau and
+// its share of the keys == tau (lower positions first).
 constexpr int kTopkCl = 8;                       // CTAs per problem
 constexpr int kTopkClThreads = 512;
-constexpr int kTopkClWarps = kTopkClThreads / 32;
 constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
-constexpr int kTopkHistRow = kTopkBins + 4;      // histogram row as copied: 256 bins, one count, padding
-__host__ inline size_t topk_cl_smem_bytes() { return sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1); }
+constexpr int kTopkLvlBins = 4096;               // bins of levels 0 and 1
+constexpr int kTopkGather = 2048;                // keys of the threshold bin gathered into every rank at most
+static_assert(kTopkLvlBins == kExpBins && kExpShift == 19, "level-0 digits are the scoring histogram's bins");
 
 struct __align__(16) TopkClShared {
-  uint32_t hist[kTopkBins];                 // summed histogram of the current pass
-  uint32_t lhist[4][kTopkBins];             // this rank's histogram (warp w adds into copy w % 4)
-  uint32_t out_hist[2][kTopkHistRow];       // the summed copy sent to every rank, two passes in flight
-  uint64_t hbar[4];                         // per pass: every rank's histogram has arrived
-  // Every rank's histogram (copied in by that rank), two passes in flight.
-  // Word kTopkBins carries the sender's count of keys above the exponent
-  // chosen from the scoring kernel's histogram (pass 1 only).
-  uint32_t g_hist[2][kTopkCl][kTopkHistRow];
-  uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau so far / in the chosen bin
+  uint32_t hist[kTopkLvlBins];              // summed histogram of the current level
+  uint32_t pub_hist[2][kTopkLvlBins];       // this rank's histogram of a level (two in flight), read by every rank
+  uint2 pub_cand[kTopkGather];              // this rank's keys of the threshold bin (key, position), position order
+  uint2 gath[kTopkGather];                  // every rank's keys of the bin, rank order
+  uint32_t pub_hdr[4];                      // this rank's count of keys above the bin, of keys in it
+  uint32_t g_gt[kTopkCl], g_n[kTopkCl], g_off[kTopkCl + 1];
+  uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau / == tau
+  uint32_t sel_hist[256];
   uint32_t warp_tot[32];
-  uint32_t total, digit, above, my_gt0;
-  // The threshold, how many keys equal to it are taken overall, and this
-  // rank's output offset and equal keys before it.
-  uint32_t tau, take_eq, out_before, eq_before;
+  uint32_t total, digit, above, mode, out_before, eq_before;
 };
+__host__ inline size_t topk_cl_smem_bytes() {
+  return sizeof(TopkClShared) + sizeof(uint32_t) * ((size_t)kpad(kTopkClKeys) + 1);
+}
 
-// Warp 0: the digit (from the top) whose bin holds the remaining-th largest
-// key of sh.hist, and how many keys lie in higher bins.
-__device__ __forceinline__ void cl_pick_digit(TopkClShared &sh, uint32_t remaining) {
+// Shift and number of bins of digit level l.
+__device__ __forceinline__ int cl_shift(int l) { return l == 0 ? 19 : (l == 1 ? 7 : 0); }
+__device__ __forceinline__ int cl_bins(int l) { return l < 2 ? kTopkLvlBins : 128; }
+
+// The bin (from the top) of `hist` holding the remaining-th largest key, and
+// how many keys lie in higher bins: sh.digit, sh.above.  Thread t owns bins
+// nbins-1-8t .. nbins-8-8t; a block scan orders the threads' counts.
+__device__ __forceinline__ void cl_pick_bin(TopkClShared &sh, const uint32_t *hist, int nbins, uint32_t remaining) {
+  uint32_t cnt[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int b = nbins - 1 - (8 * (int)threadIdx.x + j);
+    cnt[j] = b >= 0 ? hist[b] : 0u;
+    sum += cnt[j];
+  }
+  uint32_t run = block_excl_scan(sum, sh.warp_tot, &sh.total);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (run < remaining && run + cnt[j] >= remaining) {
+      sh.digit = (uint32_t)(nbins - 1 - (8 * (int)threadIdx.x + j));
+      sh.above = run;
+    }
+    run += cnt[j];
+  }
+  __syncthreads();
+}
+
+// Warp 0: the digit (from the top) of a 256-bin histogram holding the
+// remaining-th largest key, and the count in higher bins.
+__device__ __forceinline__ void cl_pick_digit256(TopkClShared &sh, const uint32_t *hist, uint32_t remaining) {
   const int lane = threadIdx.x & 31;
   uint32_t cnt[8], sum = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) { cnt[j] = sh.hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
+  for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - (lane * 8 + j)]; sum += cnt[j]; }
   uint32_t incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -435,28 +463,34 @@ __device__ __forceinline__ void cl_pick_digit(TopkClShared &sh, uint32_t remaini
   }
 }
 
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 ld_cluster_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr) : "memory");
+  return v;
+}
+
 __global__ void __cluster_dims__(kTopkCl, 1, 1) __launch_bounds__(kTopkClThreads, 1)
 topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restrict__ keys_all,
                     const uint32_t *__restrict__ ehist, int32_t *__restrict__ idx, uint32_t *__restrict__ status) {
-  extern __shared__ __align__(16) uint32_t tcl_dyn[];
-  __shared__ TopkClShared sh;
-  uint32_t *keys_s = tcl_dyn;                                   // this rank's keys (padded)
-  // The ranks exchange histograms by bulk copies completing on per-pass
-  // mbarriers; they are initialised, and the cluster synchronised once,
-  // before waiting for the scoring kernel.
-  if (threadIdx.x == 0) {
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(&sh.hbar[q], 1);
-      mbar_arrive_expect_tx(&sh.hbar[q], (uint32_t)(kTopkCl * kTopkHistRow * sizeof(uint32_t)));
-    }
-    mbar_fence_init();
-  }
-  cluster_sync();
+  extern __shared__ __align__(16) unsigned char tcl_dyn[];
+  TopkClShared &sh = *reinterpret_cast<TopkClShared *>(tcl_dyn);
+  uint32_t *keys_s = reinterpret_cast<uint32_t *>(tcl_dyn + sizeof(TopkClShared));   // this rank's keys (padded)
   pdl_wait();      // scores come from the preceding kernel
   pdl_trigger();
   const uint32_t rank = cluster_ctarank();
   const int b = blockIdx.y;
-  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t Lraw = lengths[b];
   if (rank == 0 && threadIdx.x == 0 && (Lraw < 0 || Lraw > s.cache_rows)) set_status(status, kDevStatusCheck);
   const int64_t L = valid_length(Lraw, s.cache_rows);
@@ -475,128 +509,164 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   const int chunk = (nc + kTopkCl - 1) / kTopkCl;
   const int i_begin = min(nc, (int)rank * chunk), i_end = min(nc, i_begin + chunk);
   const int my_n = i_end - i_begin;
-  // The scoring kernel's exponent histogram is read while the keys stage.
-  uint32_t eh = 0u;
-  if (ehist != nullptr && threadIdx.x < kTopkBins) eh = __ldcg(ehist + (int64_t)b * kExpBins + threadIdx.x);
   // Asynchronous 4-byte copies: every load of the share is in flight at once.
   for (int i = threadIdx.x; i < my_n; i += blockDim.x)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(keys_s + kpad(i))),
                  "l"(gkeys + i_begin + i)
                  : "memory");
-  for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
-  if (threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] = 0u;
-  if (threadIdx.x == 0) {
-    sh.my_gt0 = 0u;
-  }
+  // Level 0 from the scoring kernel's histogram, read while the keys stage.
+  if (ehist != nullptr)
+    for (int i = threadIdx.x; i < kTopkLvlBins; i += blockDim.x) sh.hist[i] = __ldcg(ehist + (int64_t)b * kExpBins + i);
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
-  // This rank's histogram of the keys matching (prefix, mask) at digit
-  // `shift`, copied into slot `pass & 1` of every rank (completing on their
-  // hbar[pass]).  Scores are >= 0, so their bit patterns order like the
-  // values and bit 31 is clear.  A slot is refilled two passes later, after
-  // this rank has received the pass in between from every rank, which each
-  // rank sent only after reading the slot.
-  // With exp_above < 256 the same loop also counts the keys whose exponent
-  // lies above it (into my_gt0, copied with the histogram).
-  auto histogram_and_store = [&](uint32_t prefix, uint32_t mask, int shift, int pass, uint32_t exp_above) {
-    const int buf = pass & 1;
-    uint32_t above = 0u;
-    for (int i = threadIdx.x; i < my_n; i += blockDim.x) {
-      const uint32_t v = keys_s[kpad(i)];
-      if ((v & mask) == prefix) atomicAdd(&sh.lhist[wid & 3][(v >> shift) & 255u], 1u);
-      above += ((v >> 23) & 255u) > exp_above;
-    }
-    if (exp_above < 256u) {
-      above = warp_sum_u32(above);
-      if (lane == 0 && above) atomicAdd(&sh.my_gt0, above);
-    }
-    __syncthreads();
-    if (threadIdx.x < kTopkBins)
-      sh.out_hist[buf][threadIdx.x] = sh.lhist[0][threadIdx.x] + sh.lhist[1][threadIdx.x] + sh.lhist[2][threadIdx.x] +
-                                      sh.lhist[3][threadIdx.x];
-    else if (threadIdx.x < kTopkHistRow)
-      sh.out_hist[buf][threadIdx.x] = threadIdx.x == kTopkBins ? sh.my_gt0 : 0u;
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the copies read it through the async proxy
-    __syncthreads();
-    if (threadIdx.x < kTopkCl)
-      bulk_copy_to_peer(cluster_map(&sh.g_hist[buf][rank][0], threadIdx.x), &sh.out_hist[buf][0],
-                        (uint32_t)(kTopkHistRow * sizeof(uint32_t)), cluster_map(&sh.hbar[pass], threadIdx.x));
-    for (int j = threadIdx.x; j < 4 * kTopkBins; j += blockDim.x) (&sh.lhist[0][0])[j] = 0u;
-  };
+  // Per-thread contiguous chunk of the rank's keys (the compactions walk it).
+  const int per = (my_n + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int j0 = min(my_n, (int)threadIdx.x * per), j1 = min(my_n, j0 + per);
 
-  uint32_t prefix = 0u, mask = 0x80000000u, remaining = (uint32_t)need;
-  uint32_t tau = 0u, take_eq = 0u, exp_above = 256u;
-  int first_pass = 0;
-  if (ehist != nullptr) {
-    // Pass 0 (the exponent) from the histogram the scoring kernel left for
-    // these candidates; every rank counts its own keys above that exponent
-    // in its pass-1 histogram loop and sends the count along with it.
-    if (threadIdx.x < kTopkBins) sh.hist[threadIdx.x] = eh;
-    __syncthreads();
-    if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
-    __syncthreads();
-    exp_above = sh.digit;
-    remaining -= sh.above;
-    prefix = exp_above << 23;
-    mask |= 255u << 23;
-    first_pass = 1;
-  } else {
-    histogram_and_store(prefix, mask, 23, 0, 256u);
-    mbar_wait(&sh.hbar[0], 0, status);
-  }
-  for (int pass = first_pass;; ++pass) {
-    const int buf = pass & 1, shift = pass < 3 ? 23 - 8 * pass : 0;   // 23, 15, 7, 0
-    if (pass > 0) {
-      histogram_and_store(prefix, mask, shift, pass, pass == first_pass ? exp_above : 256u);
-      mbar_wait(&sh.hbar[pass], 0, status);
-      if (pass == first_pass && threadIdx.x < kTopkCl) sh.gt_acc[threadIdx.x] += sh.g_hist[buf][threadIdx.x][kTopkBins];
+  uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)need;
+  uint32_t tau = 0u, take_eq = 0u;
+  int mode = 0;              // 1: bin taken whole; 2: every bit fixed; 3: threshold bin gathered
+  for (int level = 0; level < 3 && mode == 0; ++level) {
+    const int shift = cl_shift(level), nbins = cl_bins(level);
+    if (level > 0 || ehist == nullptr) {
+      // This rank's histogram of the keys that match the digits fixed so far,
+      // summed over the ranks through distributed shared memory.
+      uint32_t *ph = sh.pub_hist[level & 1];
+      for (int i = threadIdx.x; i < nbins; i += blockDim.x) ph[i] = 0u;
+      __syncthreads();
+      for (int i = threadIdx.x; i < my_n; i += blockDim.x) {
+        const uint32_t v = keys_s[kpad(i)];
+        if ((v & mask) == prefix) atomicAdd(&ph[(v >> shift) & (uint32_t)(nbins - 1)], 1u);
+      }
+      cluster_sync();
+      for (int i = 4 * (int)threadIdx.x; i < nbins; i += 4 * (int)blockDim.x) {
+        uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+        for (int rr = 0; rr < kTopkCl; ++rr) {
+          const uint4 v = ld_cluster_v4(cluster_map(&ph[i], (uint32_t)rr));
+          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        *reinterpret_cast<uint4 *>(&sh.hist[i]) = acc;
+      }
+      __syncthreads();
     }
-    // Every rank holds every rank's histogram and takes the same decisions.
-    if (threadIdx.x < kTopkBins) {
-      uint32_t h = 0;
-#pragma unroll
-      for (int c = 0; c < kTopkCl; ++c) h += sh.g_hist[buf][c][threadIdx.x];
-      sh.hist[threadIdx.x] = h;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) cl_pick_digit(sh, remaining);
-    __syncthreads();
+    cl_pick_bin(sh, sh.hist, nbins, remaining);
     const uint32_t d = sh.digit, in_bin = sh.hist[d];
     remaining -= sh.above;
-    if (threadIdx.x < kTopkBins) {
-#pragma unroll
-      for (int c = 0; c < kTopkCl; ++c) {
-        const uint32_t g = __reduce_add_sync(0xffffffffu, (uint32_t)threadIdx.x > d ? sh.g_hist[buf][c][threadIdx.x] : 0u);
-        if (lane == 0 && g) atomicAdd(&sh.gt_acc[c], g);
-      }
-    }
-    if (threadIdx.x < kTopkCl) sh.eq_acc[threadIdx.x] = sh.g_hist[buf][threadIdx.x][d];
     prefix |= d << shift;
-    mask |= 255u << shift;
+    mask |= (uint32_t)(nbins - 1) << shift;
     __syncthreads();
     if (in_bin == remaining && prefix != 0u) {
-      // Every key of the bin is taken: they are exactly the keys >= prefix
-      // within it, so tau = prefix - 1 and no equal key is rationed.
-      if (threadIdx.x < kTopkCl) {
-        sh.gt_acc[threadIdx.x] += sh.eq_acc[threadIdx.x];
-        sh.eq_acc[threadIdx.x] = 0u;
-      }
+      mode = 1;                    // every key >= prefix is taken
       tau = prefix - 1u;
       take_eq = 0u;
-      break;
-    }
-    if (pass == 3) {
-      tau = prefix;        // all 31 bits resolved: eq_acc counts the keys == tau
+    } else if (level == 2) {
+      mode = 2;                    // all 31 bits fixed
+      tau = prefix;
       take_eq = remaining;
-      break;
+    } else if (in_bin <= (uint32_t)kTopkGather) {
+      mode = 3;
     }
   }
-  // Every histogram copy into this rank has landed; the senders learn that
+
+  const uint32_t hi_bound = prefix | (~mask & 0x7fffffffu);   // largest key in the threshold bin
+  if (mode == 3) {
+    // Publish this rank's keys of the bin (stable, in position order) and
+    // its count of keys above the bin; gather every rank's.
+    uint32_t n_in = 0, n_above = 0;
+    for (int i = j0; i < j1; ++i) {
+      const uint32_t v = keys_s[kpad(i)];
+      n_in += (v & mask) == prefix;
+      n_above += v > hi_bound;
+    }
+    const uint32_t before = block_excl_scan(n_in, sh.warp_tot, &sh.total);
+    uint32_t at = before;
+    for (int i = j0; i < j1; ++i) {
+      const uint32_t v = keys_s[kpad(i)];
+      if ((v & mask) == prefix) sh.pub_cand[at++] = make_uint2(v, (uint32_t)(i_begin + i));
+    }
+    n_above = warp_sum_u32(n_above);
+    if (threadIdx.x == 0) { sh.pub_hdr[0] = 0u; sh.pub_hdr[1] = sh.total; }
+    __syncthreads();
+    if (lane == 0 && n_above) atomicAdd(&sh.pub_hdr[0], n_above);
+    cluster_sync();
+    if (threadIdx.x < kTopkCl) {
+      sh.g_gt[threadIdx.x] = ld_cluster_u32(cluster_map(&sh.pub_hdr[0], threadIdx.x));
+      sh.g_n[threadIdx.x] = ld_cluster_u32(cluster_map(&sh.pub_hdr[1], threadIdx.x));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t o = 0;
+      for (int rr = 0; rr < kTopkCl; ++rr) { sh.g_off[rr] = o; o += sh.g_n[rr]; }
+      sh.g_off[kTopkCl] = o;
+    }
+    __syncthreads();
+    const uint32_t n_g = sh.g_off[kTopkCl];   // == in_bin <= kTopkGather
+    for (uint32_t e = threadIdx.x; e < n_g; e += blockDim.x) {
+      int rr = 0;
+      while (rr + 1 < kTopkCl && e >= sh.g_off[rr + 1]) ++rr;
+      sh.gath[e] = ld_cluster_v2(cluster_map(&sh.pub_cand[e - sh.g_off[rr]], (uint32_t)rr));
+    }
+    __syncthreads();
+    // tau: the remaining-th largest gathered key (radix select on the bits below the bin).
+    uint32_t pfx = prefix, msk = mask, rem = remaining;
+    for (int sel_shift = cl_shift(0) - 8; sel_shift > -8; sel_shift -= 8) {
+      const int sh8 = sel_shift < 0 ? 0 : sel_shift;
+      if ((msk | (255u << sh8)) == msk) continue;   // these bits are fixed already
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.sel_hist[i] = 0u;
+      __syncthreads();
+      for (uint32_t e = threadIdx.x; e < n_g; e += blockDim.x) {
+        const uint32_t v = sh.gath[e].x;
+        if ((v & msk) == pfx) atomicAdd(&sh.sel_hist[(v >> sh8) & 255u], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) cl_pick_digit256(sh, sh.sel_hist, rem);
+      __syncthreads();
+      rem -= sh.above;
+      pfx |= sh.digit << sh8;
+      msk |= 255u << sh8;
+      __syncthreads();
+    }
+    tau = pfx;
+    take_eq = rem;
+    // Every rank's keys > tau and == tau: those above the bin plus its gathered keys.
+    if (threadIdx.x < kTopkCl) { sh.gt_acc[threadIdx.x] = sh.g_gt[threadIdx.x]; sh.eq_acc[threadIdx.x] = 0u; }
+    __syncthreads();
+    for (uint32_t e = threadIdx.x; e < n_g; e += blockDim.x) {
+      int rr = 0;
+      while (rr + 1 < kTopkCl && e >= sh.g_off[rr + 1]) ++rr;
+      const uint32_t v = sh.gath[e].x;
+      if (v > tau) atomicAdd(&sh.gt_acc[rr], 1u);
+      else if (v == tau) atomicAdd(&sh.eq_acc[rr], 1u);
+    }
+  } else {
+    // Modes 1 and 2: only every rank's counts of keys > tau and == tau.
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int i = j0; i < j1; ++i) {
+      const uint32_t v = keys_s[kpad(i)];
+      n_gt += v > tau;
+      n_eq += v == tau;
+    }
+    n_gt = warp_sum_u32(n_gt);
+    n_eq = warp_sum_u32(n_eq);
+    if (threadIdx.x == 0) { sh.pub_hdr[2] = 0u; sh.pub_hdr[3] = 0u; }
+    __syncthreads();
+    if (lane == 0) {
+      if (n_gt) atomicAdd(&sh.pub_hdr[2], n_gt);
+      if (n_eq) atomicAdd(&sh.pub_hdr[3], n_eq);
+    }
+    cluster_sync();
+    if (threadIdx.x < kTopkCl) {
+      sh.gt_acc[threadIdx.x] = ld_cluster_u32(cluster_map(&sh.pub_hdr[2], threadIdx.x));
+      sh.eq_acc[threadIdx.x] = ld_cluster_u32(cluster_map(&sh.pub_hdr[3], threadIdx.x));
+    }
+  }
+  // Every read of another rank's shared memory is done; the ranks learn that
   // theirs have been read only here, so no rank leaves before all arrive.
   // The arrive publishes no data, hence relaxed.
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   __syncthreads();
+  (void)wid;
   if (threadIdx.x == 0) {
     uint32_t out_before = 0, eq_before = 0;
     for (uint32_t c = 0; c < rank; ++c) {
@@ -613,8 +683,6 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   // Per-thread contiguous chunks: one scan of (n_gt << 16 | n_eq), which
   // cannot carry between the halves because a rank holds < 65536 keys.
   static_assert(kTopkClKeys < 65536, "packed counts");
-  const int per = (my_n + (int)blockDim.x - 1) / (int)blockDim.x;
-  const int j0 = min(my_n, (int)threadIdx.x * per), j1 = min(my_n, j0 + per);
   uint32_t n_gt = 0, n_eq = 0;
   for (int i = j0; i < j1; ++i) {
     const uint32_t key = keys_s[kpad(i)];

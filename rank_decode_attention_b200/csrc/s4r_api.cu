@@ -37,15 +37,15 @@ inline size_t esize(s4r_dtype dt) { return dt == S4R_BF16 ? 2 : 4; }
 
 // Byte offsets of the decode workspace regions.
 struct Layout {
-  size_t status, barrier, cq, cqs, qt, tstat, rstat, rowsum, ehist, scores, pooled, total;
+  size_t status, counters, cq, cqs, qt, tstat, rstat, rowsum, ehist, scores, pooled, total;
 };
 
 Layout layout_for(const Shape &s) {
   Layout l{};
   size_t off = 0;
   l.status = off;
-  l.barrier = off + 64;
   off += kAlign;
+  l.counters = off; off += round_up(sizeof(uint32_t) * (size_t)s.batch);
   l.cq = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_rows * s.rank_k);
   const size_t n_cb = (size_t)ceil_div(s.rank_k, kProjColBlock);
   l.cqs = off; off += round_up((size_t)s.batch * n_cb * cqs_block_bytes(s.n_rows));
@@ -222,14 +222,13 @@ s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const vo
 // Which latent-scoring kernel a decode call uses.
 struct ScorePlan {
   bool tc = false;   // tensor-core kernel (else fp64 CUDA-core passes)
-  bool two_pass = false;  // grid larger than what is resident at once: row sums, then scores
   int R = 0;         // rows per problem (template argument of the TC kernel)
-  int grid = 0;
+  int grid = 0;      // persistent cooperative grid
   size_t smem = 0;
 };
 
-// CTAs of the tensor-core scoring kernel that fit on the device at once
-// (cached per device and rank; 0 if they cannot be launched).
+// CTAs of the tensor-core scoring kernel resident at once on this device
+// (cached per device and rank; 0 if it cannot be launched).
 template <int R>
 int tc_capacity(int rank) {
   static std::atomic<int> cache[kMaxDevices][S4R_MAX_RANK / 8 + 1];   // capacity + 1; 0 = unknown
@@ -247,22 +246,10 @@ int tc_capacity(int rank) {
     cudaGetLastError();
     return 0;
   }
-  if (dev >= 0) cache[dev][slot].store(per_sm * sms + 1, std::memory_order_relaxed);
-  return per_sm * sms;
-}
-
-// 1: the fused single pass fits; 2: only the two-pass form does; 0: neither.
-template <int R>
-int tc_fits(int rank, int grid, size_t *smem_out) {
-  *smem_out = (size_t)stc_smem_bytes(R, rank);
-  const int cap = tc_capacity<R>(rank);
-  if (cap <= 0) return 0;
-  if (ensure_smem<score_tc_kernel<R, 1>>(*smem_out) != cudaSuccess ||
-      ensure_smem<score_tc_kernel<R, 2>>(*smem_out) != cudaSuccess) {
-    cudaGetLastError();
-    return grid <= cap ? 1 : 0;
-  }
-  return grid <= cap ? 1 : 2;
+  // One CTA per SM: each holds all 512 TMEM columns.
+  const int cap = per_sm > 0 ? sms : 0;
+  if (dev >= 0) cache[dev][slot].store(cap + 1, std::memory_order_relaxed);
+  return cap;
 }
 
 ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
@@ -270,45 +257,23 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   if (dt != S4R_BF16 || s.cache_rows == 0 || s.batch == 0) return p;
   if (s.n_rows != 32 && s.n_rows != 64) return p;
   if ((int64_t)s.batch * s.cache_rows >= INT32_MAX) return p;
-  const int64_t grid = (int64_t)s.batch * ceil_div(ceil_div(s.cache_rows, kStcTile), kStcTiles);
-  if (grid > (int64_t)1 << 30) return p;
-  size_t smem = 0;
-  const int fits = s.n_rows == 64 ? tc_fits<64>(s.rank_k, (int)grid, &smem) : tc_fits<32>(s.rank_k, (int)grid, &smem);
-  if (!fits) {
+  const int cap = s.n_rows == 64 ? tc_capacity<64>(s.rank_k) : tc_capacity<32>(s.rank_k);
+  if (cap <= 0) {
     cudaGetLastError();
     return p;
   }
+  const int64_t tiles = (int64_t)s.batch * ceil_div(s.cache_rows, kStcTile);
   p.tc = true;
-  p.two_pass = fits == 2;
   p.R = s.n_rows;
-  p.grid = (int)grid;
-  p.smem = smem;
+  p.grid = (int)smin<int64_t>(tiles, cap);
+  p.smem = (size_t)stc_smem_bytes(p.R, s.rank_k);
   return p;
 }
 
 template <int R>
-s4r_status launch_score_tc_two_pass(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s,
-                                    const int32_t *lengths, const unsigned char *cqs, float *scores, double *rowsum,
-                                    uint32_t *ehist, unsigned int *bar, uint32_t *status, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3(kStcThreads);
-  cfg.dynamicSmemBytes = p.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1] = {pdl_attr()};
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R, 1>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
-  if (err != cudaSuccess) return fail("score_tc_kernel (row sums)", err);
-  err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R, 2>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
-  return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (scores)", err);
-}
-
-template <int R>
 s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s, const int32_t *lengths,
-                           const unsigned char *cqs, float *scores, double *rowsum, uint32_t *ehist, unsigned int *bar,
-                           uint32_t *status,
-                           cudaStream_t st) {
+                           const unsigned char *cqs, float *scores, double *rowsum, uint32_t *ehist,
+                           unsigned int *counters, uint32_t *status, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
   cfg.blockDim = dim3(kStcThreads);
@@ -320,7 +285,8 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
   attr[1] = pdl_attr();
   cfg.attrs = attr;
   cfg.numAttrs = g_coop_pdl == 0 ? 1 : 2;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
+  cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist,
+                                       counters, status);
   if (cfg.numAttrs == 2 && g_coop_pdl < 0) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     cudaStreamIsCapturing(st, &cap);
@@ -330,7 +296,8 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
       cudaGetLastError();   // not supported together: launch without it from now on
       g_coop_pdl = 0;
       cfg.numAttrs = 1;
-      err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
+      err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, counters,
+                               status);
     }
   }
   return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (cooperative launch)", err);
@@ -347,7 +314,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
   double *rowsum = reinterpret_cast<double *>(ws + ly.rowsum);
   uint32_t *ehist = reinterpret_cast<uint32_t *>(ws + ly.ehist);
   unsigned char *cqs = ws + ly.cqs;
-  unsigned int *bar = reinterpret_cast<unsigned int *>(ws + ly.barrier);
+  unsigned int *counters = reinterpret_cast<unsigned int *>(ws + ly.counters);
   float *scores = a->scores ? a->scores : reinterpret_cast<float *>(ws + ly.scores);
   float *pooled = reinterpret_cast<float *>(ws + ly.pooled);
   const T *q = static_cast<const T *>(a->q);
@@ -374,7 +341,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    const cudaError_t err = cudaLaunchKernelEx(&cfg, project_kernel<T>, s, q, bk, cq, cqs, qt, rowsum, ehist, bar);
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, project_kernel<T>, s, q, bk, cq, cqs, qt, rowsum, ehist, counters);
     if (err != cudaSuccess) return fail("project_kernel (cluster launch)", err);
     if (check_launch("project_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
@@ -391,11 +358,8 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       return S4R_ERR_CUDA;
     }
     const s4r_status rc =
-        plan.two_pass
-            ? (plan.R == 64 ? launch_score_tc_two_pass<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st)
-                            : launch_score_tc_two_pass<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st))
-            : (plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st)
-                            : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, bar, status, st));
+        plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st)
+                     : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st);
     if (rc != S4R_OK) return rc;
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
@@ -578,7 +542,7 @@ int32_t s4r_decode_kernel_launches(const s4r_decode_args *args) {
   if (s.batch == 0) return 0;
   int32_t n = 1;                                  // projection
   const ScorePlan plan = plan_scoring(s, args->dtype);
-  if (plan.tc) n += plan.two_pass ? 2 : 1;        // scoring: tensor cores, fused or row sums + scores
+  if (plan.tc) n += 1;                            // scoring: one persistent tensor-core launch
   else if (s.cache_rows > 0) n += 3;              // scoring: stats, merge, final
   if (s.pool_kernel > 1 && s.cache_rows > 0) n += 1;
   if (s.top_k > 0) n += 1;

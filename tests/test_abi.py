@@ -115,7 +115,8 @@ def test_decode_argument_errors_are_reported_before_launch():
     ok = s4r.s4r_decode_workspace_bytes(good_args())
     assert call_decode(good_args(n_heads_q=30)) == s4r.S4R_ERR_INVALID_ARG
     assert call_decode(good_args(rank_k=12)) == s4r.S4R_ERR_UNSUPPORTED
-    assert call_decode(good_args(query_window=80)) == s4r.S4R_ERR_UNSUPPORTED   # 320 scoring rows
+    assert call_decode(good_args(query_window=160)) == s4r.S4R_ERR_UNSUPPORTED   # 640 scoring rows
+    assert call_decode(good_args(query_window=16, row_mode=1, workspace_bytes=0)) == s4r.S4R_ERR_WORKSPACE   # 512 per-head rows
     assert call_decode(good_args(q=0x2004, workspace_bytes=ok)) == s4r.S4R_ERR_INVALID_ARG
     assert call_decode(good_args(out=None, workspace_bytes=ok)) == s4r.S4R_ERR_INVALID_ARG
     assert call_decode(good_args(sink_k=None, workspace_bytes=ok)) == s4r.S4R_ERR_INVALID_ARG

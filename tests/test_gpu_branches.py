@@ -72,13 +72,13 @@ def _run(batch, y_max=None):
 
 
 def test_wide_range_every_tile():
-    # The query window scaled by a power of two (exact in bf16) until the
-    # largest |y| of the problem is near 200: every tile is past the limit,
-    # and every row's normaliser lies far above the fp32 range (2^k with k
-    # well over 128 before the offsets).
+    # The query window scaled by a power of two (exact in bf16), the smallest
+    # that takes every tile's largest |y| past 110: every tile is past the
+    # limit, and some row's normaliser lies far above the fp32 range (2^k
+    # with k over 128 before the offsets).
     batch = make_batch(W1, lengths=[5003], top_k=16, local_window=32, tag="wide-all")
-    y0 = np.abs(base2_logits(batch, 0)).max()
-    scale = 2.0 ** np.round(np.log2(200.0 / y0))
+    y0 = tile_ranges(base2_logits(batch, 0)).min()
+    scale = 2.0 ** np.ceil(np.log2(110.0 / y0))
     batch = dataclasses.replace(batch, q=(batch.q.double() * scale).to(batch.q.dtype))
     y = base2_logits(batch, 0)
     ranges = tile_ranges(y)

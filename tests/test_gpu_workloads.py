@@ -104,6 +104,15 @@ def test_ragged_append_decode_256_steps():
     assert s4r.s4r_read_device_status(ws) == s4r.S4R_OK
 
 
+def test_per_head_rows_at_the_llama_shape_32k():
+    """Per-head scoring rows (W * H_q = 16 * 32 = 512 rows, each head projected
+    with its kv group's d_h rows of the key basis) on a full-size 32K layer."""
+    batch = make_batch(W1, lengths=[W1.prompt_len - W1.n_sink], layer=5, row_mode=1, tag="per-head-32k")
+    res = run_gpu(batch)
+    assert res["status"] == 0
+    check_batch(batch, res)
+
+
 def test_bulk_encode_65536_tokens():
     import rank_decode_attention_b200 as s4r
     n, D, r = synth.BULK_ENCODE_TOKENS, 1024, 256
