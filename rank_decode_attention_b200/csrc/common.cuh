@@ -93,10 +93,33 @@ __device__ __forceinline__ int64_t n_candidates(int64_t L, int32_t w) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Bins of the histogram of the candidate scores' leading bits: the IEEE bit
-// pattern of a non-negative float orders like its value, and bits 30..19
-// (exponent and the top 4 mantissa bits) index 4096 bins.
+// Level-0 bins of the candidate scores of a problem for the top-k search.
+// The scores of a problem sum to its number of scoring rows R (each row's
+// softmax sums to 1), so their mean is R / L_c.  A score's bin is its IEEE
+// bit pattern (which orders non-negative floats like their values) minus
+// that of the mean, in steps of 2^15 (1/256 of a binade), offset by
+// kExpBins / 2 and clamped to [0, kExpBins): monotone in the score, fine
+// around the mean, and the two edge bins take everything beyond +-8 binades.
 constexpr int kExpBins = 4096;
-constexpr int kExpShift = 19;
+constexpr int kExpStep = 15;
+__host__ __device__ inline uint32_t score_center(int R, int64_t L) {
+  const float m = L > 0 ? (float)R / (float)L : 1.0f;
+  union { float f; uint32_t u; } v;
+  v.f = m;
+  return v.u;
+}
+__host__ __device__ inline int score_bin(uint32_t key, uint32_t center) {
+  const int64_t d = ((int64_t)key - (int64_t)center) >> kExpStep;   // floor for negative differences
+  const int64_t b = d + kExpBins / 2;
+  return (int)(b < 0 ? 0 : (b >= kExpBins ? kExpBins - 1 : b));
+}
+// Key range [lo, hi] of bin b.
+__host__ __device__ inline void score_bin_range(int b, uint32_t center, uint32_t &lo, uint32_t &hi) {
+  const int64_t base = (int64_t)center + ((int64_t)(b - kExpBins / 2) << kExpStep);
+  const int64_t l = b == 0 ? 0 : base;
+  const int64_t h = b == kExpBins - 1 ? 0x7fffffffLL : base + (1LL << kExpStep) - 1;
+  lo = (uint32_t)(l < 0 ? 0 : (l > 0x7fffffffLL ? 0x7fffffffLL : l));
+  hi = (uint32_t)(h < 0 ? 0 : (h > 0x7fffffffLL ? 0x7fffffffLL : h));
+}
 
 }  // namespace s4r

@@ -23,27 +23,28 @@
 //           into a ring of stages; per problem switch, the split C_Q operand
 //           (one bulk copy per k-block) into one of one or two buffers;
 //   warp 5  MMA issuer (tcgen05.mma kind::f16, M = 128);
+//   warp 6  counter watcher (arrivals and completions of the problems);
 //   warps 0-3  epilogue, one TMEM lane (position) per thread.
 // Pass 1, per tile: y, e, the tile's per-row sums (a shuffle transpose-
 // reduction, then four warps in a fixed order) added in fp64 to the CTA's sums
-// of the problem.  After its last tile of problem p the CTA adds those sums to
-// the problem's row normalisers (fp64 atomics, 16 slots per row) and arrives
-// on p's counter.  The e of a CTA's first kRetained tiles of p stay in their
+// of the problem.  After its last tile of problem p the CTA's counter watcher
+// (warp 6) adds those sums to the problem's row normalisers (fp64 atomics, 16
+// slots per row), arrives on p's counter and, once every CTA that owns tiles
+// of p has arrived, forms 1 / l_row for the epilogue.  The e of a CTA's first kRetained tiles of p stay in their
 // TMEM slot; once all min(T_p, G) CTAs that own tiles of p have arrived, the
 // epilogue forms alpha_row = 2^k / l_row (fp64) and score = sum_row alpha e
 // from the slot.  Tiles of p beyond the first kRetained keep no e: pass 2
 // streams them again (most recently loaded, so mostly from L2) and
 // recomputes e with the same arithmetic.  Problems complete independently,
 // so one problem's wait overlaps the next problem's stream.
-// It also accumulates, per problem, the histogram of the candidate scores'
-// leading 12 bits for the top-k kernel.
+// It also accumulates, per problem, the level-0 histogram of the candidate
+// scores (score_bin) for the top-k kernel.
 #pragma once
 #include "umma.cuh"
 
 namespace s4r {
 
 constexpr int kStcTile = 128;
-constexpr int kStcThreads = 192;       // warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA issuer
 constexpr float kStcRangeLimit = 100.f;
 constexpr int kStcSumSlots = 16;       // row-sum atomics spread over 16 copies per row
 constexpr int kStcMaxSmem = 232448;    // 227 KB per block on sm_100
@@ -51,7 +52,7 @@ constexpr int kStcKbBytes = kStcTile * 128;   // one 64-column k-block of a tile
 constexpr int kStcMaxStages = 12;
 constexpr int kStcMinStages = 4;
 constexpr int kStcTransient = 2;       // TMEM slots of tiles whose e is not kept
-constexpr int kStcControlBytes = 6144;
+constexpr int kStcControlBytes = 10240;
 
 template <int R>
 struct StcCfg {
@@ -60,29 +61,36 @@ struct StcCfg {
   static constexpr int kSlots = kRetained + kStcTransient;
   static constexpr int kScratchCol = kSlots * R;                 // (mid, lo) accumulator columns
   static_assert(kScratchCol + 2 * R <= 512, "TMEM columns");
+  // Epilogue: four warps per 32 scoring rows (warp w reads TMEM lanes
+  // 32 (w % 4) ...; warps w and w + 4 take rows 0-31 and 32-63).
+  static constexpr int kHalves = R / 32;
+  static constexpr int kEpiWarps = 4 * kHalves;
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kProducer = kEpiWarps, kMma = kEpiWarps + 1, kWatcher = kEpiWarps + 2;
+  static constexpr int kThreads = 32 * (kEpiWarps + 3);
 };
 
 __host__ __device__ constexpr int stc_kblocks(int r) { return (r + 63) / 64; }
 __host__ __device__ constexpr int stc_b_bytes(int R, int r) { return stc_kblocks(r) * 3 * R * 128; }
-// Split C_Q buffers: two when at least kStcMinStages ring stages still fit.
-__host__ __device__ constexpr int stc_b_buffers(int R, int r) {
-  return 1024 + 2 * stc_b_bytes(R, r) + kStcMinStages * kStcKbBytes + kStcControlBytes <= kStcMaxSmem ? 2 : 1;
+// Split C_Q buffers: one, or two (the next problem's operand loads while the
+// current one is in use) when at least kStcMinStages ring stages still fit.
+__host__ __device__ constexpr bool stc_two_b_fit(int R, int r) {
+  return 1024 + 2 * stc_b_bytes(R, r) + kStcMinStages * kStcKbBytes + kStcControlBytes <= kStcMaxSmem;
 }
-__host__ __device__ constexpr int stc_stages(int R, int r) {
-  return (kStcMaxSmem - 1024 - kStcControlBytes - stc_b_buffers(R, r) * stc_b_bytes(R, r)) / kStcKbBytes >
-                 kStcMaxStages
+__host__ __device__ constexpr int stc_stages(int R, int r, int nB) {
+  return (kStcMaxSmem - 1024 - kStcControlBytes - nB * stc_b_bytes(R, r)) / kStcKbBytes > kStcMaxStages
              ? kStcMaxStages
-             : (kStcMaxSmem - 1024 - kStcControlBytes - stc_b_buffers(R, r) * stc_b_bytes(R, r)) / kStcKbBytes;
+             : (kStcMaxSmem - 1024 - kStcControlBytes - nB * stc_b_bytes(R, r)) / kStcKbBytes;
 }
-__host__ __device__ constexpr int stc_smem_bytes(int R, int r) {
-  return 1024 + stc_b_buffers(R, r) * stc_b_bytes(R, r) + stc_stages(R, r) * kStcKbBytes + kStcControlBytes;
+__host__ __device__ constexpr int stc_smem_bytes(int R, int r, int nB) {
+  return 1024 + nB * stc_b_bytes(R, r) + stc_stages(R, r, nB) * kStcKbBytes + kStcControlBytes;
 }
-static_assert(stc_stages(64, 256) >= kStcMinStages && stc_smem_bytes(64, 256) <= kStcMaxSmem, "smem budget");
+static_assert(stc_stages(64, 256, 1) >= kStcMinStages && stc_smem_bytes(64, 256, 1) <= kStcMaxSmem, "smem budget");
 
 template <int R>
 struct StcControl {
   uint64_t full[kStcMaxStages], empty[kStcMaxStages];
-  uint64_t b_full[2], b_empty[2];
+  uint64_t b_full[2][4], b_empty[2];           // per operand buffer: each 64-column k-block landed / buffer free
   uint64_t acc_full;                         // MMA -> epilogue: the tile's accumulators are complete
   uint64_t scratch_free;                     // epilogue -> MMA: (mid, lo) columns read
   uint64_t slot_free[StcCfg<R>::kSlots];     // epilogue -> MMA: the slot may be overwritten
@@ -94,10 +102,17 @@ struct StcControl {
   int slot_p[StcCfg<R>::kRetained];          // problem of the tile in each kept slot
   int64_t slot_row0[StcCfg<R>::kRetained];   // its first row
   int kofs[R];                               // offsets of the tile in the epilogue
-  float red[4][R];                           // per-warp partial sums / maxima
-  float alpha[R];
-  double inv_l[R];
+  float red[2][4][R];                        // per lane quarter partial sums (two tiles in flight) / maxima
+  float alpha[StcCfg<R>::kRetained][R];      // per kept slot, of the problem being finished
+  float sc_part[StcCfg<R>::kHalves == 2 ? StcCfg<R>::kRetained : 1][kStcTile];   // rows 32-63's part of a score
+  double inv_l[R];                           // 1 / l of the problem in pass 2
+  double inv_q[StcCfg<R>::kRetained + 1][R]; // 1 / l of the problems the watcher saw complete (ring)
+  int ok_q[StcCfg<R>::kRetained + 1];
   int pend[StcCfg<R>::kRetained + 1];        // problems arrived on, not yet finished (FIFO)
+  int64_t pend_L[StcCfg<R>::kRetained + 1];  // and their lengths
+  volatile int arrived_seq;                  // problems the epilogue has arrived on
+  volatile int done_seq;                     // problems the watcher has seen complete
+  int done_snap;
 };
 static_assert(sizeof(StcControl<64>) <= kStcControlBytes && sizeof(StcControl<32>) <= kStcControlBytes,
               "control block");
@@ -107,90 +122,116 @@ struct StcTile {
   int p;            // problem
   int64_t row0;     // first coefficient row
   int64_t L;        // L_c of the problem
-  int k, n;         // index among the CTA's tiles of p, and their number
   int T;            // tiles of p
+  int k;            // index among the CTA's tiles of p (in this pass)
+  bool last;        // the CTA's last tile of p (pass 1)
   bool pass2;       // a second pass over a tile whose e was not kept
 };
 
-// The CTA's tiles: pass 1 visits global tiles c, c + G, ... in order; pass 2
-// revisits, problem by problem, the tiles with k >= kept.  Every role walks
-// the same sequence.
+// The CTA's tiles.  The active tiles of all problems form one list in
+// problem order (global tile g); chunks of K consecutive tiles go round-robin
+// to the CTAs: CTA c owns chunks c, c + G, c + 2G, ...  Pass 1 visits the
+// CTA's tiles in order; pass 2 revisits, problem by problem, the tiles with
+// k >= kept.  Every role walks the same sequence.
 struct StcWalker {
   const int32_t *lengths;
   int64_t cap;
-  int batch, G, c, kept;
-  int pass, p, T, n, k;
-  int64_t S, L, g0;
+  int batch, G, c, K, kept;
+  int pass;
+  int p, T, k;           // problem of the current tile, its tiles, count in this pass
+  int64_t S, L;          // first global tile and length of problem p
+  int64_t gc, g;         // next chunk and next global tile of this CTA
+  bool have_next;        // lookahead tile present
+  int64_t g_next;
 
-  __device__ void start(const int32_t *len, int64_t cap_, int batch_, int G_, int c_, int kept_) {
+  __device__ void start(const int32_t *len, int64_t cap_, int batch_, int G_, int c_, int K_, int kept_) {
     lengths = len;
     cap = cap_;
     batch = batch_;
     G = G_;
     c = c_;
+    K = K_;
     kept = kept_;
     pass = 1;
-    p = -1;
-    S = 0;
-    T = 0;
-    n = 0;
-    k = 0;
+    rewind();
   }
-  // Advance to the next problem holding tiles for this pass; false at the end.
-  __device__ bool next_problem() {
-    while (true) {
+  __device__ void rewind() {
+    p = -1;
+    T = 0;
+    S = 0;
+    k = 0;
+    gc = c;
+    g = (int64_t)c * K;
+    g_next = raw_next();
+  }
+  __device__ int64_t raw_next() {
+    if (g >= gc * K + K) {
+      gc += G;
+      g = gc * K;
+    }
+    return g++;
+  }
+  // Move the problem cursor forward to the problem holding global tile gt;
+  // false when gt lies past the last problem.
+  __device__ bool locate(int64_t gt) {
+    while (gt >= S + T) {
       S += T;
       ++p;
       T = 0;
+      k = 0;
       if (p >= batch) return false;
       const int64_t Lraw = __ldg(lengths + p);
       L = (Lraw >= 0 && Lraw <= cap) ? Lraw : 0;
       T = (int)ceil_div(L, kStcTile);
-      if (T == 0) continue;
-      const int64_t off = (((int64_t)c - S) % G + G) % G;
-      g0 = S + off;
-      n = g0 < S + T ? (int)((S + T - 1 - g0) / G) + 1 : 0;
-      const int kmin = pass == 1 ? 0 : kept;
-      if (n > kmin) {
-        k = kmin;
-        return true;
-      }
     }
+    return true;
   }
   __device__ bool next(StcTile &t) {
     while (true) {
-      if (p >= 0 && p < batch && k < n) {
-        t.p = p;
-        t.row0 = (g0 + (int64_t)k * G - S) * kStcTile;
-        t.L = L;
-        t.k = k;
-        t.n = n;
-        t.T = T;
-        t.pass2 = pass == 2;
-        ++k;
-        return true;
+      const int64_t gt = g_next;
+      const int p_before = p;
+      if (p >= batch || !locate(gt)) {
+        if (pass == 2) return false;
+        pass = 2;
+        rewind();
+        continue;
       }
-      if (next_problem()) continue;
-      if (pass == 2) return false;
-      pass = 2;
-      p = -1;
-      S = 0;
-      T = 0;
+      if (p != p_before) k = 0;
+      g_next = raw_next();
+      const int kk = k++;
+      if (pass == 2 && kk < kept) continue;   // kept in pass 1
+      t.p = p;
+      t.row0 = (gt - S) * kStcTile;
+      t.L = L;
+      t.T = T;
+      t.k = kk;
+      t.last = g_next >= S + T;
+      t.pass2 = pass == 2;
+      return true;
     }
   }
 };
 
-// Named barrier of the four epilogue warps (barrier 1, 128 threads).
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// CTAs that own tiles of a problem whose tiles are global tiles [S, S + T):
+// the chunks intersecting it, at most G.
+__device__ __forceinline__ int stc_participants(int64_t S, int T, int K, int G) {
+  const int64_t n = (S + T - 1) / K - S / K + 1;
+  return (int)(n < G ? n : G);
+}
+
+// Named barrier of the epilogue warps (barrier 1, N threads).
+template <int N>
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory"); }
+template <int N>
 __device__ __forceinline__ bool epi_or(bool v) {
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "n"(N)
       : "memory");
   return out != 0;
 }
@@ -213,27 +254,28 @@ __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32]) {
   }
 }
 
-// Arrival target of problem p's counter: every CTA that owns one of its T
+// Arrival target of a problem's counter: every CTA that owns one of its
 // tiles (one more when the test hook makes it unreachable).
-__device__ __forceinline__ uint32_t stc_target(int T, int G) {
-  return (uint32_t)(T < G ? T : G) + (*reinterpret_cast<volatile uint32_t *>(&g_barrier_unreachable) ? 1u : 0u);
+__device__ __forceinline__ uint32_t stc_target(int participants) {
+  return (uint32_t)participants + (*reinterpret_cast<volatile uint32_t *>(&g_barrier_unreachable) ? 1u : 0u);
 }
 
 template <int R>
-__global__ void __launch_bounds__(kStcThreads, 1)
+__global__ void __launch_bounds__(StcCfg<R>::kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
                 const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
-                uint32_t *__restrict__ ehist, unsigned int *__restrict__ counters, uint32_t *__restrict__ status) {
+                uint32_t *__restrict__ ehist, unsigned int *__restrict__ counters, uint32_t *__restrict__ status,
+                int K, int nB) {
   using Cfg = StcCfg<R>;
   constexpr int kR = Cfg::kRetained;
+  constexpr int EN = Cfg::kEpiThreads;
   extern __shared__ __align__(1024) unsigned char stc_smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(stc_smem_raw) + 1023) & ~uintptr_t(1023));
   const int r = s.rank_k;
   const int nkb = stc_kblocks(r);
   const int b_bytes = stc_b_bytes(R, r);
-  const int nB = stc_b_buffers(R, r);
-  const int NS = stc_stages(R, r);
+  const int NS = stc_stages(R, r, nB);
   unsigned char *b_op = smem;
   unsigned char *ring = smem + nB * b_bytes;
   StcControl<R> *ctl = reinterpret_cast<StcControl<R> *>(ring + NS * kStcKbBytes);
@@ -246,7 +288,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       mbar_init(&ctl->empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ctl->b_full[i], 1);
+      for (int kb = 0; kb < 4; ++kb) mbar_init(&ctl->b_full[i][kb], 1);
       mbar_init(&ctl->b_empty[i], 1);
     }
     mbar_init(&ctl->acc_full, 1);
@@ -254,7 +296,30 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
     for (int i = 0; i < Cfg::kSlots; ++i) mbar_init(&ctl->slot_free[i], 1);
     mbar_init(&ctl->mma_final, 1);
     ctl->abort = 0;
+    ctl->arrived_seq = 0;
+    ctl->done_seq = 0;
     mbar_fence_init();
+  }
+  __syncthreads();
+  // The cache is a call input: the first problem's first k-blocks go out
+  // before the wait for the projection kernel (which writes the split C_Q
+  // operand), as far as the ring holds them, and before TMEM is allocated.
+  uint32_t pre = 0;
+  if (warp == Cfg::kProducer && lane == 0) {
+    tma_prefetch_desc(&tmap_ck);
+    StcWalker wa;
+    wa.start(lengths, s.cache_rows, s.batch, G, c, K, kR);
+    StcTile a;
+    int p_first = -1;
+    while (pre < (uint32_t)NS && wa.next(a)) {
+      if (p_first < 0) p_first = a.p;
+      if (a.p != p_first || a.pass2) break;
+      for (int kb = 0; kb < nkb && pre < (uint32_t)NS; ++kb, ++pre) {
+        mbar_arrive_expect_tx(&ctl->full[pre], (uint32_t)kStcKbBytes);
+        tma_load_2d(ring + pre * kStcKbBytes, &tmap_ck, &ctl->full[pre], kb * 64,
+                    (int32_t)((int64_t)a.p * s.cache_rows + a.row0));
+      }
+    }
   }
   if (warp == 0) tmem_alloc(&ctl->tmem_base, 512);
   tc_fence_before();
@@ -262,7 +327,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp == 4) {
+  if (warp == Cfg::kProducer) {
     // ------------------------------------------------------- TMA producer
     if (lane == 0) {
       auto issue = [&](uint32_t idx, const StcTile &t, int kb) {
@@ -271,25 +336,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
         tma_load_2d(ring + st * kStcKbBytes, &tmap_ck, &ctl->full[st], kb * 64,
                     (int32_t)((int64_t)t.p * s.cache_rows + t.row0));
       };
-      // The cache is a call input: the first problem's first k-blocks go out
-      // before the wait for the projection kernel (which writes the split C_Q
-      // operand), as far as the ring holds them.
-      uint32_t pre = 0;
-      int p_first = -1;
-      {
-        StcWalker wa;
-        wa.start(lengths, s.cache_rows, s.batch, G, c, kR);
-        StcTile a;
-        while (pre < (uint32_t)NS && wa.next(a)) {
-          if (p_first < 0) p_first = a.p;
-          if (a.p != p_first) break;
-          for (int kb = 0; kb < nkb && pre < (uint32_t)NS; ++kb, ++pre) issue(pre, a, kb);
-        }
-      }
       pdl_wait();
       pdl_trigger();
       StcWalker w;
-      w.start(lengths, s.cache_rows, s.batch, G, c, kR);
+      w.start(lengths, s.cache_rows, s.batch, G, c, K, kR);
       StcTile t;
       int prev_p = -1;
       uint32_t n_switch = 0, issued = 0;
@@ -302,11 +352,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
           const int buf = (int)(n_switch % nB);
           if (n_switch >= (uint32_t)nB) ok = mbar_wait(&ctl->b_empty[buf], ((n_switch / nB) - 1) & 1, status);
           if (!ok) break;
-          mbar_arrive_expect_tx(&ctl->b_full[buf], (uint32_t)b_bytes);
           const unsigned char *src = cqs + (int64_t)t.p * b_bytes;
-          for (int kb = 0; kb < nkb; ++kb)
+          for (int kb = 0; kb < nkb; ++kb) {
+            mbar_arrive_expect_tx(&ctl->b_full[buf][kb], (uint32_t)(3 * R * 128));
             bulk_load(b_op + buf * b_bytes + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128,
-                      &ctl->b_full[buf]);
+                      &ctl->b_full[buf][kb]);
+          }
           ++n_switch;
           prev_p = t.p;
         }
@@ -326,19 +377,19 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       }
       for (uint32_t i = 0; i < (uint32_t)nB && i < n_switch; ++i) {
         const uint32_t last = i + ((n_switch - 1 - i) / nB) * nB;
-        mbar_wait(&ctl->b_full[i], (last / nB) & 1, status);
+        for (int kb = 0; kb < nkb; ++kb) mbar_wait(&ctl->b_full[i][kb], (last / nB) & 1, status);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == Cfg::kMma) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       StcWalker w;
-      w.start(lengths, s.cache_rows, s.batch, G, c, kR);
+      w.start(lengths, s.cache_rows, s.batch, G, c, K, kR);
       StcTile t;
       int prev_p = -1;
       uint32_t n_switch = 0, used = 0, n_tile = 0, j_ret = 0, u_tr = 0;
-      uint32_t b_base = 0;
+      uint32_t b_base = 0, b_buf = 0, b_par = 0;
       bool ok = true;
       const uint32_t idesc_hi = idesc_bf16_f32(128, R, 0, 0);
       const uint32_t idesc_ml = idesc_bf16_f32(128, 2 * R, 0, 0);
@@ -346,10 +397,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
         if (*reinterpret_cast<volatile int *>(&ctl->abort)) break;
         if (t.p != prev_p) {
           if (prev_p >= 0) umma_commit(&ctl->b_empty[(n_switch - 1) % nB]);   // previous operand free once done
-          const int buf = (int)(n_switch % nB);
-          ok = mbar_wait(&ctl->b_full[buf], (n_switch / nB) & 1, status);
-          if (!ok) break;
-          b_base = smem_u32(b_op + buf * b_bytes);
+          b_buf = n_switch % nB;
+          b_par = (n_switch / nB) & 1;
+          b_base = smem_u32(b_op + b_buf * b_bytes);
           ++n_switch;
           prev_p = t.p;
         }
@@ -371,7 +421,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
         const uint32_t d_ml = tmem + (uint32_t)Cfg::kScratchCol;
         for (int kb = 0; kb < nkb && ok; ++kb, ++used) {
           const uint32_t st = used % NS;
-          ok = mbar_wait(&ctl->full[st], (used / NS) & 1, status);
+          ok = mbar_wait(&ctl->full[st], (used / NS) & 1, status) &&
+               mbar_wait(&ctl->b_full[b_buf][kb], b_par, status);   // at once after the problem's first tile
           if (!ok) break;
           tc_fence_after();
           const uint32_t a_base = smem_u32(ring + st * kStcKbBytes);
@@ -396,269 +447,335 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       mbar_wait(&ctl->mma_final, 0, status);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------- epilogue (warps 0-3)
-    pdl_wait();      // the row sums, counters and histogram were zeroed by the projection kernel
-    pdl_trigger();
-    const int pos = threadIdx.x;                         // TMEM lane = position within the tile
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    StcWalker w;
-    w.start(lengths, s.cache_rows, s.batch, G, c, kR);
-    StcTile t;
-    uint32_t n_tile = 0, j_ret = 0, u_tr = 0;
-    int ret_head = 0;                                    // oldest kept use not yet finished
-    int n_pend = 0, pend_head = 0;                       // pending problems (FIFO in ctl->pend)
-    double psum = 0.0;                                   // this CTA's sum of row `pos` (pos < R) for the current problem
-    int cur_p2 = -1;                                     // problem whose inv_l is loaded (pass 2)
-    bool ok = true;
+  } else if (warp == Cfg::kWatcher) {
+    // ------------------------------------------------------- counter watcher
+    // For each problem of the CTA's list, once the epilogue has arrived on
+    // it: wait (bounded) until every CTA that owns tiles of it has arrived,
+    // then form 1 / l_row from its 16 row-sum slots (fp64, fixed order) into
+    // the ring slot of that problem and publish its completion.  The epilogue
+    // reads only shared memory.
+    pdl_wait();
+    constexpr int Q = kR + 1;
     const uint32_t my_slot_sum = (uint32_t)(c % kStcSumSlots);
-
-    // alpha_row = 2^k / l_row from the problem's finished row sums (fp64).
-    auto load_inv_l = [&](int p) {
-      if (pos < R) {
-        double l = 0.0;
-        if (pos < s.n_rows) {
-          double part[kStcSumSlots];
-#pragma unroll
-          for (int q = 0; q < kStcSumSlots; ++q)
-            part[q] = __ldcg(&row_sum[((int64_t)p * kStcSumSlots + q) * s.n_rows + pos]);
-#pragma unroll
-          for (int q = 0; q < kStcSumSlots; ++q) l += part[q];
-        }
-        ctl->inv_l[pos] = l > 0.0 ? 1.0 / l : 0.0;
-      }
-    };
-    // Histogram of the candidates' leading score bits (kExpBins bins of the
-    // problem), one atomic per distinct bin of the warp.
-    auto hist_add = [&](int p, float sc, bool cand) {
-      const uint32_t bin = cand ? (__float_as_uint(sc) >> kExpShift) & (kExpBins - 1) : 0xffffffffu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (cand && lane == __ffs(peers) - 1) atomicAdd(&ehist[(int64_t)p * kExpBins + bin], (uint32_t)__popc(peers));
-    };
-    // Wait (bounded) until problem p's counter is complete.
-    auto wait_problem = [&](int p, int T) -> bool {
-      if (pos == 0) {
-        const uint32_t target = stc_target(T, G);
+    StcWalker w;
+    w.start(lengths, s.cache_rows, s.batch, G, c, K, kR);
+    StcTile t;
+    int q = 0;
+    bool ok = true;
+    while (w.next(t) && !t.pass2) {
+      if (!t.last) continue;
+      // The epilogue's arrival on this problem (bounded; the epilogue may stop early).
+      int good = 1;
+      if (lane == 0) {
         const long long limit = wait_limit();
         const long long t0 = clock64();
-        int good = 1;
+        while (ctl->arrived_seq <= q) {
+          if (*reinterpret_cast<volatile int *>(&ctl->abort) || clock64() - t0 > limit) { good = 0; break; }
+          __nanosleep(32);
+        }
+      }
+      good = __shfl_sync(0xffffffffu, good, 0) && ok;
+      __threadfence_block();
+      // This CTA's row sums into the problem's normalisers (one of 16 slots
+      // per row), then the arrival.
+      if (good) {
+        for (int row = lane; row < R && row < s.n_rows; row += 32)
+          atomicAdd(&row_sum[((int64_t)t.p * kStcSumSlots + my_slot_sum) * s.n_rows + row], ctl->inv_q[q % Q][row]);
+        __threadfence();
+      }
+      __syncwarp();
+      if (lane == 0 && good) {
+        atomicAdd(counters + t.p, 1u);
+        const uint32_t target = stc_target(stc_participants(w.S, t.T, K, G));
+        const long long limit = wait_limit();
+        const long long t1 = clock64();
         while (true) {
           uint32_t v;
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counters + p) : "memory");
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counters + t.p) : "memory");
           if (v >= target) break;
-          if (clock64() - t0 > limit) {
+          if (*reinterpret_cast<volatile int *>(&ctl->abort) || clock64() - t1 > limit) {
             set_status(status, kDevStatusTimeout);
             good = 0;
             break;
           }
           __nanosleep(32);
         }
-        ctl->flag = good;
       }
-      epi_sync();
-      return ctl->flag != 0;
-    };
-    // Scores of every kept tile of the oldest pending problem, then its slots
-    // are released.
-    auto finish_oldest = [&](bool ok_p) {
-      const int p = ctl->pend[pend_head % (kR + 1)];
-      load_inv_l(p);
-      epi_sync();
-      int64_t Lp = 0;
-      while (ret_head < (int)j_ret && ctl->slot_p[ret_head % kR] == p) {
-        const int sl = ret_head % kR;
-        if (pos < R) ctl->alpha[pos] = ok_p ? (float)ldexp(ctl->inv_l[pos], ctl->kofs_slot[sl][pos]) : 0.f;
-        epi_sync();
-        const int64_t row0 = ctl->slot_row0[sl];
-        Lp = valid_length(__ldg(lengths + p), s.cache_rows);
-        float acc = 0.f;
+      good = __shfl_sync(0xffffffffu, good, 0);
+      for (int row = lane; row < R; row += 32) {
+        double l = 0.0;
+        if (good && row < s.n_rows) {
+          double part[kStcSumSlots];
 #pragma unroll
-        for (int c32 = 0; c32 < R / 32; ++c32) {
-          uint32_t ev[32];
-          tmem_ld32(tmem + lane_base + (uint32_t)(sl * R + c32 * 32), ev);
-          tmem_wait_ld();
+          for (int sl = 0; sl < kStcSumSlots; ++sl)
+            part[sl] = __ldcg(&row_sum[((int64_t)t.p * kStcSumSlots + sl) * s.n_rows + row]);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc = fmaf(ctl->alpha[c32 * 32 + j], __uint_as_float(ev[j]), acc);
+          for (int sl = 0; sl < kStcSumSlots; ++sl) l += part[sl];
         }
-        const int64_t i = row0 + pos;
-        if (i < Lp) scores[(int64_t)p * s.cache_rows + i] = acc;
-        hist_add(p, acc, i < Lp - s.local_window);
-        tc_fence_before();
-        epi_sync();
-        if (pos == 0) mbar_arrive(&ctl->slot_free[sl]);
-        ++ret_head;
+        ctl->inv_q[q % Q][row] = l > 0.0 ? 1.0 / l : 0.0;
       }
+      if (lane == 0) ctl->ok_q[q % Q] = good;
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0) ctl->done_seq = q + 1;
+      if (!good) ok = false;
+      ++q;
+    }
+  } else if (warp < Cfg::kEpiWarps) {
+    // ------------------------------------------------------- epilogue
+    pdl_wait();      // the row sums, counters and histogram were zeroed by the projection kernel
+    pdl_trigger();
+    constexpr int Q = kR + 1;
+    const int ep = threadIdx.x;                          // epilogue thread
+    const int quarter = warp & 3, half = warp >> 2;
+    const int pos = quarter * 32 + lane;                 // TMEM lane = position within the tile
+    const int rh = half * 32;                            // this thread's rows rh .. rh+31
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    StcWalker w;
+    w.start(lengths, s.cache_rows, s.batch, G, c, K, kR);
+    StcTile t;
+    uint32_t n_tile = 0, j_ret = 0, u_tr = 0;
+    int ret_head = 0;                                    // oldest kept use not yet finished
+    int n_pend = 0, pend_head = 0;                       // pending problems (FIFO in ctl->pend, index q)
+    double psum = 0.0;                                   // this CTA's sum of row ep (ep < R) for the current problem
+    int cur_p2 = -1;                                     // problem whose inv_l is loaded (pass 2)
+    bool ok = true;
+
+    // Level-0 histogram of the candidates' scores (score_bin around the mean
+    // R / L_c), one atomic per distinct bin of the warp (warps of rows 0-31).
+    auto hist_add = [&](int p, int64_t Lp, float sc, bool cand) {
+      const uint32_t bin = cand ? (uint32_t)score_bin(__float_as_uint(sc), score_center(s.n_rows, Lp)) : 0xffffffffu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (cand && lane == __ffs(peers) - 1) atomicAdd(&ehist[(int64_t)p * kExpBins + bin], (uint32_t)__popc(peers));
+    };
+    // Scores of every kept tile of the oldest pending problem (the watcher
+    // has published its 1 / l), then its slots are released.  Each thread
+    // sums its 32 rows; with two row halves, the second half's parts go
+    // through shared memory to the first half's threads, which write.
+    auto finish_oldest = [&]() {
+      const int qq = pend_head % Q;
+      const int p = ctl->pend[qq];
+      const bool okp = ctl->ok_q[qq] != 0;
+      const int first = ret_head;
+      int n_sl = 0;
+      while (first + n_sl < (int)j_ret && ctl->slot_p[(first + n_sl) % kR] == p) ++n_sl;
+      if (ep < R)
+        for (int u = 0; u < n_sl; ++u) {
+          const int sl = (first + u) % kR;
+          ctl->alpha[sl][ep] = okp ? (float)ldexp(ctl->inv_q[qq][ep], ctl->kofs_slot[sl][ep]) : 0.f;
+        }
+      epi_sync<EN>();
+      float part[kR];
+#pragma unroll
+      for (int u = 0; u < kR; ++u) part[u] = 0.f;
+#pragma unroll
+      for (int u = 0; u < kR; ++u) {
+        if (u < n_sl) {
+          const int sl = (first + u) % kR;
+          uint32_t ev[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)(sl * R + rh), ev);
+          tmem_wait_ld();
+          float a = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a = fmaf(ctl->alpha[sl][rh + j], __uint_as_float(ev[j]), a);
+          part[u] = a;
+          if (half == 1) ctl->sc_part[u][pos] = a;
+        }
+      }
+      tc_fence_before();
+      epi_sync<EN>();
+      if (half == 0) {
+        const int64_t Lp = ctl->pend_L[qq];
+#pragma unroll
+        for (int u = 0; u < kR; ++u) {
+          if (u < n_sl) {
+            const int sl = (first + u) % kR;
+            const float acc = Cfg::kHalves == 2 ? part[u] + ctl->sc_part[u][pos] : part[u];
+            const int64_t i = ctl->slot_row0[sl] + pos;
+            if (i < Lp) scores[(int64_t)p * s.cache_rows + i] = acc;
+            hist_add(p, Lp, acc, i < Lp - s.local_window);
+          }
+        }
+      }
+      if (ep == 0)
+        for (int u = 0; u < n_sl; ++u) mbar_arrive(&ctl->slot_free[(first + u) % kR]);
+      epi_sync<EN>();   // sc_part and alpha are rewritten by the next finish
+      ret_head += n_sl;
       ++pend_head;
       --n_pend;
     };
-
-    // Wait for and finish every pending problem, oldest first.
-    auto finish_all_pending = [&]() {
-      while (n_pend > 0) {
-        const int p_old = ctl->pend[pend_head % (kR + 1)];
-        const int64_t Lo = valid_length(__ldg(lengths + p_old), s.cache_rows);
-        const bool okp = ok && wait_problem(p_old, (int)ceil_div(Lo, kStcTile));
-        finish_oldest(okp);
-        if (!okp) ok = false;
+    // Wait (bounded) until the watcher has published the oldest pending problem.
+    auto wait_oldest = [&]() {
+      if (ep == 0) {
+        const long long limit = wait_limit();
+        const long long t0 = clock64();
+        while (ctl->done_seq <= pend_head) {
+          if (clock64() - t0 > 2 * limit) {
+            set_status(status, kDevStatusTimeout);
+            ctl->ok_q[pend_head % Q] = 0;
+            ctl->done_seq = pend_head + 1;   // give up on it (its scores become 0)
+            break;
+          }
+          __nanosleep(32);
+        }
       }
+      epi_sync<EN>();
     };
 
     while (w.next(t)) {
       if (*reinterpret_cast<volatile int *>(&ctl->abort)) ok = false;
       if (!ok) break;
-      // Pass 2 needs every problem's normalisers.
-      if (t.pass2 && cur_p2 < 0) finish_all_pending();
+      if (t.pass2 && cur_p2 < 0) {
+        // Pass 2 needs every problem's normalisers.
+        while (n_pend > 0) {
+          wait_oldest();
+          finish_oldest();
+        }
+      }
       const bool kept = !t.pass2 && t.k < kR;
       // A kept tile reuses the slot of the kept tile kR uses earlier, which
       // belongs to an older problem: finish problems until it is released.
       while (kept && (int)j_ret - kR >= ret_head && n_pend > 0) {
-        const int p_old = ctl->pend[pend_head % (kR + 1)];
-        const int64_t Lo = valid_length(__ldg(lengths + p_old), s.cache_rows);
-        const bool okp = ok && wait_problem(p_old, (int)ceil_div(Lo, kStcTile));
-        finish_oldest(okp);
-        if (!okp) ok = false;
+        wait_oldest();
+        finish_oldest();
       }
       if (t.pass2 && t.p != cur_p2) {
-        // Every problem was finished before pass 2: its normalisers are complete.
-        load_inv_l(t.p);
+        // 1 / l of the problem, from its finished row sums (fp64, fixed order).
+        if (ep < R) {
+          double l = 0.0;
+          if (ep < s.n_rows) {
+            double ps[kStcSumSlots];
+#pragma unroll
+            for (int sl = 0; sl < kStcSumSlots; ++sl)
+              ps[sl] = __ldcg(&row_sum[((int64_t)t.p * kStcSumSlots + sl) * s.n_rows + ep]);
+#pragma unroll
+            for (int sl = 0; sl < kStcSumSlots; ++sl) l += ps[sl];
+          }
+          ctl->inv_l[ep] = l > 0.0 ? 1.0 / l : 0.0;
+        }
         cur_p2 = t.p;
       }
       const int slot = kept ? (int)(j_ret % kR) : kR + (int)(u_tr % kStcTransient);
       ok = mbar_wait(&ctl->acc_full, n_tile & 1, status) && ok;
       tc_fence_after();
-      // y = (lo + mid) + hi for this position's R rows
-      float y[R];
+      // y = (lo + mid) + hi for this position's rows rh .. rh+31
+      float y[32];
       const int64_t i = t.row0 + pos;
       const bool valid = i < t.L;
-#pragma unroll
-      for (int c32 = 0; c32 < R / 32; ++c32) {
+      float amax = 0.f;
+      {
         uint32_t hi[32], mid[32], lo[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(slot * R + c32 * 32), hi);
-        tmem_ld32(tmem + lane_base + (uint32_t)(Cfg::kScratchCol + c32 * 32), mid);
-        tmem_ld32(tmem + lane_base + (uint32_t)(Cfg::kScratchCol + R + c32 * 32), lo);
+        tmem_ld32(tmem + lane_base + (uint32_t)(slot * R + rh), hi);
+        tmem_ld32(tmem + lane_base + (uint32_t)(Cfg::kScratchCol + rh), mid);
+        tmem_ld32(tmem + lane_base + (uint32_t)(Cfg::kScratchCol + R + rh), lo);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          y[c32 * 32 + j] = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
+        for (int j = 0; j < 32; ++j) {
+          y[j] = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
+          amax = fmaxf(amax, fabsf(y[j]));
+        }
       }
-      // The scratch (and a transient slot) may take the next tile's MMAs.
+      // One barrier: the accumulators are read (the scratch, and a transient
+      // slot, may take the next tile's MMAs), and the range check's vote.
       tc_fence_before();
-      epi_sync();
-      if (pos == 0) {
+      const bool wide = epi_or<EN>(valid && amax > kStcRangeLimit);
+      if (ep == 0) {
         mbar_arrive(&ctl->scratch_free);
         if (!kept) mbar_arrive(&ctl->slot_free[slot]);
       }
       ++n_tile;
       if (kept) ++j_ret; else ++u_tr;
-      // Range check: offsets only for a tile with some |y| beyond the limit.
-      float amax = 0.f;
-#pragma unroll
-      for (int j = 0; j < R; ++j) amax = fmaxf(amax, fabsf(y[j]));
-      const bool wide = epi_or(valid && amax > kStcRangeLimit);
+      const int rb = (int)(n_tile & 1);   // partial-sum buffer of this tile
       if (wide) {
-        // k_row = floor(max over the tile's valid positions of y_row)
+        // Offsets only for a tile with some |y| beyond the limit:
+        // k_row = floor(max over the tile's valid positions of y_row).
+        float v[32];
 #pragma unroll
-        for (int c32 = 0; c32 < R / 32; ++c32) {
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = valid ? y[c32 * 32 + j] : -INFINITY;
-          warp_transpose_reduce32<true>(v);
-          ctl->red[warp][c32 * 32 + lane] = v[0];
+        for (int j = 0; j < 32; ++j) v[j] = valid ? y[j] : -INFINITY;
+        warp_transpose_reduce32<true>(v);
+        ctl->red[rb][quarter][rh + lane] = v[0];
+        epi_sync<EN>();
+        if (ep < R) {
+          const float m = fmaxf(fmaxf(ctl->red[rb][0][ep], ctl->red[rb][1][ep]),
+                                fmaxf(ctl->red[rb][2][ep], ctl->red[rb][3][ep]));
+          ctl->kofs[ep] = (m == -INFINITY) ? 0 : (int)floorf(m);
         }
-        epi_sync();
-        if (pos < R) {
-          const float m = fmaxf(fmaxf(ctl->red[0][pos], ctl->red[1][pos]), fmaxf(ctl->red[2][pos], ctl->red[3][pos]));
-          ctl->kofs[pos] = (m == -INFINITY) ? 0 : (int)floorf(m);
-        }
-        epi_sync();
-      } else if (pos < R) {
-        ctl->kofs[pos] = 0;
-      }
-      if (wide) {
+        epi_sync<EN>();
 #pragma unroll
-        for (int j = 0; j < R; ++j) y[j] = valid ? ex2_approx(y[j] - (float)ctl->kofs[j]) : 0.f;
+        for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j] - (float)ctl->kofs[rh + j]) : 0.f;
       } else {
+        if (ep < R) ctl->kofs[ep] = 0;
 #pragma unroll
-        for (int j = 0; j < R; ++j) y[j] = valid ? ex2_approx(y[j]) : 0.f;
+        for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j]) : 0.f;
       }
       // y now holds e.
       if (t.pass2) {
-        // Second pass: the problem is finished; score straight from e.
-        if (pos < R) ctl->alpha[pos] = (float)ldexp(ctl->inv_l[pos], ctl->kofs[pos]);
-        epi_sync();
-        float acc = 0.f;
+        // Second pass: the problem is finished; score straight from e with
+        // alpha_row = 2^k / l_row (each thread forms its 32 rows' factors).
+        float a = 0.f;
 #pragma unroll
-        for (int j = 0; j < R; ++j) acc = fmaf(ctl->alpha[j], y[j], acc);
-        if (valid) scores[(int64_t)t.p * s.cache_rows + i] = acc;
-        hist_add(t.p, acc, i < t.L - s.local_window);
-        epi_sync();   // alpha is rewritten by the next tile
+        for (int j = 0; j < 32; ++j) a = fmaf((float)ldexp(ctl->inv_l[rh + j], wide ? ctl->kofs[rh + j] : 0), y[j], a);
+        if (Cfg::kHalves == 2) {
+          if (half == 1) ctl->sc_part[0][pos] = a;
+          epi_sync<EN>();
+          if (half == 0) a += ctl->sc_part[0][pos];
+        }
+        if (half == 0) {
+          if (valid) scores[(int64_t)t.p * s.cache_rows + i] = a;
+          hist_add(t.p, t.L, a, i < t.L - s.local_window);
+        }
+        epi_sync<EN>();   // inv_l and sc_part may be rewritten for the next tile
         continue;
       }
       if (kept) {
         // Keep e in the slot (the hi columns just read), with its offsets.
+        uint32_t ev[32];
 #pragma unroll
-        for (int c32 = 0; c32 < R / 32; ++c32) {
-          uint32_t ev[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) ev[j] = __float_as_uint(y[c32 * 32 + j]);
-          tmem_st32(tmem + lane_base + (uint32_t)(slot * R + c32 * 32), ev);
-        }
+        for (int j = 0; j < 32; ++j) ev[j] = __float_as_uint(y[j]);
+        tmem_st32(tmem + lane_base + (uint32_t)(slot * R + rh), ev);
         tmem_wait_st();
-        if (pos < R) ctl->kofs_slot[slot][pos] = ctl->kofs[pos];
-        if (pos == 0) {
+        if (ep < R) ctl->kofs_slot[slot][ep] = ctl->kofs[ep];
+        if (ep == 0) {
           ctl->slot_p[slot] = t.p;
           ctl->slot_row0[slot] = t.row0;
         }
       }
       // Per-row sums of e over the tile's 128 positions: within the warp by a
-      // transpose-reduction, then the four warps in order.
-#pragma unroll
-      for (int c32 = 0; c32 < R / 32; ++c32) {
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = y[c32 * 32 + j];
-        warp_transpose_reduce32<false>(v);
-        ctl->red[warp][c32 * 32 + lane] = v[0];
-      }
-      epi_sync();
-      if (pos < R) {
-        const float ts = (ctl->red[0][pos] + ctl->red[1][pos]) + (ctl->red[2][pos] + ctl->red[3][pos]);
-        const int kk = ctl->kofs[pos];
+      // transpose-reduction, then the four lane quarters in order.
+      warp_transpose_reduce32<false>(y);
+      ctl->red[rb][quarter][rh + lane] = y[0];
+      if (ep == 0) ctl->done_snap = ctl->done_seq;   // one consistent view for every thread
+      epi_sync<EN>();
+      const int done_snap = ctl->done_snap;
+      if (ep < R) {
+        const float ts = (ctl->red[rb][0][ep] + ctl->red[rb][1][ep]) + (ctl->red[rb][2][ep] + ctl->red[rb][3][ep]);
+        const int kk = ctl->kofs[ep];
         psum += kk ? ldexp((double)ts, kk) : (double)ts;
       }
-      if (t.k == t.n - 1) {
-        // The CTA's last tile of the problem: publish its row sums, arrive.
-        if (pos < R && pos < s.n_rows)
-          atomicAdd(&row_sum[((int64_t)t.p * kStcSumSlots + my_slot_sum) * s.n_rows + pos], psum);
+      if (t.last) {
+        // The CTA's last tile of the problem: its row sums go to the
+        // problem's ring slot (which later holds 1 / l); the watcher adds
+        // them to the row normalisers and arrives on the problem's counter.
+        const int qn = pend_head + n_pend;
+        if (ep < R) ctl->inv_q[qn % Q][ep] = psum;
         psum = 0.0;
-        __threadfence();
-        epi_sync();
-        if (pos == 0) {
-          atomicAdd(counters + t.p, 1u);
-          ctl->pend[(pend_head + n_pend) % (kR + 1)] = t.p;
+        epi_sync<EN>();
+        if (ep == 0) {
+          ctl->pend[qn % Q] = t.p;
+          ctl->pend_L[qn % Q] = t.L;
+          __threadfence_block();
+          ctl->arrived_seq = qn + 1;
         }
         ++n_pend;
-        epi_sync();
-      } else {
-        epi_sync();   // red[] is rewritten by the next tile
       }
-      // Finish problems whose counters completed meanwhile (not blocking).
-      while (n_pend > 0) {
-        const int p_old = ctl->pend[pend_head % (kR + 1)];
-        if (pos == 0) {
-          const int64_t Lo = valid_length(__ldg(lengths + p_old), s.cache_rows);
-          uint32_t v;
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counters + p_old) : "memory");
-          ctl->flag = v >= stc_target((int)ceil_div(Lo, kStcTile), G) ? 1 : 0;
-        }
-        epi_sync();
-        const bool done = ctl->flag != 0;
-        epi_sync();
-        if (!done) break;
-        finish_oldest(true);
-      }
+      // Finish the problems the watcher has seen complete (no waiting).
+      while (n_pend > 0 && done_snap > pend_head) finish_oldest();
     }
-    finish_all_pending();
+    while (ok && n_pend > 0) {
+      wait_oldest();
+      finish_oldest();
+    }
+    if (!ok && ep == 0) atomicExch(&ctl->abort, 1);
   }
   tc_fence_before();
   __syncthreads();

@@ -373,34 +373,41 @@ topk_kernel(Shape s, const int32_t *__restrict__ lengths, const float *__restric
 // ---------------------------------------------------------------------------
 // Cluster variant: the kTopkCl CTAs of a cluster split one problem's
 // candidates into contiguous shares held in shared memory.  The threshold
-// key tau is found from histograms of the float bit patterns in up to three
-// levels of digits (bits 30-19 and 18-7 in 4096 bins, bits 6-0 in 128):
-//   * level 0 comes from the histogram the scoring kernel leaves for these
-//     candidates (or, without it, from every rank's histogram of its keys,
-//     exchanged through distributed shared memory); every rank takes the
-//     same decision: the bin holding the remaining-th largest key;
-//   * if that bin holds at most kTopkGather keys, every rank publishes its
-//     keys of the bin (with their positions, in position order) and its count
-//     of keys above the bin; after one cluster barrier every rank reads them
-//     all, finds tau among the gathered keys by a radix select and knows
-//     every rank's counts of keys > tau and == tau;
-//   * a bin taken whole needs only the ranks' counts; a fuller bin goes down
-//     one level; at the last level every bit of tau is fixed.
-// Usually that is one exchange.  No keys move except the threshold bin's.
+// key tau (of the IEEE bit patterns, which order like the scores) is found
+// by narrowing a key range [lo, hi] that holds it:
+//   * level 0 bins the keys around the mean score (score_bin: steps of 1/256
+//     of a binade); its histogram comes from the scoring kernel, or from
+//     every rank's histogram of its keys exchanged through distributed shared
+//     memory; every rank takes the same decision: the bin holding the
+//     remaining-th largest key, and so its key range;
+//   * if that range holds at most kTopkGather keys, every rank publishes its
+//     keys in it (with their positions, in position order) and its count of
+//     keys above it; after one cluster barrier every rank reads them all,
+//     finds tau among the gathered keys by a radix select and knows every
+//     rank's counts of keys > tau and == tau;
+//   * a range taken whole needs only the ranks' counts; a single key value
+//     fixes tau; a fuller range is split again into at most 4096 bins.
+// Usually that is one exchange.  No keys move except those in the range.
 // A stable compaction in index order then writes the rank's keys > tau and
 // its share of the keys == tau (lower positions first).
 constexpr int kTopkCl = 8;                       // CTAs per problem
 constexpr int kTopkClThreads = 512;
 constexpr int kTopkClKeys = 16384;               // keys per CTA (64 KB)
 constexpr int kTopkLvlBins = 4096;               // bins of levels 0 and 1
-constexpr int kTopkGather = 2048;                // keys of the threshold bin gathered into every rank at most
-static_assert(kTopkLvlBins == kExpBins && kExpShift == 19, "level-0 digits are the scoring histogram's bins");
+constexpr int kTopkGather = 8192;                // keys of the threshold bin gathered into every rank at most
+static_assert(kTopkLvlBins == kExpBins, "level 0 uses the scoring histogram's bins");
 
 struct __align__(16) TopkClShared {
   uint32_t hist[kTopkLvlBins];              // summed histogram of the current level
-  uint32_t pub_hist[2][kTopkLvlBins];       // this rank's histogram of a level (two in flight), read by every rank
+  union {
+    // this rank's histogram of a level (two in flight), read by every rank
+    uint32_t pub_hist[2][kTopkLvlBins];
+    // every rank's keys of the threshold bin, rank order: written only after
+    // the exchange barrier, which every rank passes after its last read of
+    // the histograms
+    uint2 gath[kTopkGather];
+  };
   uint2 pub_cand[kTopkGather];              // this rank's keys of the threshold bin (key, position), position order
-  uint2 gath[kTopkGather];                  // every rank's keys of the bin, rank order
   uint32_t pub_hdr[4];                      // this rank's count of keys above the bin, of keys in it
   uint32_t g_gt[kTopkCl], g_n[kTopkCl], g_off[kTopkCl + 1];
   uint32_t gt_acc[kTopkCl], eq_acc[kTopkCl];  // every rank's keys > tau / == tau
@@ -509,35 +516,65 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   const int chunk = (nc + kTopkCl - 1) / kTopkCl;
   const int i_begin = min(nc, (int)rank * chunk), i_end = min(nc, i_begin + chunk);
   const int my_n = i_end - i_begin;
-  // Asynchronous 4-byte copies: every load of the share is in flight at once.
-  for (int i = threadIdx.x; i < my_n; i += blockDim.x)
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(keys_s + kpad(i))),
-                 "l"(gkeys + i_begin + i)
-                 : "memory");
+  // Stage the share with 16-byte loads, all in flight at once.  The share
+  // starts at key i_begin of a row that starts at b * cache_rows floats, so
+  // it need not be 16-byte aligned: the head up to the first aligned key and
+  // the tail go one by one.
+  {
+    const uint32_t *src = gkeys + i_begin;
+    const int head = min(my_n, (int)(((16u - (reinterpret_cast<uintptr_t>(src) & 15u)) & 15u) / 4));
+    const int n4 = (my_n - head) / 4;
+    const uint4 *src4 = reinterpret_cast<const uint4 *>(src + head);
+    for (int i = threadIdx.x; i < head; i += blockDim.x) keys_s[kpad(i)] = __ldcg(src + i);
+    for (int i0 = 0; i0 < n4; i0 += 4 * (int)blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+        if (i < n4) v[u] = __ldcg(src4 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+        if (i < n4) {
+          const int j = head + 4 * i;
+          keys_s[kpad(j)] = v[u].x;
+          keys_s[kpad(j + 1)] = v[u].y;
+          keys_s[kpad(j + 2)] = v[u].z;
+          keys_s[kpad(j + 3)] = v[u].w;
+        }
+      }
+    }
+    for (int i = head + 4 * n4 + (int)threadIdx.x; i < my_n; i += blockDim.x) keys_s[kpad(i)] = __ldcg(src + i);
+  }
   // Level 0 from the scoring kernel's histogram, read while the keys stage.
   if (ehist != nullptr)
     for (int i = threadIdx.x; i < kTopkLvlBins; i += blockDim.x) sh.hist[i] = __ldcg(ehist + (int64_t)b * kExpBins + i);
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
   // Per-thread contiguous chunk of the rank's keys (the compactions walk it).
   const int per = (my_n + (int)blockDim.x - 1) / (int)blockDim.x;
   const int j0 = min(my_n, (int)threadIdx.x * per), j1 = min(my_n, j0 + per);
 
-  uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)need;
+  const uint32_t center = score_center(s.n_rows, L);
+  uint32_t lo = 0u, hi = 0x7fffffffu, remaining = (uint32_t)need, in_bin = 0u;
   uint32_t tau = 0u, take_eq = 0u;
-  int mode = 0;              // 1: bin taken whole; 2: every bit fixed; 3: threshold bin gathered
-  for (int level = 0; level < 3 && mode == 0; ++level) {
-    const int shift = cl_shift(level), nbins = cl_bins(level);
+  int mode = 0;              // 1: range taken whole; 2: a single key value; 3: range gathered
+  for (int level = 0; level < 6; ++level) {
+    // Bins of this level: score_bin at level 0, else (key - lo) >> sh over [lo, hi].
+    const uint32_t w = hi - lo;
+    const int bsh = level == 0 ? 0 : ((w >> 12) == 0u ? 0 : 32 - __clz(w >> 12));
+    const int nbins = level == 0 ? kTopkLvlBins : (int)(w >> bsh) + 1;
     if (level > 0 || ehist == nullptr) {
-      // This rank's histogram of the keys that match the digits fixed so far,
-      // summed over the ranks through distributed shared memory.
+      // This rank's histogram of its keys in [lo, hi], summed over the ranks
+      // through distributed shared memory.
       uint32_t *ph = sh.pub_hist[level & 1];
-      for (int i = threadIdx.x; i < nbins; i += blockDim.x) ph[i] = 0u;
+      for (int i = threadIdx.x; i < kTopkLvlBins; i += blockDim.x) ph[i] = 0u;
       __syncthreads();
       for (int i = threadIdx.x; i < my_n; i += blockDim.x) {
         const uint32_t v = keys_s[kpad(i)];
-        if ((v & mask) == prefix) atomicAdd(&ph[(v >> shift) & (uint32_t)(nbins - 1)], 1u);
+        if (level == 0) atomicAdd(&ph[score_bin(v, center)], 1u);
+        else if (v >= lo && v <= hi) atomicAdd(&ph[(v - lo) >> bsh], 1u);
       }
       cluster_sync();
       for (int i = 4 * (int)threadIdx.x; i < nbins; i += 4 * (int)blockDim.x) {
@@ -551,39 +588,50 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       __syncthreads();
     }
     cl_pick_bin(sh, sh.hist, nbins, remaining);
-    const uint32_t d = sh.digit, in_bin = sh.hist[d];
+    const uint32_t d = sh.digit;
+    in_bin = sh.hist[d];
     remaining -= sh.above;
-    prefix |= d << shift;
-    mask |= (uint32_t)(nbins - 1) << shift;
+    if (level == 0) {
+      score_bin_range((int)d, center, lo, hi);
+    } else {
+      const uint32_t nlo = lo + (d << bsh);
+      const uint32_t top = nlo + ((1u << bsh) - 1u);
+      hi = top < hi ? top : hi;
+      lo = nlo;
+    }
     __syncthreads();
-    if (in_bin == remaining && prefix != 0u) {
-      mode = 1;                    // every key >= prefix is taken
-      tau = prefix - 1u;
+    if (in_bin == remaining && lo > 0u) {
+      mode = 1;                    // every key >= lo is taken
+      tau = lo - 1u;
       take_eq = 0u;
-    } else if (level == 2) {
-      mode = 2;                    // all 31 bits fixed
-      tau = prefix;
+      break;
+    }
+    if (lo == hi) {
+      mode = 2;                    // the range is a single key value
+      tau = lo;
       take_eq = remaining;
-    } else if (in_bin <= (uint32_t)kTopkGather) {
+      break;
+    }
+    if (in_bin <= (uint32_t)kTopkGather) {
       mode = 3;
+      break;
     }
   }
 
-  const uint32_t hi_bound = prefix | (~mask & 0x7fffffffu);   // largest key in the threshold bin
   if (mode == 3) {
     // Publish this rank's keys of the bin (stable, in position order) and
     // its count of keys above the bin; gather every rank's.
     uint32_t n_in = 0, n_above = 0;
     for (int i = j0; i < j1; ++i) {
       const uint32_t v = keys_s[kpad(i)];
-      n_in += (v & mask) == prefix;
-      n_above += v > hi_bound;
+      n_in += v >= lo && v <= hi;
+      n_above += v > hi;
     }
     const uint32_t before = block_excl_scan(n_in, sh.warp_tot, &sh.total);
     uint32_t at = before;
     for (int i = j0; i < j1; ++i) {
       const uint32_t v = keys_s[kpad(i)];
-      if ((v & mask) == prefix) sh.pub_cand[at++] = make_uint2(v, (uint32_t)(i_begin + i));
+      if (v >= lo && v <= hi) sh.pub_cand[at++] = make_uint2(v, (uint32_t)(i_begin + i));
     }
     n_above = warp_sum_u32(n_above);
     if (threadIdx.x == 0) { sh.pub_hdr[0] = 0u; sh.pub_hdr[1] = sh.total; }
@@ -608,15 +656,15 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       sh.gath[e] = ld_cluster_v2(cluster_map(&sh.pub_cand[e - sh.g_off[rr]], (uint32_t)rr));
     }
     __syncthreads();
-    // tau: the remaining-th largest gathered key (radix select on the bits below the bin).
-    uint32_t pfx = prefix, msk = mask, rem = remaining;
-    for (int sel_shift = cl_shift(0) - 8; sel_shift > -8; sel_shift -= 8) {
-      const int sh8 = sel_shift < 0 ? 0 : sel_shift;
-      if ((msk | (255u << sh8)) == msk) continue;   // these bits are fixed already
+    // tau: the remaining-th largest gathered key, by a radix select on the
+    // offsets v = key - lo (at most hi - lo), 8 bits at a time from the top.
+    uint32_t pfx = 0u, msk = 0u, rem = remaining;
+    for (int top = 31 - __clz(hi - lo); top >= 0;) {
+      const int sh8 = top >= 7 ? top - 7 : 0;
       for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.sel_hist[i] = 0u;
       __syncthreads();
       for (uint32_t e = threadIdx.x; e < n_g; e += blockDim.x) {
-        const uint32_t v = sh.gath[e].x;
+        const uint32_t v = sh.gath[e].x - lo;
         if ((v & msk) == pfx) atomicAdd(&sh.sel_hist[(v >> sh8) & 255u], 1u);
       }
       __syncthreads();
@@ -626,8 +674,9 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
       pfx |= sh.digit << sh8;
       msk |= 255u << sh8;
       __syncthreads();
+      top = sh8 - 1;
     }
-    tau = pfx;
+    tau = lo + pfx;
     take_eq = rem;
     // Every rank's keys > tau and == tau: those above the bin plus its gathered keys.
     if (threadIdx.x < kTopkCl) { sh.gt_acc[threadIdx.x] = sh.g_gt[threadIdx.x]; sh.eq_acc[threadIdx.x] = 0u; }

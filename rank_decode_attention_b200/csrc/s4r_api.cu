@@ -20,6 +20,7 @@
 #include "k_encode_tc.cuh"
 #include "k_project.cuh"
 #include "k_score_simt.cuh"
+#include "k_score_pair.cuh"
 #include "k_score_tc.cuh"
 #include "k_topk.cuh"
 
@@ -222,34 +223,72 @@ s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const vo
 // Which latent-scoring kernel a decode call uses.
 struct ScorePlan {
   bool tc = false;   // tensor-core kernel (else fp64 CUDA-core passes)
+  bool pair = false; // the fused two-tiles-per-CTA kernel (one problem, one resident wave)
   int R = 0;         // rows per problem (template argument of the TC kernel)
   int grid = 0;      // persistent cooperative grid
+  int K = 1;         // consecutive tiles per chunk of the round-robin
+  int nB = 1;        // split C_Q operand buffers
   size_t smem = 0;
 };
 
-// CTAs of the tensor-core scoring kernel resident at once on this device
-// (cached per device and rank; 0 if it cannot be launched).
+// Whether the tensor-core scoring kernel can run with this much dynamic shared
+// memory on the current device: the kernel's limit is raised to it (once per
+// size) and one CTA must fit an SM.  Results are cached per device and size.
 template <int R>
-int tc_capacity(int rank) {
-  static std::atomic<int> cache[kMaxDevices][S4R_MAX_RANK / 8 + 1];   // capacity + 1; 0 = unknown
+bool tc_launchable(size_t smem) {
+  constexpr int kSizes = 8;
+  static std::mutex mu;
+  static int known[kMaxDevices][kSizes][2];   // (size, 1 yes / -1 no)
+  const int dev = current_device();
+  if (ensure_smem<score_tc_kernel<R>>(smem) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (dev >= 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSizes; ++i)
+      if (known[dev][i][0] == (int)smem) return known[dev][i][1] > 0;
+  }
+  int per_sm = 0;
+  const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, StcCfg<R>::kThreads, smem) ==
+                      cudaSuccess &&
+                  per_sm > 0;
+  if (!ok) cudaGetLastError();
+  if (dev >= 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSizes; ++i)
+      if (known[dev][i][0] == 0) {
+        known[dev][i][0] = (int)smem;
+        known[dev][i][1] = ok ? 1 : -1;
+        break;
+      }
+  }
+  return ok;
+}
+
+// Whether the fused two-tiles-per-CTA kernel can run with `grid` CTAs, all
+// resident at once (one per SM: each holds all 512 TMEM columns).
+template <int R>
+bool pair_launchable(size_t smem, int rank, int grid) {
+  if (grid > sm_count()) return false;
+  static std::atomic<int> ok_cache[kMaxDevices][S4R_MAX_RANK / 8 + 1];   // per rank: 0 unknown, 1 no, 2 yes
   const int dev = current_device();
   const int slot = rank / 8;
-  if (dev >= 0) {
-    const int c = cache[dev][slot].load(std::memory_order_relaxed);
-    if (c > 0) return c - 1;
-  }
-  const size_t smem = (size_t)stc_smem_bytes(R, rank);
-  int sms = 0, per_sm = 0, d = 0;
-  if (cudaGetDevice(&d) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess ||
-      ensure_smem<score_tc_kernel<R>>(smem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<R>, kStcThreads, smem) != cudaSuccess) {
+  if (ensure_smem<score_pair_kernel<R>>(smem) != cudaSuccess) {
     cudaGetLastError();
-    return 0;
+    return false;
   }
-  // One CTA per SM: each holds all 512 TMEM columns.
-  const int cap = per_sm > 0 ? sms : 0;
-  if (dev >= 0) cache[dev][slot].store(cap + 1, std::memory_order_relaxed);
-  return cap;
+  if (dev >= 0) {
+    const int c = ok_cache[dev][slot].load(std::memory_order_relaxed);
+    if (c > 0) return c == 2;
+  }
+  int per_sm = 0;
+  const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_pair_kernel<R>, kSpThreads, smem) ==
+                      cudaSuccess &&
+                  per_sm > 0;
+  if (!ok) cudaGetLastError();
+  if (dev >= 0) ok_cache[dev][slot].store(ok ? 2 : 1, std::memory_order_relaxed);
+  return ok;
 }
 
 ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
@@ -257,16 +296,34 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   if (dt != S4R_BF16 || s.cache_rows == 0 || s.batch == 0) return p;
   if (s.n_rows != 32 && s.n_rows != 64) return p;
   if ((int64_t)s.batch * s.cache_rows >= INT32_MAX) return p;
-  const int cap = s.n_rows == 64 ? tc_capacity<64>(s.rank_k) : tc_capacity<32>(s.rank_k);
-  if (cap <= 0) {
-    cudaGetLastError();
-    return p;
+  const int R = s.n_rows;
+  if (s.batch == 1) {
+    // One problem whose tile pairs fit one resident wave: the fused kernel
+    // (fewer fixed latencies for a latency-bound single layer).
+    const int64_t pairs = ceil_div(ceil_div(s.cache_rows, kStcTile), kSpTiles);
+    const size_t psmem = (size_t)sp_smem_bytes(R, s.rank_k);
+    if (pairs <= sm_count() &&
+        (R == 64 ? pair_launchable<64>(psmem, s.rank_k, (int)pairs) : pair_launchable<32>(psmem, s.rank_k, (int)pairs))) {
+      p.tc = true;
+      p.pair = true;
+      p.R = R;
+      p.grid = (int)pairs;
+      p.smem = psmem;
+      return p;
+    }
   }
+  // A second operand buffer pays when the CTAs switch problems.
+  const int nB = (s.batch > 1 && stc_two_b_fit(R, s.rank_k)) ? 2 : 1;
+  const size_t smem = (size_t)stc_smem_bytes(R, s.rank_k, nB);
+  if (!(R == 64 ? tc_launchable<64>(smem) : tc_launchable<32>(smem))) return p;
+  // One CTA per SM: each holds all 512 TMEM columns.
   const int64_t tiles = (int64_t)s.batch * ceil_div(s.cache_rows, kStcTile);
   p.tc = true;
-  p.R = s.n_rows;
-  p.grid = (int)smin<int64_t>(tiles, cap);
-  p.smem = (size_t)stc_smem_bytes(p.R, s.rank_k);
+  p.R = R;
+  p.grid = (int)smin<int64_t>(tiles, sm_count());
+  p.K = tiles > 2 * (int64_t)p.grid ? 2 : 1;
+  p.nB = nB;
+  p.smem = smem;
   return p;
 }
 
@@ -276,7 +333,7 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
                            unsigned int *counters, uint32_t *status, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3(kStcThreads);
+  cfg.blockDim = dim3(StcCfg<R>::kThreads);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -286,7 +343,7 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
   cfg.attrs = attr;
   cfg.numAttrs = g_coop_pdl == 0 ? 1 : 2;
   cudaError_t err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist,
-                                       counters, status);
+                                       counters, status, p.K, p.nB);
   if (cfg.numAttrs == 2 && g_coop_pdl < 0) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     cudaStreamIsCapturing(st, &cap);
@@ -297,10 +354,42 @@ s4r_status launch_score_tc(const ScorePlan &p, const CUtensorMap &tmap, const Sh
       g_coop_pdl = 0;
       cfg.numAttrs = 1;
       err = cudaLaunchKernelEx(&cfg, score_tc_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, counters,
-                               status);
+                               status, p.K, p.nB);
     }
   }
   return err == cudaSuccess ? S4R_OK : fail("score_tc_kernel (cooperative launch)", err);
+}
+
+template <int R>
+s4r_status launch_score_pair(const ScorePlan &p, const CUtensorMap &tmap, const Shape &s, const int32_t *lengths,
+                             const unsigned char *cqs, float *scores, double *rowsum, uint32_t *ehist,
+                             unsigned int *bar, uint32_t *status, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3(kSpThreads);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1] = pdl_attr();
+  cfg.attrs = attr;
+  cfg.numAttrs = g_coop_pdl == 0 ? 1 : 2;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, score_pair_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar,
+                                       status);
+  if (cfg.numAttrs == 2 && g_coop_pdl < 0) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cap);
+    if (err == cudaSuccess) {
+      g_coop_pdl = 1;
+    } else if (cap == cudaStreamCaptureStatusNone) {
+      cudaGetLastError();   // not supported together: launch without it from now on
+      g_coop_pdl = 0;
+      cfg.numAttrs = 1;
+      err = cudaLaunchKernelEx(&cfg, score_pair_kernel<R>, tmap, s, lengths, cqs, scores, rowsum, ehist, bar, status);
+    }
+  }
+  return err == cudaSuccess ? S4R_OK : fail("score_pair_kernel (cooperative launch)", err);
 }
 
 template <typename T>
@@ -357,9 +446,14 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed for the key-coefficient cache");
       return S4R_ERR_CUDA;
     }
+    // The fused kernel's grid barrier counts on the problem's counter word.
     const s4r_status rc =
-        plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st)
-                     : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st);
+        plan.pair ? (plan.R == 64 ? launch_score_pair<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters,
+                                                          status, st)
+                                  : launch_score_pair<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters,
+                                                          status, st))
+        : plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st)
+                       : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st);
     if (rc != S4R_OK) return rc;
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);

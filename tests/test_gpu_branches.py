@@ -6,10 +6,11 @@ reach, through the C ABI against the fp64 oracle:
     per-row integer offsets 2^(y - k) so that nothing overflows or flushes.
     Each case first checks, from the stored inputs, that it really drives
     tiles past that limit (Eqs. 8-10, major comment 2, §3.2.2);
-  * a bounded device wait that runs out: the scoring kernel's grid barrier is
-    made unreachable through the library's test hook, the kernel gives up
-    after a short limit and reports S4R_ERR_TIMEOUT, and the next call on
-    the same workspace matches the oracle again;
+  * a bounded device wait that runs out: the scoring kernel's grid barrier
+    (or per-problem arrival counter) is made unreachable through the
+    library's test hook, the kernel gives up after a short limit and reports
+    S4R_ERR_TIMEOUT, and the next call on the same workspace matches the
+    oracle again;
   * average pooling of the candidate scores ("free parameters": kernel 7),
     with exact ties that pooling creates.
 
@@ -127,9 +128,12 @@ def test_wide_range_rows_far_below_zero():
     _run(batch, np.abs(y).max())
 
 
-def test_bounded_wait_runs_out_and_the_next_call_recovers():
+@pytest.mark.parametrize("lengths", [[5003], [5003, 777, 130]], ids=["one-problem", "three-problems"])
+def test_bounded_wait_runs_out_and_the_next_call_recovers(lengths):
+    # One problem takes the fused two-tiles-per-CTA scoring kernel (its grid
+    # barrier), several the persistent one (its per-problem counters).
     import rank_decode_attention_b200 as s4r
-    batch = make_batch(W1, lengths=[5003, 777, 130], top_k=256, tag="timeout")
+    batch = make_batch(W1, lengths=lengths, top_k=256, tag="timeout")
     ws = workspace_for(batch)
     s4r.s4r_debug_waits(2_000_000, True)          # ~1 ms limit, grid barrier never completes
     try:
