@@ -12,9 +12,11 @@
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "k_attend.cuh"
+#include "k_attend_rows.cuh"
 #include "k_basis.cuh"
 #include "k_encode_simt.cuh"
 #include "k_encode_tc.cuh"
@@ -291,6 +293,77 @@ bool pair_launchable(size_t smem, int rank, int grid) {
   return ok;
 }
 
+// How many clusters of `nc` CTAs of the row-split attention kernel can be
+// resident at once with `smem` bytes each (0: not launchable).  Cached per
+// device, cluster size and shared-memory size.
+int ar_active_clusters(int nc, size_t smem) {
+  constexpr int kSizes = 16;
+  static std::mutex mu;
+  static int known[kMaxDevices][kSizes][3];   // (nc, smem, clusters + 1)
+  const int dev = current_device();
+  if (ensure_smem<attend_rows_kernel>(smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSizes; ++i)
+      if (known[dev][i][0] == nc && known[dev][i][1] == (int)smem) return known[dev][i][2] - 1;
+  }
+  int n = 0;
+  if (nc > 8 && cudaFuncSetAttribute(attend_rows_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                    cudaSuccess) {
+    cudaGetLastError();
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nc, 1, 1);
+    cfg.blockDim = dim3(kArThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, attend_rows_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  if (dev >= 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSizes; ++i)
+      if (known[dev][i][0] == 0) {
+        known[dev][i][0] = nc;
+        known[dev][i][1] = (int)smem;
+        known[dev][i][2] = n + 1;
+        break;
+      }
+  }
+  return n;
+}
+
+// Plan of the row-split attention kernel (bf16 storage); nc == 0 when the
+// shape or the pointers do not suit it and the per-group kernel runs.
+// Clusters of 16 CTAs halve each CTA's rows; they are taken while every
+// problem's cluster can be resident at once, else clusters of 8.
+ArPlan plan_attend_rows(const Shape &s, const void *ck, const void *cv, const void *bv) {
+  ArPlan none{};
+  if (!ar_supported(s, 2) || !aligned16(ck) || !aligned16(cv) || !aligned16(bv)) return none;
+  for (int nc : {16, 8, 4, 2, 1}) {
+    if (s.n_heads_q % nc != 0) continue;
+    const ArPlan pl = ar_plan(s, nc);
+    const size_t smem = ar_layout(s, pl).total;
+    if (!ar_plan_ok(pl) || smem > kArSmemBudget) continue;
+    const int n = ar_active_clusters(nc, smem);
+    if (n <= 0) continue;
+    if (nc == 16 && s.batch > n) continue;
+    return pl;
+  }
+  return none;
+}
+
 ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   ScorePlan p;
   if (dt != S4R_BF16 || s.cache_rows == 0 || s.batch == 0) return p;
@@ -505,8 +578,32 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
     }
     if (check_launch("topk_kernel") != S4R_OK) return S4R_ERR_CUDA;
   }
-  // 4. rebuild + exact attention (one cluster of CTAs per kv group)
-  {
+  // 4. rebuild + exact attention: the row-split kernel (one cluster per
+  // problem, every head in every CTA) for bf16 storage, else one cluster of
+  // CTAs per kv group
+  ArPlan ap{};
+  if constexpr (std::is_same<T, bf16>::value) ap = plan_attend_rows(s, ck, cv, bv);
+  if (ap.nc > 0) {
+    if constexpr (std::is_same<T, bf16>::value) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)ap.nc, (unsigned)s.batch);
+      cfg.blockDim = dim3(kArThreads);
+      cfg.dynamicSmemBytes = ar_layout(s, ap).total;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)ap.nc;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1] = pdl_attr();
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      const cudaError_t err = cudaLaunchKernelEx(&cfg, attend_rows_kernel, s, ap, a->lengths, a->idx, ck, cv, qt, q,
+                                                 bv, sk, sv, a->out, status);
+      if (err != cudaSuccess) return fail("attend_rows_kernel (cluster launch)", err);
+      if (check_launch("attend_rows_kernel") != S4R_OK) return S4R_ERR_CUDA;
+    }
+  } else {
     AttPlan pl = att_plan(s, (int)sizeof(T), att_ranks(s, sm_count()));
     if (att_smem_bytes(s, (int)sizeof(T), pl) > kAttSmemBudget) pl = att_plan(s, (int)sizeof(T));   // the checked plan
     const size_t smem = att_smem_bytes(s, (int)sizeof(T), pl);
