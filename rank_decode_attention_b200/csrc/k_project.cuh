@@ -38,7 +38,7 @@ __host__ __device__ inline int proj_cluster(int n_heads_kv) { return n_heads_kv 
 // Write scoring row i, columns c0 .. c0+63, from its fp64 values x (already
 // scaled by 1/sqrt(r)): fp32 copy for the CUDA-core path and the bf16 split.
 __device__ __forceinline__ void proj_finish(double x, int b, int R, int r, int i, int c, int kk, float *cq,
-                                            unsigned char *blk) {
+                                            unsigned char *blk, int64_t copy_stride) {
   if (c < r) cq[((int64_t)b * R + i) * r + c] = (float)x;
   // y = x log2(e) as y1 + y2 (fp32 pair, |y2| <= ulp(y1)/2), then three bf16
   // terms whose residuals are exact fp32 differences.
@@ -49,9 +49,13 @@ __device__ __forceinline__ void proj_finish(double x, int b, int R, int r, int i
   const float r1 = (y1 - __bfloat162float(hi)) + y2;
   const bf16 mid = __float2bfloat16_rn(r1);
   const bf16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-  *reinterpret_cast<bf16 *>(blk + sw128_offset(i, kk)) = hi;
-  *reinterpret_cast<bf16 *>(blk + sw128_offset(R + i, kk)) = mid;
-  *reinterpret_cast<bf16 *>(blk + sw128_offset(2 * R + i, kk)) = lo;
+#pragma unroll
+  for (int cp = 0; cp < kCqsCopies; ++cp) {
+    unsigned char *dst = blk + cp * copy_stride;
+    *reinterpret_cast<bf16 *>(dst + sw128_offset(i, kk)) = hi;
+    *reinterpret_cast<bf16 *>(dst + sw128_offset(R + i, kk)) = mid;
+    *reinterpret_cast<bf16 *>(dst + sw128_offset(2 * R + i, kk)) = lo;
+  }
 }
 
 // Per-head results of group g: qt (current query, scaled by 1/sqrt(d_h)) and,
@@ -70,7 +74,7 @@ __device__ __forceinline__ void proj_head_writes(const Shape &s, const double (&
       const int kk = tx + 16 * jj, c = c0 + kk;
       const double v = acc[i][jj];
       if (w == W - 1 && c < r) qt[((int64_t)b * Hq + h) * r + c] = (float)(v / sqrt((double)dh));
-      if (s.row_mode == S4R_ROWS_PER_HEAD) proj_finish(c < r ? v * scale : 0.0, b, R, r, w * Hq + h, c, kk, cq, blk);
+      if (s.row_mode == S4R_ROWS_PER_HEAD) proj_finish(c < r ? v * scale : 0.0, b, R, r, w * Hq + h, c, kk, cq, blk, (int64_t)s.batch * stc_b_bytes(R, r));
     }
   }
 }
@@ -231,7 +235,7 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int kk = tx + 16 * jj, c = c0 + kk;
-        if (row < W * G) proj_finish(c < r ? x[i][jj] * scale : 0.0, b, R, r, row, c, kk, cq, blk);
+        if (row < W * G) proj_finish(c < r ? x[i][jj] * scale : 0.0, b, R, r, row, c, kk, cq, blk, (int64_t)s.batch * stc_b_bytes(R, r));
       }
     }
 }

@@ -18,9 +18,10 @@
 // columns and the three are added in fp32 by the epilogue.  C_Q is scaled by
 // log2(e), so the epilogue works in base 2: e = 2^y with y = z log2(e).
 //
-// One cooperative launch, one CTA per pair of 128-position tiles (5 warps:
-// warps 0-3 run the epilogue, one per 32 TMEM lanes; one thread of warp 4
-// issues the TMA copies and the tcgen05.mma):
+// One cooperative launch, one CTA per pair of 128-position tiles: R / 8
+// epilogue warps (warp w reads TMEM lanes 32 (w % 4) .. + 31 and scoring rows
+// 32 (w / 4) .. + 31) and one more warp whose first thread issues the TMA
+// copies and the tcgen05.mma:
 //   A. TMA both C_K tiles (before the wait for the projection kernel), then
 //      bulk-copy the split C_Q operand (its shared-memory image, written by the
 //      projection kernel); MMA each tile into its own 256-column TMEM region.
@@ -71,10 +72,13 @@ struct SpControl {
 static_assert(sizeof(SpControl) <= kSpControlBytes, "control block");
 static_assert(sp_smem_bytes(64, 256) <= kStcMaxSmem && sp_smem_bytes(32, 256) <= kStcMaxSmem, "smem budget");
 
-constexpr int kSpThreads = 160;  // warps 0-3: epilogue (one TMEM lane each); warp 4: TMA + MMA issue
+// Threads of the kernel for R scoring rows: 4 R / 32 epilogue warps (each 32
+// TMEM lanes x 32 rows) and the TMA / MMA warp.
+__host__ __device__ constexpr int sp_epi_threads(int R) { return 4 * R; }
+__host__ __device__ constexpr int sp_threads(int R) { return sp_epi_threads(R) + 32; }
 
 template <int R>
-__global__ void __launch_bounds__(kSpThreads, 1)
+__global__ void __launch_bounds__(sp_threads(R), 1)
 score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int32_t *__restrict__ lengths,
                 const unsigned char *__restrict__ cqs, float *__restrict__ scores, double *__restrict__ row_sum,
                 uint32_t *__restrict__ ehist, unsigned int *__restrict__ bar, uint32_t *__restrict__ status) {
@@ -89,8 +93,10 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
   float *red = reinterpret_cast<float *>(sp_red_aliased(R, r) ? a_op : a_op + kSpTiles * sp_a_bytes(r));
   SpControl *ctl = reinterpret_cast<SpControl *>(a_op + kSpTiles * sp_a_bytes(r) +
                                                    (sp_red_aliased(R, r) ? 0 : sp_red_bytes(R)));
+  constexpr int kEpi = sp_epi_threads(R);   // epilogue threads; thread kEpi issues TMA and MMA
   const int warp = threadIdx.x >> 5;
-  const bool epi = warp < 4;
+  const bool epi = threadIdx.x < kEpi;
+  const int cg = warp >> 2;                  // epilogue: scoring rows 32cg .. 32cg + 31
   const int64_t tiles_cap = ceil_div(s.cache_rows, kStcTile);
   const int64_t ctas_per_problem = ceil_div(tiles_cap, kSpTiles);
   const int b = (int)(blockIdx.x / ctas_per_problem);
@@ -101,7 +107,7 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
   for (int t = 0; t < kSpTiles; ++t)
     if ((tile0 + t) < tiles_cap && (tile0 + t) * kStcTile < L) n_tiles = t + 1;
 
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == kEpi) {
     mbar_init(&ctl->b_full, 1);
     for (int t = 0; t < kSpTiles; ++t) {
       for (int kb = 0; kb < 4; ++kb) mbar_init(&ctl->tma_full[t][kb], 1);
@@ -124,10 +130,10 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
   // query operand, the zeroed row sums and barrier words).
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == kEpi) {
     // The split query operand, already in its shared-memory image.
     mbar_arrive_expect_tx(&ctl->b_full, (uint32_t)stc_b_bytes(R, r));
-    const unsigned char *src = cqs + (int64_t)b * stc_b_bytes(R, r);
+    const unsigned char *src = cqs + ((int64_t)(blockIdx.x % kCqsCopies) * s.batch + b) * stc_b_bytes(R, r);
     for (int kb = 0; kb < nkb; ++kb)
       bulk_load(b_op + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128, &ctl->b_full);
   }
@@ -137,7 +143,7 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
   const uint32_t tmem = ctl->tmem_base;
   bool ok = true;
 
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == kEpi) {
     // MMA issuer: D_t[128 x 3R] = A_t[128 x r] . B[3R x r]^T
     const uint32_t idesc = idesc_bf16_f32(128, 3 * R, 0, 0);
     const uint32_t b_base = smem_u32(b_op);
@@ -160,51 +166,49 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
   }
   __syncwarp();
 
-  // B: per-tile exponentials and row sums (warps 0-3; warp 4 only joins the barriers).
+  // B: per-tile exponentials and row sums (the epilogue warps; the TMA /
+  // MMA warp only joins the barriers).
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const int p = threadIdx.x;  // position within the tile (epilogue warps)
-  constexpr int TPR = 128 / R;  // threads per row in the reductions
+  const int p = (warp & 3) * 32 + (threadIdx.x & 31);   // position within the tile (epilogue threads)
   for (int t = 0; t < n_tiles; ++t) {
     const int64_t pos = (tile0 + t) * kStcTile + p;
     const bool valid = epi && pos < L;
     const uint32_t col0 = tmem + lane_base + t * kSpTileCols;
     float amax = 0.f;
+    float ev[32];   // e of this thread's position for rows 32cg .. 32cg + 31
     if (epi) {
       ok = mbar_wait(&ctl->mma_done[t], 0, status) && ok;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < R / 32; ++c) {
-        uint32_t hi[32], mid[32], lo[32];
-        tmem_ld32(col0 + c * 32, hi);
-        tmem_ld32(col0 + R + c * 32, mid);
-        tmem_ld32(col0 + 2 * R + c * 32, lo);
-        tmem_wait_ld();
-        uint32_t ev[32];
+      const int c = cg;
+      uint32_t hi[32], mid[32], lo[32];
+      tmem_ld32(col0 + c * 32, hi);
+      tmem_ld32(col0 + R + c * 32, mid);
+      tmem_ld32(col0 + 2 * R + c * 32, lo);
+      tmem_wait_ld();
+      uint32_t eb[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float y = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
-          hi[j] = __float_as_uint(y);
-          amax = valid ? fmaxf(amax, fabsf(y)) : amax;
-          const float e = valid ? ex2_approx(y) : 0.f;
-          ev[j] = __float_as_uint(e);
-          red[p * (R + 1) + c * 32 + j] = e;
-        }
-        tmem_st32(col0 + c * 32, hi);      // y
-        tmem_st32(col0 + R + c * 32, ev);  // e
-        tmem_wait_st();
+      for (int j = 0; j < 32; ++j) {
+        const float y = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
+        hi[j] = __float_as_uint(y);
+        amax = valid ? fmaxf(amax, fabsf(y)) : amax;
+        ev[j] = valid ? ex2_approx(y) : 0.f;
+        eb[j] = __float_as_uint(ev[j]);
       }
+      tmem_st32(col0 + c * 32, hi);      // y
+      tmem_st32(col0 + R + c * 32, eb);  // e
+      tmem_wait_st();
     }
     const bool wide = __syncthreads_or(amax > kSpRangeLimit) != 0;
     if (wide) {
       // Rare path: per-row integer offsets k = floor(max_i y) for this tile.
-      if (epi)
-        for (int c = 0; c < R / 32; ++c) {
-          uint32_t yv[32];
-          tmem_ld32(col0 + c * 32, yv);
-          tmem_wait_ld();
+      const int c = cg;
+      if (epi) {
+        uint32_t yv[32];
+        tmem_ld32(col0 + c * 32, yv);
+        tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) red[p * (R + 1) + c * 32 + j] = valid ? __uint_as_float(yv[j]) : -INFINITY;
-        }
+        for (int j = 0; j < 32; ++j) red[p * (R + 1) + c * 32 + j] = valid ? __uint_as_float(yv[j]) : -INFINITY;
+      }
       __syncthreads();
       if (threadIdx.x < R) {
         float m = -INFINITY;
@@ -212,44 +216,45 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
         ctl->kofs[t][threadIdx.x] = (m == -INFINITY) ? 0 : (int)floorf(m);
       }
       __syncthreads();
-      if (epi)
-        for (int c = 0; c < R / 32; ++c) {
-          uint32_t yv[32], ev[32];
-          tmem_ld32(col0 + c * 32, yv);
-          tmem_wait_ld();
+      if (epi) {
+        uint32_t yv[32], eb[32];
+        tmem_ld32(col0 + c * 32, yv);
+        tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float e = valid ? ex2_approx(__uint_as_float(yv[j]) - (float)ctl->kofs[t][c * 32 + j]) : 0.f;
-            ev[j] = __float_as_uint(e);
-            red[p * (R + 1) + c * 32 + j] = e;
-          }
-          tmem_st32(col0 + R + c * 32, ev);
-          tmem_wait_st();
+        for (int j = 0; j < 32; ++j) {
+          ev[j] = valid ? ex2_approx(__uint_as_float(yv[j]) - (float)ctl->kofs[t][c * 32 + j]) : 0.f;
+          eb[j] = __float_as_uint(ev[j]);
         }
+        tmem_st32(col0 + R + c * 32, eb);
+        tmem_wait_st();
+      }
+      __syncthreads();   // the scratch is read before it takes the partial sums
     } else if (threadIdx.x < R) {
       ctl->kofs[t][threadIdx.x] = 0;
     }
+    // Row sums over the tile's 128 positions.  Within a warp (32 positions)
+    // by a transposing butterfly: at step w the lanes with bit w set keep the
+    // upper half of their rows and add their partner's, so lane j ends with
+    // the sum of row 32cg + j (a fixed order); the four warps of a column
+    // group are then added in a fixed order.
+    if (epi) {
+      const int lane = threadIdx.x & 31;
+#pragma unroll
+      for (int w = 16; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int j = 0; j < w; ++j) {
+          const float send = upper ? ev[j] : ev[j + w];
+          const float keep = upper ? ev[j + w] : ev[j];
+          ev[j] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+      }
+      red[(warp & 3) * R + cg * 32 + lane] = ev[0];
+    }
     __syncthreads();
-    // Row sums over the tile's 128 positions: TPR threads per row, four
-    // independent fp32 partial sums each, combined in a fixed order.
-    {
-      const int row = threadIdx.x % R, part = threadIdx.x / R;
-      constexpr int kPer = kStcTile / TPR;
-      float mine = 0.f;
-      if (epi) {
-        float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int q = 0; q < kPer; ++q) a4[q & 3] += red[(part * kPer + q) * (R + 1) + row];
-        mine = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-      }
-      __syncthreads();
-      if (epi) red[p * (R + 1) + R] = mine;   // column R of the scratch is free
-      __syncthreads();
-      if (epi && part == 0) {
-        float l = 0.f;
-        for (int pp = 0; pp < TPR; ++pp) l += red[(pp * R + row) * (R + 1) + R];
-        ctl->tile_sum[t][row] = l;
-      }
+    if (threadIdx.x < R) {
+      const int row = threadIdx.x;
+      ctl->tile_sum[t][row] = (red[row] + red[R + row]) + (red[2 * R + row] + red[3 * R + row]);
     }
     __syncthreads();
   }
@@ -285,17 +290,16 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
     const double inv = (l > 0.0) ? 1.0 / l : 0.0;
     for (int t = 0; t < n_tiles; ++t) ctl->alpha[t][row] = (float)ldexp(inv, ctl->kofs[t][row]);
   }
-  // Level-0 histogram of this CTA's candidate scores (rows before the local
-  // window; score_bin around the mean R / L_c) for the top-k kernel, in the
-  // now idle reduction scratch.
-  static_assert(kStcTile * 33 * 4 >= kExpBins * 4, "histogram fits the reduction scratch");
-  uint32_t *hist = reinterpret_cast<uint32_t *>(red);
+  // Level-0 histogram of the candidate scores (rows before the local window;
+  // score_bin around the mean R / L_c) for the top-k kernel: neighbouring
+  // positions mostly share a bin, so each warp adds one count per distinct
+  // bin straight into the problem's histogram.
   const uint32_t center = score_center(s.n_rows, L);
-  for (int i = threadIdx.x; i < kExpBins; i += blockDim.x) hist[i] = 0u;
+  uint32_t *hist = ehist + (int64_t)b * kExpBins;
   const int64_t n_cand = L > s.local_window ? L - s.local_window : 0;
-  __syncthreads();
+  __syncthreads();   // alpha is written
   if (epi)
-    for (int t = 0; t < n_tiles; ++t) {
+    for (int t = cg; t < n_tiles; t += R / 32) {
       const int64_t pos = (tile0 + t) * kStcTile + p;
       const uint32_t col0 = tmem + lane_base + t * kSpTileCols;
       float acc = 0.f;
@@ -310,12 +314,10 @@ score_pair_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
       if (pos < L) scores[(int64_t)b * s.cache_rows + pos] = acc;
       const bool cand = pos < n_cand;
       const uint32_t bin = cand ? (uint32_t)score_bin(__float_as_uint(acc), center) : 0xffffffffu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);   // neighbours mostly share a bin
-      if (cand && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (cand && (threadIdx.x & 31) == __ffs(peers) - 1)
+        asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(hist + bin), "r"((uint32_t)__popc(peers)) : "memory");
     }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kExpBins; i += blockDim.x)
-    if (hist[i]) atomicAdd(&ehist[(int64_t)b * kExpBins + i], hist[i]);
   }
   tc_fence_before();
   __syncthreads();

@@ -72,6 +72,11 @@ struct StcCfg {
 
 __host__ __device__ constexpr int stc_kblocks(int r) { return (r + 63) / 64; }
 __host__ __device__ constexpr int stc_b_bytes(int R, int r) { return stc_kblocks(r) * 3 * R * 128; }
+// The projection kernel writes kCqsCopies identical images of the split
+// C_Q operand (copy c of every problem at c * batch * stc_b_bytes): the CTAs
+// of a scoring launch read copy (CTA % kCqsCopies), so the L2 lines each
+// image is read from serve a quarter of the CTAs.
+constexpr int kCqsCopies = 4;
 // Split C_Q buffers: one, or two (the next problem's operand loads while the
 // current one is in use) when at least kStcMinStages ring stages still fit.
 __host__ __device__ constexpr bool stc_two_b_fit(int R, int r) {
@@ -352,7 +357,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
           const int buf = (int)(n_switch % nB);
           if (n_switch >= (uint32_t)nB) ok = mbar_wait(&ctl->b_empty[buf], ((n_switch / nB) - 1) & 1, status);
           if (!ok) break;
-          const unsigned char *src = cqs + (int64_t)t.p * b_bytes;
+          const unsigned char *src = cqs + ((int64_t)(blockIdx.x % kCqsCopies) * s.batch + t.p) * b_bytes;
           for (int kb = 0; kb < nkb; ++kb) {
             mbar_arrive_expect_tx(&ctl->b_full[buf][kb], (uint32_t)(3 * R * 128));
             bulk_load(b_op + buf * b_bytes + kb * (3 * R * 128), src + kb * (3 * R * 128), 3 * R * 128,

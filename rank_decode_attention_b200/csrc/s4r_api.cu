@@ -51,7 +51,7 @@ Layout layout_for(const Shape &s) {
   l.counters = off; off += round_up(sizeof(uint32_t) * (size_t)s.batch);
   l.cq = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_rows * s.rank_k);
   const size_t n_cb = (size_t)ceil_div(s.rank_k, kProjColBlock);
-  l.cqs = off; off += round_up((size_t)s.batch * n_cb * cqs_block_bytes(s.n_rows));
+  l.cqs = off; off += round_up((size_t)kCqsCopies * s.batch * n_cb * cqs_block_bytes(s.n_rows));
   l.qt = off; off += round_up(sizeof(float) * s.batch * (size_t)s.n_heads_q * s.rank_k);
   const size_t n_tiles = (size_t)ceil_div(s.cache_rows, kScoreTile);
   l.tstat = off; off += round_up(sizeof(double) * 2 * s.batch * n_tiles * s.n_rows);
@@ -285,7 +285,7 @@ bool pair_launchable(size_t smem, int rank, int grid) {
     if (c > 0) return c == 2;
   }
   int per_sm = 0;
-  const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_pair_kernel<R>, kSpThreads, smem) ==
+  const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_pair_kernel<R>, sp_threads(R), smem) ==
                       cudaSuccess &&
                   per_sm > 0;
   if (!ok) cudaGetLastError();
@@ -439,7 +439,7 @@ s4r_status launch_score_pair(const ScorePlan &p, const CUtensorMap &tmap, const 
                              unsigned int *bar, uint32_t *status, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3(kSpThreads);
+  cfg.blockDim = dim3(sp_threads(R));
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];

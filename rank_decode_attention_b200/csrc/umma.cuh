@@ -188,14 +188,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // Grid-wide barrier for a cooperative launch.  `bar` points at kBarWords
 // words that an earlier launch on the same stream zeroed; every CTA adds one
 // arrival to bar[0] and waits (bounded) until all gridDim.x CTAs arrived.
+// The arrival is a release at gpu scope (cumulative over what the CTA's
+// threads wrote before the CTA barrier), the polling loads are acquires.
 // Returns false on timeout.
 constexpr int kBarWords = 2;
 __device__ __forceinline__ bool grid_barrier(unsigned int *bar, uint32_t *status, int *flag_smem) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    __threadfence();
-    atomicAdd(bar, 1u);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
     const unsigned int target = gridDim.x + (*reinterpret_cast<volatile uint32_t *>(&g_barrier_unreachable) ? 1u : 0u);
     const long long limit = wait_limit();
     const long long t0 = clock64();
