@@ -217,7 +217,8 @@ s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const vo
     return S4R_ERR_CUDA;
   const size_t smem = enc_smem_bytes(r);
   ensure_smem<encode_tc_kernel<bf16>>(smem);
-  encode_tc_kernel<bf16><<<(unsigned)ceil_div(n, kEncBM), 128, smem, st>>>(ms, mb, static_cast<bf16 *>(coeffs),
+  const unsigned grid = (unsigned)smin<int64_t>(ceil_div(n, kEncBM), sm_count());
+  encode_tc_kernel<bf16><<<grid, kEncThreads, smem, st>>>(ms, mb, static_cast<bf16 *>(coeffs),
                                                                             ldc, n, d, r);
   return last_cuda();
 }
