@@ -106,6 +106,18 @@ s4r_status s4r_encode(const void *states, int64_t n_tokens, int64_t states_ld,
                       const void *basis, int32_t d_model, int32_t rank,
                       void *coeffs, int64_t coeffs_ld, s4r_dtype dtype, void *stream);
 
+/* Encode two token sets against their own bases in one launch: the K and V
+ * halves of a prompt (Eq. 3, "What carries the argument"), for p = 0, 1:
+ *   coeffs_p[t][j] = sum_d states_p[t][d] * basis_p[d][j],  t < n_tokens.
+ * Each (states_p, basis_p, coeffs_p) follows the layout, type, rounding and
+ * alignment rules of s4r_encode; both share n_tokens, the strides, d_model
+ * and rank.  The result equals two s4r_encode calls (the tensor-core path
+ * runs both in one persistent grid, so the second problem's tiles fill the
+ * SMs the first leaves idle).  Inputs and outputs stay owned by the caller. */
+s4r_status s4r_encode2(const void *states0, const void *states1, int64_t n_tokens, int64_t states_ld,
+                       const void *basis0, const void *basis1, int32_t d_model, int32_t rank,
+                       void *coeffs0, void *coeffs1, int64_t coeffs_ld, s4r_dtype dtype, void *stream);
+
 /* Append one new token per problem to the coefficient caches (Eq. 3 applied
  * to the token a decode step adds).  For each problem b, with n = lengths[b]
  * read on the device:

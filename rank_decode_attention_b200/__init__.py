@@ -79,6 +79,7 @@ class BasisArgs(ctypes.Structure):
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 SIGNATURES = {
     "s4r_encode": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i32, _vp, _i64, ctypes.c_int, _vp]),
+    "s4r_encode2": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _vp, _vp, _i64, ctypes.c_int, _vp]),
     "s4r_append": (ctypes.c_int, [ctypes.POINTER(AppendArgs), _vp]),
     "s4r_decode_workspace_bytes": (_sz, [ctypes.POINTER(DecodeArgs)]),
     "s4r_decode_kernel_launches": (_i32, [ctypes.POINTER(DecodeArgs)]),
@@ -156,6 +157,20 @@ def s4r_encode(states: torch.Tensor, basis: torch.Tensor, coeffs: torch.Tensor, 
     return _check(lib().s4r_encode(_ptr(states), n, states.stride(0), _ptr(basis), d, r,
                                    _ptr(coeffs), coeffs.stride(0), _DTYPE[states.dtype],
                                    _stream(stream)), "s4r_encode")
+
+
+def s4r_encode2(states, bases, coeffs, stream=None) -> int:
+    """coeffs[p][t] = states[p][t] . bases[p] for p = 0, 1 (Eq. 3), one
+    launch: two token sets of the same shape and strides with their own
+    bases (the K and V halves of a prompt)."""
+    s0, s1 = states
+    n, d = s0.shape
+    r = bases[0].shape[1]
+    if s1.shape != s0.shape or s1.stride(0) != s0.stride(0) or coeffs[1].stride(0) != coeffs[0].stride(0):
+        raise ValueError("s4r_encode2: both problems need the same shape and strides")
+    return _check(lib().s4r_encode2(_ptr(s0), _ptr(s1), n, s0.stride(0), _ptr(bases[0]), _ptr(bases[1]), d, r,
+                                    _ptr(coeffs[0]), _ptr(coeffs[1]), coeffs[0].stride(0), _DTYPE[s0.dtype],
+                                    _stream(stream)), "s4r_encode2")
 
 
 def append_args(*, state_k, state_v, basis_k, basis_v, coeff_k, coeff_v, lengths,

@@ -5,7 +5,9 @@
 // a dense GEMM, M = tokens, N = rank, K = D'.
 //
 // Persistent: one CTA per SM loops over 128-token tiles (tile = CTA, CTA +
-// grid, ...), with three roles that run ahead of one another:
+// grid, ...) of one or two independent problems (the K and V halves of a
+// prompt, each with its own basis: tiles 0 .. n_tiles - 1 are problem 0's),
+// with three roles that run ahead of one another:
 //   * warp 0 streams K-blocks of 64 with TMA (S tile: 128 x 64, K-major;
 //     basis tile: 64 x rank, N-major; both 128-byte swizzled) through a
 //     kEncStages-deep mbarrier ring, across tile boundaries;
@@ -34,10 +36,18 @@ __host__ __device__ constexpr int enc_stage_bytes(int rank) { return kEncABytes 
 __host__ __device__ constexpr int enc_tmem_cols(int rank) { return rank <= 32 ? 32 : rank <= 64 ? 64 : rank <= 128 ? 128 : 256; }
 __host__ inline size_t enc_smem_bytes(int rank) { return (size_t)kEncStages * enc_stage_bytes(rank) + 1024 + 256; }
 
+// Outputs of the (at most two) problems of a launch.
+template <typename OutT>
+struct EncOut {
+  OutT *C[2];
+  int64_t ldc[2];
+};
+
 template <typename OutT>
 __global__ void __launch_bounds__(kEncThreads, 1)
-encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_b,
-                 OutT *__restrict__ C, int64_t ldc, int64_t n, int d, int r) {
+encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s0, const __grid_constant__ CUtensorMap tmap_b0,
+                 const __grid_constant__ CUtensorMap tmap_s1, const __grid_constant__ CUtensorMap tmap_b1,
+                 EncOut<OutT> o, int n_prob, int64_t n, int d, int r) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -50,7 +60,8 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (d + kEncBK - 1) / kEncBK;
   const int nb = (r + 63) / 64;
-  const int64_t n_tiles = (n + kEncBM - 1) / kEncBM;
+  const int64_t n_tiles = (n + kEncBM - 1) / kEncBM;   // per problem
+  const int64_t all_tiles = n_prob * n_tiles;
   const uint32_t acc_cols = enc_tmem_cols(r);
 
   if (threadIdx.x == 0) {
@@ -63,8 +74,12 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_consta
       mbar_init(&acc_empty[a], 4);   // one arrival per epilogue warp
     }
     mbar_fence_init();
-    tma_prefetch_desc(&tmap_s);
-    tma_prefetch_desc(&tmap_b);
+    tma_prefetch_desc(&tmap_s0);
+    tma_prefetch_desc(&tmap_b0);
+    if (n_prob > 1) {
+      tma_prefetch_desc(&tmap_s1);
+      tma_prefetch_desc(&tmap_b1);
+    }
   }
   if (warp == 0) tmem_alloc(tmem_slot, 2 * acc_cols);
   tc_fence_before();
@@ -76,7 +91,11 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_consta
     // TMA producer: every K-block of every tile of this CTA, in order.
     bool ok = true;
     uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+    for (int64_t tile = blockIdx.x; tile < all_tiles && ok; tile += gridDim.x) {
+      const bool p1 = tile >= n_tiles;
+      const CUtensorMap *ms = p1 ? &tmap_s1 : &tmap_s0;
+      const CUtensorMap *mb = p1 ? &tmap_b1 : &tmap_b0;
+      const int32_t m0 = (int32_t)((p1 ? tile - n_tiles : tile) * kEncBM);
       for (int kb = 0; kb < nk && ok; ++kb, ++it) {
         const int s = (int)(it % kEncStages);
         if (it >= (uint32_t)kEncStages) ok = mbar_wait(&empty[s], ((it / kEncStages) - 1) & 1, nullptr);
@@ -84,8 +103,8 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_consta
         unsigned char *a = smem + s * stage_bytes;
         unsigned char *b = a + kEncABytes;
         mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
-        tma_load_2d(a, &tmap_s, &full[s], kb * kEncBK, (int32_t)(tile * kEncBM));
-        for (int j = 0; j < nb; ++j) tma_load_2d(b + j * (kEncBK * 128), &tmap_b, &full[s], j * 64, kb * kEncBK);
+        tma_load_2d(a, ms, &full[s], kb * kEncBK, m0);
+        for (int j = 0; j < nb; ++j) tma_load_2d(b + j * (kEncBK * 128), mb, &full[s], j * 64, kb * kEncBK);
       }
     }
   } else if (threadIdx.x == 32) {
@@ -93,7 +112,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_consta
     bool ok = true;
     const uint32_t idesc = idesc_bf16_f32(128, r, 0, 1);
     uint32_t it = 0, lt = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+    for (int64_t tile = blockIdx.x; tile < all_tiles && ok; tile += gridDim.x, ++lt) {
       const uint32_t a = lt & 1;
       if (lt >= 2) ok = mbar_wait(&acc_empty[a], ((lt / 2) - 1) & 1, nullptr);
       if (!ok) break;
@@ -121,12 +140,15 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_consta
     const int quad = warp & 3;
     bool ok = true;
     uint32_t lt = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+    for (int64_t tile = blockIdx.x; tile < all_tiles && ok; tile += gridDim.x, ++lt) {
       const uint32_t a = lt & 1;
       ok = mbar_wait(&acc_full[a], (lt / 2) & 1, nullptr);
       if (!ok) break;
       tc_fence_after();
-      const int64_t row = tile * kEncBM + quad * 32 + lane;
+      const int p = tile >= n_tiles ? 1 : 0;
+      OutT *C = o.C[p];
+      const int64_t ldc = o.ldc[p];
+      const int64_t row = (tile - p * n_tiles) * kEncBM + quad * 32 + lane;
       for (int c0 = 0; c0 < r; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + a * acc_cols + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);

@@ -208,18 +208,29 @@ bool make_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor-core encode of bf16 states: requires rank % 32 == 0.
-s4r_status encode_tc_launch(const void *states, int64_t n, int64_t lds, const void *basis, int d, int r,
-                            void *coeffs, int64_t ldc, cudaStream_t st) {
-  CUtensorMap ms, mb;
-  if (!make_tmap_bf16(&ms, states, (uint64_t)d, (uint64_t)n, (uint64_t)lds * 2, kEncBK, kEncBM) ||
-      !make_tmap_bf16(&mb, basis, (uint64_t)r, (uint64_t)d, (uint64_t)r * 2, 64, kEncBK))
-    return S4R_ERR_CUDA;
+// Tensor-core encode of bf16 states (rank % 32 == 0) for n_prob (1 or 2)
+// problems of the same shape in one persistent launch.
+s4r_status encode_tc_launch(int n_prob, const void *const *states, int64_t n, int64_t lds,
+                            const void *const *basis, int d, int r, void *const *coeffs, int64_t ldc,
+                            cudaStream_t st) {
+  CUtensorMap ms[2], mb[2];
+  for (int p = 0; p < n_prob; ++p)
+    if (!make_tmap_bf16(&ms[p], states[p], (uint64_t)d, (uint64_t)n, (uint64_t)lds * 2, kEncBK, kEncBM) ||
+        !make_tmap_bf16(&mb[p], basis[p], (uint64_t)r, (uint64_t)d, (uint64_t)r * 2, 64, kEncBK))
+      return S4R_ERR_CUDA;
+  if (n_prob == 1) {
+    ms[1] = ms[0];
+    mb[1] = mb[0];
+  }
+  EncOut<bf16> o;
+  for (int p = 0; p < 2; ++p) {
+    o.C[p] = static_cast<bf16 *>(coeffs[p < n_prob ? p : 0]);
+    o.ldc[p] = ldc;
+  }
   const size_t smem = enc_smem_bytes(r);
   ensure_smem<encode_tc_kernel<bf16>>(smem);
-  const unsigned grid = (unsigned)smin<int64_t>(ceil_div(n, kEncBM), sm_count());
-  encode_tc_kernel<bf16><<<grid, kEncThreads, smem, st>>>(ms, mb, static_cast<bf16 *>(coeffs),
-                                                                            ldc, n, d, r);
+  const unsigned grid = (unsigned)smin<int64_t>(n_prob * ceil_div(n, kEncBM), sm_count());
+  encode_tc_kernel<bf16><<<grid, kEncThreads, smem, st>>>(ms[0], mb[0], ms[1], mb[1], o, n_prob, n, d, r);
   return last_cuda();
 }
 
@@ -781,7 +792,7 @@ s4r_status s4r_encode(const void *states, int64_t n_tokens, int64_t states_ld, c
   if (d_model > S4R_MAX_D_MODEL || rank > S4R_MAX_RANK) return S4R_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == S4R_BF16 && rank % 32 == 0)
-    return encode_tc_launch(states, n_tokens, states_ld, basis, d_model, rank, coeffs, coeffs_ld, st);
+    return encode_tc_launch(1, &states, n_tokens, states_ld, &basis, d_model, rank, &coeffs, coeffs_ld, st);
   dim3 grid((unsigned)ceil_div(n_tokens, kEncTileM), (unsigned)ceil_div(rank, kEncTileN));
   if (dtype == S4R_BF16)
     encode_simt<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16 *>(states), n_tokens, states_ld,
@@ -792,6 +803,32 @@ s4r_status s4r_encode(const void *states, int64_t n_tokens, int64_t states_ld, c
                                              static_cast<const float *>(basis), d_model, rank,
                                              static_cast<float *>(coeffs), coeffs_ld);
   return last_cuda();
+}
+
+s4r_status s4r_encode2(const void *states0, const void *states1, int64_t n_tokens, int64_t states_ld,
+                       const void *basis0, const void *basis1, int32_t d_model, int32_t rank,
+                       void *coeffs0, void *coeffs1, int64_t coeffs_ld, s4r_dtype dtype, void *stream) {
+  if (dtype != S4R_F32 && dtype != S4R_BF16) return S4R_ERR_INVALID_ARG;
+  if (n_tokens < 0 || d_model <= 0 || rank <= 0 || states_ld < d_model || coeffs_ld < rank)
+    return S4R_ERR_INVALID_ARG;
+  if (n_tokens == 0) return S4R_OK;
+  const void *st_[2] = {states0, states1}, *bs_[2] = {basis0, basis1};
+  void *cs_[2] = {coeffs0, coeffs1};
+  for (int p = 0; p < 2; ++p)
+    if (!st_[p] || !bs_[p] || !cs_[p] || !aligned16(st_[p]) || !aligned16(bs_[p]) || !aligned16(cs_[p]))
+      return S4R_ERR_INVALID_ARG;
+  const size_t e = esize(dtype);
+  if ((states_ld * e) % 16 || (coeffs_ld * e) % 16 || ((int64_t)rank * e) % 16) return S4R_ERR_INVALID_ARG;
+  if (d_model > S4R_MAX_D_MODEL || rank > S4R_MAX_RANK) return S4R_ERR_UNSUPPORTED;
+  if (dtype == S4R_BF16 && rank % 32 == 0)
+    return encode_tc_launch(2, st_, n_tokens, states_ld, bs_, d_model, rank, cs_, coeffs_ld,
+                            static_cast<cudaStream_t>(stream));
+  for (int p = 0; p < 2; ++p) {
+    const s4r_status rc = s4r_encode(st_[p], n_tokens, states_ld, bs_[p], d_model, rank, cs_[p], coeffs_ld,
+                                     dtype, stream);
+    if (rc != S4R_OK) return rc;
+  }
+  return S4R_OK;
 }
 
 s4r_status s4r_append(const s4r_append_args *a, void *stream) {

@@ -46,6 +46,23 @@ def test_encode_matches_oracle(dtype, n, d, r):
     check_encode(S, B, C.cpu(), dtype)
 
 
+@pytest.mark.parametrize("dtype,n,d,r", [("bf16", 3000, 1024, 256), ("bf16", 129, 1024, 192),
+                                         ("bf16", 1, 128, 32), ("f32", 300, 128, 32), ("bf16", 500, 256, 48)])
+def test_encode2_matches_oracle_for_both_problems(dtype, n, d, r):
+    """The two-problem launch (K and V halves, each with its own basis) gives
+    each half exactly the oracle's encode; tile counts that are not a multiple
+    of the grid put both problems' tiles on one CTA."""
+    import rank_decode_attention_b200 as s4r
+    g = torch.Generator().manual_seed(n * 11 + r)
+    S = [synth.store(torch.randn(n, d, generator=g, dtype=torch.float64), dtype) for _ in range(2)]
+    B = [synth.store(torch.randn(d, r, generator=g, dtype=torch.float64) / d ** 0.5, dtype) for _ in range(2)]
+    C = [torch.full((n, r), float("nan"), dtype=S[0].dtype, device="cuda") for _ in range(2)]
+    s4r.s4r_encode2([x.cuda() for x in S], [x.cuda() for x in B], C)
+    torch.cuda.synchronize()
+    for p in range(2):
+        check_encode(S[p], B[p], C[p].cpu(), dtype)
+
+
 def test_encode_strided_rows():
     import rank_decode_attention_b200 as s4r
     g = torch.Generator().manual_seed(5)
