@@ -39,6 +39,7 @@ cores instead (rank 0 only), on the same workload and config.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -674,6 +675,32 @@ def run_s4r(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args, w: synth.Workload):
+    """A short untimed run for ncu captures (committed so that every profile
+    summary names a command of this repository): `decode` makes four
+    s4r_decode_step calls on one layer of the workload (every problem of that
+    layer), `encode` three s4r_encode2 calls of the bulk K + V encode."""
+    import rank_decode_attention_b200 as s4r
+    dev = torch.device("cuda", 0)
+    if args.profile_case == "encode":
+        n, D, r = synth.BULK_ENCODE_TOKENS, 1024, 256
+        g = torch.Generator(device=dev).manual_seed(1234)
+        S = [synth.store(torch.randn(n, D, generator=g, device=dev, dtype=torch.float32), "bf16") for _ in range(2)]
+        Bs = [synth.store(torch.randn(D, r, generator=g, device=dev, dtype=torch.float32) / 32, "bf16")
+              for _ in range(2)]
+        C = [torch.empty(n, r, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        for _ in range(3):
+            s4r.s4r_encode2(S, Bs, C)
+        calls = 3
+    else:
+        wl = GpuWorkload(dataclasses.replace(w, layers=1), 0, dev, 1)
+        for _ in range(4):
+            wl.step_calls(0)
+        calls = 4
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": args.profile_case, "workload": w.name, "calls": calls}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -686,8 +713,13 @@ def main():
     ap.add_argument("--no-encode", action="store_true")
     ap.add_argument("--no-basis", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["decode", "encode"],
+                    help="untimed small case for ncu: one layer of --workload, or the bulk encode")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.profile_case:
+        run_profile_case(args, w)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -56,6 +56,7 @@ struct ArPlan {
   int hpc;     // heads finished per CTA (H_q / nc)
   int e_cap;   // selected rows per chunk, a multiple of 16
   int n_grp;   // kv groups spanned by one CTA's heads (rows of B^V staged: n_grp * d_h)
+  int late_bv; // 1: B^V is copied into the spent row buffers after the last chunk (frees its region for rows)
 };
 
 // Kv groups spanned by the heads c*hpc .. c*hpc + hpc - 1.
@@ -66,31 +67,44 @@ __host__ __device__ inline int ar_groups_of(int G, int hpc, int c) {
 
 // Shared-memory regions (byte offsets, each 16-byte aligned).
 struct ArLayout {
-  size_t qb, rows, bv, pb, recv, ob, oacc, fl, rows_idx, total;
+  size_t qb, rows, part, bv, pb, recv, ob, oacc, fl, rows_idx, total;
 };
 __host__ __device__ inline ArLayout ar_layout(const Shape &s, const ArPlan &pl) {
   const int pk = att_pitch(s.rank_k, 2), pv = att_pitch(s.rank_v, 2), ppb = att_pitch(pl.e_cap, 2);
+  const size_t qbytes = (size_t)2 * kArMaxHeads * pk * 2;              // split latent queries
+  const size_t rbytes = (size_t)pl.e_cap * (pk + pv) * 2;              // a chunk's C_K and C_V rows
+  const size_t part = (size_t)s.n_heads_q * (s.rank_v + 4) * 4;        // this CTA's partials
+  const size_t bvb = (size_t)pl.n_grp * s.head_dim * pv * 2;           // rows of B^V
+  const size_t obb = (size_t)16 * pv * 2;                               // merged acc, three bf16 terms per head
+  const size_t oab = (size_t)16 * pl.n_grp * s.head_dim * 4;           // output products per term
   ArLayout ly;
   size_t o = 0;
-  // [2 * kArMaxHeads][pk] split latent queries; after the last chunk's
-  // logits the output product's operands: [16][pv] merged acc (three bf16
-  // terms per head) and [16][n_grp * d_h] fp32 products per term
   ly.qb = o;
-  ly.ob = o;
-  ly.oacc = o + (size_t)16 * pv * 2;
-  const size_t qbytes = (size_t)2 * kArMaxHeads * pk * 2;
-  const size_t obytes = (size_t)16 * pv * 2 + (size_t)16 * pl.n_grp * s.head_dim * 4;
-  o += qbytes > obytes ? qbytes : obytes;
-  ly.rows = o;                                                  // [e_cap][pk] C_K, [e_cap][pv] C_V; later the partials
-  const size_t rows = (size_t)pl.e_cap * (pk + pv) * 2;
-  const size_t part = (size_t)s.n_heads_q * (s.rank_v + 4) * 4;
-  o += rows > part ? rows : part;
-  ly.bv = o;                                                    // [n_grp * d_h][pv] rows of B^V
-  o += (size_t)pl.n_grp * s.head_dim * pv * 2;
+  if (!pl.late_bv) {
+    // [qb | ob oacc] [rows | part] [bv] ...
+    ly.ob = o;
+    ly.oacc = o + obb;
+    o += qbytes > obb + oab ? qbytes : obb + oab;
+    ly.rows = o;
+    o += rbytes > part ? rbytes : part;
+    ly.bv = o;
+    o += bvb;
+  } else {
+    // [qb | part] [rows | bv ob oacc] ...: after the last chunk the partials
+    // take the query region and B^V, then the output operands, the rows'
+    ly.part = o;
+    o += qbytes > part ? qbytes : part;
+    ly.rows = o;
+    ly.bv = o;
+    ly.ob = o + bvb;
+    ly.oacc = o + bvb + obb;
+    o += rbytes > bvb + obb + oab ? rbytes : bvb + obb + oab;
+  }
+  if (!pl.late_bv) ly.part = ly.rows;
   ly.pb = o;                                                    // [2 * kArMaxHeads][ppb] split weights
   o += (size_t)2 * kArMaxHeads * ppb * 2;
   ly.recv = o;                                                  // [nc][hpc][rv + 4] partials of the heads finished here
-  o += (size_t)s.n_heads_q * (s.rank_v + 4) * 4;
+  o += part;
   ly.fl = o;
   size_t nf = (size_t)2 * kArMaxMt * kArMaxHeads               // per-m-tile maxima and sums
               + 3 * kArMaxHeads                                 // running max, running sum, rescale
@@ -114,6 +128,9 @@ __host__ inline bool ar_supported(const Shape &s, int esize) {
 // two kv groups.
 __host__ inline bool ar_plan_ok(const ArPlan &pl) { return pl.hpc >= 1 && 3 * pl.hpc <= 16 && pl.n_grp <= 2; }
 
+// The chunk size is the largest that fits (at most the CTA's rows); B^V is
+// prefetched before the wait for the top-k kernel unless copying it after
+// the last chunk lets the rows fit in fewer chunks.
 __host__ inline ArPlan ar_plan(const Shape &s, int nc) {
   ArPlan pl;
   pl.nc = nc;
@@ -121,9 +138,21 @@ __host__ inline ArPlan ar_plan(const Shape &s, int nc) {
   pl.n_grp = 1;
   for (int c = 0; c < nc; ++c) pl.n_grp = smax(pl.n_grp, ar_groups_of(s.group, pl.hpc, c));
   const int64_t per = ceil_div((int64_t)s.top_k + s.local_window, nc);   // rows per CTA at most
-  pl.e_cap = (int)smin<int64_t>(kArMaxRows, smax<int64_t>(16, (per + 15) / 16 * 16));
-  while (pl.e_cap > 16 && ar_layout(s, pl).total > kArSmemBudget) pl.e_cap -= 16;
-  return pl;
+  const int want = (int)smin<int64_t>(kArMaxRows, smax<int64_t>(16, (per + 15) / 16 * 16));
+  ArPlan best = pl;
+  int64_t best_chunks = 0;
+  for (int late = 0; late < 2; ++late) {
+    ArPlan c = pl;
+    c.late_bv = late;
+    c.e_cap = want;
+    while (c.e_cap > 16 && ar_layout(s, c).total > kArSmemBudget) c.e_cap -= 16;
+    const int64_t chunks = ceil_div(per, c.e_cap);
+    if (late == 0 || chunks < best_chunks) {
+      best = c;
+      best_chunks = chunks;
+    }
+  }
+  return best;
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -174,7 +203,7 @@ attend_rows_kernel(Shape s, ArPlan pl, const int32_t *__restrict__ lengths, cons
   bf16 *qb = reinterpret_cast<bf16 *>(ar_smem + ly.qb);
   bf16 *ck = reinterpret_cast<bf16 *>(ar_smem + ly.rows);
   bf16 *cv = ck + (size_t)E * pk;
-  float *part = reinterpret_cast<float *>(ar_smem + ly.rows);   // after the last chunk: [H_q][pr] = (m, l, -, -, acc)
+  float *part = reinterpret_cast<float *>(ar_smem + ly.part);   // after the last chunk: [H_q][pr] = (m, l, -, -, acc)
   bf16 *bvs = reinterpret_cast<bf16 *>(ar_smem + ly.bv);
   bf16 *pb = reinterpret_cast<bf16 *>(ar_smem + ly.pb);
   float *red_m = reinterpret_cast<float *>(ar_smem + ly.fl);    // [kArMaxMt][kArMaxHeads]
@@ -219,14 +248,16 @@ attend_rows_kernel(Shape s, ArPlan pl, const int32_t *__restrict__ lengths, cons
   const int64_t per = ceil_div(n_sel, nc);
   const int64_t e_begin = smin<int64_t>(n_sel, (int64_t)rank * per);
   const int64_t e_end = smin<int64_t>(n_sel, e_begin + per);
-  {
-    // rows of B^V for the heads finished here: warp per row, lane per 16 bytes
+  // Rows of B^V for the heads finished here: warp per row, lane per 16
+  // bytes; before the wait, or after the last chunk in the late layout.
+  auto copy_bv = [&]() {
     const bf16 *src = basis_v + (int64_t)b * Dp * rv + (int64_t)g0 * dh * rv;
     const int cpr = rv / 8;
     for (int row = wid; row < n_grp * dh; row += kArWarps)
       if (lane < cpr) cp_async16(bvs + (size_t)row * pv + lane * 8, src + (int64_t)row * rv + lane * 8);
     cp_async_commit();
-  }
+  };
+  if (!pl.late_bv) copy_bv();
   {
     // Column n = 2h + term holds head h's latent query as two bf16 terms;
     // columns of heads >= H_q are zero.  float4 j holds k = 4j' .. 4j' + 3
@@ -481,6 +512,7 @@ attend_rows_kernel(Shape s, ArPlan pl, const int32_t *__restrict__ lengths, cons
     part[(size_t)tid * pr] = m_run[tid];
     part[(size_t)tid * pr + 1] = l_run[tid];
   }
+  if (pl.late_bv) copy_bv();   // the row buffers are spent; lands while the partials are exchanged
   // 2. Push the partial rows of the heads rank r finishes into rank r's
   // receive buffer (slot of this rank); the bulk copies read what the
   // threads just wrote.
