@@ -18,17 +18,19 @@
 //
 // Work.  The active tiles of every problem of the call (ceil(L_p / 128) each,
 // from the device-side lengths) form one list in problem order; CTA c of the
-// G-CTA cooperative grid takes tiles c, c + G, c + 2G, ...  Warp roles:
-//   warp 4  TMA producer: per 64-column k-block of a tile, one 16 KB TMA load
+// G-CTA cooperative grid takes chunks of K consecutive tiles, round robin.
+// Warp roles (E = R / 8 epilogue warps):
+//   warps 0 .. E-1  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31
+//           (one position per thread) and scoring rows 32 (w / 4) .. + 31;
+//   warp E  TMA producer: per 64-column k-block of a tile, one 16 KB TMA load
 //           into a ring of stages; per problem switch, the split C_Q operand
 //           (one bulk copy per k-block) into one of one or two buffers;
-//   warp 5  MMA issuer (tcgen05.mma kind::f16, M = 128);
-//   warp 6  counter watcher (arrivals and completions of the problems);
-//   warps 0-3  epilogue, one TMEM lane (position) per thread.
+//   warp E+1  MMA issuer (tcgen05.mma kind::f16, M = 128);
+//   warp E+2  counter watcher (arrivals and completions of the problems).
 // Pass 1, per tile: y, e, the tile's per-row sums (a shuffle transpose-
-// reduction, then four warps in a fixed order) added in fp64 to the CTA's sums
-// of the problem.  After its last tile of problem p the CTA's counter watcher
-// (warp 6) adds those sums to the problem's row normalisers (fp64 atomics, 16
+// reduction, then the epilogue warps in a fixed order) added in fp64 to the
+// CTA's sums of the problem.  After its last tile of problem p the CTA's
+// counter watcher adds those sums to the problem's row normalisers (fp64 atomics, 16
 // slots per row), arrives on p's counter and, once every CTA that owns tiles
 // of p has arrived, forms 1 / l_row for the epilogue.  The e of a CTA's first kRetained tiles of p stay in their
 // TMEM slot; once all min(T_p, G) CTAs that own tiles of p have arrived, the

@@ -12,7 +12,9 @@ reach, through the C ABI against the fp64 oracle:
     S4R_ERR_TIMEOUT, and the next call on the same workspace matches the
     oracle again;
   * average pooling of the candidate scores ("free parameters": kernel 7),
-    with exact ties that pooling creates.
+    with exact ties that pooling creates;
+  * a cache with more candidates than the 8-CTA cluster select holds, which
+    the single-CTA select takes (Eqs. 13-15).
 
 Comparators are those of every decode parity test (tests/problems.py).
 """
@@ -151,6 +153,17 @@ def test_bounded_wait_runs_out_and_the_next_call_recovers(lengths):
     assert s4r.s4r_read_device_status(ws) == s4r.S4R_ERR_TIMEOUT
     s4r.s4r_clear_device_status(ws)
     res = run_gpu(batch, workspace=ws)
+    assert res["status"] == 0
+    check_batch(batch, res)
+
+
+def test_cache_beyond_the_cluster_top_k():
+    """More candidates than the 8-CTA cluster select holds (8 x 16384 keys):
+    the single-CTA radix select over keys in global memory takes the top-k
+    (small-model shape with fp32 storage, so the inputs stay light)."""
+    W0 = synth.WORKLOADS[0]
+    batch = make_batch(W0, lengths=[140000], top_k=1024, local_window=64, tag="beyond-cluster")
+    res = run_gpu(batch)
     assert res["status"] == 0
     check_batch(batch, res)
 

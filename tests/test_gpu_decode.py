@@ -177,7 +177,8 @@ def test_ragged_append_then_decode_steps():
 
 
 def test_many_small_problems_single_cta_clusters():
-    # G = 1 (as many query heads as kv heads) and 40 problems: the attention
-    # launch shrinks its clusters to a single CTA per (kv group, problem).
+    # G = 1 (as many query heads as kv heads) and 40 problems: one head per
+    # CTA of each problem's attention cluster, and more clusters than fit on
+    # the device at once.
     w = synth.Workload(**{**W1.__dict__, "n_heads_q": 8})
     _run(make_batch(w, lengths=[600 + 37 * i for i in range(40)], top_k=64, local_window=32, tag="g1"))
