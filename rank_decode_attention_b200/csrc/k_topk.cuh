@@ -516,6 +516,16 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
   const int chunk = (nc + kTopkCl - 1) / kTopkCl;
   const int i_begin = min(nc, (int)rank * chunk), i_end = min(nc, i_begin + chunk);
   const int my_n = i_end - i_begin;
+  // Level 0 from the scoring kernel's histogram: 16-byte loads issued before
+  // the keys', stored after them, so the two reads overlap.
+  constexpr int kHistV = kTopkLvlBins / 4 / kTopkClThreads;   // 16-byte words per thread
+  static_assert(kTopkLvlBins % (4 * kTopkClThreads) == 0, "histogram words per thread");
+  uint4 hv[kHistV];
+  if (ehist != nullptr) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(ehist + (int64_t)b * kExpBins);
+#pragma unroll
+    for (int u = 0; u < kHistV; ++u) hv[u] = __ldcg(src + u * kTopkClThreads + threadIdx.x);
+  }
   // Stage the share with 16-byte loads, all in flight at once.  The share
   // starts at key i_begin of a row that starts at b * cache_rows floats, so
   // it need not be 16-byte aligned: the head up to the first aligned key and
@@ -547,9 +557,10 @@ topk_cluster_kernel(Shape s, const int32_t *__restrict__ lengths, const float *_
     }
     for (int i = head + 4 * n4 + (int)threadIdx.x; i < my_n; i += blockDim.x) keys_s[kpad(i)] = __ldcg(src + i);
   }
-  // Level 0 from the scoring kernel's histogram, read while the keys stage.
-  if (ehist != nullptr)
-    for (int i = threadIdx.x; i < kTopkLvlBins; i += blockDim.x) sh.hist[i] = __ldcg(ehist + (int64_t)b * kExpBins + i);
+  if (ehist != nullptr) {
+#pragma unroll
+    for (int u = 0; u < kHistV; ++u) reinterpret_cast<uint4 *>(sh.hist)[u * kTopkClThreads + threadIdx.x] = hv[u];
+  }
   __syncthreads();
 
   // Per-thread contiguous chunk of the rank's keys (the compactions walk it).
