@@ -58,7 +58,7 @@ import synth  # noqa: E402
 
 METRIC = "compressed-KV decode steps/s and achieved HBM GB/s (% of roofline) at L=32K"
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
-EXTRA_DEFAULT = "0,2,3,4,1b,3b"
+EXTRA_DEFAULT = "0,2,3,4,1b,3b,1h"
 MAX_WINDOWS = 32          # distinct query windows per workload (steps cycle through them)
 
 
@@ -265,7 +265,7 @@ class GpuWorkload:
                                local_window=self.w.local_window, top_k=self.w.top_k,
                                out=self.out[sl], idx=self.idx[sl], workspace=getattr(self, "ws", None),
                                workspace_bytes=getattr(self, "ws_bytes", None),
-                               pool_kernel=self.w.pool_kernel, profile_events=events)
+                               pool_kernel=self.w.pool_kernel, row_mode=self.w.row_mode, profile_events=events)
 
     def append(self, layer, window):
         import rank_decode_attention_b200 as s4r
@@ -299,7 +299,7 @@ def algorithmic_bytes(w: synth.Workload, Lc: list):
     C_V rows) + 2*D'*r*e (bases) + 2*s*D'*e (sinks) + W*H_q*d_h*e (queries).
     Scoring kernel per problem: L_c*r*e + R*r*4 (C_Q) + L_c*4 (scores out)."""
     e = 2 if w.dtype == "bf16" else 4
-    R = w.query_window * (w.n_heads_q // w.n_heads_kv)
+    R = w.query_window * (w.n_heads_q if w.row_mode else w.n_heads_q // w.n_heads_kv)
     step = score = 0
     for L in Lc:
         nsel = min(w.top_k, max(0, L - w.local_window)) + min(w.local_window, L)
@@ -456,7 +456,7 @@ def oracle_problem(w: synth.Workload, seq: int = 0, tag="cpu-sample"):
                           basis_k=pin.basis_k.double().numpy(), basis_v=pin.basis_v.double().numpy(),
                           sink_k=pin.states_k[:s].double().numpy(), sink_v=pin.states_v[:s].double().numpy(),
                           n_heads_kv=w.n_heads_kv, local_window=w.local_window, top_k=w.top_k,
-                          pool_kernel=w.pool_kernel)
+                          pool_kernel=w.pool_kernel, row_mode=w.row_mode)
 
 
 def time_oracle(w, budget_s=15.0, max_calls=50, min_calls=1, threads=None):
@@ -596,14 +596,18 @@ def run_basis_bench(w, device, reps=3):
 def run_extra(key, args, device):
     """One entry of `workloads`: a configuration other than the headline."""
     batched = key.endswith("b")
-    w = synth.WORKLOADS[int(key.rstrip("b"))]
+    per_head = key.endswith("h")
+    w = synth.WORKLOADS[int(key.rstrip("bh"))]
+    if per_head:
+        # the per-head reading of the scoring rows (W * H_q of them)
+        w = dataclasses.replace(w, row_mode=1)
     steps = min(args.steps, w.steps) if w.append else args.steps
     n_win = max(1, min(steps, w.steps, MAX_WINDOWS))
     append_rows = (args.warmup + 3 * steps + 8) if w.append else 0
     wl = GpuWorkload(w, 0, device, n_win, append_rows=append_rows)
     res = time_decode(wl, steps, args.warmup, batched, None, device, 1)
     hbm, _, src = peaks()
-    label = w.name + ("/layers-in-one-call" if batched else "")
+    label = w.name + ("/layers-in-one-call" if batched else "") + ("/per-head-rows" if per_head else "")
     step_bytes, roof = roofline_entry(w, wl, batched, res, steps, hbm, src, label)
     calls = (f"all {w.layers * w.batch} (layer, sequence) problems in ONE call per step (layers batched, "
              "not a model's sequential order), CUDA graph per step") if batched else \
@@ -709,7 +713,7 @@ def main():
     ap.add_argument("--impl", default="s4r", choices=["s4r", "reference"])
     ap.add_argument("--workload", type=int, default=1)
     ap.add_argument("--extra", default=EXTRA_DEFAULT,
-                    help="comma list of other workloads to time on one GPU (0,2,3,4,1b,3b) or 'none'")
+                    help="comma list of other workloads to time on one GPU (0,2,3,4,1b,3b,1h) or 'none'")
     ap.add_argument("--no-encode", action="store_true")
     ap.add_argument("--no-basis", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

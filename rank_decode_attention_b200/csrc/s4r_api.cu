@@ -23,6 +23,7 @@
 #include "k_project.cuh"
 #include "k_score_simt.cuh"
 #include "k_score_pair.cuh"
+#include "k_score_rows.cuh"
 #include "k_score_tc.cuh"
 #include "k_topk.cuh"
 
@@ -238,6 +239,7 @@ s4r_status encode_tc_launch(int n_prob, const void *const *states, int64_t n, in
 struct ScorePlan {
   bool tc = false;   // tensor-core kernel (else fp64 CUDA-core passes)
   bool pair = false; // the fused two-tiles-per-CTA kernel (one problem, one resident wave)
+  bool rows = false; // the two-pass kernel for R > 64 rows (per-head rows)
   int R = 0;         // rows per problem (template argument of the TC kernel)
   int grid = 0;      // persistent cooperative grid
   int K = 1;         // consecutive tiles per chunk of the round-robin
@@ -277,6 +279,21 @@ bool tc_launchable(size_t smem) {
         break;
       }
   }
+  return ok;
+}
+
+// Whether a pass of the many-rows kernel can be resident (one CTA per SM).
+template <int PASS>
+bool rows_launchable(size_t smem) {
+  if (ensure_smem<score_rows_kernel<PASS>>(smem) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  int per_sm = 0;
+  const bool ok =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_rows_kernel<PASS>, kSrThreads, smem) == cudaSuccess &&
+      per_sm > 0;
+  if (!ok) cudaGetLastError();
   return ok;
 }
 
@@ -379,6 +396,18 @@ ArPlan plan_attend_rows(const Shape &s, const void *ck, const void *cv, const vo
 ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   ScorePlan p;
   if (dt != S4R_BF16 || s.cache_rows == 0 || s.batch == 0) return p;
+  if (s.n_rows > 64 && s.n_rows % kSrRc == 0 && s.n_rows <= S4R_MAX_SCORE_ROWS &&
+      (int64_t)s.batch * s.cache_rows < INT32_MAX) {
+    // many rows (per-head): chunks of 64 rows, two passes over the cache
+    const size_t smem = (size_t)sr_smem_bytes(s.rank_k, sr_buffers(s.rank_k));
+    if (rows_launchable<1>(smem) && rows_launchable<2>(smem)) {
+      p.tc = true;
+      p.rows = true;
+      p.R = s.n_rows;
+      p.smem = smem;
+      return p;
+    }
+  }
   if (s.n_rows != 32 && s.n_rows != 64) return p;
   if ((int64_t)s.batch * s.cache_rows >= INT32_MAX) return p;
   const int R = s.n_rows;
@@ -532,6 +561,34 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
       return S4R_ERR_CUDA;
     }
     // The fused kernel's grid barrier counts on the problem's counter word.
+    if (plan.rows) {
+      // pass 1 (row sums), 1 / l, pass 2 (scores); the SIMT path's row
+      // statistics region holds 1 / l
+      double *inv_l = rstat;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)ceil_div(s.cache_rows, kStcTile), (unsigned)s.batch);
+      cfg.blockDim = dim3(kSrThreads);
+      cfg.dynamicSmemBytes = plan.smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1] = {pdl_attr()};
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cudaError_t err = cudaLaunchKernelEx(&cfg, score_rows_kernel<1>, tmap, s, a->lengths, cqs, rowsum, inv_l, scores,
+                                           ehist, status);
+      if (err != cudaSuccess) return fail("score_rows_kernel (pass 1)", err);
+      cudaLaunchConfig_t fcfg = {};
+      fcfg.gridDim = dim3((unsigned)s.batch);
+      fcfg.blockDim = dim3(256);
+      fcfg.stream = st;
+      fcfg.attrs = attr;
+      fcfg.numAttrs = 1;
+      err = cudaLaunchKernelEx(&fcfg, score_rows_finish, s, (const double *)rowsum, inv_l);
+      if (err != cudaSuccess) return fail("score_rows_finish", err);
+      err = cudaLaunchKernelEx(&cfg, score_rows_kernel<2>, tmap, s, a->lengths, cqs, rowsum, (const double *)inv_l,
+                               scores, ehist, status);
+      if (err != cudaSuccess) return fail("score_rows_kernel (pass 2)", err);
+      if (check_launch("score_rows_kernel") != S4R_OK) return S4R_ERR_CUDA;
+    } else {
     const s4r_status rc =
         plan.pair ? (plan.R == 64 ? launch_score_pair<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters,
                                                           status, st)
@@ -540,6 +597,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
         : plan.R == 64 ? launch_score_tc<64>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st)
                        : launch_score_tc<32>(plan, tmap, s, a->lengths, cqs, scores, rowsum, ehist, counters, status, st);
     if (rc != S4R_OK) return rc;
+    }
   } else if (n_tiles > 0) {
     const size_t smem = ScoreSmem::bytes(s.rank_k);
     ensure_smem<score_stats_simt<T>>(smem);
@@ -745,7 +803,8 @@ int32_t s4r_decode_kernel_launches(const s4r_decode_args *args) {
   if (s.batch == 0) return 0;
   int32_t n = 1;                                  // projection
   const ScorePlan plan = plan_scoring(s, args->dtype);
-  if (plan.tc) n += 1;                            // scoring: one persistent tensor-core launch
+  if (plan.rows) n += 3;                          // scoring: pass 1, 1 / l, pass 2
+  else if (plan.tc) n += 1;                       // scoring: one tensor-core launch
   else if (s.cache_rows > 0) n += 3;              // scoring: stats, merge, final
   if (s.pool_kernel > 1 && s.cache_rows > 0) n += 1;
   if (s.top_k > 0) n += 1;

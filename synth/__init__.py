@@ -57,6 +57,7 @@ class Workload:
     ragged: tuple = ()      # (lo, hi) for U[lo, hi] lengths; empty = fixed
     append: bool = False    # each step first appends one encoded token
     pool_kernel: int = 1
+    row_mode: int = 0       # scoring rows: 0 CONCAT (W * G), 1 per head (W * H_q)
 
     @property
     def d_model(self) -> int:

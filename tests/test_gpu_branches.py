@@ -45,12 +45,23 @@ def concat_rows(batch, b):
     return qc.reshape(W * G, Hkv * dh) @ batch.basis_k[b].double().numpy()
 
 
+def per_head_rows(batch, b):
+    """C_Q of problem b (PER_HEAD rows, row w * H_q + h): q[w][h] . B^K[g d_h ..
+    (g + 1) d_h], g = h / G; fp64 [W H_q][r]."""
+    q = batch.q[b].double().numpy()                       # [W][H_q][d_h]
+    W, Hq, dh = q.shape
+    G = Hq // batch.n_heads_kv
+    bk = batch.basis_k[b].double().numpy()
+    return np.stack([q[w, h] @ bk[(h // G) * dh:(h // G + 1) * dh] for w in range(W) for h in range(Hq)])
+
+
 def base2_logits(batch, b):
     """y[row][i] = (C_Q[row] . C_K[i]) / sqrt(r) * log2(e), to check which
     branch a case reaches."""
     L = batch.lengths[b]
     ck = batch.coeff_k[b, :L].double().numpy()
-    return (concat_rows(batch, b) @ ck.T) / np.sqrt(ck.shape[1]) * np.log2(np.e)
+    cq = per_head_rows(batch, b) if batch.row_mode == 1 else concat_rows(batch, b)
+    return (cq @ ck.T) / np.sqrt(ck.shape[1]) * np.log2(np.e)
 
 
 def tile_ranges(y):
@@ -87,6 +98,19 @@ def test_wide_range_every_tile():
     ranges = tile_ranges(y)
     assert ranges.min() > RANGE_LIMIT, ranges.min()
     assert y.max(axis=1).max() > 128.0
+    _run(batch, ranges.max())
+
+
+def test_wide_range_every_tile_per_head_rows():
+    # The per-head reading (W * H_q = 512 rows) takes the many-rows scoring
+    # kernel (chunks of 64 rows, two passes); the same scaling drives every
+    # tile past the limit, so both passes take the per-row offsets.
+    batch = make_batch(W1, lengths=[3001], top_k=16, local_window=32, row_mode=1, tag="wide-heads")
+    y0 = tile_ranges(base2_logits(batch, 0)).min()
+    scale = 2.0 ** np.ceil(np.log2(110.0 / y0))
+    batch = dataclasses.replace(batch, q=(batch.q.double() * scale).to(batch.q.dtype))
+    ranges = tile_ranges(base2_logits(batch, 0))
+    assert ranges.min() > RANGE_LIMIT, ranges.min()
     _run(batch, ranges.max())
 
 
