@@ -18,19 +18,20 @@
 // All arithmetic is fp64.  The SVD goes through the smaller Gram matrix of
 // the sample, m = min(T', D') rounded up to even: A A^T (T' x T', then
 // B = A^T U Sigma^-1) when T' <= D', else A^T A (D' x D', B = its
-// eigenvectors).  Its eigenvectors come from a two-sided cyclic Jacobi
-// method in parallel rounds: the m/2 disjoint pairs of a round (round-robin
-// order, every pair once per sweep) rotate together, so M' = J^T M J splits
-// into independent 2x2 blocks R_a^T M[a][b] R_b.  The matrix is stored in
-// the round's slot order (pair a in slots 2a, 2a+1), so a block is two
-// 16-byte loads; each round writes its result into the other buffer already
-// in the next round's slot order, and keeps only the upper blocks' work
-// (the lower ones are their transposes).  The eigenvectors are kept as the
-// rows of V^T in the same slot order, so their rotation is a pair of
-// contiguous rows.  The rounds of all problems are separated by a grid-wide
-// barrier of one cooperative launch.  The sweep in which every pair meets
-// an off-diagonal entry below 1e-8 of its diagonal scale is the last one:
-// its rotations leave them near their squares.
+// eigenvectors).  Its eigenvectors come from a two-sided block Jacobi
+// method.  The Gram matrix is padded with zeros to mp = m rounded up to 32
+// and its indices are cut into nb = mp / 16 blocks of 16; in each round the
+// blocks meet in disjoint pairs (round-robin order, every pair of blocks
+// once in nb - 1 rounds).  A round first applies, for every pair, one
+// cyclic Jacobi sweep to the 32 x 32 principal submatrix on its indices in
+// shared memory (Rutishauser's rotations, parallel order over its 16 index
+// pairs), keeping the product Q of its rotations; then every off-diagonal
+// 32 x 32 tile becomes Q_a^T M[a][c] Q_c and the eigenvector rows of the
+// pair become Q_a^T V^T[a].  Matrix and eigenvectors stay in natural index
+// order and are updated in place.  Rounds are separated by a grid-wide
+// barrier of one cooperative launch.  The outer sweep in which no rotation
+// meets an off-diagonal entry above 1e-8 of its diagonal scale is the last
+// one: its rotations leave them near their squares.
 // Near the rank cut the eigenvalues of the workloads' samples differ by
 // 1e-5 .. 1e-3 of the largest, so single precision would mix kept and
 // dropped directions; fp64 keeps them apart to ~1e-10.
@@ -46,6 +47,11 @@ constexpr double kJacobiTol = 1e-12;   // rotate while |a_pq| > tol * sqrt(a_pp 
 // A sweep in which no pair starts above this relative size leaves every
 // off-diagonal entry near its square (quadratic convergence): the last sweep.
 constexpr double kJacobiLastSweep = 1e-8;
+// Block Jacobi geometry: blocks of 16 indices; a pair of blocks (32 indices)
+// is the submatrix one work item rotates in shared memory.
+constexpr int kBjBlock = 16;
+constexpr int kBjPair = 2 * kBjBlock;
+constexpr int kBjMaxRounds = kBasisMaxSweeps * (S4R_MAX_D_MODEL / kBjBlock - 1) + 1;
 
 struct BasisShape {
   int32_t P;         // problems
@@ -54,6 +60,7 @@ struct BasisShape {
   int32_t s;         // sinks
   int32_t T;         // requested sample rows T'
   int32_t m;         // Gram dimension (even)
+  int32_t mp;        // m rounded up to 32: stride of M and V^T, zero padded
   int32_t t_side;    // 1: Gram of the rows (A A^T), 0: Gram of the columns (A^T A)
   int64_t state_rows;
 };
@@ -62,9 +69,9 @@ struct BasisShape {
 struct BasisCtl {
   uint32_t status;
   uint32_t bar;                   // grid barrier arrivals (monotone)
-  uint32_t final_buf;             // buffer of M and V^T holding the converged result
-  uint32_t pad;
+  uint32_t pad[2];
   uint32_t rot[kBasisMaxSweeps];  // CTAs that met a pair above kJacobiLastSweep in sweep i
+  uint32_t vq[kBjMaxRounds];      // work tickets of the eigenvector rows of round g
 };
 
 // Row of sample j (< n) of a problem with L rows ("Core claim", 7:3 split).
@@ -81,19 +88,11 @@ __host__ __device__ __forceinline__ int64_t basis_sample_row(int64_t L, int64_t 
 // Round-robin schedule (circle method): player m-1 is fixed, the others sit
 // on a circle of n1 = m-1 places; in round k (< n1) pair 0 is (m-1, k) and
 // pair a >= 1 is ((k+a) mod n1, (k-a) mod n1).  Every pair meets once in n1
-// rounds.  Pair a occupies slots 2a (first) and 2a+1 (second).
+// rounds.  Pair a is the players of slots 2a and 2a+1.
 __host__ __device__ __forceinline__ int jac_player(int m, int k, int u) {
   const int n1 = m - 1, a = u >> 1;
   if ((u & 1) == 0) return a == 0 ? m - 1 : (k + a) % n1;
   return a == 0 ? k % n1 : (k - a + n1) % n1;
-}
-__host__ __device__ __forceinline__ int jac_slot(int m, int k, int x) {
-  const int n1 = m - 1, h = m / 2;
-  if (x == m - 1) return 0;
-  const int d = ((x - k) % n1 + n1) % n1;
-  if (d == 0) return 1;
-  if (d <= h - 1) return 2 * d;
-  return 2 * (n1 - d) + 1;
 }
 
 __device__ __forceinline__ int64_t basis_n(const BasisShape &bs, const int32_t *lengths, int p) {
@@ -113,10 +112,8 @@ __global__ void __launch_bounds__(256) basis_prep_kernel(BasisShape bs, const in
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (p == 0 && blockIdx.x == 0) {
     for (int i = threadIdx.x; i < kBasisMaxSweeps; i += blockDim.x) ctl->rot[i] = 0u;
-    if (threadIdx.x == 0) {
-      ctl->bar = 0u;
-      ctl->final_buf = 0u;
-    }
+    for (int i = threadIdx.x; i < kBjMaxRounds; i += blockDim.x) ctl->vq[i] = 0u;
+    if (threadIdx.x == 0) ctl->bar = 0u;
   }
   const int64_t Lraw = lengths[p];
   const int64_t n = basis_n(bs, lengths, p);
@@ -151,7 +148,7 @@ __device__ __forceinline__ double basis_a(const BasisShape &bs, const T *states,
   return (double)to_f(states[((int64_t)p * bs.state_rows + row) * bs.D + d]) * inv_p[j];
 }
 
-// 2. Gram matrix M (buffer 0, slot order of round 0) and V^T = I.  32 x 32 output tile per CTA, four
+// 2. Gram matrix M (mp x mp, zero padded) and V^T = I.  32 x 32 output tile per CTA, four
 // outputs per thread, inner dimension in chunks of 32 staged in shared
 // memory.  Gram of the rows: M[i][j] = sum_d a[i][d] a[j][d]; of the
 // columns: M[i][j] = sum_t a[t][i] a[t][j].
@@ -164,7 +161,6 @@ __global__ void __launch_bounds__(256) basis_gram_kernel(BasisShape bs, const T 
   const int p = blockIdx.z;
   const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // ty < 8
-  const int m = bs.m;
   const int64_t *rows_p = rows + (int64_t)p * bs.T;
   const double *inv_p = inv + (int64_t)p * bs.T;
   const int K = bs.t_side ? bs.D : bs.T;
@@ -190,17 +186,14 @@ __global__ void __launch_bounds__(256) basis_gram_kernel(BasisShape bs, const T 
     }
     __syncthreads();
   }
-  // Round 0's slot order; row slot(i) of V^T starts as e_i.
-  double *Mp = M + (int64_t)p * 2 * m * m;
-  double *Vp = V + (int64_t)p * 2 * m * m;
-  const int sj = (j0 + tx < m) ? jac_slot(m, 0, j0 + tx) : 0;
+  double *Mp = M + (int64_t)p * bs.mp * bs.mp;
+  double *Vp = V + (int64_t)p * bs.mp * bs.mp;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int i = i0 + ty + 8 * u, j = j0 + tx;
-    if (i < m && j < m) {
-      const int si = jac_slot(m, 0, i);
-      Mp[(int64_t)si * m + sj] = acc[u];
-      Vp[(int64_t)si * m + j] = (i == j) ? 1.0 : 0.0;
+    if (i < bs.mp && j < bs.mp) {
+      Mp[(int64_t)i * bs.mp + j] = acc[u];
+      Vp[(int64_t)i * bs.mp + j] = (i == j) ? 1.0 : 0.0;
     }
   }
 }
@@ -233,146 +226,318 @@ __device__ __forceinline__ bool basis_grid_sync(BasisCtl *ctl, uint32_t gen, int
   return *flag_smem != 0;
 }
 
-// Rotation of pair (p, q) that zeroes M[p][q] (Rutishauser's form): returns
-// t (0 = no rotation), c, s with J[p][p] = J[q][q] = c, J[p][q] = s,
-// J[q][p] = -s.
-__device__ __forceinline__ double jacobi_angle(const double *Mc, int m, int p, int q, double &c, double &s,
-                                               double &app, double &aqq, double &apq) {
-  app = Mc[(int64_t)p * m + p];
-  aqq = Mc[(int64_t)q * m + q];
-  apq = Mc[(int64_t)p * m + q];
+// Rotation of pair (p, q) that zeroes S[p][q] (Rutishauser's form), S a
+// symmetric matrix with row stride ld: returns t (0 = no rotation), c, s
+// with J[p][p] = J[q][q] = c, J[p][q] = s, J[q][p] = -s; big tells whether
+// |S[p][q]| is above kJacobiLastSweep of sqrt|S[p][p] S[q][q]|.  The tests
+// compare squares, so only the angle itself takes a root:
+// t = sign(theta) / (|theta| + sqrt(1 + theta^2)), theta = (a_qq - a_pp) / (2 a_pq),
+// with t = 1 / (2 theta) once theta^2 would overflow.
+__device__ __forceinline__ double jacobi_angle(const double *S, int ld, int p, int q, double &c, double &s,
+                                               bool &big) {
+  const double app = S[p * ld + p], aqq = S[q * ld + q], apq = S[p * ld + q];
   c = 1.0;
   s = 0.0;
-  const double aabs = fabs(apq);
-  if (!(aabs > 1e-300) || aabs <= kJacobiTol * sqrt(fabs(app) * fabs(aqq))) return 0.0;
+  const double a2 = apq * apq, d2 = fabs(app * aqq);
+  big = a2 > (kJacobiLastSweep * kJacobiLastSweep) * d2;
+  if (!(fabs(apq) > 1e-300) || a2 <= (kJacobiTol * kJacobiTol) * d2) {
+    big = false;
+    return 0.0;
+  }
   const double theta = (aqq - app) / (2.0 * apq);
-  const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + hypot(1.0, theta));
-  c = 1.0 / sqrt(1.0 + t * t);
+  const double at = fabs(theta);
+  double t = at < 1e150 ? 1.0 / (at + sqrt(fma(at, at, 1.0))) : 0.5 / at;
+  t = theta >= 0.0 ? t : -t;
+  c = rsqrt(fma(t, t, 1.0));
   s = t * c;
   return t;
 }
 
-// Upper-triangle block t (< h(h+1)/2, row-major over a <= b) -> (a, b): a
-// single-precision root (exact operands below 2^24), then integer steps.
-__device__ __forceinline__ void upper_block(int h, int t, int &a, int &b) {
-  const float w = 2.0f * (float)h + 1.0f;
-  int x = (int)floorf((w - sqrtf(w * w - 8.0f * (float)t)) * 0.5f);
-  x = x < 0 ? 0 : (x >= h ? h - 1 : x);
-  auto start = [h](int r) { return r * h - r * (r - 1) / 2; };
-  while (x > 0 && start(x) > t) --x;
-  while (x + 1 < h && start(x + 1) <= t) ++x;
-  a = x;
-  b = x + (t - start(x));
+// Shared tiles are 32 x 32 doubles with a row stride of 36: the fragment
+// loads of the tensor-core products below (lanes g = lane / 4 and
+// q = lane % 4 reading [8 r + g][k + q] or [k + q][8 c + g]) then fall on
+// distinct banks, and rows start on 16-byte boundaries.
+constexpr int kBjLd = 36;
+constexpr int kBjThreads = 256;
+// Inner rounds over the 16 index pairs of a submatrix (blocks I and J):
+// 15 rounds inside the blocks (a round-robin of 16 on each), then 16
+// rounds across them (i with 16 + (i + r) mod 16).  The rounds inside the
+// blocks run in the first round of each outer sweep only, so every index
+// pair still meets once per sweep; the other rounds of the sweep run the
+// 16 across.
+constexpr int kBjInner = 2 * kBjBlock - 1;
+constexpr int kBjCross0 = kBjBlock - 1;
+
+// Global index of local index l (< 32) of block pair a in round k with nb
+// blocks: l < 16 in the block of slot 2a, the others in that of slot 2a+1.
+__device__ __forceinline__ int bj_index(int nb, int k, int a, int l) {
+  return jac_player(nb, k, 2 * a + (l >> 4)) * kBjBlock + (l & (kBjBlock - 1));
 }
 
-// 3. Jacobi sweeps for every problem (cooperative launch).  M and V^T are
-// [P][2][m][m]; round g reads buffer g & 1 and writes the other one.  CTA c
-// owns the items [c N / G, (c+1) N / G) of the N = P (h(h+1)/2 + h m) items
-// of a round (upper blocks of M, then the rotated row pairs of V^T, problem
-// by problem), so it meets one or two problems per round and computes their
-// h rotations once, into shared memory.
-__global__ void __launch_bounds__(256) basis_jacobi_kernel(BasisShape bs, double *__restrict__ M,
-                                                           double *__restrict__ V, BasisCtl *ctl) {
-  __shared__ int flag_s, rot_s;
-  __shared__ int ns_s[S4R_MAX_D_MODEL];            // next-round slot of the player in slot u
-  __shared__ double c_s[S4R_MAX_D_MODEL / 2], s_s[S4R_MAX_D_MODEL / 2], t_s[S4R_MAX_D_MODEL / 2];
-  const int m = bs.m, h = m / 2, n1 = m - 1;
-  const int64_t mm = (int64_t)m * m;
-  const int64_t nMp = (int64_t)h * (h + 1) / 2, nUp = nMp + (int64_t)h * m;   // items per problem
-  const int64_t N = (int64_t)bs.P * nUp;
-  const int64_t i_begin = N * blockIdx.x / gridDim.x, i_end = N * (blockIdx.x + 1) / gridDim.x;
-  if (threadIdx.x == 0) rot_s = 0;
-  uint32_t gen = 0, round = 0;
+// One m8n8k4 fp64 tensor-core product, {d0, d1} += a b, in the PTX
+// fragment layout of that shape: lane (g, q) = (lane / 4, lane % 4) holds
+// a = A[g][q], b = B[q][g] and d = D[g][2q], D[g][2q + 1].
+__device__ __forceinline__ void bj_dmma(double &d0, double &d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
+// Warp product of a strip of C = op(A) B (32 x 32 shared tiles, op(A) =
+// A^T when TA): rows 8 rt .. 8 rt + 7, columns c0 .. c0 + 8 NT - 1, into
+// acc[t] = C[8 rt + g][c0 + 8 t + 2 q + {0, 1}].
+template <bool TA, int NT>
+__device__ __forceinline__ void bj_strip(const double (*A)[kBjLd], const double (*B)[kBjLd], int rt, int c0,
+                                         double (&acc)[NT][2]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = 0.0;
+#pragma unroll
+  for (int k0 = 0; k0 < kBjPair; k0 += 4) {
+    const double a = TA ? A[k0 + q][8 * rt + g] : A[8 * rt + g][k0 + q];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) bj_dmma(acc[t][0], acc[t][1], a, B[k0 + q][c0 + 8 * t + g]);
+  }
+}
+
+__device__ __forceinline__ void bj_copy2(double *dst, const double *src) {
+  *reinterpret_cast<double2 *>(dst) = *reinterpret_cast<const double2 *>(src);
+}
+
+// Eigenvector rows of round gv (round kv of its sweep), taken from a ticket
+// counter until none is left: item (problem, pair a, 64-column strip) sets
+// V^T[a][strip] = Q_a^T V^T[a][strip].  Warps 0-3 form the first 32
+// columns, warps 4-7 the second.
+__device__ __forceinline__ void bj_rows_items(const BasisShape &bs, double *V, const double *Qbuf, BasisCtl *ctl,
+                                              int gv, int kv, double (*t0)[kBjLd], double (*t1)[kBjLd],
+                                              double (*t2)[kBjLd], int (*idx_s)[kBjPair], uint32_t *tk_s) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+  const int mp = bs.mp, nb = mp / kBjBlock, npb = nb / 2, ns = (mp / kBjPair + 1) / 2;
+  const uint32_t nV = (uint32_t)(bs.P * npb * ns);
+  for (;;) {
+    if (tid == 0) *tk_s = atomicAdd(&ctl->vq[gv], 1u);
+    __syncthreads();
+    const uint32_t v = *tk_s;
+    if (v >= nV) break;
+    const int p = (int)(v / (uint32_t)(npb * ns)), rem = (int)(v - (uint32_t)p * (npb * ns));
+    const int a = rem / ns, col0 = (rem - a * ns) * 2 * kBjPair;
+    const bool two = col0 + kBjPair < mp;
+    double *Vp = V + (int64_t)p * mp * mp;
+    const double *Qa = Qbuf + ((int64_t)p * npb + a) * (kBjPair * kBjPair);
+    if (tid < kBjPair) idx_s[0][tid] = bj_index(nb, kv, a, tid);
+    __syncthreads();
+    for (int e = tid; e < kBjPair * kBjPair / 2; e += blockDim.x) {
+      const int i = e >> 4, j = (e & 15) * 2;
+      const double *row = Vp + (int64_t)idx_s[0][i] * mp + col0 + j;
+      bj_copy2(&t1[i][j], Qa + i * kBjPair + j);
+      bj_copy2(&t0[i][j], row);
+      if (two) bj_copy2(&t2[i][j], row + kBjPair);
+    }
+    __syncthreads();
+    if (warp < 4 || two) {
+      double acc[4][2];
+      bj_strip<true, 4>(t1, warp < 4 ? t0 : t2, warp & 3, 0, acc);
+      double *row = Vp + (int64_t)idx_s[0][8 * (warp & 3) + g] * mp + col0 + (warp >> 2) * kBjPair + 2 * q;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) *reinterpret_cast<double2 *>(row + 8 * t) = make_double2(acc[t][0], acc[t][1]);
+    }
+    __syncthreads();   // tiles, indices and the ticket are reused
+  }
+}
+
+// 3. Block Jacobi sweeps for every problem (cooperative launch).  M and V^T
+// are [P][mp][mp]; Qg holds two buffers [P][mp / 32][32][32] of the pair
+// rotations, round g writing buffer g & 1.  Round g (round k of its sweep):
+//   phase 1, items (problem, pair a): load S = M[a][a], rotate it by one
+//      sweep of inner rounds, accumulate Q_a = J_1 J_2 ..., write S back
+//      into M[a][a] and Q_a; a CTA done with its items then takes the
+//      eigenvector rows of round g - 1 from their ticket counter (they are
+//      needed by nothing before the end);
+//   grid barrier;
+//   phase 2, items (problem, tile a < c): M[a][c] = Q_a^T M[a][c] Q_c on
+//      the tensor cores, and its transpose into M[c][a];
+//   grid barrier.
+// The eigenvector rows of the last round follow the last sweep.  A 2 x 2
+// block of an inner round is only read and written by the thread that owns
+// it (the upper one, mirrored into the lower), so S stays exactly
+// symmetric and needs no second buffer.
+__global__ void __launch_bounds__(kBjThreads) basis_jacobi_kernel(BasisShape bs, double *__restrict__ M,
+                                                                  double *__restrict__ V, double *__restrict__ Qg,
+                                                                  BasisCtl *ctl) {
+  __shared__ __align__(16) double t0[kBjPair][kBjLd];
+  __shared__ __align__(16) double t1[kBjPair][kBjLd];
+  __shared__ __align__(16) double t2[kBjPair][kBjLd];
+  __shared__ __align__(16) double t3[kBjPair][kBjLd];
+  __shared__ double c_s[kBjBlock], s_s[kBjBlock], tt_s[kBjBlock];
+  __shared__ unsigned char sched_s[kBjInner][kBjPair];            // index pairs of each inner round
+  __shared__ unsigned char ut_s[kBjBlock * (kBjBlock + 1) / 2];   // upper (a, c) pairs of 2 x 2 blocks
+  __shared__ int idx_s[2][kBjPair];
+  __shared__ int flag_s;
+  __shared__ uint32_t tk_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, qq = lane & 3;
+  const int mp = bs.mp, nb = mp / kBjBlock, npb = nb / 2, rps = nb - 1;
+  const int64_t mm = (int64_t)mp * mp;
+  const int64_t qbuf = (int64_t)bs.P * npb * (kBjPair * kBjPair);
+  const int nA = bs.P * npb;
+  const int nMt = npb * (npb - 1) / 2, nM = bs.P * nMt;
+  for (int e = tid; e < kBjInner * kBjBlock; e += blockDim.x) {
+    const int kk = e / kBjBlock, u = e % kBjBlock;
+    int x, y;
+    if (kk < kBjCross0) {   // inside the blocks: pairs 0..7 in I, 8..15 in J
+      const int off = u < 8 ? 0 : kBjBlock, w = u & 7;
+      x = off + jac_player(kBjBlock, kk, 2 * w);
+      y = off + jac_player(kBjBlock, kk, 2 * w + 1);
+    } else {                // across: i with 16 + (i + r) mod 16
+      x = u;
+      y = kBjBlock + (u + kk - kBjCross0) % kBjBlock;
+    }
+    sched_s[kk][2 * u] = (unsigned char)x;
+    sched_s[kk][2 * u + 1] = (unsigned char)y;
+  }
+  if (tid < kBjBlock * (kBjBlock + 1) / 2) {
+    int t = tid, a = 0;
+    while (t >= kBjBlock - a) { t -= kBjBlock - a; ++a; }
+    ut_s[tid] = (unsigned char)((a << 4) | (a + t));
+  }
+  __syncthreads();
+  uint32_t gen = 0;
+  int g = 0;
   bool converged = false;
   for (int sweep = 0; sweep < kBasisMaxSweeps && !converged; ++sweep) {
-    for (int k = 0; k < n1; ++k, ++round) {
-      const int cur = (int)(round & 1u);
-      const int kn = (k + 1) % n1;
-      for (int u = threadIdx.x; u < m; u += blockDim.x) ns_s[u] = jac_slot(m, kn, jac_player(m, k, u));
-      for (int64_t p0 = i_begin / nUp; p0 * nUp < i_end; ++p0) {
-        const int p = (int)p0;
-        const double *Mc = M + ((int64_t)p * 2 + cur) * mm;
-        double *Mn = M + ((int64_t)p * 2 + (cur ^ 1)) * mm;
-        const double *Vc = V + ((int64_t)p * 2 + cur) * mm;
-        double *Vn = V + ((int64_t)p * 2 + (cur ^ 1)) * mm;
-        __syncthreads();   // ns_s written; the previous problem's rotations consumed
-        for (int a = threadIdx.x; a < h; a += blockDim.x) {
-          double c, sn, app, aqq, apq;
-          const double t = jacobi_angle(Mc, m, 2 * a, 2 * a + 1, c, sn, app, aqq, apq);
-          c_s[a] = c;
-          s_s[a] = sn;
-          t_s[a] = t;
-          if (t != 0.0 && fabs(apq) > kJacobiLastSweep * sqrt(fabs(app) * fabs(aqq))) rot_s = 1;
+    for (int k = 0; k < rps; ++k, ++g) {
+      double *Qcur = Qg + (g & 1) * qbuf;
+      // ---- phase 1: rotate the pairs' submatrices
+      const int kk0 = k == 0 ? 0 : kBjCross0;
+      for (int item = blockIdx.x; item < nA; item += gridDim.x) {
+        const int p = item / npb, a = item - p * npb;
+        double *Mp = M + (int64_t)p * mm;
+        if (tid < kBjPair) idx_s[0][tid] = bj_index(nb, k, a, tid);
+        __syncthreads();
+        for (int e = tid; e < kBjPair * kBjPair / 2; e += blockDim.x) {
+          const int i = e >> 4, j = (e & 15) * 2;
+          bj_copy2(&t0[i][j], Mp + (int64_t)idx_s[0][i] * mp + idx_s[0][j]);
+          t1[i][j] = (i == j) ? 1.0 : 0.0;
+          t1[i][j + 1] = (i == j + 1) ? 1.0 : 0.0;
         }
         __syncthreads();
-        // Item indices within one problem stay below 2^31 (32-bit arithmetic).
-        const int lo = (int)(i_begin > p0 * nUp ? i_begin - p0 * nUp : 0);
-        const int hi = (int)(i_end < (p0 + 1) * nUp ? i_end - p0 * nUp : nUp);
-        const int nM32 = (int)nMp;
-        for (int it = lo + (int)threadIdx.x; it < hi; it += blockDim.x) {
-          if (it < nM32) {
-            int a, b;
-            upper_block(h, it, a, b);
-            const int r0 = ns_s[2 * a], r1 = ns_s[2 * a + 1];
-            const double ca = c_s[a], sa = s_s[a], ta = t_s[a];
-            if (a == b) {
-              const double app = Mc[(int64_t)(2 * a) * m + 2 * a], aqq = Mc[(int64_t)(2 * a + 1) * m + 2 * a + 1];
-              const double apq = Mc[(int64_t)(2 * a) * m + 2 * a + 1];
-              double z00 = app, z01 = apq, z10 = Mc[(int64_t)(2 * a + 1) * m + 2 * a], z11 = aqq;
-              if (ta != 0.0) {
-                z00 = app - ta * apq;
-                z11 = aqq + ta * apq;
-                z01 = z10 = 0.0;
+        int big = 0;
+        for (int kk = kk0; kk < kBjInner; ++kk) {
+          if (tid < kBjBlock) {
+            double c, sn;
+            bool bg;
+            const double t = jacobi_angle(&t0[0][0], kBjLd, sched_s[kk][2 * tid], sched_s[kk][2 * tid + 1], c, sn,
+                                          bg);
+            c_s[tid] = c;
+            s_s[tid] = sn;
+            tt_s[tid] = t;
+            big |= bg ? 1 : 0;
+          }
+          __syncthreads();
+          if (tid < kBjBlock * (kBjBlock + 1) / 2) {
+            const int ab = ut_s[tid], ea = ab >> 4, ec = ab & 15;
+            const int pa = sched_s[kk][2 * ea], qa = sched_s[kk][2 * ea + 1];
+            if (ea == ec) {
+              const double t = tt_s[ea];
+              if (t != 0.0) {
+                const double apq = t0[pa][qa];
+                t0[pa][pa] -= t * apq;
+                t0[qa][qa] += t * apq;
+                t0[pa][qa] = 0.0;
+                t0[qa][pa] = 0.0;
               }
-              Mn[(int64_t)r0 * m + r0] = z00;
-              Mn[(int64_t)r0 * m + r1] = z01;
-              Mn[(int64_t)r1 * m + r0] = z10;
-              Mn[(int64_t)r1 * m + r1] = z11;
             } else {
-              const double cb = c_s[b], sb = s_s[b];
-              const double2 x0 = *reinterpret_cast<const double2 *>(Mc + (int64_t)(2 * a) * m + 2 * b);
-              const double2 x1 = *reinterpret_cast<const double2 *>(Mc + (int64_t)(2 * a + 1) * m + 2 * b);
-              // y = R_a^T x, then z = y R_b, R = [[c, s], [-s, c]].
-              const double y00 = ca * x0.x - sa * x1.x, y01 = ca * x0.y - sa * x1.y;
-              const double y10 = sa * x0.x + ca * x1.x, y11 = sa * x0.y + ca * x1.y;
+              const int pc = sched_s[kk][2 * ec], qc = sched_s[kk][2 * ec + 1];
+              const double ca = c_s[ea], sa = s_s[ea], cb = c_s[ec], sb = s_s[ec];
+              const double x00 = t0[pa][pc], x01 = t0[pa][qc], x10 = t0[qa][pc], x11 = t0[qa][qc];
+              // y = R_a^T x, then z = y R_c, R = [[c, s], [-s, c]].
+              const double y00 = ca * x00 - sa * x10, y01 = ca * x01 - sa * x11;
+              const double y10 = sa * x00 + ca * x10, y11 = sa * x01 + ca * x11;
               const double z00 = y00 * cb - y01 * sb, z01 = y00 * sb + y01 * cb;
               const double z10 = y10 * cb - y11 * sb, z11 = y10 * sb + y11 * cb;
-              const int c0 = ns_s[2 * b], c1 = ns_s[2 * b + 1];
-              Mn[(int64_t)r0 * m + c0] = z00;
-              Mn[(int64_t)r0 * m + c1] = z01;
-              Mn[(int64_t)r1 * m + c0] = z10;
-              Mn[(int64_t)r1 * m + c1] = z11;
-              Mn[(int64_t)c0 * m + r0] = z00;
-              Mn[(int64_t)c1 * m + r0] = z01;
-              Mn[(int64_t)c0 * m + r1] = z10;
-              Mn[(int64_t)c1 * m + r1] = z11;
+              t0[pa][pc] = z00;
+              t0[pa][qc] = z01;
+              t0[qa][pc] = z10;
+              t0[qa][qc] = z11;
+              t0[pc][pa] = z00;
+              t0[qc][pa] = z01;
+              t0[pc][qa] = z10;
+              t0[qc][qa] = z11;
             }
-          } else {
-            // V' = V J on the rows of V^T: rows 2a, 2a+1 (column i) into the
-            // rows of their next slots.
-            const int v = it - nM32;
-            const int a = v / m, i = v - a * m;
-            const double c = c_s[a], sn = s_s[a];
-            const bool rot = t_s[a] != 0.0;
-            const double v0 = Vc[(int64_t)(2 * a) * m + i], v1 = Vc[(int64_t)(2 * a + 1) * m + i];
-            Vn[(int64_t)ns_s[2 * a] * m + i] = rot ? c * v0 - sn * v1 : v0;
-            Vn[(int64_t)ns_s[2 * a + 1] * m + i] = rot ? sn * v0 + c * v1 : v1;
+          }
+          {
+            // Q = Q J on the columns of index pair e, rows i and i + 16.
+            const int e = tid & 15, i = tid >> 4;
+            if (tt_s[e] != 0.0) {
+              const int pe = sched_s[kk][2 * e], qe = sched_s[kk][2 * e + 1];
+              const double c = c_s[e], sn = s_s[e];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const double q0 = t1[i + 16 * h][pe], q1 = t1[i + 16 * h][qe];
+                t1[i + 16 * h][pe] = c * q0 - sn * q1;
+                t1[i + 16 * h][qe] = sn * q0 + c * q1;
+              }
+            }
+          }
+          __syncthreads();
+        }
+        double *Qp = Qcur + ((int64_t)p * npb + a) * (kBjPair * kBjPair);
+        for (int e = tid; e < kBjPair * kBjPair / 2; e += blockDim.x) {
+          const int i = e >> 4, j = (e & 15) * 2;
+          bj_copy2(Mp + (int64_t)idx_s[0][i] * mp + idx_s[0][j], &t0[i][j]);
+          bj_copy2(Qp + i * kBjPair + j, &t1[i][j]);
+        }
+        if (__syncthreads_or(big) && tid == 0) atomicAdd(&ctl->rot[sweep], 1u);   // also frees the tiles
+      }
+      if (g > 0) bj_rows_items(bs, V, Qg + ((g - 1) & 1) * qbuf, ctl, g - 1, (k + rps - 1) % rps, t0, t1, t2, idx_s,
+                               &tk_s);
+      if (!basis_grid_sync(ctl, ++gen, &flag_s)) return;
+      // ---- phase 2: rotate the off-diagonal tiles
+      for (int item = blockIdx.x; item < nM; item += gridDim.x) {
+        const int p = item / nMt;
+        int a = 0, r = item - p * nMt;
+        while (r >= npb - 1 - a) { r -= npb - 1 - a; ++a; }
+        const int c = a + 1 + r;
+        double *Mp = M + (int64_t)p * mm;
+        const double *Qp = Qcur + (int64_t)p * npb * (kBjPair * kBjPair);
+        if (tid < 2 * kBjPair) idx_s[tid >> 5][tid & 31] = bj_index(nb, k, (tid >> 5) ? c : a, tid & 31);
+        __syncthreads();
+        for (int e = tid; e < kBjPair * kBjPair / 2; e += blockDim.x) {
+          const int i = e >> 4, j = (e & 15) * 2;
+          bj_copy2(&t0[i][j], Mp + (int64_t)idx_s[0][i] * mp + idx_s[1][j]);
+          bj_copy2(&t1[i][j], Qp + (int64_t)a * (kBjPair * kBjPair) + i * kBjPair + j);
+          bj_copy2(&t2[i][j], Qp + (int64_t)c * (kBjPair * kBjPair) + i * kBjPair + j);
+        }
+        __syncthreads();
+        const int rt = warp & 3, c0 = (warp >> 2) * kBjBlock;
+        {
+          double acc[2][2];
+          bj_strip<false, 2>(t0, t2, rt, c0, acc);   // Y = X Q_c
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            *reinterpret_cast<double2 *>(&t3[8 * rt + gq][c0 + 8 * t + 2 * qq]) = make_double2(acc[t][0], acc[t][1]);
+        }
+        __syncthreads();
+        {
+          double acc[2][2];
+          bj_strip<true, 2>(t1, t3, rt, c0, acc);    // Z = Q_a^T Y
+          const int i = 8 * rt + gq;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int j = c0 + 8 * t + 2 * qq;
+            *reinterpret_cast<double2 *>(Mp + (int64_t)idx_s[0][i] * mp + idx_s[1][j]) =
+                make_double2(acc[t][0], acc[t][1]);
+            Mp[(int64_t)idx_s[1][j] * mp + idx_s[0][i]] = acc[t][0];
+            Mp[(int64_t)idx_s[1][j + 1] * mp + idx_s[0][i]] = acc[t][1];
           }
         }
-      }
-      __syncthreads();
-      if (threadIdx.x == 0 && rot_s) {
-        atomicAdd(&ctl->rot[sweep], 1u);
-        rot_s = 0;
+        __syncthreads();   // tiles reused by the next item
       }
       if (!basis_grid_sync(ctl, ++gen, &flag_s)) return;
     }
     converged = *(volatile uint32_t *)&ctl->rot[sweep] == 0u;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    ctl->final_buf = round & 1u;
-    if (!converged) set_status(&ctl->status, kDevStatusCheck);
-  }
+  if (blockIdx.x == 0 && tid == 0 && !converged) set_status(&ctl->status, kDevStatusCheck);
+  if (g > 0) bj_rows_items(bs, V, Qg + ((g - 1) & 1) * qbuf, ctl, g - 1, (g - 1) % rps, t0, t1, t2, idx_s, &tk_s);
 }
 
 // 4. Order of the eigenvalues (decreasing, lower index first on ties), the
@@ -383,8 +548,8 @@ __global__ void __launch_bounds__(1024) basis_order_kernel(BasisShape bs, const 
                                                            double *__restrict__ sigma_out, BasisCtl *ctl) {
   __shared__ double lam_s[S4R_MAX_D_MODEL];
   const int p = blockIdx.x, m = bs.m;
-  const double *Mf = M + ((int64_t)p * 2 + ctl->final_buf) * m * m;
-  for (int i = threadIdx.x; i < m; i += blockDim.x) lam_s[i] = Mf[(int64_t)i * m + i];
+  const double *Mf = M + (int64_t)p * bs.mp * bs.mp;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) lam_s[i] = Mf[(int64_t)i * bs.mp + i];
   __syncthreads();
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
     const double li = lam_s[i];
@@ -417,15 +582,15 @@ __global__ void __launch_bounds__(256) basis_columns_kernel(BasisShape bs, const
                                                             const double *__restrict__ inv,
                                                             const double *__restrict__ V,
                                                             const int32_t *__restrict__ order,
-                                                            const double *__restrict__ sig, const BasisCtl *ctl,
+                                                            const double *__restrict__ sig,
                                                             double *__restrict__ Bw) {
   __shared__ double a_s[32][33], u_s[32][33];
   __shared__ int ord_s[32];
   const int p = blockIdx.z;
   const int d0 = blockIdx.y * 32, k0 = blockIdx.x * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int m = bs.m;
-  const double *Vp = V + ((int64_t)p * 2 + ctl->final_buf) * m * m;   // V^T, rows in slot order
+  const int m = bs.m, mp = bs.mp;
+  const double *Vp = V + (int64_t)p * mp * mp;   // V^T: row i is the eigenvector of M[i][i]
   if (threadIdx.x < 32) ord_s[threadIdx.x] = (k0 + threadIdx.x < bs.r) ? order[(int64_t)p * bs.r + k0 + threadIdx.x] : 0;
   __syncthreads();
   double *Bp = Bw + (int64_t)p * bs.D * bs.r;
@@ -433,7 +598,7 @@ __global__ void __launch_bounds__(256) basis_columns_kernel(BasisShape bs, const
     for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
       const int dd = e >> 5, kk = e & 31;
       const int d = d0 + dd, k = k0 + kk;
-      if (d < bs.D && k < bs.r) Bp[(int64_t)d * bs.r + k] = Vp[(int64_t)ord_s[kk] * m + d];
+      if (d < bs.D && k < bs.r) Bp[(int64_t)d * bs.r + k] = Vp[(int64_t)ord_s[kk] * mp + d];
     }
     return;
   }
@@ -444,7 +609,7 @@ __global__ void __launch_bounds__(256) basis_columns_kernel(BasisShape bs, const
     for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
       const int hi = e >> 5, lo = e & 31;
       a_s[lo][hi] = basis_a(bs, states, rows_p, inv_p, p, j0 + hi, d0 + lo);     // consecutive threads walk d
-      u_s[lo][hi] = (j0 + lo < m && k0 + hi < bs.r) ? Vp[(int64_t)ord_s[hi] * m + j0 + lo] : 0.0;   // ... and j
+      u_s[lo][hi] = (j0 + lo < m && k0 + hi < bs.r) ? Vp[(int64_t)ord_s[hi] * mp + j0 + lo] : 0.0;   // ... and j
     }
     __syncthreads();
 #pragma unroll 8

@@ -701,7 +701,7 @@ s4r_status decode_launch(const s4r_decode_args *a, const Shape &s, const Layout 
 
 // ---- prefill bases
 struct BasisLayout {
-  size_t ctl, rows, inv, M, V, order, sig, Bw, total;
+  size_t ctl, rows, inv, M, V, Q, order, sig, Bw, total;
 };
 
 s4r_status basis_shape(const s4r_basis_args *a, BasisShape *bs) {
@@ -721,20 +721,22 @@ s4r_status basis_shape(const s4r_basis_args *a, BasisShape *bs) {
   bs->t_side = a->n_sample <= a->d_model ? 1 : 0;
   const int mm = bs->t_side ? a->n_sample : a->d_model;
   bs->m = (mm + 1) & ~1;
+  bs->mp = (mm + 31) & ~31;
   bs->state_rows = a->state_rows;
   return S4R_OK;
 }
 
 BasisLayout basis_layout(const BasisShape &bs) {
   BasisLayout l;
-  const size_t P = (size_t)bs.P, m = (size_t)bs.m;
+  const size_t P = (size_t)bs.P, mp = (size_t)bs.mp;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off += round_up(bytes); return o; };
   l.ctl = take(sizeof(BasisCtl));
   l.rows = take(P * bs.T * sizeof(int64_t));
   l.inv = take(P * bs.T * sizeof(double));
-  l.M = take(P * 2 * m * m * sizeof(double));
-  l.V = take(P * 2 * m * m * sizeof(double));
+  l.M = take(P * mp * mp * sizeof(double));
+  l.V = take(P * mp * mp * sizeof(double));
+  l.Q = take(2 * P * (mp / 32) * 32 * 32 * sizeof(double));
   l.order = take(P * bs.r * sizeof(int32_t));
   l.sig = take(P * bs.r * sizeof(double));
   l.Bw = take(P * bs.D * bs.r * sizeof(double));
@@ -750,6 +752,7 @@ s4r_status basis_launch(const s4r_basis_args *a, const BasisShape &bs, const Bas
   double *inv = reinterpret_cast<double *>(ws + ly.inv);
   double *M = reinterpret_cast<double *>(ws + ly.M);
   double *V = reinterpret_cast<double *>(ws + ly.V);
+  double *Q = reinterpret_cast<double *>(ws + ly.Q);
   int32_t *order = reinterpret_cast<int32_t *>(ws + ly.order);
   double *sig = reinterpret_cast<double *>(ws + ly.sig);
   double *Bw = reinterpret_cast<double *>(ws + ly.Bw);
@@ -757,30 +760,31 @@ s4r_status basis_launch(const s4r_basis_args *a, const BasisShape &bs, const Bas
   const unsigned P = (unsigned)bs.P;
   basis_prep_kernel<T><<<dim3((unsigned)ceil_div(bs.T, 8), P), 256, 0, st>>>(bs, a->lengths, states, rows, inv, ctl);
   if (check_launch("basis_prep_kernel") != S4R_OK) return S4R_ERR_CUDA;
-  const unsigned mt = (unsigned)ceil_div(bs.m, 32);
+  const unsigned mt = (unsigned)(bs.mp / 32);
   basis_gram_kernel<T><<<dim3(mt, mt, P), 256, 0, st>>>(bs, states, rows, inv, M, V);
   if (check_launch("basis_gram_kernel") != S4R_OK) return S4R_ERR_CUDA;
   {
-    // One cooperative grid for the Jacobi rounds of every problem.
+    // One cooperative grid for the block Jacobi rounds of every problem.
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, basis_jacobi_kernel, 256, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, basis_jacobi_kernel, kBjThreads, 0) != cudaSuccess ||
         per_sm < 1)
       return fail("basis_jacobi_kernel occupancy", cudaGetLastError());
-    const int64_t h = bs.m / 2;
-    const int64_t work = (int64_t)bs.P * (h * (h + 1) / 2 + (int64_t)bs.m * h);
-    const int64_t want = ceil_div(work, (int64_t)256);
+    const int64_t npb = bs.mp / 32;
+    const int64_t items_a = (int64_t)bs.P * npb;
+    const int64_t items_b = (int64_t)bs.P * (npb * (npb - 1) / 2 + npb * ((npb + 1) / 2));
+    const int64_t want = items_a > items_b ? items_a : items_b;
     const int64_t cap = (int64_t)per_sm * sm_count();
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
     BasisShape bsv = bs;
-    void *kargs[] = {&bsv, &M, &V, &ctl};
+    void *kargs[] = {&bsv, &M, &V, &Q, &ctl};
     const cudaError_t err = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(basis_jacobi_kernel),
-                                                        dim3(grid), dim3(256), kargs, 0, st);
+                                                        dim3(grid), dim3(kBjThreads), kargs, 0, st);
     if (err != cudaSuccess) return fail("basis_jacobi_kernel (cooperative launch)", err);
   }
   basis_order_kernel<<<P, 1024, 0, st>>>(bs, M, order, sig, a->sigma, ctl);
   if (check_launch("basis_order_kernel") != S4R_OK) return S4R_ERR_CUDA;
   basis_columns_kernel<T><<<dim3((unsigned)ceil_div(bs.r, 32), (unsigned)ceil_div(bs.D, 32), P), 256, 0, st>>>(
-      bs, states, rows, inv, V, order, sig, ctl, Bw);
+      bs, states, rows, inv, V, order, sig, Bw);
   if (check_launch("basis_columns_kernel") != S4R_OK) return S4R_ERR_CUDA;
   basis_output_kernel<T><<<dim3((unsigned)bs.r, P), 256, 0, st>>>(bs, Bw, a->basis_f64,
                                                                    static_cast<T *>(a->basis_out));

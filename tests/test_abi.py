@@ -158,11 +158,11 @@ def basis_good(**over):
 
 def test_basis_workspace_bytes_and_validation():
     n = s4r.s4r_basis_workspace_bytes(basis_good())
-    # Gram of the 256 sampled rows: two buffers of it and two of its eigenvectors per problem, plus
-    # the fp64 columns, in fp64
-    assert n >= 4 * (4 * 256 * 256 + 1024 * 192) * 8 and n % 256 == 0
+    # Gram of the 256 sampled rows and its eigenvectors per problem, two buffers of the 32 x 32
+    # rotations of its 8 block pairs, plus the fp64 columns, in fp64
+    assert n >= 4 * (2 * 256 * 256 + 2 * 8 * 32 * 32 + 1024 * 192) * 8 and n % 256 == 0
     # more samples than D': the Gram of the 1024 columns instead
-    assert s4r.s4r_basis_workspace_bytes(basis_good(n_sample=2048)) >= 4 * 4 * 1024 * 1024 * 8
+    assert s4r.s4r_basis_workspace_bytes(basis_good(n_sample=2048)) >= 4 * 2 * 1024 * 1024 * 8
     for bad in (dict(rank=0), dict(rank=257, n_sample=300), dict(rank=300, n_sample=200), dict(dtype=7),
                 dict(d_model=0), dict(n_sample=0), dict(n_problems=-1), dict(d_model=2048),
                 dict(n_sink=-1), dict(state_rows=-5)):
