@@ -71,6 +71,13 @@ def test_llama_shape_L32k_one_layer():
         _run(make_batch(W1, lengths=[32768 - 4], layer=3, step=step))
 
 
+def test_llama_shape_L32k_two_problems_one_call():
+    """Two full-size 32K problems in one call (the shape of the
+    all-layers-in-one-call variant): the row-split attention with 16-CTA
+    clusters at full size."""
+    _run(make_batch(W1, lengths=[32768 - 4, 32768 - 4], layer=5))
+
+
 def test_batched_16x8k():
     _run(make_batch(W2, lengths=[8192 - 4] * 16, layer=1))
 
@@ -136,8 +143,11 @@ def test_ranks_off_the_tensor_core_tiles(rank_k, rank_v):
 
 
 def test_many_selected_rows_take_several_chunks():
-    # k + w large enough that a CTA of the attention cluster stages its rows
-    # in more than one pass (rank 256 shrinks the staging capacity).
+    # k + w large enough that a CTA of the row-split attention cluster (two
+    # problems per call) stages its rows in more than one pass (rank 256
+    # shrinks the staging capacity); the single problem takes the per-group
+    # kernel with the same selection size.
+    _run(make_batch(W3, lengths=[40000, 36000], top_k=3000, local_window=512, tag="chunks"))
     _run(make_batch(W3, lengths=[40000], top_k=3000, local_window=512, tag="chunks"))
 
 
