@@ -99,7 +99,7 @@ struct StcControl {
   uint64_t full[kStcMaxStages], empty[kStcMaxStages];
   uint64_t b_full[2][4], b_empty[2];           // per operand buffer: each 64-column k-block landed / buffer free
   uint64_t acc_full;                         // MMA -> epilogue: the tile's accumulators are complete
-  uint64_t scratch_free;                     // epilogue -> MMA: (mid, lo) columns read
+  uint64_t scratch_free;                     // epilogue warps -> MMA: (mid, lo) columns read
   uint64_t slot_free[StcCfg<R>::kSlots];     // epilogue -> MMA: the slot may be overwritten
   uint64_t mma_final;                        // every MMA of the CTA has completed (teardown)
   uint32_t tmem_base;
@@ -113,6 +113,7 @@ struct StcControl {
   float alpha[StcCfg<R>::kRetained][R];      // per kept slot, of the problem being finished
   float sc_part[StcCfg<R>::kHalves == 2 ? StcCfg<R>::kRetained : 1][kStcTile];   // rows 32-63's part of a score
   double inv_l[R];                           // 1 / l of the problem in pass 2
+  float alpha2[R];                           // 2^k / l of the tile in pass 2
   double inv_q[StcCfg<R>::kRetained + 1][R]; // 1 / l of the problems the watcher saw complete (ring)
   int ok_q[StcCfg<R>::kRetained + 1];
   int pend[StcCfg<R>::kRetained + 1];        // problems arrived on, not yet finished (FIFO)
@@ -299,7 +300,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       mbar_init(&ctl->b_empty[i], 1);
     }
     mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->scratch_free, 1);
+    mbar_init(&ctl->scratch_free, Cfg::kEpiWarps);   // one arrival per epilogue warp
     for (int i = 0; i < Cfg::kSlots; ++i) mbar_init(&ctl->slot_free[i], 1);
     mbar_init(&ctl->mma_final, 1);
     ctl->abort = 0;
@@ -676,20 +677,22 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
         tmem_ld32(tmem + lane_base + (uint32_t)(Cfg::kScratchCol + rh), mid);
         tmem_ld32(tmem + lane_base + (uint32_t)(Cfg::kScratchCol + R + rh), lo);
         tmem_wait_ld();
+        // This warp's reads of the (mid, lo) columns are done: the next
+        // tile's MMAs may overwrite them once every epilogue warp says so.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->scratch_free);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           y[j] = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
           amax = fmaxf(amax, fabsf(y[j]));
         }
       }
-      // One barrier: the accumulators are read (the scratch, and a transient
-      // slot, may take the next tile's MMAs), and the range check's vote.
+      // One barrier: the hi columns are read (a transient slot may take the
+      // next tile's MMAs), and the range check's vote.
       tc_fence_before();
       const bool wide = epi_or<EN>(valid && amax > kStcRangeLimit);
-      if (ep == 0) {
-        mbar_arrive(&ctl->scratch_free);
-        if (!kept) mbar_arrive(&ctl->slot_free[slot]);
-      }
+      if (ep == 0 && !kept) mbar_arrive(&ctl->slot_free[slot]);
       ++n_tile;
       if (kept) ++j_ret; else ++u_tr;
       const int rb = (int)(n_tile & 1);   // partial-sum buffer of this tile
@@ -718,10 +721,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
       // y now holds e.
       if (t.pass2) {
         // Second pass: the problem is finished; score straight from e with
-        // alpha_row = 2^k / l_row (each thread forms its 32 rows' factors).
+        // alpha_row = 2^k / l_row, formed once per row and tile.
+        if (ep < R) ctl->alpha2[ep] = (float)ldexp(ctl->inv_l[ep], wide ? ctl->kofs[ep] : 0);
+        epi_sync<EN>();
         float a = 0.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) a = fmaf((float)ldexp(ctl->inv_l[rh + j], wide ? ctl->kofs[rh + j] : 0), y[j], a);
+        for (int j = 0; j < 32; ++j) a = fmaf(ctl->alpha2[rh + j], y[j], a);
         if (Cfg::kHalves == 2) {
           if (half == 1) ctl->sc_part[0][pos] = a;
           epi_sync<EN>();
@@ -731,7 +736,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const int3
           if (valid) scores[(int64_t)t.p * s.cache_rows + i] = a;
           hist_add(t.p, t.L, a, i < t.L - s.local_window);
         }
-        epi_sync<EN>();   // inv_l and sc_part may be rewritten for the next tile
+        epi_sync<EN>();   // inv_l, alpha2 and sc_part may be rewritten for the next tile
         continue;
       }
       if (kept) {
