@@ -44,6 +44,7 @@ struct SrControl {
   int pad;
   float part[4][32];    // per-warp row sums (pass 1) or maxima (wide tiles)
   int kofs[32];         // offsets of the current 32 rows
+  float alpha[32];      // pass 2: 2^k / l of the current 32 rows
   double inv_l[S4R_MAX_SCORE_ROWS];   // pass 2: 1 / l of every row
 };
 __host__ __device__ constexpr int sr_smem_bytes(int r, int nB) {
@@ -180,12 +181,16 @@ score_rows_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
           if (threadIdx.x < 32) {
             const float m = fmaxf(fmaxf(ctl->part[0][lane], ctl->part[1][lane]), fmaxf(ctl->part[2][lane], ctl->part[3][lane]));
             ctl->kofs[lane] = (m == -INFINITY) ? 0 : (int)floorf(m);
+            if (PASS == 2) ctl->alpha[lane] = (float)ldexp(ctl->inv_l[c * kSrRc + h * 32 + lane], ctl->kofs[lane]);
           }
           epi_sync<kSrEpi>();
 #pragma unroll
           for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j] - (float)ctl->kofs[j]) : 0.f;
         } else {
-          if (threadIdx.x < 32) ctl->kofs[lane] = 0;
+          if (threadIdx.x < 32) {
+            ctl->kofs[lane] = 0;
+            if (PASS == 2) ctl->alpha[lane] = (float)ctl->inv_l[c * kSrRc + h * 32 + lane];
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j]) : 0.f;
           epi_sync<kSrEpi>();
@@ -205,10 +210,10 @@ score_rows_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
         } else {
           float a = 0.f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) a = fmaf((float)ldexp(ctl->inv_l[row0 + j], ctl->kofs[j]), y[j], a);
+          for (int j = 0; j < 32; ++j) a = fmaf(ctl->alpha[j], y[j], a);   // 2^k_j / l_j, formed once per row
           score += a;
         }
-        epi_sync<kSrEpi>();   // part and kofs are rewritten by the next rows
+        epi_sync<kSrEpi>();   // part, kofs and alpha are rewritten by the next rows
       }
       // The accumulator buffer has been read.
       tc_fence_before();
