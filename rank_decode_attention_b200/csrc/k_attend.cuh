@@ -408,8 +408,9 @@ attend_kernel(Shape s, AttPlan pl, const int32_t *__restrict__ lengths, const in
     }
     __syncthreads();
     if (tc_acc) {
-      // Split weights into the B operand, then one m16n8k16 per (tile, 16 entries).
-      for (int t = threadIdx.x; t < 16 * E; t += blockDim.x) {
+      // Split weights into the B operand (the 8 n_nt columns the products
+      // read), then one m16n8k16 per (tile, 16 entries).
+      for (int t = threadIdx.x; t < 8 * n_nt * E; t += blockDim.x) {
         const int n = t / E, e = t - n * E, j = n >> 1;
         const float pv_ = j < G ? p_s[e * kAttMaxGroup + j] : 0.f;
         const float hi = __bfloat162float(__float2bfloat16_rn(pv_));
