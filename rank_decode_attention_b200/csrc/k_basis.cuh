@@ -359,8 +359,7 @@ __device__ __forceinline__ void bj_rows_items(const BasisShape &bs, double *V, c
 //   grid barrier.
 // The eigenvector rows of the last round follow the last sweep.  A 2 x 2
 // block of an inner round is only read and written by the thread that owns
-// it (the upper one, mirrored into the lower), so S stays exactly
-// symmetric and needs no second buffer.
+// it, and S is kept in its upper triangle, so it needs no second buffer.
 __global__ void __launch_bounds__(kBjThreads) basis_jacobi_kernel(BasisShape bs, double *__restrict__ M,
                                                                   double *__restrict__ V, double *__restrict__ Qg,
                                                                   BasisCtl *ctl) {
@@ -425,8 +424,16 @@ __global__ void __launch_bounds__(kBjThreads) basis_jacobi_kernel(BasisShape bs,
           if (tid < kBjBlock) {
             double c, sn;
             bool bg;
-            const double t = jacobi_angle(&t0[0][0], kBjLd, sched_s[kk][2 * tid], sched_s[kk][2 * tid + 1], c, sn,
-                                          bg);
+            // S holds its upper triangle: a pair listed as (x, y) with x > y
+            // is solved as (y, x), whose theta, t and s are the negatives of
+            // those of (x, y) (the same rotation J).
+            const int x = sched_s[kk][2 * tid], y = sched_s[kk][2 * tid + 1];
+            double t = x < y ? jacobi_angle(&t0[0][0], kBjLd, x, y, c, sn, bg)
+                             : jacobi_angle(&t0[0][0], kBjLd, y, x, c, sn, bg);
+            if (x > y) {
+              t = -t;
+              sn = -sn;
+            }
             c_s[tid] = c;
             s_s[tid] = sn;
             tt_s[tid] = t;
@@ -436,32 +443,29 @@ __global__ void __launch_bounds__(kBjThreads) basis_jacobi_kernel(BasisShape bs,
           if (tid < kBjBlock * (kBjBlock + 1) / 2) {
             const int ab = ut_s[tid], ea = ab >> 4, ec = ab & 15;
             const int pa = sched_s[kk][2 * ea], qa = sched_s[kk][2 * ea + 1];
+            // S is kept in its upper triangle: entry (i, j) lives at
+            // (min, max).
+            auto up = [&](int i, int j) -> double & { return i < j ? t0[i][j] : t0[j][i]; };
             if (ea == ec) {
               const double t = tt_s[ea];
               if (t != 0.0) {
-                const double apq = t0[pa][qa];
+                double &apq = up(pa, qa);
                 t0[pa][pa] -= t * apq;
                 t0[qa][qa] += t * apq;
-                t0[pa][qa] = 0.0;
-                t0[qa][pa] = 0.0;
+                apq = 0.0;
               }
             } else {
               const int pc = sched_s[kk][2 * ec], qc = sched_s[kk][2 * ec + 1];
               const double ca = c_s[ea], sa = s_s[ea], cb = c_s[ec], sb = s_s[ec];
-              const double x00 = t0[pa][pc], x01 = t0[pa][qc], x10 = t0[qa][pc], x11 = t0[qa][qc];
+              double &e00 = up(pa, pc), &e01 = up(pa, qc), &e10 = up(qa, pc), &e11 = up(qa, qc);
+              const double x00 = e00, x01 = e01, x10 = e10, x11 = e11;
               // y = R_a^T x, then z = y R_c, R = [[c, s], [-s, c]].
               const double y00 = ca * x00 - sa * x10, y01 = ca * x01 - sa * x11;
               const double y10 = sa * x00 + ca * x10, y11 = sa * x01 + ca * x11;
-              const double z00 = y00 * cb - y01 * sb, z01 = y00 * sb + y01 * cb;
-              const double z10 = y10 * cb - y11 * sb, z11 = y10 * sb + y11 * cb;
-              t0[pa][pc] = z00;
-              t0[pa][qc] = z01;
-              t0[qa][pc] = z10;
-              t0[qa][qc] = z11;
-              t0[pc][pa] = z00;
-              t0[qc][pa] = z01;
-              t0[pc][qa] = z10;
-              t0[qc][qa] = z11;
+              e00 = y00 * cb - y01 * sb;
+              e01 = y00 * sb + y01 * cb;
+              e10 = y10 * cb - y11 * sb;
+              e11 = y10 * sb + y11 * cb;
             }
           }
           {
@@ -483,7 +487,8 @@ __global__ void __launch_bounds__(kBjThreads) basis_jacobi_kernel(BasisShape bs,
         double *Qp = Qcur + ((int64_t)p * npb + a) * (kBjPair * kBjPair);
         for (int e = tid; e < kBjPair * kBjPair / 2; e += blockDim.x) {
           const int i = e >> 4, j = (e & 15) * 2;
-          bj_copy2(Mp + (int64_t)idx_s[0][i] * mp + idx_s[0][j], &t0[i][j]);
+          const double v0 = i <= j ? t0[i][j] : t0[j][i], v1 = i <= j + 1 ? t0[i][j + 1] : t0[j + 1][i];
+          *reinterpret_cast<double2 *>(Mp + (int64_t)idx_s[0][i] * mp + idx_s[0][j]) = make_double2(v0, v1);
           bj_copy2(Qp + i * kBjPair + j, &t1[i][j]);
         }
         if (__syncthreads_or(big) && tid == 0) atomicAdd(&ctl->rot[sweep], 1u);   // also frees the tiles

@@ -91,6 +91,8 @@ CASES = [
     # Gram of the columns when T' > D'
     ("tiny-columns", synth.F32, 2, [2048, 1500], 128, 32, 32, 4, 256),
     ("full-width-columns", synth.BF16, 1, [4096], 64, 16, 64, 4, 300),
+    # the largest Gram matrix: D' = 1024 columns, 64 index blocks, 63 block rounds per sweep
+    ("max-gram-columns", synth.BF16, 1, [4096], 1024, 64, 256, 4, 2048),
 ]
 
 
