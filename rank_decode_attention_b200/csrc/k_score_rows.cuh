@@ -16,14 +16,15 @@
 // tile cannot be kept until the row normalisers are known.  Hence two
 // passes, each one CTA per 128-position tile:
 //   pass 1  per chunk: MMA (three N = 64 products) into one of two TMEM
-//           buffers while the epilogue reduces the previous chunk; per-row
-//           sums of e over the tile (a transposing warp butterfly, then the
-//           four warps in a fixed order) added in fp64 to the row's 16 slots;
+//           buffers while the epilogue reduces the previous chunk (its two
+//           32-row halves side by side, four warps each); per-row sums of e
+//           over the tile (a transposing warp butterfly, then the four warps
+//           in a fixed order) added in fp64 to the row's 16 slots;
 //   finish  1 / l_row = 1 / (sum of the row's slots, fixed order);
 //   pass 2  the same MMAs and e (the same offsets: the same y), and
 //           score = sum over the chunks and rows of e * 2^k / l_row;
 //           the level-0 histogram of the candidates' scores for the top-k.
-// One thread of the fifth warp issues the TMA copy of the tile (kept for
+// One thread of the ninth warp issues the TMA copy of the tile (kept for
 // every chunk), the chunks' operand copies (two buffers when they fit) and
 // the MMAs.
 #pragma once
@@ -32,7 +33,8 @@
 namespace s4r {
 
 constexpr int kSrRc = 64;           // scoring rows per chunk
-constexpr int kSrEpi = 128;         // epilogue threads (4 warps, one TMEM lane quadrant each)
+constexpr int kSrHalf = 128;        // epilogue threads of one 32-row half of a chunk (4 warps, one TMEM lane quadrant each)
+constexpr int kSrEpi = 2 * kSrHalf; // epilogue threads: warp w reads lane quadrant w % 4 and rows of half w / 4
 constexpr int kSrThreads = kSrEpi + 32;
 constexpr int kSrAccCols = 256;     // TMEM columns per accumulator buffer (hi, mid, lo at +0, +64, +128)
 
@@ -42,9 +44,10 @@ struct SrControl {
   uint64_t a_full, b_full[2], b_empty[2], acc_full[2], acc_empty[2];
   uint32_t tmem_base;
   int pad;
-  float part[4][32];    // per-warp row sums (pass 1) or maxima (wide tiles)
-  int kofs[32];         // offsets of the current 32 rows
-  float alpha[32];      // pass 2: 2^k / l of the current 32 rows
+  float part[2][4][32]; // per half and warp: row sums (pass 1) or maxima (wide tiles)
+  int kofs[2][32];      // per half: offsets of its current 32 rows
+  float alpha[2][32];   // pass 2, per half: 2^k / l of its current 32 rows
+  float sc2[kStcTile];  // pass 2: the second half's part of each position's score
   double inv_l[S4R_MAX_SCORE_ROWS];   // pass 2: 1 / l of every row
 };
 __host__ __device__ constexpr int sr_smem_bytes(int r, int nB) {
@@ -52,6 +55,21 @@ __host__ __device__ constexpr int sr_smem_bytes(int r, int nB) {
 }
 // Operand buffers: two when they fit.
 __host__ __device__ constexpr int sr_buffers(int r) { return sr_smem_bytes(r, 2) <= kStcMaxSmem ? 2 : 1; }
+
+// Named barrier `id` over n threads, and its OR-reduction of a predicate.
+__device__ __forceinline__ void sr_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ bool sr_or(int id, int n, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return out != 0;
+}
 
 template <int PASS>
 __global__ void __launch_bounds__(kSrThreads, 1)
@@ -92,7 +110,7 @@ score_rows_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
       mbar_init(&ctl->b_full[q], 1);
       mbar_init(&ctl->b_empty[q], 1);
       mbar_init(&ctl->acc_full[q], 1);
-      mbar_init(&ctl->acc_empty[q], 4);   // one arrival per epilogue warp
+      mbar_init(&ctl->acc_empty[q], kSrEpi / 32);   // one arrival per epilogue warp
     }
     mbar_fence_init();
     const int32_t row0 = (int32_t)((int64_t)b * s.cache_rows + (int64_t)tile * kStcTile);
@@ -142,91 +160,100 @@ score_rows_kernel(const __grid_constant__ CUtensorMap tmap_ck, Shape s, const in
       }
     }
   } else if (epi) {
-    const int p = threadIdx.x;                                // position within the tile
+    // Warp w: TMEM lane quadrant w % 4 (positions), rows 32 h .. 32 h + 31 of
+    // every 64-row chunk (h = w / 4); each half has its own named barrier.
+    const int quarter = warp & 3, h = warp >> 2, bid = 1 + h;
+    const int p = quarter * 32 + lane;                        // position within the tile
     const int64_t pos = (int64_t)tile * kStcTile + p;
     const bool valid = pos < L;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int slot = tile % kStcSumSlots;
     float score = 0.f;
     bool ok = true;
     for (int c = 0; c < nch; ++c) {
       const int d = c & 1;
+      const int row0 = c * kSrRc + h * 32;
       ok = mbar_wait(&ctl->acc_full[d], (c / 2) & 1, status) && ok;
       tc_fence_after();
-      for (int h = 0; h < 2; ++h) {   // rows 64c + 32h .. + 31
-        float y[32];
-        float amax = 0.f;
-        {
-          uint32_t hi[32], mid[32], lo[32];
-          const uint32_t col = tmem + lane_base + (uint32_t)(d * kSrAccCols + h * 32);
-          tmem_ld32(col, hi);
-          tmem_ld32(col + kSrRc, mid);
-          tmem_ld32(col + 2 * kSrRc, lo);
-          tmem_wait_ld();
+      float y[32];
+      float amax = 0.f;
+      {
+        uint32_t hi[32], mid[32], lo[32];
+        const uint32_t col = tmem + lane_base + (uint32_t)(d * kSrAccCols + h * 32);
+        tmem_ld32(col, hi);
+        tmem_ld32(col + kSrRc, mid);
+        tmem_ld32(col + 2 * kSrRc, lo);
+        tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            y[j] = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
-            amax = fmaxf(amax, fabsf(y[j]));
-          }
+        for (int j = 0; j < 32; ++j) {
+          y[j] = (__uint_as_float(lo[j]) + __uint_as_float(mid[j])) + __uint_as_float(hi[j]);
+          amax = fmaxf(amax, fabsf(y[j]));
         }
-        const bool wide = epi_or<kSrEpi>(valid && amax > kStcRangeLimit);
-        if (wide) {
-          // k_row = floor(max over the tile's valid positions of y_row)
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = valid ? y[j] : -INFINITY;
-          warp_transpose_reduce32<true>(v);
-          ctl->part[warp][lane] = v[0];
-          epi_sync<kSrEpi>();
-          if (threadIdx.x < 32) {
-            const float m = fmaxf(fmaxf(ctl->part[0][lane], ctl->part[1][lane]), fmaxf(ctl->part[2][lane], ctl->part[3][lane]));
-            ctl->kofs[lane] = (m == -INFINITY) ? 0 : (int)floorf(m);
-            if (PASS == 2) ctl->alpha[lane] = (float)ldexp(ctl->inv_l[c * kSrRc + h * 32 + lane], ctl->kofs[lane]);
-          }
-          epi_sync<kSrEpi>();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j] - (float)ctl->kofs[j]) : 0.f;
-        } else {
-          if (threadIdx.x < 32) {
-            ctl->kofs[lane] = 0;
-            if (PASS == 2) ctl->alpha[lane] = (float)ctl->inv_l[c * kSrRc + h * 32 + lane];
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j]) : 0.f;
-          epi_sync<kSrEpi>();
-        }
-        // y holds e.
-        const int row0 = c * kSrRc + h * 32;
-        if (PASS == 1) {
-          warp_transpose_reduce32<false>(y);
-          ctl->part[warp][lane] = y[0];
-          epi_sync<kSrEpi>();
-          if (threadIdx.x < 32) {
-            const float l = (ctl->part[0][lane] + ctl->part[1][lane]) + (ctl->part[2][lane] + ctl->part[3][lane]);
-            const int row = row0 + lane;
-            if (row < s.n_rows && l != 0.f)
-              atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + slot) * R + row], ldexp((double)l, ctl->kofs[lane]));
-          }
-        } else {
-          float a = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) a = fmaf(ctl->alpha[j], y[j], a);   // 2^k_j / l_j, formed once per row
-          score += a;
-        }
-        epi_sync<kSrEpi>();   // part, kofs and alpha are rewritten by the next rows
       }
-      // The accumulator buffer has been read.
+      // This warp has read its part of the accumulator buffer.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->acc_empty[d]);
+      const bool wide = sr_or(bid, kSrHalf, valid && amax > kStcRangeLimit);
+      if (wide) {
+        // k_row = floor(max over the tile's valid positions of y_row)
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = valid ? y[j] : -INFINITY;
+        warp_transpose_reduce32<true>(v);
+        ctl->part[h][quarter][lane] = v[0];
+        sr_bar(bid, kSrHalf);
+        if (quarter == 0) {
+          const float m = fmaxf(fmaxf(ctl->part[h][0][lane], ctl->part[h][1][lane]),
+                                fmaxf(ctl->part[h][2][lane], ctl->part[h][3][lane]));
+          ctl->kofs[h][lane] = (m == -INFINITY) ? 0 : (int)floorf(m);
+          if (PASS == 2) ctl->alpha[h][lane] = (float)ldexp(ctl->inv_l[row0 + lane], ctl->kofs[h][lane]);
+        }
+        sr_bar(bid, kSrHalf);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j] - (float)ctl->kofs[h][j]) : 0.f;
+      } else {
+        if (quarter == 0) {
+          ctl->kofs[h][lane] = 0;
+          if (PASS == 2) ctl->alpha[h][lane] = (float)ctl->inv_l[row0 + lane];
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = valid ? ex2_approx(y[j]) : 0.f;
+        sr_bar(bid, kSrHalf);
+      }
+      // y holds e.
+      if (PASS == 1) {
+        warp_transpose_reduce32<false>(y);
+        ctl->part[h][quarter][lane] = y[0];
+        sr_bar(bid, kSrHalf);
+        if (quarter == 0) {
+          const float l = (ctl->part[h][0][lane] + ctl->part[h][1][lane]) + (ctl->part[h][2][lane] + ctl->part[h][3][lane]);
+          const int row = row0 + lane;
+          if (row < s.n_rows && l != 0.f)
+            atomicAdd(&row_sum[((int64_t)b * kStcSumSlots + slot) * R + row], ldexp((double)l, ctl->kofs[h][lane]));
+        }
+      } else {
+        float a = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a = fmaf(ctl->alpha[h][j], y[j], a);   // 2^k_j / l_j, formed once per row
+        score += a;
+      }
+      sr_bar(bid, kSrHalf);   // part, kofs and alpha of this half are rewritten by the next chunk
     }
-    if (PASS == 2 && ok) {
-      if (valid) scores[(int64_t)b * s.cache_rows + pos] = score;
-      const int64_t n_cand = L > s.local_window ? L - s.local_window : 0;
-      const bool cand = pos < n_cand;
-      const uint32_t bin = cand ? (uint32_t)score_bin(__float_as_uint(score), score_center(s.n_rows, L)) : 0xffffffffu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (cand && lane == __ffs(peers) - 1) atomicAdd(&ehist[(int64_t)b * kExpBins + bin], (uint32_t)__popc(peers));
+    if (PASS == 2) {
+      // The two halves' parts of a position's score meet once; the write
+      // needs both halves' waits to have succeeded.
+      if (h == 1) ctl->sc2[p] = score;
+      const bool any_bad = sr_or(3, kSrEpi, !ok);
+      if (h == 0 && !any_bad) {
+        score += ctl->sc2[p];
+        if (valid) scores[(int64_t)b * s.cache_rows + pos] = score;
+        const int64_t n_cand = L > s.local_window ? L - s.local_window : 0;
+        const bool cand = pos < n_cand;
+        const uint32_t bin = cand ? (uint32_t)score_bin(__float_as_uint(score), score_center(s.n_rows, L)) : 0xffffffffu;
+        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        if (cand && lane == __ffs(peers) - 1) atomicAdd(&ehist[(int64_t)b * kExpBins + bin], (uint32_t)__popc(peers));
+      }
     }
   }
   tc_fence_before();
