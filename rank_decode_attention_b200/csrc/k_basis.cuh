@@ -270,8 +270,24 @@ constexpr int kBjCross0 = kBjBlock - 1;
 
 // Global index of local index l (< 32) of block pair a in round k with nb
 // blocks: l < 16 in the block of slot 2a, the others in that of slot 2a+1.
-__device__ __forceinline__ int bj_index(int nb, int k, int a, int l) {
+__host__ __device__ __forceinline__ int bj_index(int nb, int k, int a, int l) {
   return jac_player(nb, k, 2 * a + (l >> 4)) * kBjBlock + (l & (kBjBlock - 1));
+}
+
+// Index pair u (< 16) of inner round kk (< 31) of a 32 x 32 submatrix whose
+// first 16 local indices are block I and the others block J: rounds
+// 0 .. 14 pair the indices inside the blocks (a round-robin of 16 on each,
+// pairs 0-7 in I, 8-15 in J), rounds 15 .. 30 pair i in I with
+// 16 + (i + r) mod 16 in J (r = kk - 15).
+__host__ __device__ __forceinline__ void bj_inner_pair(int kk, int u, int &x, int &y) {
+  if (kk < kBjCross0) {
+    const int off = u < 8 ? 0 : kBjBlock, w = u & 7;
+    x = off + jac_player(kBjBlock, kk, 2 * w);
+    y = off + jac_player(kBjBlock, kk, 2 * w + 1);
+  } else {
+    x = u;
+    y = kBjBlock + (u + kk - kBjCross0) % kBjBlock;
+  }
 }
 
 // One m8n8k4 fp64 tensor-core product, {d0, d1} += a b, in the PTX
@@ -382,14 +398,7 @@ __global__ void __launch_bounds__(kBjThreads) basis_jacobi_kernel(BasisShape bs,
   for (int e = tid; e < kBjInner * kBjBlock; e += blockDim.x) {
     const int kk = e / kBjBlock, u = e % kBjBlock;
     int x, y;
-    if (kk < kBjCross0) {   // inside the blocks: pairs 0..7 in I, 8..15 in J
-      const int off = u < 8 ? 0 : kBjBlock, w = u & 7;
-      x = off + jac_player(kBjBlock, kk, 2 * w);
-      y = off + jac_player(kBjBlock, kk, 2 * w + 1);
-    } else {                // across: i with 16 + (i + r) mod 16
-      x = u;
-      y = kBjBlock + (u + kk - kBjCross0) % kBjBlock;
-    }
+    bj_inner_pair(kk, u, x, y);
     sched_s[kk][2 * u] = (unsigned char)x;
     sched_s[kk][2 * u + 1] = (unsigned char)y;
   }
