@@ -441,7 +441,14 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   p.tc = true;
   p.R = R;
   p.grid = (int)smin<int64_t>(tiles, sm_count());
-  p.K = tiles > 2 * (int64_t)p.grid ? 2 : 1;
+  // Chunks of one tile balance the CTAs best (at most ceil(tiles / G) each,
+  // so the fewest tiles beyond the kept ones); when problems are shorter
+  // than the grid, chunks of two keep each CTA on fewer problems, which
+  // waits less for problems to complete before kept slots free up.
+  // (Measured: 128K 329 -> 352 steps/s, ragged +2%, 32 x 32K in one call +3%
+  // with one-tile chunks; 16 x 8K 314 with two-tile chunks, 289 with one.)
+  const bool short_problems = ceil_div(s.cache_rows, kStcTile) < (int64_t)p.grid;
+  p.K = (tiles > 2 * (int64_t)p.grid && short_problems) ? 2 : 1;
   p.nB = nB;
   p.smem = smem;
   return p;
