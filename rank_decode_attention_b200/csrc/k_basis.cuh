@@ -22,14 +22,16 @@
 // method.  The Gram matrix is padded with zeros to mp = m rounded up to 32
 // and its indices are cut into nb = mp / 16 blocks of 16; in each round the
 // blocks meet in disjoint pairs (round-robin order, every pair of blocks
-// once in nb - 1 rounds).  A round first applies, for every pair, one
-// cyclic Jacobi sweep to the 32 x 32 principal submatrix on its indices in
-// shared memory (Rutishauser's rotations, parallel order over its 16 index
-// pairs), keeping the product Q of its rotations; then every off-diagonal
+// once in nb - 1 rounds).  A round first rotates, for every pair, the
+// 32 x 32 principal submatrix on its indices in shared memory by parallel
+// inner rounds of 16 Rutishauser rotations (in the first round of an outer
+// sweep all 31 rounds, inside each block and across the two; in the others
+// the 16 across, so every index pair meets once per outer sweep), keeping
+// the product Q of its rotations; then every off-diagonal
 // 32 x 32 tile becomes Q_a^T M[a][c] Q_c and the eigenvector rows of the
 // pair become Q_a^T V^T[a].  Matrix and eigenvectors stay in natural index
-// order and are updated in place.  Rounds are separated by a grid-wide
-// barrier of one cooperative launch.  The outer sweep in which no rotation
+// order and are updated in place.  The phases of a round are separated by
+// grid-wide barriers of one cooperative launch.  The outer sweep in which no rotation
 // meets an off-diagonal entry above 1e-8 of its diagonal scale is the last
 // one: its rotations leave them near their squares.
 // Near the rank cut the eigenvalues of the workloads' samples differ by
@@ -364,8 +366,8 @@ __device__ __forceinline__ void bj_rows_items(const BasisShape &bs, double *V, c
 // 3. Block Jacobi sweeps for every problem (cooperative launch).  M and V^T
 // are [P][mp][mp]; Qg holds two buffers [P][mp / 32][32][32] of the pair
 // rotations, round g writing buffer g & 1.  Round g (round k of its sweep):
-//   phase 1, items (problem, pair a): load S = M[a][a], rotate it by one
-//      sweep of inner rounds, accumulate Q_a = J_1 J_2 ..., write S back
+//   phase 1, items (problem, pair a): load S = M[a][a], rotate it by its
+//      inner rounds, accumulate Q_a = J_1 J_2 ..., write S back
 //      into M[a][a] and Q_a; a CTA done with its items then takes the
 //      eigenvector rows of round g - 1 from their ticket counter (they are
 //      needed by nothing before the end);
