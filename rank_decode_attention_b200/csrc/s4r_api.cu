@@ -446,7 +446,7 @@ ScorePlan plan_scoring(const Shape &s, s4r_dtype dt) {
   // than the grid, chunks of two keep each CTA on fewer problems, which
   // waits less for problems to complete before kept slots free up.
   // (Measured: 128K 329 -> 352 steps/s, ragged +2%, 32 x 32K in one call +3%
-  // with one-tile chunks; 16 x 8K 314 with two-tile chunks, 289 with one.)
+  // with one-tile chunks; 16 x 8K 314 with two-tile chunks, 289 with one, 308 with four.)
   const bool short_problems = ceil_div(s.cache_rows, kStcTile) < (int64_t)p.grid;
   p.K = (tiles > 2 * (int64_t)p.grid && short_problems) ? 2 : 1;
   p.nB = nB;
