@@ -152,7 +152,7 @@ struct StcWalker {
   bool have_next;        // lookahead tile present
   int64_t g_next;
 
-  __device__ void start(const int32_t *len, int64_t cap_, int batch_, int G_, int c_, int K_, int kept_) {
+  __host__ __device__ void start(const int32_t *len, int64_t cap_, int batch_, int G_, int c_, int K_, int kept_) {
     lengths = len;
     cap = cap_;
     batch = batch_;
@@ -163,7 +163,7 @@ struct StcWalker {
     pass = 1;
     rewind();
   }
-  __device__ void rewind() {
+  __host__ __device__ void rewind() {
     p = -1;
     T = 0;
     S = 0;
@@ -172,7 +172,7 @@ struct StcWalker {
     g = (int64_t)c * K;
     g_next = raw_next();
   }
-  __device__ int64_t raw_next() {
+  __host__ __device__ int64_t raw_next() {
     if (g >= gc * K + K) {
       gc += G;
       g = gc * K;
@@ -181,20 +181,24 @@ struct StcWalker {
   }
   // Move the problem cursor forward to the problem holding global tile gt;
   // false when gt lies past the last problem.
-  __device__ bool locate(int64_t gt) {
+  __host__ __device__ bool locate(int64_t gt) {
     while (gt >= S + T) {
       S += T;
       ++p;
       T = 0;
       k = 0;
       if (p >= batch) return false;
+#ifdef __CUDA_ARCH__
       const int64_t Lraw = __ldg(lengths + p);
+#else
+      const int64_t Lraw = lengths[p];
+#endif
       L = (Lraw >= 0 && Lraw <= cap) ? Lraw : 0;
       T = (int)ceil_div(L, kStcTile);
     }
     return true;
   }
-  __device__ bool next(StcTile &t) {
+  __host__ __device__ bool next(StcTile &t) {
     while (true) {
       const int64_t gt = g_next;
       const int p_before = p;
@@ -222,7 +226,7 @@ struct StcWalker {
 
 // CTAs that own tiles of a problem whose tiles are global tiles [S, S + T):
 // the chunks intersecting it, at most G.
-__device__ __forceinline__ int stc_participants(int64_t S, int T, int K, int G) {
+__host__ __device__ __forceinline__ int stc_participants(int64_t S, int T, int K, int G) {
   const int64_t n = (S + T - 1) / K - S / K + 1;
   return (int)(n < G ? n : G);
 }
