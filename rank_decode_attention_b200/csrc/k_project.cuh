@@ -90,15 +90,17 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
   constexpr int V = Vec16<T>::n;
   const int rank = (int)blockIdx.x, n_rank = (int)gridDim.x, cb = blockIdx.y;
   // Programmatic launch: this kernel may start while the previous decode
-  // call's attention kernel still runs.  That kernel reads qt (and, through
-  // its predecessors, the rest of this workspace had been released before
-  // it started), so only the writes of cq / cqs / qt wait for it.  A CTA that
-  // projects a single kv group computes before waiting; one with several
-  // waits first.  The next kernel (scoring) only reads caller inputs before
-  // its own wait, so it may be released right away.
+  // call's attention kernel still runs, but only once every CTA of it has
+  // passed its own wait and trigger.  Both attention kernels read qt only
+  // before that point, and every other buffer written here was last read by
+  // kernels that completed before the attention kernel passed its wait; so
+  // this kernel writes without waiting.  It still waits at its end: its
+  // completion then implies the attention kernel's, so the next kernels of
+  // this call (the top-k writes idx, which that attention kernel reads) are
+  // ordered after it.  The next kernel (scoring) only reads caller inputs
+  // before its own wait, so it may be released right away.
   const bool early = (s.n_heads_kv - rank + n_rank - 1) / n_rank <= 1;
   pdl_trigger();
-  if (!early) pdl_wait();
   const int n_rb = (int)ceil_div((int64_t)s.query_window * s.group, kProjRowBlock);
   const int rb = blockIdx.z % n_rb, b = blockIdx.z / n_rb;
   const int G = s.group, W = s.query_window, Hq = s.n_heads_q, dh = s.head_dim, r = s.rank_k;
@@ -224,10 +226,7 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
     }
     cluster_sync();  // rank 0 has read every partial
   }
-  if (early) {
-    pdl_wait();
-    proj_head_writes(s, keep, g_keep, b, pr0, c0, scale, cq, blk, qt);
-  }
+  if (early) proj_head_writes(s, keep, g_keep, b, pr0, c0, scale, cq, blk, qt);
   if (s.row_mode == S4R_ROWS_CONCAT && rank == 0)
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -238,6 +237,7 @@ project_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ basis_k, 
         if (row < W * G) proj_finish(c < r ? x[i][jj] * scale : 0.0, b, R, r, row, c, kk, cq, blk, (int64_t)s.batch * stc_b_bytes(R, r));
       }
     }
+  pdl_wait();   // complete only after the previous call's attention kernel (see above)
 }
 
 }  // namespace s4r
