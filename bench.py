@@ -147,8 +147,8 @@ def source_sha(paths) -> str:
 def profiled(kernel: str, workload: str):
     """ncu figures of one kernel on one workload from the committed summary
     (profiles/traffic.json): DRAM bytes per launch and the serialised launch
-    duration, each only while the kernel's sources are unchanged since the
-    capture (else None)."""
+    duration, each only while the sources the entry lists (the kernel's and
+    the launch plan's) are unchanged since the capture (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None, None
